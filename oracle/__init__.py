@@ -65,12 +65,12 @@ def lib():
             L.oracle_compress_regions.restype = None
             L.oracle_compress_regions.argtypes = [
                 _P(ctypes.c_uint16), ctypes.c_int64, _P(ctypes.c_int64), _P(ctypes.c_int64),
-                ctypes.c_int, _P(ctypes.c_uint8), _P(ctypes.c_float)]
+                ctypes.c_int, ctypes.c_int64, _P(ctypes.c_uint8), _P(ctypes.c_float)]
             L.oracle_indexer_scores.restype = None
             L.oracle_indexer_scores.argtypes = [
                 _P(ctypes.c_uint16), _P(ctypes.c_float), _P(ctypes.c_int32), _P(ctypes.c_int32),
                 ctypes.c_int, _P(ctypes.c_uint8), _P(ctypes.c_float), _P(ctypes.c_int64),
-                _P(ctypes.c_float), ctypes.c_int64, ctypes.c_uint32]
+                ctypes.c_int64, _P(ctypes.c_float), ctypes.c_int64, ctypes.c_uint32]
             L.oracle_topk_regions.restype = None
             L.oracle_topk_regions.argtypes = [
                 _P(ctypes.c_float), ctypes.c_int64, _P(ctypes.c_int32), ctypes.c_int, ctypes.c_int,
@@ -139,8 +139,9 @@ def get_threads() -> int:
 
 def compress_regions(index_k_bits, src_row, dst_slot, n_slots, summaries=None, scales=None):
     """index_k_bits: uint16 [tokens][4][256] (bf16 bit patterns, rows may be a 2-D
-    [tokens][row_stride] view).  Returns (summaries uint8 [n_slots][4][256],
-    scales float32 [n_slots][4]); untouched slots stay as passed (zeros by default)."""
+    [tokens][row_stride] view).  Returns the group-major pool (summaries uint8
+    [4][n_slots][256], scales float32 [4][n_slots]); untouched slots stay as passed
+    (zeros by default)."""
     k = _arr(index_k_bits, np.uint16)
     row_stride = int(np.prod(k.shape[1:]))
     src = _arr(np.asarray(src_row, np.int64), np.int64)
@@ -150,10 +151,12 @@ def compress_regions(index_k_bits, src_row, dst_slot, n_slots, summaries=None, s
         raise ValueError("src_row out of range")
     if n and (dst.min() < 0 or dst.max() >= n_slots):
         raise ValueError("dst_slot out of range")
-    S = np.zeros((n_slots, G, DI), np.uint8) if summaries is None else _arr(summaries, np.uint8)
-    C = np.zeros((n_slots, G), np.float32) if scales is None else _arr(scales, np.float32)
+    S = np.zeros((G, n_slots, DI), np.uint8) if summaries is None else _arr(summaries, np.uint8)
+    C = np.zeros((G, n_slots), np.float32) if scales is None else _arr(scales, np.float32)
+    if S.shape != (G, n_slots, DI) or C.shape != (G, n_slots):
+        raise ValueError("pool shape must be [4][n_slots][256] / [4][n_slots]")
     lib().oracle_compress_regions(_ptr(k, ctypes.c_uint16), row_stride, _ptr(src, ctypes.c_int64),
-                                  _ptr(dst, ctypes.c_int64), n, _ptr(S, ctypes.c_uint8),
+                                  _ptr(dst, ctypes.c_int64), n, int(n_slots), _ptr(S, ctypes.c_uint8),
                                   _ptr(C, ctypes.c_float))
     return S, C
 
@@ -169,20 +172,23 @@ def indexer_scores(index_q_bits, gate, q_req, q_pos, summaries, scales, sum_base
     S = _arr(summaries, np.uint8)
     C = _arr(scales, np.float32)
     base = _arr(np.asarray(sum_base, np.int64), np.int64)
+    if S.ndim != 3 or S.shape[0] != G or S.shape[2] != DI or C.shape != S.shape[:2]:
+        raise ValueError("pool shape must be [4][n_slots][256] / [4][n_slots]")
+    n_slots = int(S.shape[1])
     own = qp // REGION
     if ld is None:
         ld = max(1, int(own.max()) if nq else 1)
     if nq and int(own.max()) > ld:
         raise ValueError("ld smaller than the largest own-region index")
     for i in range(nq):
-        if own[i] > 0 and base[qr[i]] + own[i] > S.shape[0]:
+        if own[i] > 0 and base[qr[i]] + own[i] > n_slots:
             raise ValueError("summary slots out of range")
     out = np.full((nq, G, ld), fill, np.float32)
     lib().oracle_indexer_scores(_ptr(q, ctypes.c_uint16), _ptr(z, ctypes.c_float),
                                 _ptr(qr, ctypes.c_int32), _ptr(qp, ctypes.c_int32), nq,
                                 _ptr(S, ctypes.c_uint8), _ptr(C, ctypes.c_float),
-                                _ptr(base, ctypes.c_int64), _ptr(out, ctypes.c_float), int(ld),
-                                int(flags))
+                                _ptr(base, ctypes.c_int64), n_slots, _ptr(out, ctypes.c_float),
+                                int(ld), int(flags))
     return out
 
 

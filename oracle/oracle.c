@@ -169,10 +169,11 @@ static void compress_one(const uint16_t *const rows[OR_REGION], uint8_t *code, f
 
 /* index_k: bf16 token rows, row t of group g at index_k[t*row_stride + g*256 + i].
  * Region i is made of rows src_row[i] .. src_row[i]+7 and is written to pool slot
- * dst_slot[i]: summaries[(slot*4 + g)*256 + i], scales[slot*4 + g]. */
+ * dst_slot[i] of every group: the pool is group-major, summaries[(g*n_slots + slot)*256 + i],
+ * scales[g*n_slots + slot]. */
 void oracle_compress_regions(const uint16_t *index_k, int64_t row_stride,
                              const int64_t *src_row, const int64_t *dst_slot, int n_regions,
-                             uint8_t *summaries, float *scales)
+                             int64_t n_slots, uint8_t *summaries, float *scales)
 {
 #pragma omp parallel for schedule(static)
     for (int i = 0; i < n_regions; ++i) {
@@ -181,7 +182,8 @@ void oracle_compress_regions(const uint16_t *index_k, int64_t row_stride,
             for (int t = 0; t < OR_REGION; ++t)
                 rows[t] = index_k + (src_row[i] + t) * row_stride + (int64_t)g * OR_DI;
             int64_t slot = dst_slot[i];
-            compress_one(rows, summaries + (slot * OR_G + g) * OR_DI, scales + slot * OR_G + g);
+            compress_one(rows, summaries + ((int64_t)g * n_slots + slot) * OR_DI,
+                         scales + (int64_t)g * n_slots + slot);
         }
     }
 }
@@ -218,7 +220,7 @@ static void quantise_q_head(const uint16_t *qh, double *out)
 void oracle_indexer_scores(const uint16_t *index_q, const float *gate,
                            const int32_t *q_req, const int32_t *q_pos, int nq,
                            const uint8_t *summaries, const float *scales, const int64_t *sum_base,
-                           float *scores, int64_t ld, uint32_t flags)
+                           int64_t n_slots, float *scores, int64_t ld, uint32_t flags)
 {
     double *qd = (double *)malloc(sizeof(double) * (size_t)nq * OR_HI * OR_DI);
     for (int qi = 0; qi < nq; ++qi)
@@ -235,8 +237,8 @@ void oracle_indexer_scores(const uint16_t *index_q, const float *gate,
 #pragma omp parallel for schedule(static)
             for (int64_t r = 0; r < own; ++r) {
                 int64_t slot = base + r;
-                const uint8_t *s8 = summaries + (slot * OR_G + g) * OR_DI;
-                double sc = (double)scales[slot * OR_G + g];
+                const uint8_t *s8 = summaries + ((int64_t)g * n_slots + slot) * OR_DI;
+                double sc = (double)scales[(int64_t)g * n_slots + slot];
                 double acc = 0.0;
                 for (int h = OR_G * g; h < OR_G * g + OR_G; ++h) {
                     const double *qh = qd + ((int64_t)qi * OR_HI + h) * OR_DI;

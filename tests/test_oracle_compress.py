@@ -34,10 +34,12 @@ def rand_bf16(rng, shape, scale=1.0):
 
 
 def compress(tokens_bits, n_regions=None):
-    """tokens [T][4][256] -> summaries/scales of regions 0..T/8-1 in slots 0..."""
+    """tokens [T][4][256] -> summaries [r][g][256] / scales [r][g] of regions 0..T/8-1
+    (the oracle's group-major pool, transposed to region-major for indexing here)."""
     T = tokens_bits.shape[0]
     n = T // 8 if n_regions is None else n_regions
-    return oracle.compress_regions(tokens_bits, [8 * r for r in range(n)], list(range(n)), n)
+    S, C = oracle.compress_regions(tokens_bits, [8 * r for r in range(n)], list(range(n)), n)
+    return S.transpose(1, 0, 2), C.T
 
 
 def test_rows_of_region_r_are_8r_to_8r_plus_7():
@@ -130,6 +132,7 @@ def test_strided_rows_and_scattered_slots():
     Sa, Ca = oracle.compress_regions(wide, [0, 8, 24], [5, 0, 2], 7)
     Sb, Cb = oracle.compress_regions(x, [0, 8, 24], [5, 0, 2], 7)
     assert np.array_equal(Sa, Sb) and np.array_equal(Ca, Cb)
+    Sa, Ca = Sa.transpose(1, 0, 2), Ca.T
     Sr, Cr = compress(x)
     assert np.array_equal(Sa[5], Sr[0]) and np.array_equal(Sa[0], Sr[1]) and np.array_equal(Sa[2], Sr[3])
     for s in (1, 3, 4, 6):

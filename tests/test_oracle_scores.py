@@ -29,10 +29,16 @@ def rand_bf16(rng, shape):
 
 
 def one_hot_pool(n_slots, j=0, c=448.0 * 2 ** -6):
-    """Pool whose every summary is c * e_j exactly: code 0x7E at j, scale c/448."""
-    S = np.zeros((n_slots, G, DI), np.uint8)
+    """Group-major pool whose every summary is c * e_j exactly: code 0x7E at j, scale c/448."""
+    S = np.zeros((G, n_slots, DI), np.uint8)
     S[:, :, j] = 0x7E
-    C = np.full((n_slots, G), np.float32(c / 448.0), np.float32)
+    C = np.full((G, n_slots), np.float32(c / 448.0), np.float32)
+    return S, C
+
+
+def random_pool(rng, n_slots, lo=0, hi=0x7E):
+    S = rng.integers(lo, hi, (G, n_slots, DI), dtype=np.uint8)
+    C = rng.uniform(0.001, 0.01, (G, n_slots)).astype(np.float32)
     return S, C
 
 
@@ -75,8 +81,7 @@ def test_head_to_group_map():
 def test_only_regions_before_the_own_region_are_scored():
     rng = np.random.default_rng(0)
     n = 10
-    S = rng.integers(0, 0x7E, (n, G, DI), dtype=np.uint8)
-    C = rng.uniform(0.001, 0.01, (n, G)).astype(np.float32)
+    S, C = random_pool(rng, n)
     q = rand_bf16(rng, (3, HI, DI))
     z = rng.uniform(0, 1, (3, HI)).astype(np.float32)
     pos = [0, 23, 79]                          # own regions 0, 2, 9
@@ -89,20 +94,18 @@ def test_only_regions_before_the_own_region_are_scored():
 
 def test_request_base_selects_the_request_slots():
     rng = np.random.default_rng(1)
-    S = rng.integers(0, 0x7E, (12, G, DI), dtype=np.uint8)
-    C = rng.uniform(0.001, 0.01, (12, G)).astype(np.float32)
+    S, C = random_pool(rng, 12)
     q = rand_bf16(rng, (1, HI, DI))
     z = rng.uniform(0, 1, (1, HI)).astype(np.float32)
     a = oracle.indexer_scores(q, z, [1], [40], S, C, [0, 7])      # request 1: slots 7..11
-    b = oracle.indexer_scores(q, z, [0], [40], S[7:], C[7:], [0])
+    b = oracle.indexer_scores(q, z, [0], [40], S[:, 7:], C[:, 7:], [0])
     assert np.array_equal(a, b)
 
 
 def test_exact_scalings():
     # doubling every gate, or every query, doubles every score exactly (powers of two)
     rng = np.random.default_rng(2)
-    S = rng.integers(0, 0x7E, (6, G, DI), dtype=np.uint8)
-    C = rng.uniform(0.001, 0.01, (6, G)).astype(np.float32)
+    S, C = random_pool(rng, 6)
     q = rand_bf16(rng, (1, HI, DI))
     z = rng.uniform(0, 1, (1, HI)).astype(np.float32)
     s0 = oracle.indexer_scores(q, z, [0], [48], S, C, [0])
@@ -116,18 +119,17 @@ def test_brute_force_from_library_decode():
     # decoded with ml_dtypes, evaluated with numpy float64 einsum
     rng = np.random.default_rng(3)
     n, nq = 33, 4
-    S = rng.integers(0, 256, (n, G, DI), dtype=np.uint8)
+    S, C = random_pool(rng, n, 0, 256)
     S[(S & 0x7F) == 0x7F] = 0x11               # no NaN codes
-    C = rng.uniform(0.001, 0.01, (n, G)).astype(np.float32)
     q = rand_bf16(rng, (nq, HI, DI))
     z = rng.uniform(0, 1, (nq, HI)).astype(np.float32)
     pos = [8 * n + 1, 70, 8, 200]
     sc = oracle.indexer_scores(q, z, [0] * nq, pos, S, C, [0], ld=n)
-    s = S.view(ml_dtypes.float8_e4m3fn).astype(np.float64) * C[..., None].astype(np.float64)
+    s = S.view(ml_dtypes.float8_e4m3fn).astype(np.float64) * C[..., None].astype(np.float64)  # [g][r][d]
     qd = f64(q)
     for i in range(nq):
         own = pos[i] // 8
-        dots = np.einsum("hd,rgd->rgh", qd[i], s)               # [r][g][h]
+        dots = np.einsum("hd,grd->rgh", qd[i], s)               # [r][g][h]
         for g in range(G):
             h = np.arange(4 * g, 4 * g + 4)
             ref = (np.maximum(dots[:own, g, h], 0) * z[i, h]).sum(axis=1) / 16
@@ -142,8 +144,7 @@ def test_fp8_query_mode_is_exact_for_representable_queries():
     codes[..., 0] = 0x7E                      # absmax code 448 in every head
     vals = codes.view(ml_dtypes.float8_e4m3fn).astype(np.float32) * np.float32(2.0 ** -5)
     q = bits_of(vals)
-    S = rng.integers(0, 0x7E, (5, G, DI), dtype=np.uint8)
-    C = rng.uniform(0.001, 0.01, (5, G)).astype(np.float32)
+    S, C = random_pool(rng, 5)
     z = rng.uniform(0, 1, (1, HI)).astype(np.float32)
     a = oracle.indexer_scores(q, z, [0], [40], S, C, [0], flags=0)
     b = oracle.indexer_scores(q, z, [0], [40], S, C, [0], flags=oracle.Q_FP8)
