@@ -1,0 +1,411 @@
+#!/usr/bin/env python
+"""DSA decode benchmark: queries/s at 1M-token context on B200 (one JSON line).
+
+A step is one decode query through one DSA layer: compress the region the new token
+completes, score every complete region with the 16-head indexer, select the own region
+plus the top-511, and attend 64 query heads over the selected regions' K/V (4,096 tokens
+per KV group).  Workload (default): one request, L = 1,048,576 tokens, k = 512, paged
+K/V with a random page permutation, all inputs seeded synthetic N(0,1) bf16 / U(0,1).
+Four independent layer caches (each 128 MiB of summaries + 3 GiB of K/V) are used round
+robin, so consecutive steps never find their inputs in the 126 MB L2.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+--gpus N > 1 (under torchrun): every rank runs an independent replica (requests shard
+across GPUs with no data-path collective, weak scaling); timing is the max over ranks.
+--impl reference times the CPU oracle (the only other arm this method has) on the host.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "DSA decode queries/s @1M ctx; indexer+attn HBM GB/s vs B200 peak"
+UNIT = "queries/s"
+L_CTX = 1 << 20
+TOPK = 512
+N_LAYERS = 4
+KERNELS_PER_STEP = 7      # compress, scan, top-k hist/gather/final, attention, combine
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--layers", type=int, default=N_LAYERS)
+    ap.add_argument("--cpu-queries", type=int, default=3, help="oracle queries timed for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def scan_bytes(own: int) -> int:
+    """Algorithmic bytes of one indexer scan: e4m3 summaries + fp32 scales of every
+    eligible region, 4 groups."""
+    return 4 * own * (256 + 4)
+
+
+def step_bytes(own: int, k: int) -> int:
+    """Algorithmic bytes of one decode step at position L-1: scan + selected K/V (4 groups
+    x k regions x 8 tokens x 768 B) + index_q/gate + Q/O + the compressed region."""
+    kv = 4 * min(k, own + 1) * 8 * 2 * 192 * 2
+    return scan_bytes(own) + kv + 16 * 256 * 2 + 16 * 4 + 2 * 64 * 192 * 2 + 4 * 8 * 256 * 2 + 4 * 260
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML every 10 ms in a thread."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, cuda_index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            from cuda.bindings import runtime as rt
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            # NVML enumerates every GPU of the host: find ours by PCI bus id
+            bus = rt.cudaDeviceGetPCIBusId(64, cuda_index)[1]
+            bus = bus.split(b"\x00")[0].decode() if isinstance(bus, bytes) else str(bus)
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            self.sample()
+            time.sleep(0.01)
+
+    def sample(self):
+        if self.nv is None:
+            return
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            self.raw_reasons = getattr(self, "raw_reasons", 0) | int(r)
+            for bit, name in self.REASONS.items():
+                if r & bit and name != "gpu_idle":
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
+    def __enter__(self):
+        self.sample()
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        self._t.join()
+        self.sample()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+# ------------------------------------------------------------------ CPU oracle arm
+
+def oracle_inputs(seed: int, device):
+    """Host copies of one layer cache for the oracle (index_k, K/V, queries)."""
+    import numpy as np
+    import torch
+    from sparse_long_context_dsa_b200 import workloads as W
+
+    d = W.decode_batch([L_CTX], seed=seed, device=device, permute=True)
+
+    def bits(t):
+        return t.cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    host = {k: bits(d[k]) for k in ("index_k", "index_q", "q", "k_cache", "v_cache")}
+    host["gate"] = d["gate"].cpu().numpy()
+    host["block_table"] = d["block_table"].cpu().numpy()
+    host["q_pos"] = d["q_pos"].cpu().numpy()
+    host["n_slots"] = d["n_slots"]
+    del d
+    return host
+
+
+def oracle_time(host, n_queries: int):
+    """Times n oracle decode steps (compress the due region, score, select, attend)."""
+    import numpy as np
+    import oracle
+
+    own = (L_CTX - 1) // 8
+    src = [8 * r for r in range(own)]
+    S, C = oracle.compress_regions(host["index_k"], src, list(range(own)), host["n_slots"])
+    t0 = time.perf_counter()
+    for _ in range(n_queries):
+        oracle.compress_regions(host["index_k"], [8 * own], [own], host["n_slots"], S, C)
+        sc = oracle.indexer_scores(host["index_q"], host["gate"], [0], host["q_pos"], S, C, [0], ld=own)
+        idx, cnt = oracle.topk_regions(np.nan_to_num(sc), host["q_pos"], TOPK)
+        oracle.sparse_attention(host["q"], host["k_cache"], host["v_cache"], host["block_table"], [0],
+                                host["q_pos"], idx, cnt)
+    dt = time.perf_counter() - t0
+    return n_queries / dt, oracle.get_threads(), dt
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import torch
+    dev = torch.device("cuda", 0) if torch.cuda.is_available() else torch.device("cpu")
+    host = oracle_inputs(1237, dev)
+    oracle_time(host, 1 if args.warmup > 0 else 0) if args.warmup > 0 else None
+    qps, cores, dt = oracle_time(host, args.steps)
+    line = {"impl": "reference", "metric": METRIC, "value": qps, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": "decode_b1_1m", "context": L_CTX, "topk": TOPK},
+            "cpu_baseline": {"kind": "oracle", "value": qps, "unit": UNIT, "cores": cores,
+                             "sample": f"{args.steps} decode queries at 1M context, one layer cache"},
+            "e2e": {"value": qps, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def build_layers(n_layers, seed0, device):
+    import torch
+    from sparse_long_context_dsa_b200 import pipeline
+    from sparse_long_context_dsa_b200 import workloads as W
+
+    layers = []
+    for l in range(n_layers):
+        d = W.decode_batch([L_CTX], seed=seed0 + 1000 * l, device=device, permute=True)
+        n_slots = d["n_slots"]
+        S = torch.zeros((4, n_slots, 256), dtype=torch.uint8, device=device)
+        C = torch.zeros((4, n_slots), dtype=torch.float32, device=device)
+        pipeline.compress_all(d["index_k"], [L_CTX - 1], [0], d["sum_base"], S, C)
+        tail = d["index_k"][L_CTX - 8:].clone()            # the region this step completes
+        del d["index_k"]
+        torch.cuda.empty_cache()
+        own = (L_CTX - 1) // 8
+        step = pipeline.DecodeStep(S, C, d["sum_base"], d["block_table"], d["k_cache"], d["v_cache"], ld=own,
+                                   k=TOPK, max_compress=1, index_k=tail)
+        src = torch.zeros(1, dtype=torch.int64, device=device)
+        dst = torch.full((1,), own, dtype=torch.int64, device=device)
+        step.load(d["index_q"], d["gate"], d["q"], d["q_pos"], src, dst)
+        layers.append(dict(step=step, inputs=d, tail=tail))
+    torch.cuda.synchronize()
+    return layers
+
+
+def record_external(event, stream_handle: int):
+    """cudaEventRecordWithFlags(..., External): inside a stream capture this becomes an
+    event-record node, so each replay timestamps the event."""
+    from cuda.bindings import runtime as rt
+    err = rt.cudaEventRecordWithFlags(event, rt.cudaStream_t(stream_handle), int(rt.cudaEventRecordExternal))[0]
+    if err != rt.cudaError_t.cudaSuccess:
+        raise RuntimeError(f"cudaEventRecordWithFlags failed: {err}")
+
+
+def capture(layers, n_steps, ev_pairs=None, e2e=None):
+    """One CUDA graph of n_steps decode steps, layer i % len(layers) at step i.
+    ev_pairs: list of (start, end) raw cudaEvent_t recorded (external) around each scan.
+    e2e: per-layer pinned host buffers; copies in/out are captured around each step."""
+    import torch
+    from cuda.bindings import runtime as rt
+
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            raw = torch.cuda.current_stream().cuda_stream
+            for i in range(n_steps):
+                L = layers[i % len(layers)]
+                st = L["step"]
+                if e2e is not None:
+                    h = e2e[i % len(layers)]
+                    st.index_q.copy_(h["index_q"], non_blocking=True)
+                    st.gate.copy_(h["gate"], non_blocking=True)
+                    st.q.copy_(h["q"], non_blocking=True)
+                    st.q_pos.copy_(h["q_pos"], non_blocking=True)
+                    L["tail"].copy_(h["tail"], non_blocking=True)
+                pre = post = None
+                if ev_pairs is not None:
+                    a, b = ev_pairs[i]
+                    pre = lambda a=a: record_external(a, raw)
+                    post = lambda b=b: record_external(b, raw)
+                st.run(pre_scan=pre, post_scan=post)
+                if e2e is not None:
+                    e2e[i % len(layers)]["out"].copy_(st.out, non_blocking=True)
+    torch.cuda.current_stream().wait_stream(s)
+    return g
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from cuda.bindings import runtime as rt
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from sparse_long_context_dsa_b200 import dsa
+    dsa.lib()
+
+    layers = build_layers(args.layers, seed0=1237 + 7919 * rank, device=dev)
+    own = (L_CTX - 1) // 8
+    for L in layers:                 # one eager step per layer before any capture
+        L["step"].run()
+    dsa.check_device()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---- warm-up graph and timed graph(s); each graph holds at most 250 steps
+    chunk = min(args.steps, 250)
+    n_full, rem = divmod(args.steps, chunk)
+    evs = [(rt.cudaEventCreate()[1], rt.cudaEventCreate()[1]) for _ in range(chunk)]
+    g_warm = capture(layers, max(args.warmup, 3))
+    g_main = capture(layers, chunk, ev_pairs=evs)
+    g_tail = capture(layers, rem) if rem else None
+    for _ in range(2):
+        g_warm.replay()
+    dsa.check_device()
+    torch.cuda.synchronize()
+
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        start.record()
+        for _ in range(n_full):
+            g_main.replay()
+        if g_tail is not None:
+            g_tail.replay()
+        end.record()
+        torch.cuda.synchronize()
+    barrier()
+    ms = start.elapsed_time(end)
+    ms = max_over_ranks(ms)
+    scan_ms = [rt.cudaEventElapsedTime(a, b)[1] for a, b in evs]
+    scan_avg_ms = max_over_ranks(sum(scan_ms) / len(scan_ms))
+    dsa.check_device()
+
+    # ---- e2e: host (pinned) inputs in, result out, every step
+    e2e_bufs = []
+    for L in layers:
+        st, d = L["step"], L["inputs"]
+        e2e_bufs.append(dict(index_q=d["index_q"].cpu().pin_memory(), gate=d["gate"].cpu().pin_memory(),
+                             q=d["q"].cpu().pin_memory(), q_pos=d["q_pos"].cpu().pin_memory(),
+                             tail=L["tail"].cpu().pin_memory(),
+                             out=torch.empty_like(st.out, device="cpu").pin_memory()))
+    h2d = sum(t.numel() * t.element_size() for k, t in e2e_bufs[0].items() if k != "out")
+    d2h = e2e_bufs[0]["out"].numel() * e2e_bufs[0]["out"].element_size()
+    g_e2e = capture(layers, chunk, e2e=e2e_bufs)
+    g_e2e_tail = capture(layers, rem, e2e=e2e_bufs) if rem else None
+    g_e2e.replay()
+    torch.cuda.synchronize()
+    barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(n_full):
+        g_e2e.replay()
+    if g_e2e_tail is not None:
+        g_e2e_tail.replay()
+    t1.record()
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(t0.elapsed_time(t1))
+    dsa.check_device()
+    # e2e results must equal the device-resident results (same inputs)
+    assert torch.equal(e2e_bufs[0]["out"], layers[0]["step"].out.cpu())
+
+    hbm, peak_kind = peaks()
+    qps = world * args.steps / (ms / 1e3)
+    scan_gbs = scan_bytes(own) / (scan_avg_ms / 1e3) / 1e9
+    step_gbs = step_bytes(own, TOPK) * args.steps / (ms / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": qps, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3+bf16 (fp32 accumulate)", "data": "synthetic",
+        "config": {"workload": "decode_b1_1m", "context": L_CTX, "topk": TOPK, "batch_per_gpu": 1,
+                   "layer_caches": args.layers,
+                   "l2": f"inputs larger than L2: {args.layers} layer caches of "
+                         f"{scan_bytes(own) / 1e6:.0f} MB summaries + 3 GiB K/V used round robin",
+                   "graph": "each step captured in a CUDA graph"},
+        "step_hbm_gbs": step_gbs,
+        "roofline": {"kernel": "indexer scan (scan_kernel)", "bound": "hbm", "achieved": scan_gbs, "peak": hbm,
+                     "unit": "GB/s", "frac": scan_gbs / hbm, "peak_kind": peak_kind,
+                     "algorithmic_bytes_per_launch": scan_bytes(own), "avg_launch_us": scan_avg_ms * 1e3,
+                     "traffic": None},
+        "e2e": {"value": world * args.steps / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "clocks": sampler.summary(),
+    }
+    # ---- CPU baseline: the oracle on this host, rank 0 at N = 1 only
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        host = oracle_inputs(1237, dev)
+        v, cores, dt = oracle_time(host, args.cpu_queries)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": f"{args.cpu_queries} decode queries at 1M context "
+                                          f"({dt:.1f} s), one layer cache"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    for L in layers:
+        del L
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,184 @@
+/*
+ * dsa.h: C-ABI of libdsa, DSA region-sparse GQA on NVIDIA B200 (sm_100a).
+ *
+ * DSA is the sparse attention of Step-5-Preview's 23 full-attention layers.  Pages
+ * cited (title, site):
+ *   [P1] Step-5-Preview 百万 token 长上下文: 滑窗 + DSA (kwkr.cn/news/601179)
+ *   [P2] Step-5-Preview 如何实现1M长上下文？滑窗+DSA稀疏注意力混合机制完整揭秘 (yfxerp.com/news/376439)
+ *   [P3] 100 万 token 上下文实测：Step 5 Preview 一次能吞下多大的工程 (kwkr.cn/news/593658)
+ *
+ * The method has four steps, one call each (plus the fused decode selection):
+ *   dsa_compress_regions     A1  8-token regions -> 256-d e4m3 summaries     [P1 §DSA ②][P2 §区域压缩CSA]
+ *   dsa_indexer_scores       A2  16-head indexer score per (query, region)   [P1 §DSA ③][P2 §索引器打分]
+ *   dsa_topk_regions         A3  own region + top-(k-1), ties -> lower index [P2 §索引器打分]
+ *   dsa_sparse_attn_decode   A4  exact GQA over the selected regions         [P1 §DSA ④][P3 §一]
+ *   dsa_sparse_attn_prefill  A4  the same for a chunk of prefill queries     [P3 §一 sparse_attention_prefill]
+ *
+ * Conventions (every call):
+ *   - Pointers are DEVICE pointers unless stated otherwise, owned by the caller.  The
+ *     library never allocates device memory; scratch comes from a caller-provided
+ *     workspace `ws` of at least the size the matching *_workspace_size() returns,
+ *     aligned to 256 bytes.  Workspace contents need not be initialised and are
+ *     clobbered.  Calls that share a workspace must not overlap on the GPU.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy default
+ *     stream) and never synchronise it.  The return value reflects the synchronous
+ *     host-side argument checks and the launch; errors that only the kernels can see
+ *     (an index read from device memory out of range, a bounded wait that gave up)
+ *     set a per-device error word that dsa_check_device() reads and clears.
+ *   - All tensors are dense row-major with the shapes given; bf16 is IEEE bfloat16,
+ *     e4m3 is the OCP FP8 E4M3 ("fn") byte format.
+ *   - dsa_last_error() returns a thread-local message for the last failed call.
+ *
+ * Shapes: G = 4 KV groups, HI = 16 indexer heads (head h in group h/4), DI = 256,
+ * HQ = 64 query heads (head h uses KV group h/16), D = 192, regions of 8 tokens,
+ * K/V pages of 64 tokens (8 regions).
+ */
+#ifndef DSA_H
+#define DSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DSA_VERSION 100          /* 1.0.0 */
+
+#define DSA_REGION_TOKENS 8      /* [P1 §DSA ①] REGION_BLOCK_SIZE */
+#define DSA_GROUPS 4             /* [P3 §一] num_attention_groups; [P2 §索引器打分] num_provider_groups */
+#define DSA_PROXY_DIM 256        /* [P2 §第二招] proxy_dim */
+#define DSA_INDEX_HEADS 16       /* [P1 §DSA ③] 16-head sparse indexer */
+#define DSA_Q_HEADS 64           /* [P3 §一] num_attention_heads */
+#define DSA_HEAD_DIM 192         /* [P3 §三] 2 x 4 x 192 x 2 bytes per token per layer */
+#define DSA_PAGE_TOKENS 64       /* K/V page size of the paged cache ([P3 §一] block_table) */
+#define DSA_MAX_TOPK 2048        /* largest k accepted (the method uses 512, [P2 §第二招]) */
+
+/* flags for dsa_indexer_scores */
+#define DSA_Q_FP8 1u             /* quantise index_q per (query, head) to e4m3 (absmax/448
+                                    scale) before scoring: an FP8 x FP8 contraction */
+
+typedef struct CUstream_st *dsa_stream_t;   /* identical to cudaStream_t */
+
+typedef enum dsa_status {
+    DSA_OK = 0,
+    DSA_ERR_INVALID_ARG = 1,     /* a host-visible argument is out of range or NULL */
+    DSA_ERR_UNSUPPORTED = 2,     /* the device is not sm_100 or a size exceeds a limit */
+    DSA_ERR_WORKSPACE = 3,       /* ws too small or not 256-byte aligned */
+    DSA_ERR_CUDA = 4,            /* a CUDA runtime call failed (launch, attribute, ...) */
+    DSA_ERR_DEVICE = 5           /* a kernel flagged an error (dsa_check_device) */
+} dsa_status_t;
+
+/* Library version (DSA_VERSION of the build). */
+int dsa_version(void);
+
+/* Message for the last non-OK status returned on this host thread ("" if none).
+ * The pointer stays valid until the next call on this thread. */
+const char *dsa_last_error(void);
+
+/* Synchronises `stream`, then reads and clears the error word that kernels of this
+ * library set on the current device.  Returns DSA_OK or DSA_ERR_DEVICE (message via
+ * dsa_last_error), or DSA_ERR_CUDA if the synchronisation itself failed. */
+dsa_status_t dsa_check_device(dsa_stream_t stream);
+
+/* ------------------------------------------------------------------------------ */
+/* A1 region compression.  [P1 §DSA ②] every complete 8-token region is collapsed into a
+ * 256-d summary stored as FP8; [P2 §区域压缩CSA] only full regions are summarised, a
+ * tail of fewer than 8 tokens waits.  For region i and group g:
+ *   m_j   = fp32( sum_{t=0..7} index_k[src_row[i]+t][g][j] / 8 )   (sum in fp64, t = 0..7)
+ *   scale = fp32( max_j |m_j| / 448 )
+ *   code_j = e4m3_RNE_satfinite( fp32(m_j / scale) ),  all 0 when scale = 0
+ * index_k   bf16  [n_rows][row_stride]; token row t of group g is index_k[t*row_stride + g*256 + j]
+ *           (row_stride >= 1024 elements, a multiple of 8)
+ * src_row   int64 [n_regions]   first row of region i (rows src_row[i] .. +7, must be < n_rows)
+ * dst_slot  int64 [n_regions]   pool slot written for region i (0 <= slot < n_slots)
+ * summaries e4m3  [4][n_slots][256]   (group-major pool)
+ * scales    fp32  [4][n_slots]
+ * Out-of-range src_row/dst_slot values are skipped and flag DSA_ERR_DEVICE.  Regions
+ * written to the same slot in one call race.  n_regions == 0 is a no-op. */
+dsa_status_t dsa_compress_regions(const void *index_k, int64_t row_stride, int64_t n_rows,
+                                  const int64_t *src_row, const int64_t *dst_slot, int n_regions,
+                                  uint8_t *summaries, float *scales, int64_t n_slots,
+                                  dsa_stream_t stream);
+
+/* ------------------------------------------------------------------------------ */
+/* A2 indexer scores.  [P1 §DSA ③][P2 §索引器打分] the 16-head indexer scores each query
+ * against every region summary of its request; regions and heads map onto the 4 KV
+ * groups (heads 4g..4g+3 score group g):
+ *   score[q][g][r] = sum_{h=4g}^{4g+3} gate[q][h] * ReLU(index_q[q][h] . s_{r,g}) / 16,
+ *   s_{r,g} = e4m3 value of summaries[g][sum_base[b]+r] * scales[g][sum_base[b]+r],
+ * for r = 0 .. own-1 where own = q_pos[q] / 8 (the regions complete before the query's
+ * own region; the own region itself is forced by dsa_topk_regions, not scored).
+ * Entries r >= own are not written.  Accumulation is fp32 on the tensor cores.
+ * index_q   bf16  [nq][16][256]
+ * gate      fp32  [nq][16]
+ * q_req     int32 [nq]      request of each query (index into sum_base)
+ * q_pos     int32 [nq]      0-based position of the query token
+ * sum_base  int64 [n_req]   pool slot of region 0 of each request
+ * scores    fp32  [nq][4][ld_scores]
+ * flags     0 or DSA_Q_FP8
+ * A query whose own > ld_scores, q_req out of [0, n_req) or sum_base[b]+own > n_slots
+ * is skipped and flags DSA_ERR_DEVICE.  ws may be NULL (size 0 today). */
+size_t dsa_indexer_workspace_size(int nq, int64_t ld_scores);
+dsa_status_t dsa_indexer_scores(const void *index_q, const float *gate, const int32_t *q_req,
+                                const int32_t *q_pos, int nq, const uint8_t *summaries,
+                                const float *scales, int64_t n_slots, const int64_t *sum_base,
+                                int n_req, float *scores, int64_t ld_scores, uint32_t flags,
+                                void *ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* ------------------------------------------------------------------------------ */
+/* A3 top-k region selection.  [P2 §索引器打分] a radix-style top-k keeps the best regions
+ * and always includes the query's own region; [P2 §第二招] at most k = 512 per query.
+ * Per (query q, group g), own = q_pos[q] / 8: the own region plus the k-1 best of the
+ * regions r < own ordered by (score descending, region index ascending); equal values
+ * (+0 and -0 included) tie.  Output ascending region indices:
+ *   sel_idx   int32 [nq][4][k]   first sel_count entries valid, the rest -1
+ *   sel_count int32 [nq][4]      min(k, own + 1)
+ * scores    fp32  [nq][4][ld_scores]; only entries r < own are read.  NaN scores are
+ *           not supported (their rank is unspecified).
+ * 1 <= k <= DSA_MAX_TOPK.  A query with own > ld_scores flags DSA_ERR_DEVICE and gets
+ * count 0. */
+size_t dsa_topk_workspace_size(int nq, int64_t ld_scores, int k);
+dsa_status_t dsa_topk_regions(const float *scores, int64_t ld_scores, const int32_t *q_pos, int nq,
+                              int k, int32_t *sel_idx, int32_t *sel_count, void *ws,
+                              size_t ws_bytes, dsa_stream_t stream);
+
+/* ------------------------------------------------------------------------------ */
+/* A4 sparse GQA attention.  [P1 §DSA ④] exact attention over only the selected regions'
+ * real K/V; [P3 §一] the selected regions are gathered from the paged cache through the
+ * block_table.  For query q (request b = q_req[q], position p = q_pos[q]) and head h
+ * (group g = h/16): T = union of tokens 8r..8r+7 over r in sel_idx[q][g][0..cnt), kept
+ * where t <= p (the causal mask inside the own region);
+ *   out[q][h] = sum_{t in T} softmax_t(q[q][h] . K_t / sqrt(192)) V_t   (bf16, fp32 math)
+ *   lse[q][h] = ln sum_{t in T} exp(q[q][h] . K_t / sqrt(192))          (-inf if T empty)
+ * q           bf16  [nq][64][192]  (already rotated)
+ * k_cache     bf16  [n_pages][4][64][192]; token t of request b is row t%64 of page
+ * v_cache     bf16  [n_pages][4][64][192]   block_table[b*max_pages + t/64]
+ * block_table int32 [n_req][max_pages]
+ * sel_idx     int32 [nq][4][k], sel_count int32 [nq][4]  (as written by dsa_topk_regions)
+ * out         bf16  [nq][64][192]
+ * lse         fp32  [nq][64] or NULL
+ * A selected region beyond the block table, a page index outside [0, n_pages) or a
+ * q_req outside [0, n_req) is skipped and flags DSA_ERR_DEVICE.  An empty T gives
+ * out = 0.  decode: one query per request, q_req = identity (nq = n_req = batch).
+ * The workspace is needed only when few (query, group) rows must be split across CTAs;
+ * dsa_attn_workspace_size() returns 0 otherwise (it depends on the current device's
+ * SM count). */
+size_t dsa_attn_workspace_size(int nq, int k);
+dsa_status_t dsa_sparse_attn_decode(const void *q, const void *k_cache, const void *v_cache,
+                                    int64_t n_pages, const int32_t *block_table, int max_pages,
+                                    const int32_t *q_pos, int batch, const int32_t *sel_idx,
+                                    const int32_t *sel_count, int k, void *out, float *lse,
+                                    void *ws, size_t ws_bytes, dsa_stream_t stream);
+dsa_status_t dsa_sparse_attn_prefill(const void *q, const void *k_cache, const void *v_cache,
+                                     int64_t n_pages, const int32_t *block_table, int max_pages,
+                                     int n_req, const int32_t *q_req, const int32_t *q_pos, int nq,
+                                     const int32_t *sel_idx, const int32_t *sel_count, int k,
+                                     void *out, float *lse, void *ws, size_t ws_bytes,
+                                     dsa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H */

@@ -1,0 +1,397 @@
+// libdsa: the C-ABI entry points declared in include/dsa.h.  Host code here only checks
+// arguments, sizes grids, encodes TMA tensor maps and launches the kernels of
+// compress.cuh, indexer.cuh, topk.cuh and attention.cuh (one translation unit, so the
+// per-device error word is a single symbol).
+#include <mutex>
+#include <string>
+
+#include "../../include/dsa.h"
+#include "attention.cuh"
+#include "common.cuh"
+#include "compress.cuh"
+#include "indexer.cuh"
+#include "topk.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+dsa_status_t fail(dsa_status_t st, const std::string &msg)
+{
+    g_last_error = msg;
+    return st;
+}
+
+dsa_status_t cuda_fail(cudaError_t e, const char *what)
+{
+    return fail(DSA_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+#define DSA_REQUIRE(cond, msg)                                  \
+    do {                                                        \
+        if (!(cond)) return fail(DSA_ERR_INVALID_ARG, (msg));   \
+    } while (0)
+
+#define DSA_CUDA(call, what)                                    \
+    do {                                                        \
+        cudaError_t e_ = (call);                                \
+        if (e_ != cudaSuccess) return cuda_fail(e_, (what));    \
+    } while (0)
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Device facts, checked on every call (cheap attribute queries).
+dsa_status_t device_info(int &sm_count)
+{
+    int dev = 0;
+    DSA_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+    int major = 0;
+    DSA_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev), "cudaDeviceGetAttribute");
+    if (major != 10) return fail(DSA_ERR_UNSUPPORTED, "libdsa is built for sm_100a (B200); device is sm_" +
+                                                          std::to_string(major) + "x");
+    DSA_CUDA(cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev), "cudaDeviceGetAttribute");
+    return DSA_OK;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+dsa_status_t encode(CUtensorMap *map, CUtensorMapDataType dt, int rank, const void *base, const cuuint64_t *dims,
+                    const cuuint64_t *strides, const cuuint32_t *box, CUtensorMapL2promotion l2)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = fn(map, dt, (cuuint32_t)rank, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, l2, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (" + std::to_string((int)r) + ")");
+    return DSA_OK;
+}
+
+dsa_status_t launched(const char *what)
+{
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, what);
+    return DSA_OK;
+}
+
+// K/V cache viewed as [rows = n_pages*4*64][3][64] bf16: one region = box {64, 3, 8}.
+dsa_status_t kv_map(CUtensorMap *m, const void *cache, int64_t n_pages)
+{
+    const cuuint64_t dims[3] = {64, 3, (cuuint64_t)n_pages * dsa::kG * dsa::kPage};
+    const cuuint64_t strides[2] = {128, (cuuint64_t)dsa::kD * 2};
+    const cuuint32_t box[3] = {64, 3, (cuuint32_t)dsa::kRegion};
+    return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, cache, dims, strides, box, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+}
+
+struct TopkLayout {
+    size_t hist, ctr, sure, cand, total;
+};
+
+TopkLayout topk_layout(int nq, int64_t ld, int k)
+{
+    const size_t rows = (size_t)nq * dsa::kG;
+    TopkLayout L;
+    L.hist = 0;
+    L.ctr = round_up(rows * dsa::topk::kBins * 4, 256);
+    L.sure = L.ctr + round_up(rows * 16, 256);
+    L.cand = L.sure + round_up(rows * (size_t)k * 4, 256);
+    L.total = L.cand + round_up(rows * (size_t)ld * 8, 256);
+    return L;
+}
+
+// attention split policy: few rows -> split each selection into chunks of 16 regions
+struct AttnPlan {
+    int rps, n_splits;
+    size_t ws;
+};
+
+AttnPlan attn_plan(int nq, int k, int sm_count)
+{
+    AttnPlan a;
+    const int rows = nq * dsa::kG;
+    if (rows >= 2 * sm_count) {
+        a.rps = k;
+        a.n_splits = 1;
+        a.ws = 0;
+    } else {
+        a.rps = 16;
+        a.n_splits = (k + a.rps - 1) / a.rps;
+        const size_t n = (size_t)rows * a.n_splits * 16;
+        a.ws = round_up(n * dsa::kD * 4, 256) + round_up(n * 2 * 4, 256);
+    }
+    return a;
+}
+
+dsa_status_t attn_common(const void *q, const void *k_cache, const void *v_cache, int64_t n_pages,
+                         const int32_t *block_table, int max_pages, const int32_t *q_req, int n_req,
+                         const int32_t *q_pos, int nq, const int32_t *sel_idx, const int32_t *sel_count, int k,
+                         void *out, float *lse, void *ws, size_t ws_bytes, dsa_stream_t stream)
+{
+    DSA_REQUIRE(nq >= 0, "nq must be >= 0");
+    DSA_REQUIRE(k >= 1 && k <= DSA_MAX_TOPK, "k out of [1, DSA_MAX_TOPK]");
+    DSA_REQUIRE(n_pages >= 1 && n_pages <= (INT32_MAX / (dsa::kG * dsa::kPage)), "n_pages out of range");
+    DSA_REQUIRE(max_pages >= 1, "max_pages must be >= 1");
+    DSA_REQUIRE(n_req >= 1, "n_req must be >= 1");
+    if (nq == 0) return DSA_OK;
+    DSA_REQUIRE(q && k_cache && v_cache && block_table && q_pos && sel_idx && sel_count && out, "NULL pointer");
+    DSA_REQUIRE(aligned(q, 16) && aligned(k_cache, 16) && aligned(v_cache, 16) && aligned(out, 4),
+                "q, k_cache, v_cache must be 16-byte aligned, out 4-byte aligned");
+    int sms = 0;
+    dsa_status_t st = device_info(sms);
+    if (st != DSA_OK) return st;
+    const AttnPlan plan = attn_plan(nq, k, sms);
+    if (plan.ws > 0) {
+        if (!ws || ws_bytes < plan.ws || !aligned(ws, 256))
+            return fail(DSA_ERR_WORKSPACE, "attention workspace too small or not 256-byte aligned (need " +
+                                               std::to_string(plan.ws) + " bytes)");
+    }
+    CUtensorMap mk, mv;
+    if ((st = kv_map(&mk, k_cache, n_pages)) != DSA_OK) return st;
+    if ((st = kv_map(&mv, v_cache, n_pages)) != DSA_OK) return st;
+
+    dsa::attn::Params p{};
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.block_table = block_table;
+    p.q_req = q_req;
+    p.q_pos = q_pos;
+    p.sel_idx = sel_idx;
+    p.sel_count = sel_count;
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.lse = lse;
+    const size_t n = (size_t)nq * dsa::kG * plan.n_splits * 16;
+    p.part_o = plan.ws ? static_cast<float *>(ws) : nullptr;
+    p.part_ml = plan.ws ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + round_up(n * dsa::kD * 4, 256))
+                        : nullptr;
+    p.n_pages = n_pages;
+    p.max_pages = max_pages;
+    p.n_req = n_req;
+    p.nq = nq;
+    p.k = k;
+    p.rps = plan.rps;
+    p.n_splits = plan.n_splits;
+    p.scale_log2 = dsa::attn::kLog2e / sqrtf((float)dsa::kD);
+
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(dsa::attn::sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)dsa::attn::kSmemBytes);
+    });
+    DSA_CUDA(attr_err, "cudaFuncSetAttribute(sparse_attn_kernel)");
+    dim3 grid(plan.n_splits, nq * dsa::kG);
+    dsa::attn::sparse_attn_kernel<<<grid, dsa::attn::kThreads, dsa::attn::kSmemBytes, stream>>>(mk, mv, p);
+    if ((st = launched("sparse_attn_kernel")) != DSA_OK) return st;
+    if (plan.n_splits > 1) {
+        dsa::attn::combine_kernel<<<nq * dsa::kG * 16, dsa::kD, 0, stream>>>(p);
+        if ((st = launched("combine_kernel")) != DSA_OK) return st;
+    }
+    return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dsa_version(void) { return DSA_VERSION; }
+
+const char *dsa_last_error(void) { return g_last_error.c_str(); }
+
+dsa_status_t dsa_check_device(dsa_stream_t stream)
+{
+    DSA_CUDA(cudaStreamSynchronize(stream), "cudaStreamSynchronize");
+    unsigned word = 0;
+    DSA_CUDA(cudaMemcpyFromSymbol(&word, dsa::g_error_word, sizeof(word)), "read error word");
+    if (word == 0) return DSA_OK;
+    const unsigned zero = 0;
+    DSA_CUDA(cudaMemcpyToSymbol(dsa::g_error_word, &zero, sizeof(zero)), "clear error word");
+    std::string msg = "device error word 0x" + [&] {
+        char b[16];
+        snprintf(b, sizeof b, "%x", word);
+        return std::string(b);
+    }() + ":";
+    if (word & dsa::kErrCompressIndex) msg += " compress src_row/dst_slot out of range;";
+    if (word & dsa::kErrIndexerQuery) msg += " indexer query out of range (q_req, own > ld, slots);";
+    if (word & dsa::kErrTopkRow) msg += " top-k own region beyond ld_scores;";
+    if (word & dsa::kErrAttnIndex) msg += " attention region/page index out of range;";
+    if (word & dsa::kErrWaitTimeout) msg += " bounded wait timed out;";
+    if (word & dsa::kErrTopkInternal) msg += " top-k internal inconsistency;";
+    return fail(DSA_ERR_DEVICE, msg);
+}
+
+dsa_status_t dsa_compress_regions(const void *index_k, int64_t row_stride, int64_t n_rows, const int64_t *src_row,
+                                  const int64_t *dst_slot, int n_regions, uint8_t *summaries, float *scales,
+                                  int64_t n_slots, dsa_stream_t stream)
+{
+    DSA_REQUIRE(n_regions >= 0, "n_regions must be >= 0");
+    if (n_regions == 0) return DSA_OK;
+    DSA_REQUIRE(index_k && src_row && dst_slot && summaries && scales, "NULL pointer");
+    DSA_REQUIRE(row_stride >= dsa::kG * dsa::kDI && row_stride % 8 == 0, "row_stride must be >= 1024 and a multiple of 8");
+    DSA_REQUIRE(n_rows >= dsa::kRegion && n_slots >= 1, "n_rows >= 8 and n_slots >= 1 required");
+    DSA_REQUIRE(aligned(index_k, 16) && aligned(summaries, 8) && aligned(scales, 4), "misaligned pointer");
+    int sms = 0;
+    dsa_status_t st = device_info(sms);
+    if (st != DSA_OK) return st;
+    const int grid = (int)std::min<int64_t>(n_regions, (int64_t)sms * 16);
+    dsa::compress_regions_kernel<<<grid, 128, 0, stream>>>(static_cast<const __nv_bfloat16 *>(index_k), row_stride,
+                                                          n_rows, src_row, dst_slot, n_regions, summaries, scales,
+                                                          n_slots);
+    return launched("compress_regions_kernel");
+}
+
+size_t dsa_indexer_workspace_size(int nq, int64_t ld_scores)
+{
+    (void)nq;
+    (void)ld_scores;
+    return 0;
+}
+
+dsa_status_t dsa_indexer_scores(const void *index_q, const float *gate, const int32_t *q_req, const int32_t *q_pos,
+                                int nq, const uint8_t *summaries, const float *scales, int64_t n_slots,
+                                const int64_t *sum_base, int n_req, float *scores, int64_t ld_scores, uint32_t flags,
+                                void *ws, size_t ws_bytes, dsa_stream_t stream)
+{
+    (void)ws;
+    (void)ws_bytes;
+    DSA_REQUIRE(nq >= 0, "nq must be >= 0");
+    DSA_REQUIRE((flags & ~DSA_Q_FP8) == 0, "unknown flag");
+    DSA_REQUIRE(ld_scores >= 1 && ld_scores <= (1ll << 26), "ld_scores out of [1, 2^26]");
+    DSA_REQUIRE(n_slots >= 1 && n_slots <= (1ll << 28), "n_slots out of [1, 2^28]");
+    DSA_REQUIRE(n_req >= 1, "n_req must be >= 1");
+    if (nq == 0) return DSA_OK;
+    DSA_REQUIRE(index_q && gate && q_req && q_pos && summaries && scales && sum_base && scores, "NULL pointer");
+    DSA_REQUIRE(aligned(index_q, 16) && aligned(summaries, 16), "index_q and summaries must be 16-byte aligned");
+    int sms = 0;
+    dsa_status_t st = device_info(sms);
+    if (st != DSA_OK) return st;
+
+    CUtensorMap map;
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)dsa::kDI, (cuuint64_t)n_slots * dsa::kG};
+        const cuuint64_t strides[1] = {(cuuint64_t)dsa::kDI};
+        const cuuint32_t box[2] = {128, (cuuint32_t)dsa::idx::kChunk};
+        if ((st = encode(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, summaries, dims, strides, box,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B)) != DSA_OK)
+            return st;
+    }
+    dsa::idx::Params p{};
+    p.index_q = static_cast<const __nv_bfloat16 *>(index_q);
+    p.gate = gate;
+    p.q_req = q_req;
+    p.q_pos = q_pos;
+    p.scales = scales;
+    p.sum_base = sum_base;
+    p.scores = scores;
+    p.n_slots = n_slots;
+    p.ld = ld_scores;
+    p.units_per_query = (int)((ld_scores + dsa::idx::kChunk - 1) / dsa::idx::kChunk);
+    p.total_units = (int64_t)nq * p.units_per_query;
+    p.nq = nq;
+    p.n_req = n_req;
+    p.flags = flags;
+
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(dsa::idx::scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)dsa::idx::kSmemBytes);
+    });
+    DSA_CUDA(attr_err, "cudaFuncSetAttribute(scan_kernel)");
+    const int grid = (int)std::min<int64_t>(p.total_units, (int64_t)sms * 2);
+    dsa::idx::scan_kernel<<<grid, dsa::idx::kThreads, dsa::idx::kSmemBytes, stream>>>(map, p);
+    return launched("scan_kernel");
+}
+
+size_t dsa_topk_workspace_size(int nq, int64_t ld_scores, int k)
+{
+    if (nq <= 0 || ld_scores < 1 || k < 1) return 0;
+    return topk_layout(nq, ld_scores, k).total;
+}
+
+dsa_status_t dsa_topk_regions(const float *scores, int64_t ld_scores, const int32_t *q_pos, int nq, int k,
+                              int32_t *sel_idx, int32_t *sel_count, void *ws, size_t ws_bytes, dsa_stream_t stream)
+{
+    DSA_REQUIRE(nq >= 0, "nq must be >= 0");
+    DSA_REQUIRE(k >= 1 && k <= DSA_MAX_TOPK, "k out of [1, DSA_MAX_TOPK]");
+    DSA_REQUIRE(ld_scores >= 1 && ld_scores < dsa::topk::kMaxRegions, "ld_scores out of [1, 2^20)");
+    if (nq == 0) return DSA_OK;
+    DSA_REQUIRE(scores && q_pos && sel_idx && sel_count, "NULL pointer");
+    const TopkLayout L = topk_layout(nq, ld_scores, k);
+    if (!ws || ws_bytes < L.total || !aligned(ws, 256))
+        return fail(DSA_ERR_WORKSPACE, "top-k workspace too small or not 256-byte aligned (need " +
+                                           std::to_string(L.total) + " bytes)");
+    int sms = 0;
+    dsa_status_t st = device_info(sms);
+    if (st != DSA_OK) return st;
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    dsa::topk::Ws tw;
+    tw.hist = reinterpret_cast<uint32_t *>(w + L.hist);
+    tw.ctr = reinterpret_cast<uint32_t *>(w + L.ctr);
+    tw.sure = reinterpret_cast<int32_t *>(w + L.sure);
+    tw.cand = reinterpret_cast<uint2 *>(w + L.cand);
+    DSA_CUDA(cudaMemsetAsync(w, 0, L.sure, stream), "cudaMemsetAsync(top-k histograms)");
+    const int rows = nq * dsa::kG;
+    const dim3 grid((unsigned)((ld_scores + dsa::topk::kChunk - 1) / dsa::topk::kChunk), (unsigned)rows);
+    dsa::topk::hist_kernel<<<grid, dsa::topk::kThreads, 0, stream>>>(scores, ld_scores, q_pos, k, tw);
+    if ((st = launched("topk hist_kernel")) != DSA_OK) return st;
+    dsa::topk::gather_kernel<<<grid, dsa::topk::kThreads, 0, stream>>>(scores, ld_scores, q_pos, k, tw);
+    if ((st = launched("topk gather_kernel")) != DSA_OK) return st;
+    const size_t bitmap = round_up((size_t)((ld_scores + 1 + 31) / 32) * 4, 16);
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(dsa::topk::final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)((dsa::topk::kMaxRegions / 32 + 16) * 4));
+    });
+    DSA_CUDA(attr_err, "cudaFuncSetAttribute(topk final_kernel)");
+    dsa::topk::final_kernel<<<rows, dsa::topk::kFinalThreads, bitmap, stream>>>(q_pos, ld_scores, k, tw, sel_idx,
+                                                                               sel_count);
+    return launched("topk final_kernel");
+}
+
+size_t dsa_attn_workspace_size(int nq, int k)
+{
+    if (nq <= 0 || k < 1) return 0;
+    int sms = 0;
+    if (device_info(sms) != DSA_OK) sms = 148;
+    return attn_plan(nq, k, sms).ws;
+}
+
+dsa_status_t dsa_sparse_attn_decode(const void *q, const void *k_cache, const void *v_cache, int64_t n_pages,
+                                    const int32_t *block_table, int max_pages, const int32_t *q_pos, int batch,
+                                    const int32_t *sel_idx, const int32_t *sel_count, int k, void *out, float *lse,
+                                    void *ws, size_t ws_bytes, dsa_stream_t stream)
+{
+    return attn_common(q, k_cache, v_cache, n_pages, block_table, max_pages, nullptr, batch, q_pos, batch, sel_idx,
+                       sel_count, k, out, lse, ws, ws_bytes, stream);
+}
+
+dsa_status_t dsa_sparse_attn_prefill(const void *q, const void *k_cache, const void *v_cache, int64_t n_pages,
+                                     const int32_t *block_table, int max_pages, int n_req, const int32_t *q_req,
+                                     const int32_t *q_pos, int nq, const int32_t *sel_idx, const int32_t *sel_count,
+                                     int k, void *out, float *lse, void *ws, size_t ws_bytes, dsa_stream_t stream)
+{
+    DSA_REQUIRE(q_req != nullptr || nq == 0, "q_req must not be NULL");
+    return attn_common(q, k_cache, v_cache, n_pages, block_table, max_pages, q_req, n_req, q_pos, nq, sel_idx,
+                       sel_count, k, out, lse, ws, ws_bytes, stream);
+}
+
+}  // extern "C"

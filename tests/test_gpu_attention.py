@@ -1,0 +1,105 @@
+"""GPU sparse attention (A4) against the oracle on the same selections: bf16 outputs
+within 2e-2 absolute + 1e-2 relative, lse within 1e-3."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_long_context_dsa_b200 import dsa
+from sparse_long_context_dsa_b200 import workloads as W
+
+from _util import bits, bf16_from_bits_np
+
+pytestmark = pytest.mark.gpu
+G = 4
+
+
+def random_selection(q_pos, k, seed, force_own=True):
+    rng = np.random.default_rng(seed)
+    nq = len(q_pos)
+    idx = np.full((nq, G, k), -1, np.int32)
+    cnt = np.zeros((nq, G), np.int32)
+    for i, p in enumerate(q_pos):
+        own = p // 8
+        for g in range(G):
+            n = min(k, own + 1)
+            pick = rng.choice(own, size=n - 1, replace=False) if n > 1 else np.array([], np.int64)
+            s = np.sort(np.concatenate([pick, [own]]).astype(np.int32))
+            idx[i, g, :n] = s
+            cnt[i, g] = n
+    return idx, cnt
+
+
+def run(d, idx, cnt, q_req=None, prefill=False):
+    dev = "cuda"
+    si = torch.from_numpy(idx).to(dev)
+    sc = torch.from_numpy(cnt).to(dev)
+    nq = idx.shape[0]
+    lse = torch.empty((nq, 64), dtype=torch.float32, device=dev)
+    q = d["q"][:nq].contiguous()
+    if prefill:
+        out = dsa.sparse_attn_prefill(q, d["k_cache"], d["v_cache"], d["block_table"], q_req, d["q_pos"], si, sc,
+                                      lse=lse)
+    else:
+        out = dsa.sparse_attn_decode(q, d["k_cache"], d["v_cache"], d["block_table"], d["q_pos"], si, sc, lse=lse)
+    dsa.check_device()
+    qr = np.arange(nq) if q_req is None else q_req.cpu().numpy()
+    oo, lo = oracle.sparse_attention(bits(q), bits(d["k_cache"]), bits(d["v_cache"]), d["block_table"].cpu().numpy(),
+                                     qr, d["q_pos"].cpu().numpy(), idx, cnt)
+    og = out.float().cpu().numpy()
+    of = bf16_from_bits_np(oo)
+    err = np.abs(og - of)
+    assert np.all(err <= 2e-2 + 1e-2 * np.abs(of)), err.max()
+    lg = lse.cpu().numpy()
+    fin = np.isfinite(lo)
+    assert np.array_equal(np.isfinite(lg), fin)
+    np.testing.assert_allclose(lg[fin], lo[fin], rtol=1e-3, atol=1e-3)
+    return err.max()
+
+
+@pytest.mark.parametrize("k", [1, 5, 16, 64, 512])
+def test_decode_random_selections(k):
+    lengths = [16384, 9000 + 3, 600 + 7]
+    d = W.decode_batch(lengths, seed=30 + k, device="cuda", permute=True)
+    idx, cnt = random_selection(d["q_pos"].cpu().numpy(), k, seed=k)
+    e = run(d, idx, cnt)
+    print(f"k={k} max abs err {e:.3e}")
+
+
+def test_prefill_many_rows_single_pass():
+    # >= 2 * SMs (query, group) rows: each CTA covers a whole selection (no split)
+    ctx = 4096
+    d = W.prefill_chunk(ctx, 160, seed=33, device="cuda", permute=True)
+    qp = d["q_pos"].cpu().numpy()
+    idx, cnt = random_selection(qp, 64, seed=3)
+    run(d, idx, cnt, q_req=d["q_req"], prefill=True)
+
+
+def test_causal_mask_inside_the_own_region():
+    # queries at every offset of a region; the own region alone is selected
+    d = W.decode_batch([8 * 20 + 8], seed=34, device="cuda", permute=False)
+    dev = "cuda"
+    nq = 8
+    pos = torch.arange(8 * 20, 8 * 21, dtype=torch.int32, device=dev)
+    d["q_pos"] = pos
+    d["q"] = W.normal_bf16((nq, 64, 192), W.generator(9, dev), dev)
+    idx = np.full((nq, G, 2), -1, np.int32)
+    idx[:, :, 0] = 20
+    cnt = np.ones((nq, G), np.int32)
+    run(d, idx, cnt, q_req=torch.zeros(nq, dtype=torch.int32, device=dev), prefill=True)
+
+
+def test_empty_selection_and_bad_region():
+    d = W.decode_batch([1000], seed=35, device="cuda")
+    idx = np.full((1, G, 4), -1, np.int32)
+    cnt = np.zeros((1, G), np.int32)
+    idx[0, 1, :2] = [3, 124]
+    cnt[0, 1] = 2
+    run(d, idx, cnt)
+    idx[0, 2, 0] = 99999                       # beyond the block table: flagged, skipped
+    cnt[0, 2] = 1
+    si = torch.from_numpy(idx).cuda()
+    sc = torch.from_numpy(cnt).cuda()
+    dsa.sparse_attn_decode(d["q"], d["k_cache"], d["v_cache"], d["block_table"], d["q_pos"], si, sc)
+    with pytest.raises(dsa.DsaError):
+        dsa.check_device()

@@ -1,0 +1,82 @@
+"""GPU top-k (A3) fed the oracle's fp32 scores must reproduce the oracle's selection
+bit for bit (indices, order, counts, padding)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_long_context_dsa_b200 import dsa
+
+pytestmark = pytest.mark.gpu
+G = 4
+
+
+def both(scores, q_pos, k):
+    s = torch.from_numpy(np.ascontiguousarray(scores)).cuda()
+    qp = torch.tensor(q_pos, dtype=torch.int32, device="cuda")
+    ig, cg = dsa.topk_regions(s, qp, k)
+    dsa.check_device()
+    io, co = oracle.topk_regions(scores, q_pos, k)
+    return ig.cpu().numpy(), cg.cpu().numpy(), io, co
+
+
+def check(scores, q_pos, k):
+    ig, cg, io, co = both(scores, q_pos, k)
+    assert np.array_equal(cg, co)
+    assert np.array_equal(ig, io)
+
+
+@pytest.mark.parametrize("k", [1, 2, 64, 512, 2048])
+def test_random_rows(k):
+    rng = np.random.default_rng(k)
+    ld = 20000
+    s = rng.standard_normal((4, G, ld)).astype(np.float32)
+    check(s, [8 * ld - 1, 8 * 3000 + 4, 7, 8 * 511], k)
+
+
+def test_scores_like_the_indexer():
+    # non-negative, ReLU zeros, gated sums: the distribution the decode path produces
+    rng = np.random.default_rng(1)
+    ld = 16383
+    d = rng.standard_normal((2, G, 4, ld)) * 5.6
+    z = rng.uniform(0, 1, (2, G, 4, 1))
+    s = (np.maximum(d, 0) * z).sum(axis=2).astype(np.float32) / 16
+    check(s, [8 * ld + 7, 8 * ld], 512)
+
+
+def test_heavy_ties_and_all_zero_rows():
+    rng = np.random.default_rng(2)
+    s = rng.integers(0, 5, (2, G, 9000)).astype(np.float32)
+    s[1] = 0.0
+    s[1, 2, 100:200] = -0.0
+    check(s, [8 * 9000, 8 * 9000 + 3], 512)
+
+
+def test_negative_and_mixed_sign_scores():
+    rng = np.random.default_rng(3)
+    s = (rng.standard_normal((1, G, 5000)) * 1e3).astype(np.float32)
+    s[0, 1] = -np.abs(s[0, 1])
+    check(s, [8 * 5000], 300)
+
+
+def test_own_region_smaller_than_k():
+    rng = np.random.default_rng(4)
+    s = rng.standard_normal((3, G, 600)).astype(np.float32)
+    check(s, [0, 8 * 100 + 1, 8 * 511 + 7], 512)
+
+
+def test_one_million_token_row():
+    rng = np.random.default_rng(5)
+    ld = 131071
+    d = rng.standard_normal((1, G, 4, ld)).astype(np.float32) * 5.6
+    s = (np.maximum(d, 0) * rng.uniform(0, 1, (1, G, 4, 1)).astype(np.float32)).sum(axis=2) / 16
+    check(s.astype(np.float32), [8 * 131072 - 1], 512)
+
+
+def test_own_beyond_ld_is_flagged():
+    s = np.zeros((1, G, 10), np.float32)
+    sc = torch.from_numpy(s).cuda()
+    idx, cnt = dsa.topk_regions(sc, torch.tensor([8 * 50], dtype=torch.int32, device="cuda"), 4)
+    with pytest.raises(dsa.DsaError):
+        dsa.check_device()
+    assert np.all(cnt.cpu().numpy() == 0) and np.all(idx.cpu().numpy() == -1)
