@@ -143,6 +143,27 @@ dsa_status_t dsa_topk_regions(const float *scores, int64_t ld_scores, const int3
                               int k, int32_t *sel_idx, int32_t *sel_count, void *ws,
                               size_t ws_bytes, dsa_stream_t stream);
 
+/* Allocation-free top-k (no counterpart in the pages: a library convenience).  Same
+ * computation and results as dsa_topk_regions, for callers that cannot allocate device
+ * memory at the point of the call: code running while another component owns the
+ * device allocator (a serving runtime whose memory pool is fully reserved), or a
+ * plain-C host without a device allocator of its own.  The caller passes only inputs
+ * and outputs; the scratch lives in one static device array inside libdsa,
+ * DSA_TOPK_STATIC_SCRATCH_BYTES (8 MiB) per GPU, held by every GPU that loads the library
+ * until the process exits.  A call needs dsa_topk_workspace_size(nq, ld_scores, k)
+ * bytes of it (a 1M-token request, k = 512: about 4.3 MB); larger calls return
+ * DSA_ERR_UNSUPPORTED.  No cudaMalloc/cudaFree or allocating routine is called.
+ *   - The first call on a device resolves the array's device address (once per device,
+ *     with that device current); make that first call before any stream capture.
+ *   - Every call on a device shares the one array and it keeps the previous call's
+ *     contents (the call clears what must start at zero itself): calls whose kernels
+ *     overlap on the GPU (different streams, concurrent graphs) race and must be
+ *     serialised by the caller. */
+#define DSA_TOPK_STATIC_SCRATCH_BYTES (8u << 20)
+dsa_status_t dsa_topk_regions_noalloc(const float *scores, int64_t ld_scores, const int32_t *q_pos,
+                                      int nq, int k, int32_t *sel_idx, int32_t *sel_count,
+                                      dsa_stream_t stream);
+
 /* ------------------------------------------------------------------------------ */
 /* A4 sparse GQA attention.  [P1 §DSA ④] exact attention over only the selected regions'
  * real K/V; [P3 §一] the selected regions are gathered from the paged cache through the

@@ -207,6 +207,27 @@ dsa_status_t attn_common(const void *q, const void *k_cache, const void *v_cache
     return DSA_OK;
 }
 
+// Scratch of dsa_topk_regions_noalloc: one static array per GPU that loads the library.
+static __device__ __align__(256) uint8_t g_topk_static_scratch[DSA_TOPK_STATIC_SCRATCH_BYTES];
+
+// Device address of g_topk_static_scratch on `dev` (looked up once per device with that
+// device current; in host code the symbol itself is only a host-side stand-in).
+dsa_status_t static_scratch(int dev, void **ptr)
+{
+    constexpr int kMaxDevices = 64;
+    static void *addr[kMaxDevices] = {};
+    static std::mutex mu;
+    if (dev < 0 || dev >= kMaxDevices) return fail(DSA_ERR_UNSUPPORTED, "device ordinal out of range");
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        DSA_CUDA(cudaGetSymbolAddress(&p, g_topk_static_scratch), "cudaGetSymbolAddress(top-k static scratch)");
+        addr[dev] = p;
+    }
+    *ptr = addr[dev];
+    return DSA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -365,6 +386,27 @@ dsa_status_t dsa_topk_regions(const float *scores, int64_t ld_scores, const int3
     dsa::topk::final_kernel<<<rows, dsa::topk::kFinalThreads, bitmap, stream>>>(q_pos, ld_scores, k, tw, sel_idx,
                                                                                sel_count);
     return launched("topk final_kernel");
+}
+
+dsa_status_t dsa_topk_regions_noalloc(const float *scores, int64_t ld_scores, const int32_t *q_pos, int nq, int k,
+                                      int32_t *sel_idx, int32_t *sel_count, dsa_stream_t stream)
+{
+    DSA_REQUIRE(nq >= 0, "nq must be >= 0");
+    DSA_REQUIRE(k >= 1 && k <= DSA_MAX_TOPK, "k out of [1, DSA_MAX_TOPK]");
+    DSA_REQUIRE(ld_scores >= 1 && ld_scores < dsa::topk::kMaxRegions, "ld_scores out of [1, 2^20)");
+    if (nq == 0) return DSA_OK;
+    const size_t need = topk_layout(nq, ld_scores, k).total;
+    if (need > DSA_TOPK_STATIC_SCRATCH_BYTES)
+        return fail(DSA_ERR_UNSUPPORTED, "dsa_topk_regions_noalloc: this call needs " + std::to_string(need) +
+                                             " bytes of scratch, the static buffer holds " +
+                                             std::to_string((size_t)DSA_TOPK_STATIC_SCRATCH_BYTES) +
+                                             " (use dsa_topk_regions with a workspace)");
+    int dev = 0;
+    DSA_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+    void *ws = nullptr;
+    dsa_status_t st = static_scratch(dev, &ws);
+    if (st != DSA_OK) return st;
+    return dsa_topk_regions(scores, ld_scores, q_pos, nq, k, sel_idx, sel_count, ws, need, stream);
 }
 
 size_t dsa_attn_workspace_size(int nq, int k)

@@ -47,6 +47,8 @@ _SIG = {
     "dsa_topk_workspace_size": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int64, ctypes.c_int]),
     "dsa_topk_regions": (ctypes.c_int, [_F32P, ctypes.c_int64, _I32P, ctypes.c_int, ctypes.c_int, _I32P, _I32P,
                                         _VP, ctypes.c_size_t, _VP]),
+    "dsa_topk_regions_noalloc": (ctypes.c_int, [_F32P, ctypes.c_int64, _I32P, ctypes.c_int, ctypes.c_int, _I32P,
+                                                _I32P, _VP]),
     "dsa_attn_workspace_size": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int]),
     "dsa_sparse_attn_decode": (ctypes.c_int, [_VP, _VP, _VP, ctypes.c_int64, _I32P, ctypes.c_int, _I32P,
                                               ctypes.c_int, _I32P, _I32P, ctypes.c_int, _VP, _F32P, _VP,
@@ -172,6 +174,21 @@ def topk_regions(scores, q_pos, k, sel_idx=None, sel_count=None):
     ws = _workspace(nbytes, scores.device)
     _check(lib().dsa_topk_regions(_p(scores), ld, _p(q_pos), nq, k, _p(sel_idx), _p(sel_count), _p(ws), nbytes,
                                   _stream()))
+    return sel_idx, sel_count
+
+
+def topk_regions_noalloc(scores, q_pos, k, sel_idx, sel_count):
+    """dsa_topk_regions_noalloc: the same selection with no device allocation at all, for
+    callers that cannot allocate (outputs must be passed in; scratch is the library's
+    static per-GPU buffer, so overlapping calls on one GPU race)."""
+    _need(scores, torch.float32, name="scores")
+    nq, g, ld = scores.shape
+    if g != G:
+        raise ValueError("scores must be [nq][4][ld]")
+    _need(q_pos, torch.int32, (nq,), "q_pos")
+    _need(sel_idx, torch.int32, (nq, G, k), "sel_idx")
+    _need(sel_count, torch.int32, (nq, G), "sel_count")
+    _check(lib().dsa_topk_regions_noalloc(_p(scores), ld, _p(q_pos), nq, k, _p(sel_idx), _p(sel_count), _stream()))
     return sel_idx, sel_count
 
 
