@@ -215,11 +215,10 @@ def build_layers(n_layers, seed0, device):
         torch.cuda.empty_cache()
         own = (L_CTX - 1) // 8
         step = pipeline.DecodeStep(S, C, d["sum_base"], d["block_table"], d["k_cache"], d["v_cache"], ld=own,
-                                   k=TOPK, max_compress=1, index_k=tail)
-        src = torch.zeros(1, dtype=torch.int64, device=device)
-        dst = torch.full((1,), own, dtype=torch.int64, device=device)
-        step.load(d["index_q"], d["gate"], d["q"], d["q_pos"], src, dst)
-        layers.append(dict(step=step, inputs=d, tail=tail))
+                                   k=TOPK, tail_tokens=8)
+        step.load(d["index_q"], d["gate"], d["q"], d["q_pos"], tail)
+        step.set_compress([0], [own])
+        layers.append(dict(step=step, inputs=d))
     torch.cuda.synchronize()
     return layers
 
@@ -250,12 +249,7 @@ def capture(layers, n_steps, ev_pairs=None, e2e=None):
                 L = layers[i % len(layers)]
                 st = L["step"]
                 if e2e is not None:
-                    h = e2e[i % len(layers)]
-                    st.index_q.copy_(h["index_q"], non_blocking=True)
-                    st.gate.copy_(h["gate"], non_blocking=True)
-                    st.q.copy_(h["q"], non_blocking=True)
-                    st.q_pos.copy_(h["q_pos"], non_blocking=True)
-                    L["tail"].copy_(h["tail"], non_blocking=True)
+                    st.arena.copy_(e2e[i % len(layers)]["arena"], non_blocking=True)
                 pre = post = None
                 if ev_pairs is not None:
                     a, b = ev_pairs[i]
@@ -334,12 +328,10 @@ def run_ours(args):
     # ---- e2e: host (pinned) inputs in, result out, every step
     e2e_bufs = []
     for L in layers:
-        st, d = L["step"], L["inputs"]
-        e2e_bufs.append(dict(index_q=d["index_q"].cpu().pin_memory(), gate=d["gate"].cpu().pin_memory(),
-                             q=d["q"].cpu().pin_memory(), q_pos=d["q_pos"].cpu().pin_memory(),
-                             tail=L["tail"].cpu().pin_memory(),
+        st = L["step"]
+        e2e_bufs.append(dict(arena=st.arena.cpu().pin_memory(),
                              out=torch.empty_like(st.out, device="cpu").pin_memory()))
-    h2d = sum(t.numel() * t.element_size() for k, t in e2e_bufs[0].items() if k != "out")
+    h2d = e2e_bufs[0]["arena"].numel()
     d2h = e2e_bufs[0]["out"].numel() * e2e_bufs[0]["out"].element_size()
     g_e2e = capture(layers, chunk, e2e=e2e_bufs)
     g_e2e_tail = capture(layers, rem, e2e=e2e_bufs) if rem else None

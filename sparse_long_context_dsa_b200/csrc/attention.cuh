@@ -80,17 +80,106 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int nr = min(p.rps, cnt - j0);   // regions of this CTA
     if (nr <= 0 && p.n_splits > 1) return; // combine_kernel ignores empty splits
     const bool bad_req = (b < 0 || b >= p.n_req || pos < 0);
-
     if (threadIdx.x < kWarps * kSlots) mbar_init(&bars[threadIdx.x], 1);
+
+    const int n_pairs = (max(nr, 0) + 1) >> 1;
+    uint8_t *ring = smem + warp * kWarpRing;
+    uint64_t *wbar = bars + warp * kSlots;
+    const int32_t *sel = p.sel_idx + (int64_t)row * p.k + j0;
+
+    // This warp handles pairs warp, warp + 4, ...; its local region q (pair q/2, half q%2)
+    // is region j = 2*(warp + 4*(q/2)) + q%2 of the CTA.  Lanes resolve the coordinates of
+    // 32 local regions at a time (sel_idx, then block_table) in parallel and keep them in
+    // registers; the issuing code reads them with shuffles and records, per ring slot, the
+    // region ids and validity the compute side needs.
+    int my_pairs = 0;
+    for (int pi = warp; pi < n_pairs; pi += kWarps) ++my_pairs;
+    int c_base = -64;                   // first local region held by the lane cache
+    int c_y = 0, c_r = -1;              // tensor row and region of local region c_base + lane
+    int c_v = 0;
+    auto refill = [&](int base) {       // warp-collective
+        c_base = base;
+        const int q = base + lane;
+        const int j = 2 * (warp + kWarps * (q >> 1)) + (q & 1);
+        c_v = 0;
+        c_r = -1;
+        if (!bad_req && j < nr) {
+            const int r = sel[j];
+            if (r < 0 || r / 8 >= p.max_pages) {
+                set_error(kErrAttnIndex);
+            } else {
+                const int64_t page = p.block_table[(int64_t)b * p.max_pages + r / 8];
+                if (page < 0 || page >= p.n_pages) {
+                    set_error(kErrAttnIndex);
+                } else {
+                    c_y = (int)((page * kG + g) * kPage + (r % 8) * kRegion);
+                    c_r = r;
+                    c_v = 1;
+                }
+            }
+        }
+    };
+    int slot_r[kSlots][2], slot_v[kSlots][2];
+    auto issue = [&](int i, int slot) {   // warp-collective; lane 0 issues pair i's loads
+        if (2 * i + 1 >= c_base + 32) refill(2 * i);
+        const int s0 = 2 * i - c_base, s1 = s0 + 1;
+        const int y0 = __shfl_sync(0xffffffffu, c_y, s0), y1 = __shfl_sync(0xffffffffu, c_y, s1);
+        const int r0 = __shfl_sync(0xffffffffu, c_r, s0), r1 = __shfl_sync(0xffffffffu, c_r, s1);
+        const int va = __shfl_sync(0xffffffffu, c_v, s0), vb = __shfl_sync(0xffffffffu, c_v, s1);
+#pragma unroll
+        for (int sl = 0; sl < kSlots; ++sl)
+            if (sl == slot) {
+                slot_r[sl][0] = r0;
+                slot_r[sl][1] = r1;
+                slot_v[sl][0] = va;
+                slot_v[sl][1] = vb;
+            }
+        if (lane == 0) {
+            uint8_t *dst = ring + slot * kPairBytes;
+            const unsigned bytes = (va ? 2u * kRegionBytes : 0u) + (vb ? 2u * kRegionBytes : 0u);
+            if (bytes == 0) {
+                mbar_arrive(&wbar[slot]);
+            } else {
+                mbar_arrive_expect_tx(&wbar[slot], bytes);
+                if (va) {
+                    tma_load_3d(dst, &tmap_k, 0, 0, y0, &wbar[slot]);
+                    tma_load_3d(dst + 2 * kRegionBytes, &tmap_v, 0, 0, y0, &wbar[slot]);
+                }
+                if (vb) {
+                    tma_load_3d(dst + kRegionBytes, &tmap_k, 0, 0, y1, &wbar[slot]);
+                    tma_load_3d(dst + 3 * kRegionBytes, &tmap_v, 0, 0, y1, &wbar[slot]);
+                }
+            }
+        }
+    };
+
+    // prologue: resolve this warp's first region coordinates (sel_idx -> block_table) while
+    // the Q tile loads, then issue the first pairs' TMA before building the Q fragments
+    if (lane == 0) {
+        prefetch_tensormap(&tmap_k);
+        prefetch_tensormap(&tmap_v);
+    }
+    if (my_pairs > 0) refill(0);
     // Q tile [16 heads][192] into smem with the same swizzled layout as the K/V tiles
     const __nv_bfloat16 *qsrc = p.q + ((int64_t)qi * kHQ + g * kHeadsPerGroup) * kD;
-    for (int i = threadIdx.x; i < 16 * kD / 8; i += kThreads) {
-        const int r = i / (kD / 8), c = (i % (kD / 8)) * 8;
-        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(qsrc + r * kD + c));
-        *reinterpret_cast<uint4 *>(qs + swz(r, c)) = v;
+    static_assert(16 * kD / 8 == 3 * kThreads, "Q tile: three 16-byte chunks per thread");
+    uint4 qv[3];
+#pragma unroll
+    for (int u = 0; u < 3; ++u) {
+        const int i = threadIdx.x + u * kThreads;
+        qv[u] = __ldg(reinterpret_cast<const uint4 *>(qsrc + (i / (kD / 8)) * kD + (i % (kD / 8)) * 8));
+    }
+#pragma unroll
+    for (int u = 0; u < 3; ++u) {
+        const int i = threadIdx.x + u * kThreads;
+        *reinterpret_cast<uint4 *>(qs + swz(i / (kD / 8), (i % (kD / 8)) * 8)) = qv[u];
     }
     fence_mbar_init();
     __syncthreads();
+
+#pragma unroll
+    for (int s2 = 0; s2 < kSlots; ++s2)
+        if (s2 < my_pairs) issue(s2, s2);
 
     // A fragments of Q (16 x 192): 12 k-steps
     uint32_t qa[12][4];
@@ -110,86 +199,23 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int i = 0; i < 24; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
     float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.0f, 0.0f};
 
-    const int n_pairs = (max(nr, 0) + 1) >> 1;
-    uint8_t *ring = smem + warp * kWarpRing;
-    uint64_t *wbar = bars + warp * kSlots;
-    const int32_t *sel = p.sel_idx + (int64_t)row * p.k + j0;
-
-    // region validity / tensor row of pair slot regions, decided by lane 0, broadcast
-    auto region_row = [&](int j, int &yrow) -> bool {
-        if (bad_req || j >= nr) return false;
-        const int r = sel[j];
-        if (r < 0 || r / 8 >= p.max_pages) {
-            set_error(kErrAttnIndex);
-            return false;
-        }
-        const int64_t page = p.block_table[(int64_t)b * p.max_pages + r / 8];
-        if (page < 0 || page >= p.n_pages) {
-            set_error(kErrAttnIndex);
-            return false;
-        }
-        yrow = (int)((page * kG + g) * kPage + (r % 8) * kRegion);
-        return true;
-    };
-    auto issue = [&](int pi, int slot) {
-        // lane 0 only: load K and V of regions 2pi and 2pi+1 of this warp's pair pi
-        uint8_t *dst = ring + slot * kPairBytes;
-        int y0 = 0, y1 = 0;
-        const int ja = 2 * pi, jb = 2 * pi + 1;
-        const bool va = region_row(ja, y0), vb = region_row(jb, y1);
-        const unsigned bytes = (va ? 2u * kRegionBytes : 0u) + (vb ? 2u * kRegionBytes : 0u);
-        if (bytes == 0) {
-            mbar_arrive(&wbar[slot]);
-            return;
-        }
-        mbar_arrive_expect_tx(&wbar[slot], bytes);
-        if (va) {
-            tma_load_3d(dst, &tmap_k, 0, 0, y0, &wbar[slot]);
-            tma_load_3d(dst + 2 * kRegionBytes, &tmap_v, 0, 0, y0, &wbar[slot]);
-        }
-        if (vb) {
-            tma_load_3d(dst + kRegionBytes, &tmap_k, 0, 0, y1, &wbar[slot]);
-            tma_load_3d(dst + 3 * kRegionBytes, &tmap_v, 0, 0, y1, &wbar[slot]);
-        }
-    };
-
-    // this warp handles pairs warp, warp + 4, ...
-    int my_pairs = 0;
-    for (int pi = warp; pi < n_pairs; pi += kWarps) ++my_pairs;
-    if (lane == 0) {
-        prefetch_tensormap(&tmap_k);
-        prefetch_tensormap(&tmap_v);
-        for (int s = 0; s < kSlots && s < my_pairs; ++s) issue(warp + s * kWarps, s);
-    }
 
     for (int i = 0; i < my_pairs; ++i) {
-        const int pi = warp + i * kWarps;
         const int slot = i % kSlots;
         const unsigned ph = (unsigned)(i / kSlots) & 1u;
-        if (!mbar_wait(&wbar[slot], ph)) break;
-        const uint32_t kt = smem_u32(ring + slot * kPairBytes);
-        const uint32_t vt = kt + 2 * kRegionBytes;
-
-        // validity of the 16 tokens: region ja = 2pi (n-tile 0), jb = 2pi+1 (n-tile 1)
         int rr[2];
         bool rv[2];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int j = 2 * pi + h;
-            rv[h] = false;
-            rr[h] = -1;
-            if (!bad_req && j < nr) {
-                const int r = sel[j];
-                // same checks as the loader (without flagging twice)
-                if (r >= 0 && r / 8 < p.max_pages) {
-                    const int64_t page = p.block_table[(int64_t)b * p.max_pages + r / 8];
-                    if (page >= 0 && page < p.n_pages) {
-                        rv[h] = true;
-                        rr[h] = r;
-                    }
-                }
+        for (int sl = 0; sl < kSlots; ++sl)
+            if (sl == slot) {
+                rr[0] = slot_r[sl][0];
+                rr[1] = slot_r[sl][1];
+                rv[0] = slot_v[sl][0] != 0;
+                rv[1] = slot_v[sl][1] != 0;
             }
-        }
+        if (!mbar_wait(&wbar[slot], ph)) break;
+        const uint32_t kt = smem_u32(ring + slot * kPairBytes);
+        const uint32_t vt = kt + 2 * kRegionBytes;
 
         float s[2][4];
 #pragma unroll
@@ -275,100 +301,162 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         __syncwarp();
         const int next = i + kSlots;
-        if (next < my_pairs && lane == 0) {
-            fence_proxy_async();
-            issue(warp + next * kWarps, slot);
+        if (next < my_pairs) {
+            if (lane == 0) fence_proxy_async();
+            issue(next, slot);
         }
     }
 
-    // ---- merge the 4 warps: write (m, l, O) of each warp to smem (reusing the rings)
+    // ---- merge the 4 warps: (m, l, O) of each warp to smem (reusing the rings), then
+    // element-major combine so that smem reads and global writes are contiguous
+    constexpr int kRow = kD + 8;                                         // padded row (floats)
     __syncthreads();
-    float *red_o = reinterpret_cast<float *>(smem);                      // [4][16][192]
-    float *red_ml = red_o + kWarps * 16 * kD;                            // [4][16][2]
+    float *red_o = reinterpret_cast<float *>(smem);                      // [4][16][kRow]
+    float *red_ml = red_o + kWarps * 16 * kRow;                          // [4][16][2]
+    float *hw = red_ml + kWarps * 16 * 2;                                // [16][4] weights, [16] L, [16] M
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const int hr = gq + 8 * h;
+        float *rowp = red_o + (warp * 16 + hr) * kRow + 2 * t;
 #pragma unroll
-        for (int nd = 0; nd < 24; ++nd) {
-            float *dst = red_o + ((warp * 16 + hr) * kD) + nd * 8 + 2 * t;
-            dst[0] = o[nd][2 * h];
-            dst[1] = o[nd][2 * h + 1];
-        }
+        for (int nd = 0; nd < 24; ++nd)
+            *reinterpret_cast<float2 *>(rowp + nd * 8) = make_float2(o[nd][2 * h], o[nd][2 * h + 1]);
         if (t == 0) {
             red_ml[(warp * 16 + hr) * 2 + 0] = mrow[h];
             red_ml[(warp * 16 + hr) * 2 + 1] = lrow[h];
         }
     }
     __syncthreads();
-    // thread -> (head hr, 24 consecutive dims)
-    {
-        const int hr = threadIdx.x >> 3;              // 16 heads x 8 threads
-        const int d0 = (threadIdx.x & 7) * 24;
+    if (threadIdx.x < 16) {                                              // per-head weights
+        const int hr = threadIdx.x;
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) M = fmaxf(M, red_ml[(w * 16 + hr) * 2]);
         const float Mref = (M == -INFINITY) ? 0.0f : M;
-        float wgt[kWarps], L = 0.0f;
+        float L = 0.0f;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) {
-            wgt[w] = exp2f(red_ml[(w * 16 + hr) * 2] - Mref);
-            L += wgt[w] * red_ml[(w * 16 + hr) * 2 + 1];
+            const float wt = exp2f(red_ml[(w * 16 + hr) * 2] - Mref);
+            hw[hr * 4 + w] = wt;
+            L += wt * red_ml[(w * 16 + hr) * 2 + 1];
         }
-        const int head = g * kHeadsPerGroup + hr;
-        if (p.n_splits == 1) {
+        hw[64 + hr] = L;
+        hw[80 + hr] = M;
+    }
+    __syncthreads();
+    if (p.n_splits == 1) {
+        // element e = (head, d) pair of dims: thread covers pairs e = tid + 128*j
+        for (int e = threadIdx.x; e < 16 * kD / 2; e += kThreads) {
+            const int hr = e / (kD / 2), d = 2 * (e % (kD / 2));
+            float a = 0.0f, c = 0.0f;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) {
+                const float2 v = *reinterpret_cast<const float2 *>(red_o + (w * 16 + hr) * kRow + d);
+                a += hw[hr * 4 + w] * v.x;
+                c += hw[hr * 4 + w] * v.y;
+            }
+            const float L = hw[64 + hr];
             const float inv = (L > 0.0f) ? 1.0f / L : 0.0f;
-            __nv_bfloat16 *dst = p.out + ((int64_t)qi * kHQ + head) * kD + d0;
+            const int head = g * kHeadsPerGroup + hr;
+            *reinterpret_cast<__nv_bfloat162 *>(p.out + ((int64_t)qi * kHQ + head) * kD + d) =
+                __floats2bfloat162_rn(a * inv, c * inv);
+        }
+        if (p.lse && threadIdx.x < 16) {
+            const int hr = threadIdx.x;
+            const float L = hw[64 + hr], M = hw[80 + hr];
+            p.lse[(int64_t)qi * kHQ + g * kHeadsPerGroup + hr] =
+                (L > 0.0f) ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+        }
+    } else {
+        const int64_t pbase = ((int64_t)row * p.n_splits + split) * 16;
+        for (int e = threadIdx.x; e < 16 * kD / 4; e += kThreads) {
+            const int hr = e / (kD / 4), d = 4 * (e % (kD / 4));
+            float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 #pragma unroll
-            for (int d = 0; d < 24; d += 2) {
-                float a = 0.0f, c = 0.0f;
-#pragma unroll
-                for (int w = 0; w < kWarps; ++w) {
-                    a += wgt[w] * red_o[(w * 16 + hr) * kD + d0 + d];
-                    c += wgt[w] * red_o[(w * 16 + hr) * kD + d0 + d + 1];
-                }
-                *reinterpret_cast<__nv_bfloat162 *>(dst + d) = __floats2bfloat162_rn(a * inv, c * inv);
+            for (int w = 0; w < kWarps; ++w) {
+                const float4 v = *reinterpret_cast<const float4 *>(red_o + (w * 16 + hr) * kRow + d);
+                const float wt = hw[hr * 4 + w];
+                acc.x += wt * v.x;
+                acc.y += wt * v.y;
+                acc.z += wt * v.z;
+                acc.w += wt * v.w;
             }
-            if (p.lse && (threadIdx.x & 7) == 0)
-                p.lse[(int64_t)qi * kHQ + head] = (L > 0.0f) ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
-        } else {
-            const int64_t pidx = ((int64_t)row * p.n_splits + split) * 16 + hr;
-            float *dst = p.part_o + pidx * kD + d0;
-#pragma unroll
-            for (int d = 0; d < 24; ++d) {
-                float a = 0.0f;
-#pragma unroll
-                for (int w = 0; w < kWarps; ++w) a += wgt[w] * red_o[(w * 16 + hr) * kD + d0 + d];
-                dst[d] = a;
-            }
-            if ((threadIdx.x & 7) == 0) {
-                p.part_ml[pidx * 2 + 0] = M;
-                p.part_ml[pidx * 2 + 1] = L;
-            }
+            *reinterpret_cast<float4 *>(p.part_o + (pbase + hr) * kD + d) = acc;
+        }
+        if (threadIdx.x < 16) {
+            const int hr = threadIdx.x;
+            p.part_ml[(pbase + hr) * 2 + 0] = hw[80 + hr];
+            p.part_ml[(pbase + hr) * 2 + 1] = hw[64 + hr];
         }
     }
 }
 
 // Merges the per-split partials of one (query, head): O = sum_s 2^(m_s - M) O_s / L.
-__global__ void __launch_bounds__(kD) combine_kernel(const Params p)
+// 4 x 192 threads: thread (sg, d) sums splits sg, sg+4, ... of dimension d with all its
+// loads in flight, then the 4 partial sums meet in smem.
+constexpr int kCombineThreads = 4 * kD;
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const Params p)
 {
+    __shared__ float wsm[kD];
+    __shared__ float part[kCombineThreads / 32];
+    __shared__ float red[2];
+    __shared__ float osum[4][kD];
     const int row = blockIdx.x >> 4, hr = blockIdx.x & 15;
     const int qi = row >> 2, g = row & 3;
-    const int d = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int d = tid % kD, sg = tid / kD;
     const int cnt = min(max(p.sel_count[row], 0), p.k);
-    const int ns = min(p.n_splits, (cnt + p.rps - 1) / p.rps);
-    float M = -INFINITY;
-    for (int s = 0; s < ns; ++s) M = fmaxf(M, p.part_ml[(((int64_t)row * p.n_splits + s) * 16 + hr) * 2]);
-    const float Mref = (M == -INFINITY) ? 0.0f : M;
-    float L = 0.0f, acc = 0.0f;
-    for (int s = 0; s < ns; ++s) {
-        const int64_t pidx = ((int64_t)row * p.n_splits + s) * 16 + hr;
-        const float w = exp2f(p.part_ml[pidx * 2] - Mref);
-        L += w * p.part_ml[pidx * 2 + 1];
-        acc += w * p.part_o[pidx * kD + d];
+    const int ns = min(p.n_splits, (cnt + p.rps - 1) / p.rps);   // <= kD (host-checked)
+    const int64_t pbase = (int64_t)row * p.n_splits * 16 + hr;
+    float m = -INFINITY, l = 0.0f;
+    if (tid < ns) {
+        m = p.part_ml[(pbase + (int64_t)tid * 16) * 2];
+        l = p.part_ml[(pbase + (int64_t)tid * 16) * 2 + 1];
     }
-    const int head = g * kHeadsPerGroup + hr;
-    p.out[((int64_t)qi * kHQ + head) * kD + d] = __float2bfloat16_rn(L > 0.0f ? acc / L : 0.0f);
-    if (p.lse && d == 0) p.lse[(int64_t)qi * kHQ + head] = (L > 0.0f) ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+    float mx = m;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) part[w] = mx;
+    __syncthreads();
+    if (tid == 0) {
+        float M = -INFINITY;
+        for (int i = 0; i < kCombineThreads / 32; ++i) M = fmaxf(M, part[i]);
+        red[0] = M;
+    }
+    __syncthreads();
+    const float M = red[0];
+    const float Mref = (M == -INFINITY) ? 0.0f : M;
+    const float wt = (tid < ns) ? exp2f(m - Mref) : 0.0f;
+    if (tid < kD) wsm[tid] = wt;
+    float lw = wt * l;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
+    __syncthreads();
+    if (lane == 0) part[w] = lw;
+    __syncthreads();
+    if (tid == 0) {
+        float L = 0.0f;
+        for (int i = 0; i < kCombineThreads / 32; ++i) L += part[i];
+        red[1] = L;
+    }
+    __syncthreads();
+    const float L = red[1];
+    float acc[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+    int s = sg;
+    for (; s + 28 < ns; s += 32) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) acc[u] += wsm[s + 4 * u] * p.part_o[(pbase + (int64_t)(s + 4 * u) * 16) * kD + d];
+    }
+    for (; s < ns; s += 4) acc[0] += wsm[s] * p.part_o[(pbase + (int64_t)s * 16) * kD + d];
+    osum[sg][d] = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+    __syncthreads();
+    if (sg == 0) {
+        const float o = (osum[0][d] + osum[1][d]) + (osum[2][d] + osum[3][d]);
+        const int head = g * kHeadsPerGroup + hr;
+        p.out[((int64_t)qi * kHQ + head) * kD + d] = __float2bfloat16_rn(L > 0.0f ? o / L : 0.0f);
+        if (p.lse && d == 0)
+            p.lse[(int64_t)qi * kHQ + head] = (L > 0.0f) ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+    }
 }
 
 }  // namespace attn

@@ -95,6 +95,21 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, unsigned parity)
     return true;
 }
 
+// 4-byte asynchronous global->shared copy; zero-fills (reads nothing) when !valid.
+__device__ __forceinline__ void cp_async_4(void *smem_dst, const void *gmem_src, bool valid)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src),
+                 "r"(valid ? 4 : 0)
+                 : "memory");
+}
+
+// The mbarrier receives one arrival when all cp.async copies this thread issued so far
+// have completed (the arrival is one of the barrier's expected count: .noinc).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t *bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // ------------------------------------------------------------------ TMA (no multicast)
 
 __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *map, int x, int y, uint64_t *bar)

@@ -2,6 +2,7 @@
 // arguments, sizes grids, encodes TMA tensor maps and launches the kernels of
 // compress.cuh, indexer.cuh, topk.cuh and attention.cuh (one translation unit, so the
 // per-device error word is a single symbol).
+#include <algorithm>
 #include <mutex>
 #include <string>
 
@@ -11,6 +12,7 @@
 #include "compress.cuh"
 #include "indexer.cuh"
 #include "topk.cuh"
+#include "topk_cluster.cuh"
 
 namespace {
 
@@ -133,7 +135,13 @@ AttnPlan attn_plan(int nq, int k, int sm_count)
         a.n_splits = 1;
         a.ws = 0;
     } else {
-        a.rps = 16;
+        // about 2 CTAs per SM over all rows, at least 2 regions (one pair) per CTA and at
+        // most kD splits (the combine kernel holds one split weight per thread)
+        const int want = std::max(1, (2 * sm_count + rows - 1) / rows);
+        int rps = (k + want - 1) / want;
+        rps = std::max(2, (rps + 1) & ~1);
+        while ((k + rps - 1) / rps > dsa::kD) rps += 2;
+        a.rps = rps;
         a.n_splits = (k + a.rps - 1) / a.rps;
         const size_t n = (size_t)rows * a.n_splits * 16;
         a.ws = round_up(n * dsa::kD * 4, 256) + round_up(n * 2 * 4, 256);
@@ -201,10 +209,80 @@ dsa_status_t attn_common(const void *q, const void *k_cache, const void *v_cache
     dsa::attn::sparse_attn_kernel<<<grid, dsa::attn::kThreads, dsa::attn::kSmemBytes, stream>>>(mk, mv, p);
     if ((st = launched("sparse_attn_kernel")) != DSA_OK) return st;
     if (plan.n_splits > 1) {
-        dsa::attn::combine_kernel<<<nq * dsa::kG * 16, dsa::kD, 0, stream>>>(p);
+        dsa::attn::combine_kernel<<<nq * dsa::kG * 16, dsa::attn::kCombineThreads, 0, stream>>>(p);
         if ((st = launched("combine_kernel")) != DSA_OK) return st;
     }
     return DSA_OK;
+}
+
+// Workspace path of the top-k: histogram, threshold-bin gather and last-CTA selection
+// (scales to many rows; scratch from the caller's workspace).
+dsa_status_t topk_workspace_path(const float *scores, int64_t ld_scores, const int32_t *q_pos, int nq, int k,
+                                 int32_t *sel_idx, int32_t *sel_count, void *ws, size_t ws_bytes, dsa_stream_t stream)
+{
+    const TopkLayout L = topk_layout(nq, ld_scores, k);
+    if (!ws || ws_bytes < L.total || reinterpret_cast<uintptr_t>(ws) % 256 != 0)
+        return fail(DSA_ERR_WORKSPACE, "top-k workspace too small or not 256-byte aligned (need " +
+                                           std::to_string(L.total) + " bytes)");
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    dsa::topk::Ws tw;
+    tw.hist = reinterpret_cast<uint32_t *>(w + L.hist);
+    tw.ctr = reinterpret_cast<uint32_t *>(w + L.ctr);
+    tw.sure = reinterpret_cast<int32_t *>(w + L.sure);
+    tw.cand = reinterpret_cast<uint2 *>(w + L.cand);
+    DSA_CUDA(cudaMemsetAsync(w, 0, L.sure, stream), "cudaMemsetAsync(top-k histograms)");
+    const int rows = nq * dsa::kG;
+    const dim3 grid((unsigned)((ld_scores + dsa::topk::kChunk - 1) / dsa::topk::kChunk), (unsigned)rows);
+    dsa_status_t st;
+    dsa::topk::hist_kernel<<<grid, dsa::topk::kThreads, 0, stream>>>(scores, ld_scores, q_pos, k, tw);
+    if ((st = launched("topk hist_kernel")) != DSA_OK) return st;
+    const size_t dyn = dsa::topk::kCandStage * 8 + round_up((size_t)((ld_scores + 1 + 31) / 32) * 4, 16);
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(dsa::topk::select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)(dsa::topk::kCandStage * 8 + (dsa::topk::kMaxRegions / 32 + 16) * 4));
+    });
+    DSA_CUDA(attr_err, "cudaFuncSetAttribute(topk select_kernel)");
+    dsa::topk::select_kernel<<<grid, dsa::topk::kSelectThreads, dyn, stream>>>(scores, ld_scores, q_pos, k, tw,
+                                                                              sel_idx, sel_count);
+    return launched("topk select_kernel");
+}
+
+// Cluster size for the cluster path: enough CTAs that each holds <= kPartMax keys in smem
+// (power of two, at most 8); 0 when a row is too long for it.
+int cluster_size_for(int64_t ld)
+{
+    int cl = 1;
+    while ((int64_t)cl * dsa::topkc::kPartMax < ld) cl *= 2;
+    return cl <= dsa::topkc::kMaxCluster ? cl : 0;
+}
+
+dsa_status_t topk_cluster_path(const float *scores, int64_t ld_scores, const int32_t *q_pos, int nq, int k,
+                               int32_t *sel_idx, int32_t *sel_count, int cl, dsa_stream_t stream)
+{
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(dsa::topkc::topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)dsa::topkc::kSmemBytes);
+    });
+    DSA_CUDA(attr_err, "cudaFuncSetAttribute(topk_cluster_kernel)");
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)cl, (unsigned)(nq * dsa::kG), 1);
+    cfg.blockDim = dim3(dsa::topkc::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = dsa::topkc::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cl;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    DSA_CUDA(cudaLaunchKernelEx(&cfg, dsa::topkc::topk_cluster_kernel, scores, ld_scores, q_pos, k, sel_idx, sel_count),
+             "cudaLaunchKernelEx(topk_cluster_kernel)");
+    return launched("topk_cluster_kernel");
 }
 
 // Scratch of dsa_topk_regions_noalloc: one static array per GPU that loads the library.
@@ -310,7 +388,7 @@ dsa_status_t dsa_indexer_scores(const void *index_q, const float *gate, const in
         const cuuint64_t strides[1] = {(cuuint64_t)dsa::kDI};
         const cuuint32_t box[2] = {128, (cuuint32_t)dsa::idx::kChunk};
         if ((st = encode(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, summaries, dims, strides, box,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B)) != DSA_OK)
+                         (CUtensorMapL2promotion)DSA_SCAN_L2_PROMOTION)) != DSA_OK)
             return st;
     }
     dsa::idx::Params p{};
@@ -336,7 +414,7 @@ dsa_status_t dsa_indexer_scores(const void *index_q, const float *gate, const in
                                         (int)dsa::idx::kSmemBytes);
     });
     DSA_CUDA(attr_err, "cudaFuncSetAttribute(scan_kernel)");
-    const int grid = (int)std::min<int64_t>(p.total_units, (int64_t)sms * 2);
+    const int grid = (int)std::min<int64_t>(p.total_units, (int64_t)sms * dsa::idx::kCtasPerSm);
     dsa::idx::scan_kernel<<<grid, dsa::idx::kThreads, dsa::idx::kSmemBytes, stream>>>(map, p);
     return launched("scan_kernel");
 }
@@ -355,37 +433,14 @@ dsa_status_t dsa_topk_regions(const float *scores, int64_t ld_scores, const int3
     DSA_REQUIRE(ld_scores >= 1 && ld_scores < dsa::topk::kMaxRegions, "ld_scores out of [1, 2^20)");
     if (nq == 0) return DSA_OK;
     DSA_REQUIRE(scores && q_pos && sel_idx && sel_count, "NULL pointer");
-    const TopkLayout L = topk_layout(nq, ld_scores, k);
-    if (!ws || ws_bytes < L.total || !aligned(ws, 256))
-        return fail(DSA_ERR_WORKSPACE, "top-k workspace too small or not 256-byte aligned (need " +
-                                           std::to_string(L.total) + " bytes)");
     int sms = 0;
     dsa_status_t st = device_info(sms);
     if (st != DSA_OK) return st;
-    uint8_t *w = static_cast<uint8_t *>(ws);
-    dsa::topk::Ws tw;
-    tw.hist = reinterpret_cast<uint32_t *>(w + L.hist);
-    tw.ctr = reinterpret_cast<uint32_t *>(w + L.ctr);
-    tw.sure = reinterpret_cast<int32_t *>(w + L.sure);
-    tw.cand = reinterpret_cast<uint2 *>(w + L.cand);
-    DSA_CUDA(cudaMemsetAsync(w, 0, L.sure, stream), "cudaMemsetAsync(top-k histograms)");
     const int rows = nq * dsa::kG;
-    const dim3 grid((unsigned)((ld_scores + dsa::topk::kChunk - 1) / dsa::topk::kChunk), (unsigned)rows);
-    dsa::topk::hist_kernel<<<grid, dsa::topk::kThreads, 0, stream>>>(scores, ld_scores, q_pos, k, tw);
-    if ((st = launched("topk hist_kernel")) != DSA_OK) return st;
-    dsa::topk::gather_kernel<<<grid, dsa::topk::kThreads, 0, stream>>>(scores, ld_scores, q_pos, k, tw);
-    if ((st = launched("topk gather_kernel")) != DSA_OK) return st;
-    const size_t bitmap = round_up((size_t)((ld_scores + 1 + 31) / 32) * 4, 16);
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(dsa::topk::final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)((dsa::topk::kMaxRegions / 32 + 16) * 4));
-    });
-    DSA_CUDA(attr_err, "cudaFuncSetAttribute(topk final_kernel)");
-    dsa::topk::final_kernel<<<rows, dsa::topk::kFinalThreads, bitmap, stream>>>(q_pos, ld_scores, k, tw, sel_idx,
-                                                                               sel_count);
-    return launched("topk final_kernel");
+    const int cl = cluster_size_for(ld_scores);
+    if (cl > 0 && (int64_t)rows * cl <= 2 * sms) return topk_cluster_path(scores, ld_scores, q_pos, nq, k, sel_idx,
+                                                                           sel_count, cl, stream);
+    return topk_workspace_path(scores, ld_scores, q_pos, nq, k, sel_idx, sel_count, ws, ws_bytes, stream);
 }
 
 dsa_status_t dsa_topk_regions_noalloc(const float *scores, int64_t ld_scores, const int32_t *q_pos, int nq, int k,
@@ -406,7 +461,7 @@ dsa_status_t dsa_topk_regions_noalloc(const float *scores, int64_t ld_scores, co
     void *ws = nullptr;
     dsa_status_t st = static_scratch(dev, &ws);
     if (st != DSA_OK) return st;
-    return dsa_topk_regions(scores, ld_scores, q_pos, nq, k, sel_idx, sel_count, ws, need, stream);
+    return topk_workspace_path(scores, ld_scores, q_pos, nq, k, sel_idx, sel_count, ws, need, stream);
 }
 
 size_t dsa_attn_workspace_size(int nq, int k)

@@ -28,13 +28,30 @@
 namespace dsa {
 namespace idx {
 
-constexpr int kChunk = 32;                         // regions per stage
-constexpr int kStages = 3;
+// Pipeline shape (compile-time tunables; the defaults are the measured best on B200).
+#ifndef DSA_SCAN_STAGES
+#define DSA_SCAN_STAGES 3
+#endif
+#ifndef DSA_SCAN_CTAS_PER_SM
+#define DSA_SCAN_CTAS_PER_SM 2
+#endif
+#ifndef DSA_SCAN_CHUNK
+#define DSA_SCAN_CHUNK 32
+#endif
+#ifndef DSA_SCAN_L2_PROMOTION
+#define DSA_SCAN_L2_PROMOTION 3          // CU_TENSOR_MAP_L2_PROMOTION_L2_256B
+#endif
+constexpr int kChunk = DSA_SCAN_CHUNK;             // regions per stage (multiple of 32)
+constexpr int kStages = DSA_SCAN_STAGES;
+constexpr int kCtasPerSm = DSA_SCAN_CTAS_PER_SM;
 constexpr int kHalfBytes = kChunk * 128;           // one 128-byte column half of a group tile
-constexpr int kGroupBytes = 2 * kHalfBytes;        // 8 KiB
-constexpr int kStageBytes = kG * kGroupBytes;      // 32 KiB
+constexpr int kGroupBytes = 2 * kHalfBytes;        // 8 KiB at 32 regions
+constexpr int kStageBytes = kG * kGroupBytes;      // 32 KiB at 32 regions
+constexpr int kTiles = kChunk / 16;                // m16 tiles per group per stage
 constexpr int kThreads = 160;                      // 4 consumer warps + 1 producer warp
-constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + 1024 /*align*/ + 64 /*barriers*/;
+constexpr int kScaleBytes = kG * kChunk * 4;       // fp32 scales of one stage (512 B)
+constexpr size_t kSmemBytes =
+    (size_t)kStages * (kStageBytes + kScaleBytes) + 1024 /*align*/ + 64 /*barriers*/;
 
 struct Params {
     const __nv_bfloat16 *index_q;
@@ -133,18 +150,19 @@ __device__ __forceinline__ void load_query_fragments(const Params &p, int qi, in
     z_t = __ldg(p.gate + (int64_t)qi * kHI + g * 4 + t);
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
     scan_kernel(const __grid_constant__ CUtensorMap tmap, const Params p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kStages * kStageBytes);
+    float *sscale = reinterpret_cast<float *>(smem + kStages * kStageBytes);      // [kStages][4][32]
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kStages * (kStageBytes + kScaleBytes));
     uint64_t *empty = full + kStages;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], 1 + 32);   // expect_tx arrive + one arrive per producer lane (scales)
             mbar_init(&empty[s], kG);
         }
         fence_mbar_init();
@@ -155,19 +173,22 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int64_t u_end = (int64_t)(blockIdx.x + 1) * p.total_units / gridDim.x;
 
     if (warp == kG) {
-        // ---------------- producer: one elected lane issues the TMA loads
-        if (lane == 0) {
-            prefetch_tensormap(&tmap);
-            int it = 0;
-            for (int64_t u = u_begin; u < u_end; ++u) {
-                const int qi = (int)(u / p.units_per_query);
-                const int64_t r0 = (u % p.units_per_query) * kChunk;
-                int64_t base;
-                const int64_t own = query_own(p, qi, base);
-                if (own < 0 || r0 >= own) continue;
-                const int s = it % kStages;
-                const unsigned ph = (unsigned)(it / kStages) & 1u;
-                if (!mbar_wait(&empty[s], ph ^ 1u)) break;
+        // ---------------- producer warp: lane 0 issues the TMA loads of the summaries; every
+        // lane copies 4 of the stage's 128 fp32 scales into smem asynchronously
+        if (lane == 0) prefetch_tensormap(&tmap);
+        int it = 0;
+        constexpr int kScalesPerLane = kG * kChunk / 32;          // 4 at 32 regions per stage
+        const int sg = (lane * kScalesPerLane) / kChunk, sr = (lane * kScalesPerLane) % kChunk;
+        for (int64_t u = u_begin; u < u_end; ++u) {
+            const int qi = (int)(u / p.units_per_query);
+            const int64_t r0 = (u % p.units_per_query) * kChunk;
+            int64_t base;
+            const int64_t own = query_own(p, qi, base);
+            if (own < 0 || r0 >= own) continue;
+            const int s = it % kStages;
+            const unsigned ph = (unsigned)(it / kStages) & 1u;
+            if (!mbar_wait(&empty[s], ph ^ 1u)) break;
+            if (lane == 0) {
                 mbar_arrive_expect_tx(&full[s], kStageBytes);
                 uint8_t *st = smem + s * kStageBytes;
 #pragma unroll
@@ -176,8 +197,17 @@ __global__ void __launch_bounds__(kThreads, 2)
                     tma_load_2d(st + g * kGroupBytes, &tmap, 0, y, &full[s]);
                     tma_load_2d(st + g * kGroupBytes + kHalfBytes, &tmap, 128, y, &full[s]);
                 }
-                ++it;
             }
+            // scales: asynchronous 4-byte copies that arrive on the stage's barrier when they
+            // land, so the producer never waits for them
+            const float *srow = p.scales + sg * p.n_slots + base;
+#pragma unroll
+            for (int e = 0; e < kScalesPerLane; ++e) {
+                const int64_t r = r0 + sr + e;
+                cp_async_4(sscale + (s * kG + sg) * kChunk + sr + e, srow + (r < own ? r : 0), r < own);
+            }
+            cp_async_mbar_arrive(&full[s]);
+            ++it;
         }
         return;
     }
@@ -203,23 +233,19 @@ __global__ void __launch_bounds__(kThreads, 2)
             load_query_fragments(p, qi, g, lane, bfrag, sq_t, z_t);
             cached_q = qi;
         }
-        // scales of this lane's 4 rows (tile m: rows n and n+8)
-        float sc[2][2];
-#pragma unroll
-        for (int m = 0; m < 2; ++m)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int64_t r = r0 + 16 * m + 8 * h + n;
-                sc[m][h] = (r < own) ? __ldg(p.scales + g * p.n_slots + base + r) : 0.0f;
-            }
-
         const int s = it % kStages;
         const unsigned ph = (unsigned)(it / kStages) & 1u;
         if (!mbar_wait(&full[s], ph)) break;
-        const uint32_t tile = smem_u32(smem + s * kStageBytes + g * kGroupBytes);
-        float acc[2][4];
+        // scales of this lane's 4 rows (tile m: rows n and n+8), staged by the producer
+        float sc[kTiles][2];
 #pragma unroll
-        for (int m = 0; m < 2; ++m) {
+        for (int m = 0; m < kTiles; ++m)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) sc[m][h] = sscale[(s * kG + g) * kChunk + 16 * m + 8 * h + n];
+        const uint32_t tile = smem_u32(smem + s * kStageBytes + g * kGroupBytes);
+        float acc[kTiles][4];
+#pragma unroll
+        for (int m = 0; m < kTiles; ++m) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[m][e] = 0.0f;
             // ldmatrix.x4: lane l addresses row (16m + 8*((l>>3)&1) + (l&7)), 16-byte chunk
@@ -240,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 
         float *out = p.scores + ((int64_t)qi * kG + g) * p.ld;
 #pragma unroll
-        for (int m = 0; m < 2; ++m) {
+        for (int m = 0; m < kTiles; ++m) {
             float v0 = z_t * fmaxf((acc[m][0] + acc[m][1]) * sq_t * sc[m][0], 0.0f);
             float v1 = z_t * fmaxf((acc[m][2] + acc[m][3]) * sq_t * sc[m][1], 0.0f);
             v0 += __shfl_xor_sync(0xffffffffu, v0, 1);

@@ -5,15 +5,33 @@ A decode step for a batch of requests, one query each, is
     indexer scores over every complete region     (A2)
     top-k with the own region forced              (A3)
     sparse attention over the selected regions    (A4)
-([P2] Step-5-Preview 如何实现1M长上下文 §区域压缩CSA / §索引器打分).  All buffers are
-allocated once, so a step can be captured in a CUDA graph and replayed.
+([P2] Step-5-Preview 如何实现1M长上下文 §区域压缩CSA / §索引器打分).
+
+The region a decode token completes is always the query's own region (token p completes
+region p/8 exactly when p % 8 == 7), and the own region is forced, never scored.  So this
+step's scan never reads what this step's compression writes, and the compression runs on
+a parallel branch (a side stream joined at the end of the step); the next step sees it.
+
+All buffers are allocated once, so a step can be captured in a CUDA graph and replayed.
+The per-step inputs live in one device arena (index_q, gate, q, q_pos and, optionally,
+the 8-token tails whose regions complete), so a host caller refreshes them with a single
+host-to-device copy of `arena`.
 """
 from __future__ import annotations
 
 import torch
 
 from . import dsa
-from .dsa import G, HQ, D, REGION
+from .dsa import G, HQ, D, DI, HI, REGION
+
+
+def _carve(arena: torch.Tensor, off: int, shape, dtype) -> tuple:
+    n = 1
+    for s in shape:
+        n *= s
+    nbytes = n * torch.tensor([], dtype=dtype).element_size()
+    view = arena[off: off + nbytes].view(dtype).view(*shape)
+    return view, off + (nbytes + 255) // 256 * 256
 
 
 class DecodeStep:
@@ -21,24 +39,34 @@ class DecodeStep:
 
     summaries/scales: the group-major pool; sum_base int64 [B]; block_table int32 [B][P];
     k_cache/v_cache bf16 [pages][4][64][192]; ld: score row length (>= max own region).
-    Per-step inputs (index_q, gate, q, q_pos, compress lists) are copied into the
-    step's own tensors by `load`, so graph replays see new values."""
+    tail_tokens = 8 gives the step an input tail buffer (bf16 [B*8][4][256]) whose
+    regions are compressed when `set_compress` lists them."""
 
     def __init__(self, summaries, scales, sum_base, block_table, k_cache, v_cache, ld, k=512,
-                 max_compress=0, index_k=None, flags=0):
+                 tail_tokens=0, flags=0):
         dev = summaries.device
-        self.B = int(block_table.shape[0])
+        self.B = B = int(block_table.shape[0])
         self.k = int(k)
         self.ld = int(ld)
         self.flags = flags
         self.summaries, self.scales, self.sum_base = summaries, scales, sum_base
         self.block_table, self.k_cache, self.v_cache = block_table, k_cache, v_cache
-        self.index_k = index_k
-        B = self.B
-        self.index_q = torch.zeros((B, dsa.HI, dsa.DI), dtype=torch.bfloat16, device=dev)
-        self.gate = torch.zeros((B, dsa.HI), dtype=torch.float32, device=dev)
-        self.q = torch.zeros((B, HQ, D), dtype=torch.bfloat16, device=dev)
-        self.q_pos = torch.zeros(B, dtype=torch.int32, device=dev)
+        # per-step inputs: one arena
+        size = 0
+        for shape, dt in (((B, HI, DI), torch.bfloat16), ((B, HI), torch.float32), ((B, HQ, D), torch.bfloat16),
+                          ((B,), torch.int32), ((B * max(tail_tokens, 1), G, DI), torch.bfloat16)):
+            n = 1
+            for s in shape:
+                n *= s
+            size += (n * torch.tensor([], dtype=dt).element_size() + 255) // 256 * 256
+        self.arena = torch.zeros(size, dtype=torch.uint8, device=dev)
+        off = 0
+        self.index_q, off = _carve(self.arena, off, (B, HI, DI), torch.bfloat16)
+        self.gate, off = _carve(self.arena, off, (B, HI), torch.float32)
+        self.q, off = _carve(self.arena, off, (B, HQ, D), torch.bfloat16)
+        self.q_pos, off = _carve(self.arena, off, (B,), torch.int32)
+        self.tail, off = _carve(self.arena, off, (B * max(tail_tokens, 1), G, DI), torch.bfloat16)
+        self.tail_tokens = tail_tokens
         self.q_req = torch.arange(B, dtype=torch.int32, device=dev)
         self.scores = torch.zeros((B, G, self.ld), dtype=torch.float32, device=dev)
         self.sel_idx = torch.empty((B, G, self.k), dtype=torch.int32, device=dev)
@@ -46,9 +74,9 @@ class DecodeStep:
         self.out = torch.empty((B, HQ, D), dtype=torch.bfloat16, device=dev)
         self.lse = torch.empty((B, HQ), dtype=torch.float32, device=dev)
         self.n_compress = 0
-        self.src_row = torch.zeros(max(1, max_compress), dtype=torch.int64, device=dev)
-        self.dst_slot = torch.zeros(max(1, max_compress), dtype=torch.int64, device=dev)
-        # workspaces (allocated once)
+        self.src_row = torch.zeros(max(1, B), dtype=torch.int64, device=dev)
+        self.dst_slot = torch.zeros(max(1, B), dtype=torch.int64, device=dev)
+        self.side = torch.cuda.Stream(device=dev)
         L = dsa.lib()
         self.ws_idx_n = L.dsa_indexer_workspace_size(B, self.ld)
         self.ws_topk_n = L.dsa_topk_workspace_size(B, self.ld, self.k)
@@ -57,15 +85,21 @@ class DecodeStep:
         self.ws_topk = torch.empty(max(1, self.ws_topk_n), dtype=torch.uint8, device=dev)
         self.ws_attn = torch.empty(max(1, self.ws_attn_n), dtype=torch.uint8, device=dev)
 
-    def load(self, index_q, gate, q, q_pos, src_row=None, dst_slot=None):
+    def load(self, index_q, gate, q, q_pos, tail=None):
         self.index_q.copy_(index_q, non_blocking=True)
         self.gate.copy_(gate, non_blocking=True)
         self.q.copy_(q, non_blocking=True)
         self.q_pos.copy_(q_pos, non_blocking=True)
-        n = 0 if src_row is None else int(src_row.numel())
+        if tail is not None:
+            self.tail.copy_(tail, non_blocking=True)
+
+    def set_compress(self, requests, slots):
+        """Regions to compress this step: tail block i (rows 8i..8i+7 of `tail`) of each
+        listed request goes to pool slot slots[j]."""
+        n = len(requests)
         if n:
-            self.src_row[:n].copy_(src_row, non_blocking=True)
-            self.dst_slot[:n].copy_(dst_slot, non_blocking=True)
+            self.src_row[:n].copy_(torch.tensor([REGION * int(b) for b in requests], dtype=torch.int64))
+            self.dst_slot[:n].copy_(torch.tensor([int(s) for s in slots], dtype=torch.int64))
         self.n_compress = n
 
     def run(self, pre_scan=None, post_scan=None):
@@ -73,13 +107,16 @@ class DecodeStep:
         optional callables invoked right before/after the indexer-scan launch (the
         benchmark records timing events there)."""
         L = dsa.lib()
-        st = dsa._stream()
+        main = torch.cuda.current_stream()
         p = dsa._p
         if self.n_compress:
-            ik = self.index_k
-            dsa._check(L.dsa_compress_regions(p(ik), ik[0].numel(), ik.shape[0], p(self.src_row), p(self.dst_slot),
-                                              self.n_compress, p(self.summaries), p(self.scales),
-                                              self.summaries.shape[1], st))
+            self.side.wait_stream(main)
+            with torch.cuda.stream(self.side):
+                t = self.tail
+                dsa._check(L.dsa_compress_regions(p(t), t[0].numel(), t.shape[0], p(self.src_row), p(self.dst_slot),
+                                                  self.n_compress, p(self.summaries), p(self.scales),
+                                                  self.summaries.shape[1], dsa._stream()))
+        st = dsa._stream()
         if pre_scan is not None:
             pre_scan()
         dsa._check(L.dsa_indexer_scores(p(self.index_q), p(self.gate), p(self.q_req), p(self.q_pos), self.B,
@@ -94,6 +131,8 @@ class DecodeStep:
                                             p(self.block_table), self.block_table.shape[1], p(self.q_pos), self.B,
                                             p(self.sel_idx), p(self.sel_count), self.k, p(self.out), p(self.lse),
                                             p(self.ws_attn), self.ws_attn_n, st))
+        if self.n_compress:
+            main.wait_stream(self.side)
         return self.out
 
 

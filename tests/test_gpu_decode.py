@@ -42,12 +42,14 @@ def test_decode_step_against_oracle(case):
     lengths_before = [L - 1 for L in d["lengths"]]
     pipeline.compress_all(d["index_k"], lengths_before, d["tok_base"], d["sum_base"], S, C)
     ld = max(d["lengths"]) // 8
-    due_src = [int(d["tok_base"][b]) + 8 * ((L - 1) // 8) for b, L in enumerate(d["lengths"]) if L % 8 == 0]
-    due_dst = [int(d["sum_base"][b]) + (L - 1) // 8 for b, L in enumerate(d["lengths"]) if L % 8 == 0]
     step = pipeline.DecodeStep(S, C, d["sum_base"], d["block_table"], d["k_cache"], d["v_cache"], ld, k=k,
-                               max_compress=len(due_src), index_k=d["index_k"])
-    step.load(d["index_q"], d["gate"], d["q"], d["q_pos"], torch.tensor(due_src, device=dev),
-              torch.tensor(due_dst, device=dev))
+                               tail_tokens=8)
+    # tail block b = the last 8 tokens of request b; compressed when the query completes it
+    tail = torch.cat([d["index_k"][int(d["tok_base"][b]) + L - 8: int(d["tok_base"][b]) + L]
+                      for b, L in enumerate(d["lengths"])])
+    step.load(d["index_q"], d["gate"], d["q"], d["q_pos"], tail)
+    due = [b for b, L in enumerate(d["lengths"]) if L % 8 == 0]
+    step.set_compress(due, [int(d["sum_base"][b]) + (d["lengths"][b] - 1) // 8 for b in due])
     step.run()
     dsa.check_device()
 

@@ -73,6 +73,26 @@ def test_one_million_token_row():
     check(s.astype(np.float32), [8 * 131072 - 1], 512)
 
 
+def test_many_rows_take_the_workspace_path():
+    # more (query, group) rows than the cluster path takes: histogram + select kernels
+    rng = np.random.default_rng(6)
+    nq, ld = 100, 3000
+    s = rng.standard_normal((nq, G, ld)).astype(np.float32)
+    s[::7] = np.round(s[::7])                     # some tie-heavy rows
+    q_pos = [int(x) for x in rng.integers(0, 8 * ld + 1, nq)]
+    check(s, q_pos, 512)
+
+
+def test_cluster_path_long_rows_and_ties():
+    # rows long enough for 8-CTA clusters, with a plateau of equal scores at the threshold
+    rng = np.random.default_rng(7)
+    ld = 120000
+    s = rng.standard_normal((2, G, ld)).astype(np.float32)
+    s[0, 0, :5000] = 2.5
+    s[1, 3, :] = 0.0
+    check(s, [8 * ld, 8 * 70000 + 3], 512)
+
+
 def test_own_beyond_ld_is_flagged():
     s = np.zeros((1, G, 10), np.float32)
     sc = torch.from_numpy(s).cuda()
