@@ -30,7 +30,7 @@ namespace idx {
 
 // Pipeline shape (compile-time tunables; the defaults are the measured best on B200).
 #ifndef DSA_SCAN_STAGES
-#define DSA_SCAN_STAGES 3
+#define DSA_SCAN_STAGES 2
 #endif
 #ifndef DSA_SCAN_CTAS_PER_SM
 #define DSA_SCAN_CTAS_PER_SM 2

@@ -132,6 +132,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __shared__ uint32_t sh_above, sh_binc, sh_run;
     __shared__ uint32_t slice_tot[kMaxCluster];
     __shared__ uint32_t sh_ccount, sh_L;
+    __shared__ uint32_t off_s[kMaxCluster + 1];
 
     cg::cluster_group cluster = cg::this_cluster();
     const int CL = (int)cluster.num_blocks();
@@ -148,6 +149,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int cnt = (int)(hi - lo);
     const bool in_smem = part <= kPartMax;
     const float *src = scores + (int64_t)row * ld + lo;
+    // rank 0 samples every st-th score of the row (for the fast path's lower bound); its
+    // loads are issued together with the key loads
+    const bool trivial = (need == 0 || need == own);
+    const int64_t st = max((int64_t)1, own / kSample);
+    const uint32_t ns = (uint32_t)min((int64_t)kSample, (own + st - 1) / st);
+    constexpr int kSPer = kSample / kThreads;
+    float sv[kSPer];
+    if (rank == 0 && !trivial) {
+        const float *row_src = scores + (int64_t)row * ld;
+#pragma unroll
+        for (int u = 0; u < kSPer; ++u) {
+            const uint32_t j = u * kThreads + tid;
+            sv[u] = j < ns ? __ldcg(row_src + (int64_t)j * st) : 0.0f;
+        }
+    }
     if (in_smem) {
         // all loads of this thread in flight at once (<= 32 at part <= kPartMax)
         constexpr int kMaxPer = kPartMax / kThreads;
@@ -169,25 +185,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     // rank 0, an exact selection among them there.  Used when at least `need` keys are >= L
     // and they fit (uniform decision after a barrier); otherwise the distributed radix
     // select below, which is exact for any input.
-    const bool trivial = (need == 0 || need == own);
     bool fast_ok = false;
     if (!trivial) {
         if (rank == 0) {
-            // sample every st-th score of the row
-            const int64_t st = max((int64_t)1, own / kSample);
-            const uint32_t ns = (uint32_t)min((int64_t)kSample, (own + st - 1) / st);
             uint32_t *skeys = sl_copy;
-            const float *row_src = scores + (int64_t)row * ld;
-            for (uint32_t j = tid; j < ns; j += kThreads) skeys[j] = score_key(__ldcg(row_src + (int64_t)j * st));
+#pragma unroll
+            for (int u = 0; u < kSPer; ++u) {
+                const uint32_t j = u * kThreads + tid;
+                if (j < ns) skeys[j] = score_key(sv[u]);
+            }
             __syncthreads();
-            // the sample rank whose expected row rank is ~1.5 need, plus a margin
+            // the sample rank whose expected row rank is ~1.5 need, plus a margin; the bound
+            // is the lower edge of its 12-bit key bin (any bound is fine: the count of keys
+            // above it is verified below)
             uint32_t js = (uint32_t)((3 * need + 2 * st - 1) / (2 * st)) + 8;
             js = min(max(js, 1u), ns);
-            const int sh3[3] = {20, 8, 0};
-            const int wd3[3] = {12, 12, 8};
+            const int sh1[1] = {20};
+            const int wd1[1] = {12};
             uint32_t lp, lm;
-            cta_select_desc<uint32_t, kThreads, 3>(skeys, ns, js, sh3, wd3, hist, scan_ws, lp, lm);
-            if (tid == 0) sh_L = lp;                      // prefix with low bits 0: <= the js-th key
+            cta_select_desc<uint32_t, kThreads, 1>(skeys, ns, js, sh1, wd1, hist, scan_ws, lp, lm);
+            if (tid == 0) sh_L = lp;                      // low 20 bits 0: <= the js-th sample key
         }
         cluster.sync();                                                     // L published
         const uint32_t Lk = *cluster.map_shared_rank(&sh_L, 0);
@@ -213,12 +230,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         fast_ok = !overflow && total >= (uint32_t)need && total <= (uint32_t)kCandTotal;
         if (fast_ok && rank == 0) {
             uint64_t *call = reinterpret_cast<uint64_t *>(gsl);              // all candidates
-            uint32_t n = 0;
-            for (int q = 0; q < CL; ++q) {
-                const uint32_t c = *cluster.map_shared_rank(&sh_ccount, q);
+            if (tid < CL) slice_tot[tid] = *cluster.map_shared_rank(&sh_ccount, tid);
+            __syncthreads();
+            if (tid == 0) {
+                off_s[0] = 0;
+                for (int q = 0; q < CL; ++q) off_s[q + 1] = off_s[q] + slice_tot[q];
+            }
+            __syncthreads();
+            const uint32_t n = off_s[CL];
+            // one flat parallel copy: entry i of the concatenation comes from rank q
+            for (uint32_t i = tid; i < n; i += kThreads) {
+                int q = 0;
+                while (q + 1 < CL && i >= off_s[q + 1]) ++q;
                 const uint64_t *rl = reinterpret_cast<const uint64_t *>(cluster.map_shared_rank(hist, q));
-                for (uint32_t i = tid; i < c; i += kThreads) call[n + i] = rl[i];
-                n += c;
+                call[i] = rl[i - off_s[q]];
             }
             __syncthreads();
             const int shc[5] = {52, 40, 32, 10, 0};
