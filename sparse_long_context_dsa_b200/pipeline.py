@@ -147,3 +147,41 @@ def compress_all(index_k, lengths, tok_base, sum_base, summaries, scales):
     src = torch.cat(src).to(index_k.device)
     dst = torch.cat(dst).to(index_k.device)
     dsa.compress_regions(index_k, src, dst, summaries, scales)
+
+
+def due_regions(positions):
+    """Requests whose appended token (at the given 0-based positions) completes a region:
+    token p completes region p // 8 exactly when p % 8 == 7."""
+    return [b for b, p in enumerate(positions) if int(p) % REGION == REGION - 1]
+
+
+class StreamingDecode:
+    """The streaming summary update of a ragged decode batch ([P2] Step-5-Preview 如何实现1M长上下文
+    §区域压缩CSA, update_summaries_decode): a region is summarised exactly when its 8th token
+    arrives; the tail of fewer than 8 tokens waits and is never summarised.
+
+    lengths[b] tokens of request b are cached.  Each step appends one token per request at
+    position p_b = lengths[b] (the caller writes its K/V into the paged cache and its
+    index_k row into row p_b % 8 of tail block b of `step.tail`), queries at p_b, and
+    compresses region p_b / 8 of the requests whose token completes it (p_b % 8 == 7) from
+    their tail blocks.  That region is the query's own region, which its scan never reads,
+    so the compression runs on the step's parallel branch."""
+
+    def __init__(self, summaries, scales, sum_base, block_table, k_cache, v_cache, lengths, ld, k=512):
+        self.lengths = [int(L) for L in lengths]
+        self.sum_base = [int(x) for x in sum_base.tolist()]
+        self.step = DecodeStep(summaries, scales, sum_base, block_table, k_cache, v_cache, ld, k=k, tail_tokens=8)
+
+    def positions(self):
+        """Positions of the tokens the next step appends (= its query positions)."""
+        return list(self.lengths)
+
+    def run(self, index_q, gate, q):
+        """One step: the tail blocks must already hold the new tokens' index_k rows."""
+        pos = self.positions()
+        due = due_regions(pos)
+        self.step.load(index_q, gate, q, torch.tensor(pos, dtype=torch.int32))
+        self.step.set_compress(due, [self.sum_base[b] + pos[b] // REGION for b in due])
+        out = self.step.run()
+        self.lengths = [L + 1 for L in self.lengths]
+        return out, due
