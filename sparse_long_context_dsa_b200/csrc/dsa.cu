@@ -10,6 +10,7 @@
 #include "attention.cuh"
 #include "common.cuh"
 #include "compress.cuh"
+#include "gemm_indexer.cuh"
 #include "indexer.cuh"
 #include "topk.cuh"
 #include "topk_cluster.cuh"
@@ -39,6 +40,8 @@ dsa_status_t cuda_fail(cudaError_t e, const char *what)
         cudaError_t e_ = (call);                                \
         if (e_ != cudaSuccess) return cuda_fail(e_, (what));    \
     } while (0)
+
+constexpr int kGemmMinQueries = 64;   // FP8 prefill chunks at least this long use the GEMM
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -215,6 +218,83 @@ dsa_status_t attn_common(const void *q, const void *k_cache, const void *v_cache
     return DSA_OK;
 }
 
+// Workspace of the prefill GEMM path: e4m3 query codes [nq][16][256], their scales
+// [nq][16], the validated own region of every query and the largest one of every tile.
+size_t gemm_ws_size(int nq)
+{
+    if (nq < kGemmMinQueries) return 0;
+    const size_t tiles = (size_t)(nq + dsa::gemm::kQPerTile - 1) / dsa::gemm::kQPerTile;
+    return round_up((size_t)nq * dsa::kHI * dsa::kDI, 256) + round_up((size_t)nq * dsa::kHI * 4, 256) +
+           round_up((size_t)nq * 4, 256) + round_up(tiles * 4, 256);
+}
+
+dsa_status_t indexer_gemm_path(const void *index_q, const float *gate, const int32_t *q_req, const int32_t *q_pos,
+                               int nq, const uint8_t *summaries, const float *scales, int64_t n_slots,
+                               const int64_t *sum_base, float *scores, int64_t ld, void *ws, int sms,
+                               dsa_stream_t stream)
+{
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    uint8_t *codes = w;
+    float *qscale = reinterpret_cast<float *>(w + round_up((size_t)nq * dsa::kHI * dsa::kDI, 256));
+    int32_t *q_own = reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(qscale) +
+                                                 round_up((size_t)nq * dsa::kHI * 4, 256));
+    int32_t *tile_own = reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(q_own) + round_up((size_t)nq * 4, 256));
+    const int n_mtiles = (nq + dsa::gemm::kQPerTile - 1) / dsa::gemm::kQPerTile;
+    const int qblocks = (nq * dsa::kHI + 3) / 4;
+    const int grid_q = std::max(qblocks, (n_mtiles + 127) / 128);
+    dsa::gemm::quantize_kernel<<<grid_q, 128, 0, stream>>>(static_cast<const __nv_bfloat16 *>(index_q), q_req, q_pos,
+                                                          sum_base, ld, n_slots, nq, codes, qscale, q_own,
+                                                          tile_own, n_mtiles);
+    dsa_status_t st;
+    if ((st = launched("gemm quantize_kernel")) != DSA_OK) return st;
+
+    CUtensorMap map_a, map_b;
+    {
+        const cuuint64_t dims[4] = {(cuuint64_t)dsa::kDI, 4, 4, (cuuint64_t)nq};
+        const cuuint64_t strides[3] = {(cuuint64_t)dsa::kDI, (cuuint64_t)dsa::kDI * 4, (cuuint64_t)dsa::kDI * 16};
+        const cuuint32_t box[4] = {128, 4, 1, (cuuint32_t)dsa::gemm::kQPerTile};
+        if ((st = encode(&map_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, codes, dims, strides, box,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B)) != DSA_OK)
+            return st;
+    }
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)dsa::kDI, (cuuint64_t)n_slots * dsa::kG};
+        const cuuint64_t strides[1] = {(cuuint64_t)dsa::kDI};
+        const cuuint32_t box[2] = {128, (cuuint32_t)dsa::gemm::kBN};
+        if ((st = encode(&map_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, summaries, dims, strides, box,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B)) != DSA_OK)
+            return st;
+    }
+    dsa::gemm::Params p{};
+    p.qscale = qscale;
+    p.gate = gate;
+    p.q_own = q_own;
+    p.tile_own = tile_own;
+    p.scales = scales;
+    p.sum_base = sum_base;
+    p.scores = scores;
+    p.ld = ld;
+    p.n_slots = n_slots;
+    p.nq = nq;
+    p.n_rblocks = (int)((ld + dsa::gemm::kBN - 1) / dsa::gemm::kBN);
+    p.n_mtiles = n_mtiles;
+    int parts = 1;
+    while (4 * p.n_rblocks * parts < 6 * sms && parts < n_mtiles) parts *= 2;
+    p.m_per_unit = (n_mtiles + parts - 1) / parts;
+    p.n_mparts = (n_mtiles + p.m_per_unit - 1) / p.m_per_unit;
+    p.n_units = dsa::kG * p.n_rblocks * p.n_mparts;
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(dsa::gemm::gemm_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)dsa::gemm::kSmemBytes);
+    });
+    DSA_CUDA(attr_err, "cudaFuncSetAttribute(gemm_scores_kernel)");
+    dsa::gemm::gemm_scores_kernel<<<std::min(sms, p.n_units), dsa::gemm::kThreads, dsa::gemm::kSmemBytes, stream>>>(
+        map_a, map_b, p);
+    return launched("gemm_scores_kernel");
+}
+
 // Workspace path of the top-k: histogram, threshold-bin gather and last-CTA selection
 // (scales to many rows; scratch from the caller's workspace).
 dsa_status_t topk_workspace_path(const float *scores, int64_t ld_scores, const int32_t *q_pos, int nq, int k,
@@ -358,9 +438,8 @@ dsa_status_t dsa_compress_regions(const void *index_k, int64_t row_stride, int64
 
 size_t dsa_indexer_workspace_size(int nq, int64_t ld_scores)
 {
-    (void)nq;
     (void)ld_scores;
-    return 0;
+    return gemm_ws_size(nq);
 }
 
 dsa_status_t dsa_indexer_scores(const void *index_q, const float *gate, const int32_t *q_req, const int32_t *q_pos,
@@ -368,8 +447,6 @@ dsa_status_t dsa_indexer_scores(const void *index_q, const float *gate, const in
                                 const int64_t *sum_base, int n_req, float *scores, int64_t ld_scores, uint32_t flags,
                                 void *ws, size_t ws_bytes, dsa_stream_t stream)
 {
-    (void)ws;
-    (void)ws_bytes;
     DSA_REQUIRE(nq >= 0, "nq must be >= 0");
     DSA_REQUIRE((flags & ~DSA_Q_FP8) == 0, "unknown flag");
     DSA_REQUIRE(ld_scores >= 1 && ld_scores <= (1ll << 26), "ld_scores out of [1, 2^26]");
@@ -382,6 +459,10 @@ dsa_status_t dsa_indexer_scores(const void *index_q, const float *gate, const in
     dsa_status_t st = device_info(sms);
     if (st != DSA_OK) return st;
 
+    if ((flags & DSA_Q_FP8) && n_req == 1 && nq >= kGemmMinQueries && ws && ws_bytes >= gemm_ws_size(nq) &&
+        aligned(ws, 256))
+        return indexer_gemm_path(index_q, gate, q_req, q_pos, nq, summaries, scales, n_slots, sum_base, scores,
+                                 ld_scores, ws, sms, stream);
     CUtensorMap map;
     {
         const cuuint64_t dims[2] = {(cuuint64_t)dsa::kDI, (cuuint64_t)n_slots * dsa::kG};
