@@ -10,6 +10,12 @@ Four independent layer caches (each 128 MiB of summaries + 3 GiB of K/V) are use
 robin, so consecutive steps never find their inputs in the 126 MB L2.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload decode_b1_1m|prefill_2k_256k]
+
+--workload prefill_2k_256k times the chunked-prefill step instead (2,048 new query tokens
+on a 262,144-token context: compress the 256 completed regions, FP8 indexer GEMM, top-512
+per query and group, sparse GQA prefill attention) and prints its own line (tokens/s and
+each stage's share; the indexer GEMM's roofline against the FP8 tensor peak).
 
 --gpus N > 1 (under torchrun): every rank runs an independent replica (requests shard
 across GPUs with no data-path collective, weak scaling); timing is the max over ranks.
@@ -34,7 +40,9 @@ UNIT = "queries/s"
 L_CTX = 1 << 20
 TOPK = 512
 N_LAYERS = 4
-KERNELS_PER_STEP = 7      # compress, scan, top-k hist/gather/final, attention, combine
+KERNELS_PER_STEP = 5      # compress, scan, cluster top-k, attention, split combine
+PREFILL_CTX, PREFILL_NEW = 262144, 2048
+PREFILL_KERNELS = 6       # compress, quantize, GEMM, top-k histogram, top-k select, attention
 
 
 def parse():
@@ -46,6 +54,7 @@ def parse():
     ap.add_argument("--layers", type=int, default=N_LAYERS)
     ap.add_argument("--cpu-queries", type=int, default=3, help="oracle queries timed for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=["decode_b1_1m", "prefill_2k_256k"], default="decode_b1_1m")
     return ap.parse_args()
 
 
@@ -391,10 +400,141 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+# ------------------------------------------------------------------ prefill workload
+
+def prefill_flops():
+    """Algorithmic FLOPs of the chunk: indexer 2*256*16 per (query, eligible region) and
+    attention 4*192*64 per (query, attended token); both summed exactly over the chunk."""
+    n_idx = n_att = 0
+    for i in range(PREFILL_NEW):
+        p = PREFILL_CTX + i
+        own = p // 8
+        n_idx += own
+        n_att += 8 * min(TOPK - 1, own) + (p % 8 + 1)
+    return 2 * 256 * 16 * n_idx, 4 * 192 * 16 * 4 * n_att
+
+
+def run_prefill(args):
+    import torch
+    from sparse_long_context_dsa_b200 import dsa, pipeline
+    from sparse_long_context_dsa_b200 import workloads as W
+
+    rank, world, local = dist_env()
+    if world > 1:
+        raise SystemExit("--workload prefill_2k_256k runs on one GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dsa.lib()
+    d = W.prefill_chunk(PREFILL_CTX, PREFILL_NEW, seed=1238, device=dev, permute=True)
+    n_slots = d["n_slots"]
+    S = torch.zeros((4, n_slots, 256), dtype=torch.uint8, device=dev)
+    C = torch.zeros((4, n_slots), dtype=torch.float32, device=dev)
+    pipeline.compress_all(d["index_k"], [PREFILL_CTX], [0], d["sum_base"], S, C)
+    total = PREFILL_CTX + PREFILL_NEW
+    first, last = PREFILL_CTX // 8, total // 8
+    src = torch.arange(first, last, dtype=torch.int64, device=dev) * 8
+    dst = torch.arange(first, last, dtype=torch.int64, device=dev)
+    ld = last
+    scores = torch.zeros((PREFILL_NEW, 4, ld), dtype=torch.float32, device=dev)
+    sel = torch.empty((PREFILL_NEW, 4, TOPK), dtype=torch.int32, device=dev)
+    cnt = torch.empty((PREFILL_NEW, 4), dtype=torch.int32, device=dev)
+    out = torch.empty((PREFILL_NEW, 64, 192), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step(ev=None):
+        rec = (lambda i: ev[i].record()) if ev else (lambda i: None)
+        rec(0)
+        dsa.compress_regions(d["index_k"], src, dst, S, C)
+        rec(1)
+        dsa.indexer_scores(d["index_q"], d["gate"], d["q_req"], d["q_pos"], S, C, d["sum_base"], scores, dsa.Q_FP8)
+        rec(2)
+        dsa.topk_regions(scores, d["q_pos"], TOPK, sel, cnt)
+        rec(3)
+        dsa.sparse_attn_prefill(d["q"], d["k_cache"], d["v_cache"], d["block_table"], d["q_req"], d["q_pos"],
+                                sel, cnt, out=out)
+        rec(4)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    dsa.check_device()
+    stage = [0.0] * 4
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    with sampler:
+        for i in range(args.steps):
+            flush.zero_()                      # L2 flushed between steps (outside the timed stages)
+            step(evs[i])
+        torch.cuda.synchronize()
+    for ev in evs:
+        for j in range(4):
+            stage[j] += ev[j].elapsed_time(ev[j + 1])
+    dsa.check_device()
+    ms = sum(stage)
+    f_idx, f_att = prefill_flops()
+    fp8_peak, kind = tensor_peak(fp8=True)
+    t_gemm = stage[1] / args.steps * 1e-3
+    # e2e: the chunk's host inputs (pinned) in, its output out, through the same calls
+    names = ["index_q", "gate", "q", "q_pos"]
+    host = {n: d[n].cpu().pin_memory() for n in names}
+    host_ik = d["index_k"][PREFILL_CTX:].cpu().pin_memory()
+    host_out = torch.empty_like(out, device="cpu").pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values()) + host_ik.numel() * host_ik.element_size()
+    d2h = host_out.numel() * host_out.element_size()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record()
+    for _ in range(args.steps):
+        for n in names:
+            d[n].copy_(host[n], non_blocking=True)
+        d["index_k"][PREFILL_CTX:].copy_(host_ik, non_blocking=True)
+        step()
+        host_out.copy_(out, non_blocking=True)
+    t1.record()
+    torch.cuda.synchronize()
+    e2e_ms = t0.elapsed_time(t1)
+    line = {
+        "metric": "DSA chunked-prefill query tokens/s (2,048 new on 262,144 ctx)", "value":
+            PREFILL_NEW * args.steps / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 indexer, bf16 attention (fp32 accumulate)",
+        "data": "synthetic",
+        "config": {"workload": "prefill_2k_256k", "context": PREFILL_CTX, "new_tokens": PREFILL_NEW, "topk": TOPK,
+                   "l2": "flushed (256 MiB write) before every step, outside the timed stages"},
+        "stages_ms": {"compress": stage[0] / args.steps, "indexer_gemm": stage[1] / args.steps,
+                      "topk": stage[2] / args.steps, "attention": stage[3] / args.steps},
+        "roofline": {"kernel": "indexer GEMM (quantize + gemm_scores_kernel)", "bound": "tensor",
+                     "achieved": f_idx / t_gemm / 1e12, "peak": fp8_peak, "unit": "TFLOP/s",
+                     "frac": f_idx / t_gemm / 1e12 / fp8_peak, "peak_kind": kind, "flops_per_launch": f_idx,
+                     "traffic": None},
+        "attention": {"flops": f_att, "tflops": f_att / (stage[3] / args.steps * 1e-3) / 1e12,
+                      "peak_bf16": tensor_peak(fp8=False)[0]},
+        "e2e": {"value": PREFILL_NEW * args.steps / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": PREFILL_KERNELS * args.steps,
+        "clocks": sampler.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def tensor_peak(fp8: bool):
+    """Dense tensor peak in TFLOP/s: the measured cuBLAS bf16 burst figure (x2 for e4m3,
+    the nominal fp8/bf16 ratio of the part), else the fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v, kind = float(json.load(f)["bf16_tflops"]), "measured bf16"
+    except Exception:
+        v, kind = 1590.0, "fallback bf16"
+    return (2 * v, kind + " x 2 (nominal e4m3/bf16 ratio)") if fp8 else (v, kind)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload == "prefill_2k_256k":
+        run_prefill(args)
     else:
         run_ours(args)
 
