@@ -344,8 +344,11 @@ dsa_status_t topk_cluster_path(const float *scores, int64_t ld_scores, const int
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(dsa::topkc::topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)dsa::topkc::kSmemBytes);
+        attr_err = cudaFuncSetAttribute(dsa::topkc::topk_cluster_kernel<true>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsa::topkc::kSmemBytes);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(dsa::topkc::topk_cluster_kernel<false>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsa::topkc::kSmemBytes);
     });
     DSA_CUDA(attr_err, "cudaFuncSetAttribute(topk_cluster_kernel)");
     cudaLaunchConfig_t cfg = {};
@@ -360,8 +363,14 @@ dsa_status_t topk_cluster_path(const float *scores, int64_t ld_scores, const int
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    DSA_CUDA(cudaLaunchKernelEx(&cfg, dsa::topkc::topk_cluster_kernel, scores, ld_scores, q_pos, k, sel_idx, sel_count),
-             "cudaLaunchKernelEx(topk_cluster_kernel)");
+    if (cl == 1)
+        DSA_CUDA(cudaLaunchKernelEx(&cfg, dsa::topkc::topk_cluster_kernel<true>, scores, ld_scores, q_pos, k, sel_idx,
+                                    sel_count),
+                 "cudaLaunchKernelEx(topk_cluster_kernel)");
+    else
+        DSA_CUDA(cudaLaunchKernelEx(&cfg, dsa::topkc::topk_cluster_kernel<false>, scores, ld_scores, q_pos, k, sel_idx,
+                                    sel_count),
+                 "cudaLaunchKernelEx(topk_cluster_kernel)");
     return launched("topk_cluster_kernel");
 }
 

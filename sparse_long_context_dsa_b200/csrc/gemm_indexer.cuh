@@ -36,7 +36,7 @@ constexpr int kBHalf = kBN * 128;        // 32 KiB
 constexpr int kBBytes = 2 * kBHalf;
 constexpr int kThreads = 192;            // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr int kTmemCols = 512;           // two 256-column fp32 accumulators
-constexpr size_t kSmemBytes = 1024 + kBBytes + kAStages * kABytes + 256;
+constexpr size_t kSmemBytes = 1024 + kBBytes + kAStages * kABytes + 4 * kBN * 4 + 256;
 constexpr uint32_t kIdesc = umma_idesc_e4m3(kBM, kBN);
 
 struct Params {
@@ -154,7 +154,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sb = smem;                                   // summary tile: 2 K columns x [256][128]
     uint8_t *sa = smem + kBBytes;                         // query tiles: kAStages x 2 K columns x [128][128]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sa + kAStages * kABytes);
+    float *sscale_all = reinterpret_cast<float *>(sa + kAStages * kABytes);    // [4 warps][256] scales / 16
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sscale_all + 4 * kBN);
     uint64_t *b_full = bars + 0, *b_empty = bars + 1;
     uint64_t *a_full = bars + 2, *a_empty = bars + 4;     // [kAStages]
     uint64_t *acc_full = bars + 6, *acc_empty = bars + 8; // [2]
@@ -252,12 +253,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int sp = warp & 3;
         const int qt = sp * 8 + (lane >> 2), h = lane & 3;      // this lane's row: query in tile, head
         const int cb = 16 * (h & 1) + 8 * ((h >> 1) & 1);        // its 8 finished columns in a chunk
+        float *wscale = sscale_all + (warp - 2) * kBN;
         int cit = 0;
         for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
             int g, rb, t0, t1;
             unit_coords(p, u, g, rb, t0, t1);
             if (!unit_active(p, t0, t1, rb)) continue;
-            const float *srow = p.scales + g * p.n_slots + base + (int64_t)rb * kBN;   // this unit's scales
+            // this unit's 256 region scales / 16, staged by each warp in its own smem slice
+            // (no barrier across the epilogue warps); entries past the pool read as 0
+            {
+                const int64_t s0 = g * p.n_slots + base + (int64_t)rb * kBN;
+                const int64_t lim = (int64_t)kG * p.n_slots;
+#pragma unroll
+                for (int j = 0; j < kBN / 32; ++j) {
+                    const int64_t i = s0 + j * 32 + lane;
+                    wscale[j * 32 + lane] = i < lim ? __ldg(p.scales + i) * 0.0625f : 0.0f;
+                }
+                __syncwarp();
+            }
             for (int t = t0; t < t1; ++t) {
                 if (!tile_active(p, t, rb)) continue;
                 const int buf = cit & 1;
@@ -294,9 +307,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int c0 = ch * 32 + cb;
                     const int64_t r0 = (int64_t)rb * kBN + c0;
                     if (qv && r0 < own) {
-                        float sc[8];
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) sc[j] = (r0 + j < own) ? __ldg(srow + c0 + j) * 0.0625f : 0.0f;
+                        const float4 sa4 = *reinterpret_cast<const float4 *>(wscale + c0);
+                        const float4 sb4 = *reinterpret_cast<const float4 *>(wscale + c0 + 4);
+                        const float sc[8] = {sa4.x, sa4.y, sa4.z, sa4.w, sb4.x, sb4.y, sb4.z, sb4.w};
                         if (r0 + 8 <= own && (p.ld & 3) == 0) {
                             *reinterpret_cast<float4 *>(orow + r0) =
                                 make_float4(k8[0] * sc[0], k8[1] * sc[1], k8[2] * sc[2], k8[3] * sc[3]);
@@ -314,6 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) mbar_arrive(&acc_empty[buf]);
                 ++cit;
             }
+            __syncwarp();                                   // the slice is rewritten by the next unit
         }
     }
     // every role done (or gave up): release TMEM

@@ -3,18 +3,29 @@
 // regions and always includes the query's own region).
 //
 // For few long rows (decode: 4 rows of up to 131,071 scores per query) a row is split over
-// a cluster of CL CTAs.  CTA `rank` owns the contiguous region range
-// [rank*part, rank*part + part) and keeps its order-preserving score keys in smem.  A radix
-// select finds the need-th largest key over the whole row: per digit (key bits 31..20,
-// 19..8, 7..0) every CTA histograms its keys that match the prefix found so far, the
-// cluster sums the histograms through distributed shared memory (each CTA reduces a slice
-// of the bins), and every CTA locates the digit from the slice totals.  Equal keys at the
-// threshold are taken lowest region first: the ranks own ascending ranges, so a prefix of
-// per-rank tie counts says how many ties each CTA takes, and inside a CTA an ordered block
-// scan picks the first ones.  The output (ascending region indices) is an ordered
-// compaction: each CTA writes its selected regions at the offset given by the counts of the
-// ranks before it.  No global scratch, no atomics, no waiting on other CTAs except the
-// cluster's hardware barriers.
+// a cluster of CL CTAs; CTA `rank` owns the contiguous region range [rank*part, ...).
+// Fast path, two cluster barriers in all:
+//  1. every thread's share of the CTA's range is loaded coalesced (all loads, the query
+//     position's included, in flight at once: the partition follows the row length, and
+//     entries at or beyond the own region are masked afterwards), staged in shared memory
+//     and taken back as a run of 32 consecutive order-preserving keys: a group.  The group
+//     maxima go to every CTA of the cluster;
+//  2. every CTA selects the same bound L from the group maxima: the lower edge of the (at
+//     most two) 8-bit digit bins that hold the need-th largest maximum.  At least `need`
+//     groups have a maximum >= L, so at least `need` keys are >= L, and few more (groups
+//     holding two of the best keys);
+//  3. the keys >= L are pushed in region order, with each CTA's count, into rank 0's shared
+//     memory; rank 0 gathers them densely (still in region order), selects exactly the need
+//     largest (key desc, then region asc) and writes them with one ordered compaction, the
+//     own region last.
+// When the candidates do not fit (many equal scores, or k beyond the group count) every CTA
+// sees it in the pushed counts and the cluster runs an exact distributed radix select
+// instead: per digit every CTA histograms its keys that match the prefix found so far, the
+// cluster sums the histograms through distributed shared memory (each CTA reduces a slice of
+// the bins) and every CTA locates the digit; equal keys at the threshold are taken lowest
+// region first (a prefix of per-rank tie counts, then an ordered block scan), and the output
+// is an ordered compaction over the ranks.  No global scratch, no waiting on other CTAs
+// except the cluster's hardware barriers.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -27,15 +38,35 @@ namespace topkc {
 namespace cg = cooperative_groups;
 
 constexpr int kThreads = 512;
-constexpr int kPartMax = 16384;        // keys per CTA held in smem (64 KiB)
-constexpr int kMaxCluster = 8;         // portable cluster size
-constexpr int kBins = 4096;
-constexpr int kCandMax = 2048;         // candidates per CTA on the fast path
-constexpr int kCandTotal = 4096;       // candidates gathered at rank 0
-constexpr int kSample = 4096;          // sampled scores for the lower bound
-constexpr size_t kSmemBytes = (size_t)kPartMax * 4 + 5 * kBins * 4 + 1024;
-static_assert(kCandMax * 8 <= 2 * kBins * 4 && kCandTotal * 8 <= 2 * kBins * 4 && kSample <= kBins,
-              "fast-path buffers fit");
+constexpr int kWarps = kThreads / 32;
+constexpr int kPartMax = 16384;                 // scores per CTA
+constexpr int kPer = kPartMax / kThreads;       // 32 per thread: one group
+constexpr int kPadded = kPartMax + kPartMax / 8;    // fallback: key i at i + 4*(i/32)
+constexpr int kMaxCluster = 8;                  // portable cluster size
+constexpr int kGroups = kThreads * kMaxCluster; // group maxima per row (at most)
+constexpr int kBins = 4096;                     // fallback digit bins
+constexpr int kSlots = 8192;                    // candidate slots at rank 0 (kSlots / CL per rank)
+constexpr int kDense = 2048;                    // gathered candidates at rank 0
+constexpr int kDPer = kDense / kThreads;
+// fast-path smem layout (bytes)
+constexpr size_t kOffSlots = 0;
+constexpr size_t kOffGmax = kOffSlots + (size_t)kSlots * 8;
+constexpr size_t kOffHw = kOffGmax + (size_t)kGroups * 4;
+constexpr size_t kOffHs = kOffHw + (size_t)kWarps * 256 * 4;
+constexpr size_t kOffDense = kOffHs + 256 * 4;
+constexpr size_t kFastBytes = kOffDense + (size_t)kDense * 8;
+// the staged keys [kPadded] after them; the fallback's hist [2][kBins], gsl [2][kBins] and
+// sl_copy [kBins] overlay the fast-path regions (used only after the second barrier)
+constexpr size_t kOffKeys = kFastBytes;
+constexpr size_t kFallbackBytes = 5 * (size_t)kBins * 4;
+constexpr size_t kSmemBytes = kOffKeys + (size_t)kPadded * 4 + 1024;
+static_assert(kOffDense % 16 == 0, "aligned smem regions");
+static_assert(kFallbackBytes <= kOffKeys, "fallback buffers stay clear of the staged keys");
+static_assert(kOffKeys % 16 == 0, "aligned key staging");
+
+// 4 words of padding after every 32 keys: a thread's run of 32 keys is 16-byte aligned and the
+// 8 threads of a 16-byte load phase hit distinct banks.
+__device__ __forceinline__ int padded(int i) { return i + 4 * (i >> 5); }
 
 template <int NT>
 __device__ __forceinline__ uint32_t block_scan_incl(uint32_t v, uint32_t *ws)
@@ -64,49 +95,109 @@ __device__ __forceinline__ uint32_t block_scan_incl(uint32_t v, uint32_t *ws)
 }
 
 
-// Single-CTA radix select over n smem values (descending): finds the digits of the m-th
-// largest value (1 <= m <= n).  Returns (prefix, mask) such that exactly m values v satisfy
-// (v & mask) >= prefix.  `h` needs 4096 words, `ws` 40 words.  Values are distinct or the
-// caller accepts that all values equal to the m-th are counted (the last digit decides).
-template <typename T, int NT, int ND>
-__device__ void cta_select_desc(const T *vals, uint32_t n, uint32_t m, const int (&shifts)[ND],
-                                const int (&widths)[ND], uint32_t *h, uint32_t *ws, T &prefix_out, T &mask_out)
+// Block-wide min and max (every thread gets both); `ws` needs 2 * kWarps entries.
+template <typename T>
+__device__ __forceinline__ void block_minmax(T &mn, T &mx, T *ws)
 {
-    const int tid = threadIdx.x;
-    T prefix = 0, pmask = 0;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const T a = __shfl_xor_sync(0xffffffffu, mn, o), b = __shfl_xor_sync(0xffffffffu, mx, o);
+        mn = a < mn ? a : mn;
+        mx = b > mx ? b : mx;
+    }
+    if (lane == 0) {
+        ws[warp] = mn;
+        ws[kWarps + warp] = mx;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int w = 0; w < kWarps; ++w) {
+        const T a = ws[w], b = ws[kWarps + w];
+        mn = a < mn ? a : mn;
+        mx = b > mx ? b : mx;
+    }
+    __syncthreads();
+}
+
+template <typename T>
+__device__ __forceinline__ int top_differing_bit(T a, T b)
+{
+    if (a == b) return -1;
+    if constexpr (sizeof(T) == 8) return 63 - __clzll((long long)(a ^ b));
+    else return 31 - __clz((int)(a ^ b));
+}
+
+// The m-th largest (1 <= m <= count) of the block's register-held values (v[u] of a thread
+// counts when bit u of `valid` is set), by digits of at most 8 bits from bit `top` down;
+// every value agrees with `first` on the bits above `top` (top = -1: all values equal).
+// Each warp histograms into its own 256 bins (values crowd into few bins near the top of a
+// score distribution: the conflicts stay inside a warp), 256 threads add the warps' bins
+// and one warp scans them.  Returns (prefix, mask): the values v with (v & mask) >= prefix
+// are the m largest when the values are distinct; otherwise every value equal to the m-th
+// one satisfies it too.  With max_digits the search stops early: then at least m values
+// satisfy it (those in the bins at and above the m-th one's).  `hw` needs kWarps * 256
+// words, `hs` 256, `res` 3.
+template <typename T, int R>
+__device__ void cta_select_reg(const T (&v)[R], uint32_t valid, uint32_t m, int top, T first, uint32_t *hw,
+                               uint32_t *hs, uint32_t *res, T &prefix_out, T &mask_out, int max_digits = 64)
+{
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int kBitsT = 8 * sizeof(T);
+    T pmask = top >= kBitsT - 1 ? (T)0 : (~(T)0 << (top + 1));
+    T prefix = first & pmask;
     uint32_t m_rem = m;
-    for (int d = 0; d < ND; ++d) {
-        const int sh = shifts[d], nb = 1 << widths[d];
-        for (int i = tid; i < nb; i += NT) h[i] = 0;
+    uint32_t *myh = hw + warp * 256;
+    for (int hi = top, d = 0; hi >= 0 && d < max_digits; hi -= 8, ++d) {
+        const int sh = max(hi - 7, 0);
+        const uint32_t nb = 1u << (hi - sh + 1);
+#pragma unroll
+        for (int b = lane; b < 256; b += 32) myh[b] = 0;
+        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < R; ++u)
+            if (((valid >> u) & 1u) && (v[u] & pmask) == prefix)
+                atomicAdd(&myh[(uint32_t)(v[u] >> sh) & (nb - 1)], 1u);
         __syncthreads();
-        for (uint32_t i = tid; i < n; i += NT) {
-            const T v = vals[i];
-            if ((v & pmask) == prefix) atomicAdd(&h[(uint32_t)(v >> sh) & (uint32_t)(nb - 1)], 1u);
+        if (tid < 256) {
+            uint32_t s = 0;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) s += hw[w * 256 + tid];
+            hs[tid] = s;
         }
         __syncthreads();
-        // descending scan: thread t owns bins nb-1-t*bpt ... downwards
-        const int bpt = (nb + NT - 1) / NT;
-        const int p0 = tid * bpt;
-        uint32_t c = 0;
-        for (int u = 0; u < bpt; ++u)
-            if (p0 + u < nb) c += h[nb - 1 - (p0 + u)];
-        const uint32_t incl = block_scan_incl<NT>(c, ws);
-        if (incl >= m_rem && incl - c < m_rem) {
-            uint32_t run = incl - c;
-            for (int u = 0; u < bpt; ++u) {
-                const int b = nb - 1 - (p0 + u);
-                if (run + h[b] >= m_rem) {
-                    ws[32] = (uint32_t)b;
-                    ws[33] = run;
-                    ws[34] = h[b];
-                    break;
+        if (warp == 0) {
+            // descending: lane owns bins nb-1-8*lane .. nb-8-8*lane
+            uint32_t c[8], s = 0;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int bin = (int)nb - 1 - (lane * 8 + u);
+                c[u] = bin >= 0 ? hs[bin] : 0u;
+                s += c[u];
+            }
+            uint32_t incl = s;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += x;
+            }
+            const uint32_t excl = incl - s;
+            if (excl < m_rem && incl >= m_rem) {
+                uint32_t run = excl;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    if (run + c[u] >= m_rem) {
+                        res[0] = (uint32_t)((int)nb - 1 - (lane * 8 + u));
+                        res[1] = run;
+                        res[2] = c[u];
+                        break;
+                    }
+                    run += c[u];
                 }
-                run += h[b];
             }
         }
         __syncthreads();
-        const uint32_t B = ws[32], above = ws[33], binc = ws[34];
-        __syncthreads();
+        const uint32_t B = res[0], above = res[1], binc = res[2];
         m_rem -= above;
         prefix |= (T)B << sh;
         pmask |= (T)(nb - 1) << sh;
@@ -116,181 +207,425 @@ __device__ void cta_select_desc(const T *vals, uint32_t n, uint32_t m, const int
     mask_out = pmask;
 }
 
+// One warp: the bin (scanning 256 bins from the top) that holds the m-th largest value, the
+// count above it and its own count, into res[0..2] (m <= total count).
+__device__ __forceinline__ void desc_bin_search(const uint32_t *h, uint32_t m, uint32_t *res)
+{
+    const int lane = threadIdx.x & 31;
+    uint32_t c[8], s = 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        c[u] = h[255 - (lane * 8 + u)];
+        s += c[u];
+    }
+    uint32_t incl = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += x;
+    }
+    const uint32_t excl = incl - s;
+    if (excl < m && incl >= m) {
+        uint32_t run = excl;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            if (run + c[u] >= m) {
+                res[0] = (uint32_t)(255 - (lane * 8 + u));
+                res[1] = run;
+                res[2] = c[u];
+                break;
+            }
+            run += c[u];
+        }
+    }
+}
+
+// Exact threshold of the m largest among the block's (key, region) items, each thread holding
+// R of them (item u of a thread counts when valid(u); comp(u) = key << 32 | ~region, all
+// distinct).  Up to three levels of 256-bin key histograms (power-of-two bin widths, the
+// first over [klo, max key], each next one inside the previous level's bin of the m-th
+// largest) narrow the m-th largest down to a key range [*elo, *ehi) holding at most 32 items
+// (or a single key value); those are ranked exactly, pairwise in one warp, else by a radix
+// select over them.  Afterwards an item is selected iff key >= *ehi, or key >= *elo and
+// (comp & *cm) >= *cp: exactly m items.  Needs 1 <= m <= the valid count and every valid key
+// >= klo; returns false (uniformly) when the final range holds more than kDense items.
+// hs: 256 words; list: kDense 8-byte words; sh_kmax, sh_nin: zeroed before the call.
+template <int R, typename Valid, typename Comp>
+__device__ bool block_threshold(Valid valid, Comp comp, uint32_t m, uint32_t klo, uint32_t *hs, uint64_t *list,
+                                uint32_t *hw, uint32_t *sh_kmax, uint32_t *sh_nin, uint32_t *res, uint64_t *bc,
+                                uint64_t *elo, uint64_t *ehi, uint64_t *cp, uint64_t *cm)
+{
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint32_t kmx = 0u;
+#pragma unroll
+    for (int u = 0; u < R; ++u)
+        if (valid(u)) kmx = max(kmx, (uint32_t)(comp(u) >> 32));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) kmx = max(kmx, __shfl_xor_sync(0xffffffffu, kmx, o));
+    if (lane == 0) atomicMax(sh_kmax, kmx);
+    if (tid < 256) hs[tid] = 0u;
+    __syncthreads();
+    kmx = *sh_kmax;
+    uint64_t rlo = klo;                                                     // current key range [rlo, rlo + 256 << bsh)
+    int bsh = max(0, 24 - __clz((int)(kmx - klo)));
+    uint32_t m_rem = m, n_in = 0, bin = 0;
+    for (int level = 0; level < 3; ++level) {
+        const uint64_t rhi = rlo + (256ull << bsh);
+#pragma unroll
+        for (int u = 0; u < R; ++u) {
+            if (!valid(u)) continue;
+            const uint64_t kk = comp(u) >> 32;
+            if (kk >= rlo && kk < rhi) atomicAdd(&hs[(uint32_t)((kk - rlo) >> bsh)], 1u);
+        }
+        __syncthreads();
+        if (warp == 0) desc_bin_search(hs, m_rem, res);
+        __syncthreads();
+        bin = res[0];
+        m_rem -= res[1];
+        n_in = res[2];
+        if (tid < 256) hs[tid] = 0u;                                        // for the next level
+        if (n_in <= 32 || bsh == 0) break;
+        rlo += (uint64_t)bin << bsh;
+        bsh = max(0, bsh - 8);
+        __syncthreads();
+    }
+    const uint64_t blo = rlo + ((uint64_t)bin << bsh), bhi = blo + (1ull << bsh);
+    if (n_in > (uint32_t)kDense) return false;
+#pragma unroll
+    for (int u = 0; u < R; ++u) {
+        if (!valid(u)) continue;
+        const uint64_t kk = comp(u) >> 32;
+        if (kk >= blo && kk < bhi) list[atomicAdd(sh_nin, 1u)] = comp(u);
+    }
+    __syncthreads();
+    uint64_t p, mk;
+    if (n_in <= 32) {
+        if (warp == 0) {
+            const uint64_t e = lane < (int)n_in ? list[lane] : 0ull;
+            uint32_t gt = 0;
+            for (int j = 0; j < (int)n_in; ++j) gt += __shfl_sync(0xffffffffu, e, j) > e ? 1u : 0u;
+            if (lane < (int)n_in && gt == m_rem - 1) bc[0] = e;
+        }
+        __syncthreads();
+        p = bc[0];
+        mk = ~0ull;
+    } else {
+        constexpr int kLP = kDense / kThreads;
+        uint64_t lv[kLP];
+        uint32_t lvalid = 0;
+        uint64_t lmin = ~0ull, lmax = 0ull;
+#pragma unroll
+        for (int u = 0; u < kLP; ++u) {
+            const uint32_t i = u * kThreads + tid;
+            lv[u] = i < n_in ? list[i] : 0ull;
+            if (i < n_in) {
+                lvalid |= 1u << u;
+                lmin = min(lmin, lv[u]);
+                lmax = max(lmax, lv[u]);
+            }
+        }
+        block_minmax<uint64_t>(lmin, lmax, bc);
+        cta_select_reg<uint64_t, kLP>(lv, lvalid, m_rem, top_differing_bit(lmin, lmax), lmin, hw, hs, res, p, mk);
+    }
+    *elo = blo;
+    *ehi = bhi;
+    *cp = p;
+    *cm = mk;
+    return true;
+}
+
+__device__ __forceinline__ bool threshold_selects(uint64_t c, uint64_t elo, uint64_t ehi, uint64_t cp, uint64_t cm)
+{
+    const uint64_t kk = c >> 32;
+    return kk >= ehi || (kk >= elo && (c & cm) >= cp);
+}
+
+// kSingle: one CTA per row (launched without a cluster; CL = 1), else a cluster of CL CTAs.
+template <bool kSingle>
 __global__ void __launch_bounds__(kThreads, 1)
     topk_cluster_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ q_pos, int k,
                         int32_t *__restrict__ sel_idx, int32_t *__restrict__ sel_count)
 {
-    extern __shared__ uint8_t smem_raw[];
-    uint32_t *keys = reinterpret_cast<uint32_t *>(smem_raw);                 // [kPartMax]
-    uint32_t *hist = keys + kPartMax;                                        // [2][kBins]
-    uint32_t *gsl = hist + 2 * kBins;                                        // [2][kBins] reduced slices
-    uint32_t *sl_copy = gsl + 2 * kBins;                                     // [kBins] local copy of a slice
+    extern __shared__ __align__(16) uint8_t smem_raw[];
     __shared__ uint32_t scan_ws[40];                                         // block scans + select results
     __shared__ uint32_t tot[2];                                              // slice totals (double-buffered)
     __shared__ uint32_t sh_count[2];                                         // tie count, selected count
     __shared__ int sh_bin, sh_q;
     __shared__ uint32_t sh_above, sh_binc, sh_run;
     __shared__ uint32_t slice_tot[kMaxCluster];
-    __shared__ uint32_t sh_ccount, sh_L;
-    __shared__ uint32_t off_s[kMaxCluster + 1];
+    __shared__ uint32_t cand_cnt[kMaxCluster];                               // pushed by every rank
+    __shared__ uint64_t mm_ws[2 * kWarps];
+    __shared__ uint32_t sh_kmin, sh_kmax, sh_nin;
 
     cg::cluster_group cluster = cg::this_cluster();
     const int CL = (int)cluster.num_blocks();
     const int rank = (int)cluster.block_rank();
     const int row = blockIdx.y;
     const int tid = threadIdx.x;
+    const int lane = tid & 31, warp = tid >> 5;
 
+    // ---- loads: this thread's group is the CTA's entries tid, tid+512, ... (coalesced)
     const int p = q_pos[row >> 2];
+    const int64_t part = (ld + CL - 1) / CL;
+    const int64_t lo = min(ld, (int64_t)rank * part), hi_ld = min(ld, lo + part);
+    const float *src = scores + (int64_t)row * ld + lo;
+    if (part > kPartMax) {             // the host sizes the cluster so that a part fits
+        if (rank == 0 && tid == 0) {
+            set_error(kErrTopkInternal);
+            sel_count[row] = 0;
+        }
+        return;
+    }
+    uint32_t *keys = reinterpret_cast<uint32_t *>(smem_raw + kOffKeys);      // [kPadded] staged keys
+    {
+        const int n_ld = (int)(hi_ld - lo);
+        float v[kPer];
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int i = u * kThreads + tid;
+            v[u] = i < n_ld ? __ldcg(src + i) : 0.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int i = u * kThreads + tid;
+            if (i < n_ld) keys[padded(i)] = score_key(v[u]);
+        }
+    }
     const bool valid = p >= 0 && (int64_t)(p / kRegion) <= ld;
     const int64_t own = valid ? p / kRegion : 0;
     const int64_t need = valid ? min((int64_t)(k - 1), own) : 0;
-    const int64_t part = (own + CL - 1) / CL;
-    const int64_t lo = min(own, (int64_t)rank * part), hi = min(own, lo + part);
-    const int cnt = (int)(hi - lo);
-    const bool in_smem = part <= kPartMax;
-    const float *src = scores + (int64_t)row * ld + lo;
-    // rank 0 samples every st-th score of the row (for the fast path's lower bound); its
-    // loads are issued together with the key loads
+    const int cnt = (int)max((int64_t)0, min(own, hi_ld) - lo);            // this CTA's eligible keys
     const bool trivial = (need == 0 || need == own);
-    const int64_t st = max((int64_t)1, own / kSample);
-    const uint32_t ns = (uint32_t)min((int64_t)kSample, (own + st - 1) / st);
-    constexpr int kSPer = kSample / kThreads;
-    float sv[kSPer];
-    if (rank == 0 && !trivial) {
-        const float *row_src = scores + (int64_t)row * ld;
-#pragma unroll
-        for (int u = 0; u < kSPer; ++u) {
-            const uint32_t j = u * kThreads + tid;
-            sv[u] = j < ns ? __ldcg(row_src + (int64_t)j * st) : 0.0f;
-        }
+    // this thread's group: CTA entries [tid*32, tid*32 + nmine)
+    const int nmine = max(0, min(kPer, cnt - tid * kPer));
+    if (tid == 0) {
+        sh_kmin = 0xFFFFFFFFu;
+        sh_kmax = 0u;
+        sh_nin = 0u;
     }
-    if (in_smem) {
-        // all loads of this thread in flight at once (<= 32 at part <= kPartMax)
-        constexpr int kMaxPer = kPartMax / kThreads;
-        float v[kMaxPer];
-#pragma unroll
-        for (int u = 0; u < kMaxPer; ++u) {
-            const int i = u * kThreads + tid;
-            v[u] = i < cnt ? __ldcg(src + i) : 0.0f;
-        }
-#pragma unroll
-        for (int u = 0; u < kMaxPer; ++u) {
-            const int i = u * kThreads + tid;
-            if (i < cnt) keys[i] = score_key(v[u]);
-        }
-    }
-    auto key_at = [&](int i) -> uint32_t { return in_smem ? keys[i] : score_key(__ldcg(src + i)); };
+    if (tid < 256) reinterpret_cast<uint32_t *>(smem_raw + kOffHs)[tid] = 0u;
+    __syncthreads();                                                        // keys staged
+    auto key_at = [&](int i) -> uint32_t { return keys[padded(i)]; };
 
-    // ---- fast path: a sampled lower bound L of the threshold, the keys >= L gathered at
-    // rank 0, an exact selection among them there.  Used when at least `need` keys are >= L
-    // and they fit (uniform decision after a barrier); otherwise the distributed radix
-    // select below, which is exact for any input.
+    // groups holding an eligible entry, over the cluster (the same count in every CTA)
+    uint32_t n_groups = 0;
+    for (int q = 0; q < CL; ++q) {
+        const int64_t lq = min(ld, (int64_t)q * part), hq = min(ld, lq + part);
+        const int64_t cq = max((int64_t)0, min(own, hq) - lq);
+        n_groups += (uint32_t)((cq + kPer - 1) / kPer);
+    }
     bool fast_ok = false;
-    if (!trivial) {
-        if (rank == 0) {
-            uint32_t *skeys = sl_copy;
+    uint64_t *dense = reinterpret_cast<uint64_t *>(smem_raw + kOffDense);       // [kDense]
+    uint32_t *hw = reinterpret_cast<uint32_t *>(smem_raw + kOffHw);
+    uint32_t *hs = reinterpret_cast<uint32_t *>(smem_raw + kOffHs);
+    int32_t *out = sel_idx + (int64_t)row * k;
+    if constexpr (kSingle) {
+      if (!trivial) {
+        // ---- one CTA holds the row: the exact threshold over its keys directly (entry u of
+        // a thread is u*512 + tid, as loaded), emitted in region order through a bitmap
+        // the keys stay in smem (read again per pass) to keep registers for the passes
+        auto valid_u = [&](int u) { return u * kThreads + tid < cnt; };
+        auto comp_u = [&](int u) {
+            return ((uint64_t)keys[padded(u * kThreads + tid)] << 32) |
+                   (uint64_t)(0xFFFFFFFFu - (uint32_t)(lo + u * kThreads + tid));
+        };
+        uint32_t kmin = 0xFFFFFFFFu;
 #pragma unroll
-            for (int u = 0; u < kSPer; ++u) {
-                const uint32_t j = u * kThreads + tid;
-                if (j < ns) skeys[j] = score_key(sv[u]);
-            }
-            __syncthreads();
-            // the sample rank whose expected row rank is ~1.5 need, plus a margin; the bound
-            // is the lower edge of its 12-bit key bin (any bound is fine: the count of keys
-            // above it is verified below)
-            uint32_t js = (uint32_t)((3 * need + 2 * st - 1) / (2 * st)) + 8;
-            js = min(max(js, 1u), ns);
-            const int sh1[1] = {20};
-            const int wd1[1] = {12};
-            uint32_t lp, lm;
-            cta_select_desc<uint32_t, kThreads, 1>(skeys, ns, js, sh1, wd1, hist, scan_ws, lp, lm);
-            if (tid == 0) sh_L = lp;                      // low 20 bits 0: <= the js-th sample key
-        }
-        cluster.sync();                                                     // L published
-        const uint32_t Lk = *cluster.map_shared_rank(&sh_L, 0);
-        uint64_t *clist = reinterpret_cast<uint64_t *>(hist);                // own candidates
-        if (tid == 0) sh_ccount = 0;
+        for (int u = 0; u < kPer; ++u) kmin = valid_u(u) ? min(kmin, keys[padded(u * kThreads + tid)]) : kmin;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+        if (lane == 0) atomicMin(&sh_kmin, kmin);
         __syncthreads();
-        for (int i = tid; i < cnt; i += kThreads) {
-            const uint32_t key = key_at(i);
-            if (key >= Lk) {
-                const uint32_t slot = atomicAdd(&sh_ccount, 1u);
-                if (slot < (uint32_t)kCandMax)
-                    clist[slot] = ((uint64_t)key << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)(lo + i));
-            }
-        }
-        cluster.sync();                                                     // candidate lists ready
-        uint32_t total = 0;
-        bool overflow = false;
-        for (int q = 0; q < CL; ++q) {
-            const uint32_t c = *cluster.map_shared_rank(&sh_ccount, q);
-            total += c;
-            overflow |= c > (uint32_t)kCandMax;
-        }
-        fast_ok = !overflow && total >= (uint32_t)need && total <= (uint32_t)kCandTotal;
-        if (fast_ok && rank == 0) {
-            uint64_t *call = reinterpret_cast<uint64_t *>(gsl);              // all candidates
-            if (tid < CL) slice_tot[tid] = *cluster.map_shared_rank(&sh_ccount, tid);
-            __syncthreads();
-            if (tid == 0) {
-                off_s[0] = 0;
-                for (int q = 0; q < CL; ++q) off_s[q + 1] = off_s[q] + slice_tot[q];
-            }
-            __syncthreads();
-            const uint32_t n = off_s[CL];
-            // one flat parallel copy: entry i of the concatenation comes from rank q
-            for (uint32_t i = tid; i < n; i += kThreads) {
-                int q = 0;
-                while (q + 1 < CL && i >= off_s[q + 1]) ++q;
-                const uint64_t *rl = reinterpret_cast<const uint64_t *>(cluster.map_shared_rank(hist, q));
-                call[i] = rl[i - off_s[q]];
-            }
-            __syncthreads();
-            const int shc[5] = {52, 40, 32, 10, 0};
-            const int wdc[5] = {12, 12, 8, 10, 10};
-            uint64_t cp, cm;
-            cta_select_desc<uint64_t, kThreads, 5>(call, n, (uint32_t)need, shc, wdc, sl_copy, scan_ws, cp, cm);
-            // mark the selection plus the own region in a bitmap (over this CTA's keys, now
-            // unused) and emit it in ascending order
-            uint32_t *bitmap = keys;
+        uint64_t elo, ehi, cp, cm;
+        fast_ok = block_threshold<kPer>(valid_u, comp_u, (uint32_t)need, sh_kmin, hs, dense, hw, &sh_kmax, &sh_nin,
+                                        scan_ws + 32, mm_ws, &elo, &ehi, &cp, &cm);
+        if (fast_ok) {
+            uint32_t *bitmap = hw;                                          // own + 1 <= kPartMax bits
             const int words = (int)((own + 1 + 31) / 32);
-            for (int i = tid; i < words; i += kThreads) bitmap[i] = 0;
+            __syncthreads();                                                // hw free again
+            for (int i = tid; i < words; i += kThreads) bitmap[i] = 0u;
             __syncthreads();
-            for (uint32_t i = tid; i < n; i += kThreads) {
-                const uint64_t c = call[i];
-                if ((c & cm) >= cp) {
-                    const uint32_t r = 0xFFFFFFFFu - (uint32_t)c;
-                    if (r < (uint64_t)own) atomicOr(&bitmap[r >> 5], 1u << (r & 31));
+#pragma unroll
+            for (int u = 0; u < kPer; ++u) {
+                if (valid_u(u) && threshold_selects(comp_u(u), elo, ehi, cp, cm)) {
+                    const int r = u * kThreads + tid;                       // lo = 0 with one CTA
+                    atomicOr(&bitmap[r >> 5], 1u << (r & 31));
                 }
             }
-            __syncthreads();
             if (tid == 0) atomicOr(&bitmap[own >> 5], 1u << (own & 31));
             __syncthreads();
             const int wpt = (words + kThreads - 1) / kThreads;
-            const int w0 = tid * wpt;
-            uint32_t c = 0;
+            uint32_t bc = 0;
             for (int i = 0; i < wpt; ++i)
-                if (w0 + i < words) c += __popc(bitmap[w0 + i]);
-            const uint32_t incl = block_scan_incl<kThreads>(c, scan_ws);
-            int32_t *out = sel_idx + (int64_t)row * k;
-            uint32_t pos = incl - c;
+                if (tid * wpt + i < words) bc += __popc(bitmap[tid * wpt + i]);
+            const uint32_t bincl = block_scan_incl<kThreads>(bc, scan_ws);
+            uint32_t opos = bincl - bc;
             for (int i = 0; i < wpt; ++i) {
-                if (w0 + i >= words) break;
-                uint32_t b = bitmap[w0 + i];
-                while (b) {
-                    const int bit = __ffs(b) - 1;
-                    b &= b - 1;
-                    if (pos < (uint32_t)k) out[pos] = (w0 + i) * 32 + bit;
-                    ++pos;
+                const int w = tid * wpt + i;
+                if (w >= words) break;
+                uint32_t bits = bitmap[w];
+                while (bits) {
+                    const int bit = __ffs(bits) - 1;
+                    bits &= bits - 1;
+                    if (opos < (uint32_t)k) out[opos] = w * 32 + bit;
+                    ++opos;
                 }
             }
             if (tid == kThreads - 1) {
-                if (incl != (uint32_t)(need + 1)) set_error(kErrTopkInternal);
-                sel_count[row] = (int32_t)min((int64_t)incl, (int64_t)k);
+                if (bincl != (uint32_t)(need + 1)) set_error(kErrTopkInternal);
+                sel_count[row] = (int32_t)(need + 1);
             }
             for (int i = (int)need + 1 + tid; i < k; i += kThreads) out[i] = -1;
         }
+      }
+    } else if (!trivial && (int64_t)n_groups >= need) {
+        uint32_t *gmax = reinterpret_cast<uint32_t *>(smem_raw + kOffGmax);
+        uint64_t *slots = reinterpret_cast<uint64_t *>(smem_raw + kOffSlots);
+        uint32_t key[kPer];
+        {
+            const uint4 *run = reinterpret_cast<const uint4 *>(keys + padded(tid * kPer));
+#pragma unroll
+            for (int j = 0; j < kPer / 4; ++j) {
+                const uint4 w = run[j];
+                key[4 * j] = w.x;
+                key[4 * j + 1] = w.y;
+                key[4 * j + 2] = w.z;
+                key[4 * j + 3] = w.w;
+            }
+        }
+        // ---- group maximum to every CTA (0 = no eligible entry: below every score key)
+        uint32_t gm = 0;
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) gm = (u < nmine && key[u] > gm) ? key[u] : gm;
+        for (int q = 0; q < CL; ++q) cluster.map_shared_rank(gmax, q)[rank * kThreads + tid] = gm;
+        cluster.sync();                                                     // all group maxima in place
+        // ---- the bound L (the same in every CTA): a 256-bin histogram of the group maxima over
+        // [gmin, gmax] with a power-of-two bin width; L is the lower edge of the bin that holds
+        // the need-th largest maximum (groups without an eligible entry, maximum 0, take no part)
+        uint32_t g8[kMaxCluster];
+        uint32_t gmin = 0xFFFFFFFFu, gmx = 0u;
+#pragma unroll
+        for (int q = 0; q < kMaxCluster; ++q) {
+            g8[q] = q < CL ? gmax[q * kThreads + tid] : 0u;
+            if (g8[q] != 0u) {
+                gmin = min(gmin, g8[q]);
+                gmx = max(gmx, g8[q]);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            gmin = min(gmin, __shfl_xor_sync(0xffffffffu, gmin, o));
+            gmx = max(gmx, __shfl_xor_sync(0xffffffffu, gmx, o));
+        }
+        if (lane == 0) {
+            atomicMin(&sh_kmin, gmin);
+            atomicMax(&sh_kmax, gmx);
+        }
+        __syncthreads();
+        gmin = sh_kmin;
+        gmx = sh_kmax;
+        const int gsh = max(0, 24 - __clz((int)(gmx - gmin)));                // (gmx - gmin) >> gsh < 256
+#pragma unroll
+        for (int q = 0; q < kMaxCluster; ++q)
+            if (g8[q] != 0u) atomicAdd(&hs[(g8[q] - gmin) >> gsh], 1u);
+        __syncthreads();
+        if (warp == 0) desc_bin_search(hs, (uint32_t)need, scan_ws + 32);
+        __syncthreads();
+        const uint32_t Lk = gmin + (scan_ws[32] << gsh);
+        // ---- candidates (key >= L) in region order into rank 0's slots [rank*slot_n, ...),
+        // the count to every CTA
+        const int lg_slot = __ffs(kSlots / CL) - 1;                         // CL is a power of 2
+        const uint32_t slot_n = 1u << lg_slot;
+        uint32_t c = 0;
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) c += (u < nmine && key[u] >= Lk) ? 1u : 0u;
+        const uint32_t incl = block_scan_incl<kThreads>(c, scan_ws);
+        const uint32_t cta_total = scan_ws[kWarps - 1];
+        uint64_t *dst = reinterpret_cast<uint64_t *>(cluster.map_shared_rank(slots, 0)) + ((size_t)rank << lg_slot);
+        uint32_t pos = incl - c;
+        const uint32_t rbase = 0xFFFFFFFFu - (uint32_t)(lo + tid * kPer);  // ~region of key[0]
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            if (u < nmine && key[u] >= Lk) {
+                if (pos < slot_n) dst[pos] = ((uint64_t)key[u] << 32) | (uint64_t)(rbase - (uint32_t)u);
+                ++pos;
+            }
+        }
+        if (tid < CL) *cluster.map_shared_rank(&cand_cnt[rank], tid) = cta_total;
+        if (tid == 0) {
+            sh_kmax = 0u;
+            sh_nin = 0u;
+        }
+        cluster.sync();                                                     // candidates and counts in place
+        uint32_t total = 0;
+        bool overflow = false;
+        for (int q = 0; q < CL; ++q) {
+            total += cand_cnt[q];
+            overflow |= cand_cnt[q] > slot_n;
+        }
+        fast_ok = !overflow && total >= (uint32_t)need && total <= (uint32_t)kDense;
+        if (fast_ok && rank == 0) {
+            // ---- dense gather in region order: thread t takes entries [t*kDPer, (t+1)*kDPer)
+            uint32_t *first = slice_tot;                                    // first dense entry of each rank
+            if (tid == 0) {
+                uint32_t run = 0;
+                for (int q = 0; q < CL; ++q) {
+                    first[q] = run;
+                    run += cand_cnt[q];
+                }
+            }
+            __syncthreads();
+            uint64_t cv[kDPer];
+            const uint32_t d0 = tid * kDPer;
+            int q = 0;
+            while (q + 1 < CL && d0 >= first[q + 1]) ++q;
+#pragma unroll
+            for (int u = 0; u < kDPer; ++u) {
+                const uint32_t d = d0 + u;
+                while (q + 1 < CL && d >= first[q + 1]) ++q;
+                cv[u] = d < total ? slots[((uint32_t)q << lg_slot) + (d - first[q])] : 0ull;
+            }
+            auto valid_u = [&](int u) { return d0 + (uint32_t)u < total; };
+            auto comp_u = [&](int u) { return cv[u]; };
+            uint64_t elo, ehi, cp, cm;
+            const bool ok = block_threshold<kDPer>(valid_u, comp_u, (uint32_t)need, Lk, hs, dense, hw, &sh_kmax,
+                                                   &sh_nin, scan_ws + 32, mm_ws, &elo, &ehi, &cp, &cm);
+            if (ok) {
+                // ---- ordered emit
+                uint32_t cs = 0;
+#pragma unroll
+                for (int u = 0; u < kDPer; ++u) cs += (valid_u(u) && threshold_selects(cv[u], elo, ehi, cp, cm)) ? 1u : 0u;
+                const uint32_t sincl = block_scan_incl<kThreads>(cs, scan_ws);
+                uint32_t opos = sincl - cs;
+#pragma unroll
+                for (int u = 0; u < kDPer; ++u) {
+                    if (valid_u(u) && threshold_selects(cv[u], elo, ehi, cp, cm)) {
+                        if (opos < (uint32_t)need) out[opos] = (int32_t)(0xFFFFFFFFu - (uint32_t)cv[u]);
+                        ++opos;
+                    }
+                }
+                if (tid == kThreads - 1) {
+                    if (sincl != (uint32_t)need) set_error(kErrTopkInternal);
+                    out[need] = (int32_t)own;                               // own > every eligible region
+                    sel_count[row] = (int32_t)(need + 1);
+                }
+                for (int i = (int)need + 1 + tid; i < k; i += kThreads) out[i] = -1;
+            } else {
+                // more than kDense candidates share one key: cannot happen with total <= kDense
+                if (tid == 0) {
+                    set_error(kErrTopkInternal);
+                    sel_count[row] = 0;
+                }
+            }
+        }
     }
+    if (fast_ok) return;               // nothing reads another CTA's smem after the barrier
+
+    // ---- fallback: exact distributed radix select over the staged keys
+    uint32_t *hist = reinterpret_cast<uint32_t *>(smem_raw);                 // [2][kBins]
+    uint32_t *gsl = hist + 2 * kBins;                                        // [2][kBins] reduced slices
+    uint32_t *sl_copy = gsl + 2 * kBins;                                     // [kBins] local copy of a slice
+
 
     // ---- distributed radix select of the need-th largest key (fallback and trivial rows)
     uint32_t prefix = 0, pmask = 0;
@@ -392,8 +727,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         // smem), and ballots keep index order.  Equal keys at the exact threshold (when the last
         // digit left more of them than needed) are taken lowest region first: rank by rank, warp
         // by warp, then in ballot order.
-        const int lane = tid & 31, warp = tid >> 5;
-        constexpr int kWarps = kThreads / 32;
         const int span = ((cnt + kWarps - 1) / kWarps + 31) & ~31;
         const int wb = warp * span, we = min(cnt, wb + span);
         const bool take_all = (need == own);
