@@ -62,6 +62,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                        const Params p)
 {
+    pdl_trigger();   // the next kernel may launch; it waits for this one itself
+    pdl_wait();      // the previous kernel's results are visible from here on
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *qs = smem + kWarps * kWarpRing;
@@ -397,6 +399,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 constexpr int kCombineThreads = 4 * kD;
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const Params p)
 {
+    pdl_trigger();   // the next kernel may launch; it waits for this one itself
+    pdl_wait();      // the previous kernel's results are visible from here on
     __shared__ float wsm[kD];
     __shared__ float part[kCombineThreads / 32];
     __shared__ float red[2];

@@ -294,4 +294,12 @@ __device__ __forceinline__ uint32_t score_key(float f)
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream serialization
+// may start while the previous kernel in the stream is still running.  pdl_wait() blocks until
+// that kernel has completed and its memory is visible: every kernel calls it before its first
+// global read or write.  pdl_trigger() lets the next kernel launch early (its own wait keeps it
+// correct).  Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
 }  // namespace dsa

@@ -20,6 +20,8 @@ __global__ void __launch_bounds__(128) compress_regions_kernel(
     const int64_t *__restrict__ src_row, const int64_t *__restrict__ dst_slot, int n_regions,
     uint8_t *__restrict__ summaries, float *__restrict__ scales, int64_t n_slots)
 {
+    pdl_trigger();   // the next kernel may launch; it waits for this one itself
+    pdl_wait();      // the previous kernel's results are visible from here on
     const int g = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int i = blockIdx.x; i < n_regions; i += gridDim.x) {
         const int64_t r0 = src_row[i], slot = dst_slot[i];

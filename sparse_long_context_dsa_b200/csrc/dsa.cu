@@ -4,10 +4,12 @@
 // per-device error word is a single symbol).
 #include <algorithm>
 #include <mutex>
+#include <utility>
 #include <string>
 
 #include "../../include/dsa.h"
 #include "attention.cuh"
+#include "attention_cluster.cuh"
 #include "common.cuh"
 #include "compress.cuh"
 #include "gemm_indexer.cuh"
@@ -98,6 +100,37 @@ dsa_status_t launched(const char *what)
     return DSA_OK;
 }
 
+// Every kernel is launched with programmatic stream serialization (it may start while the
+// previous kernel of the stream finishes; each kernel waits for it before touching global
+// memory), optionally as clusters of cluster_x CTAs.
+template <typename... KArgs, typename... Args>
+dsa_status_t launch_k(const char *what, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                      dsa_stream_t stream, unsigned cluster_x, Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    unsigned n = 0;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+    if (cluster_x > 0) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = cluster_x;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+    if (e != cudaSuccess) return cuda_fail(e, what);
+    return launched(what);
+}
+
 // K/V cache viewed as [rows = n_pages*4*64][3][64] bf16: one region = box {64, 3, 8}.
 dsa_status_t kv_map(CUtensorMap *m, const void *cache, int64_t n_pages)
 {
@@ -152,6 +185,51 @@ AttnPlan attn_plan(int nq, int k, int sm_count)
     return a;
 }
 
+// The clustered attention kernel (splits merged in the kernel) serves rows that get one
+// 16-CTA cluster each with every cluster resident at once: k <= 512 and rows <= the number
+// of such clusters the device holds together (queried once per process; 0 when the kernel
+// cannot take the non-portable cluster size).
+int cluster_attn_capacity()
+{
+    static std::once_flag once;
+    static int capacity = 0;
+    std::call_once(once, [] {
+        auto *fn = dsa::attnc::sparse_attn_cluster_kernel;
+        if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsa::attnc::kSmemBytes) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+            cudaGetLastError();
+            return;
+        }
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(dsa::attnc::kSplits, 1, 1);
+        cfg.blockDim = dim3(dsa::attnc::kThreads, 1, 1);
+        cfg.dynamicSmemBytes = dsa::attnc::kSmemBytes;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = dsa::attnc::kSplits;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            return;
+        }
+        capacity = n;
+    });
+    return capacity;
+}
+
+dsa_status_t attn_cluster_launch(const CUtensorMap &mk, const CUtensorMap &mv, const dsa::attn::Params &p, int nq,
+                                 dsa_stream_t stream)
+{
+    return launch_k("sparse_attn_cluster_kernel", dsa::attnc::sparse_attn_cluster_kernel,
+                    dim3(dsa::attnc::kSplits, (unsigned)(nq * dsa::kG)), dim3(dsa::attnc::kThreads),
+                    dsa::attnc::kSmemBytes, stream, (unsigned)dsa::attnc::kSplits, mk, mv, p);
+}
+
 dsa_status_t attn_common(const void *q, const void *k_cache, const void *v_cache, int64_t n_pages,
                          const int32_t *block_table, int max_pages, const int32_t *q_req, int n_req,
                          const int32_t *q_pos, int nq, const int32_t *sel_idx, const int32_t *sel_count, int k,
@@ -169,8 +247,9 @@ dsa_status_t attn_common(const void *q, const void *k_cache, const void *v_cache
     int sms = 0;
     dsa_status_t st = device_info(sms);
     if (st != DSA_OK) return st;
+    const bool clustered = k <= dsa::attnc::kMaxK && (int64_t)nq * dsa::kG <= cluster_attn_capacity();
     const AttnPlan plan = attn_plan(nq, k, sms);
-    if (plan.ws > 0) {
+    if (plan.ws > 0 && !clustered) {
         if (!ws || ws_bytes < plan.ws || !aligned(ws, 256))
             return fail(DSA_ERR_WORKSPACE, "attention workspace too small or not 256-byte aligned (need " +
                                                std::to_string(plan.ws) + " bytes)");
@@ -201,6 +280,7 @@ dsa_status_t attn_common(const void *q, const void *k_cache, const void *v_cache
     p.n_splits = plan.n_splits;
     p.scale_log2 = dsa::attn::kLog2e / sqrtf((float)dsa::kD);
 
+    if (clustered) return attn_cluster_launch(mk, mv, p, nq, stream);
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
@@ -209,11 +289,13 @@ dsa_status_t attn_common(const void *q, const void *k_cache, const void *v_cache
     });
     DSA_CUDA(attr_err, "cudaFuncSetAttribute(sparse_attn_kernel)");
     dim3 grid(plan.n_splits, nq * dsa::kG);
-    dsa::attn::sparse_attn_kernel<<<grid, dsa::attn::kThreads, dsa::attn::kSmemBytes, stream>>>(mk, mv, p);
-    if ((st = launched("sparse_attn_kernel")) != DSA_OK) return st;
+    if ((st = launch_k("sparse_attn_kernel", dsa::attn::sparse_attn_kernel, grid, dim3(dsa::attn::kThreads),
+                       dsa::attn::kSmemBytes, stream, 0, mk, mv, p)) != DSA_OK)
+        return st;
     if (plan.n_splits > 1) {
-        dsa::attn::combine_kernel<<<nq * dsa::kG * 16, dsa::attn::kCombineThreads, 0, stream>>>(p);
-        if ((st = launched("combine_kernel")) != DSA_OK) return st;
+        if ((st = launch_k("combine_kernel", dsa::attn::combine_kernel, dim3(nq * dsa::kG * 16),
+                           dim3(dsa::attn::kCombineThreads), 0, stream, 0, p)) != DSA_OK)
+            return st;
     }
     return DSA_OK;
 }
@@ -242,11 +324,11 @@ dsa_status_t indexer_gemm_path(const void *index_q, const float *gate, const int
     const int n_mtiles = (nq + dsa::gemm::kQPerTile - 1) / dsa::gemm::kQPerTile;
     const int qblocks = (nq * dsa::kHI + 3) / 4;
     const int grid_q = std::max(qblocks, (n_mtiles + 127) / 128);
-    dsa::gemm::quantize_kernel<<<grid_q, 128, 0, stream>>>(static_cast<const __nv_bfloat16 *>(index_q), q_req, q_pos,
-                                                          sum_base, ld, n_slots, nq, codes, qscale, q_own,
-                                                          tile_own, n_mtiles);
     dsa_status_t st;
-    if ((st = launched("gemm quantize_kernel")) != DSA_OK) return st;
+    if ((st = launch_k("gemm quantize_kernel", dsa::gemm::quantize_kernel, dim3(grid_q), dim3(128), 0, stream, 0,
+                       static_cast<const __nv_bfloat16 *>(index_q), q_req, q_pos, sum_base, ld, n_slots, nq, codes,
+                       qscale, q_own, tile_own, n_mtiles)) != DSA_OK)
+        return st;
 
     CUtensorMap map_a, map_b;
     {
@@ -290,9 +372,8 @@ dsa_status_t indexer_gemm_path(const void *index_q, const float *gate, const int
                                         (int)dsa::gemm::kSmemBytes);
     });
     DSA_CUDA(attr_err, "cudaFuncSetAttribute(gemm_scores_kernel)");
-    dsa::gemm::gemm_scores_kernel<<<std::min(sms, p.n_units), dsa::gemm::kThreads, dsa::gemm::kSmemBytes, stream>>>(
-        map_a, map_b, p);
-    return launched("gemm_scores_kernel");
+    return launch_k("gemm_scores_kernel", dsa::gemm::gemm_scores_kernel, dim3(std::min(sms, p.n_units)),
+                    dim3(dsa::gemm::kThreads), dsa::gemm::kSmemBytes, stream, 0, map_a, map_b, p);
 }
 
 // Workspace path of the top-k: histogram, threshold-bin gather and last-CTA selection
@@ -314,8 +395,9 @@ dsa_status_t topk_workspace_path(const float *scores, int64_t ld_scores, const i
     const int rows = nq * dsa::kG;
     const dim3 grid((unsigned)((ld_scores + dsa::topk::kChunk - 1) / dsa::topk::kChunk), (unsigned)rows);
     dsa_status_t st;
-    dsa::topk::hist_kernel<<<grid, dsa::topk::kThreads, 0, stream>>>(scores, ld_scores, q_pos, k, tw);
-    if ((st = launched("topk hist_kernel")) != DSA_OK) return st;
+    if ((st = launch_k("topk hist_kernel", dsa::topk::hist_kernel, grid, dim3(dsa::topk::kThreads), 0, stream, 0,
+                       scores, ld_scores, q_pos, k, tw)) != DSA_OK)
+        return st;
     const size_t dyn = dsa::topk::kCandStage * 8 + round_up((size_t)((ld_scores + 1 + 31) / 32) * 4, 16);
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
@@ -324,9 +406,8 @@ dsa_status_t topk_workspace_path(const float *scores, int64_t ld_scores, const i
                                         (int)(dsa::topk::kCandStage * 8 + (dsa::topk::kMaxRegions / 32 + 16) * 4));
     });
     DSA_CUDA(attr_err, "cudaFuncSetAttribute(topk select_kernel)");
-    dsa::topk::select_kernel<<<grid, dsa::topk::kSelectThreads, dyn, stream>>>(scores, ld_scores, q_pos, k, tw,
-                                                                              sel_idx, sel_count);
-    return launched("topk select_kernel");
+    return launch_k("topk select_kernel", dsa::topk::select_kernel, grid, dim3(dsa::topk::kSelectThreads), dyn,
+                    stream, 0, scores, ld_scores, q_pos, k, tw, sel_idx, sel_count);
 }
 
 // Cluster size for the cluster path: enough CTAs that each holds <= kPartMax keys in smem
@@ -351,27 +432,12 @@ dsa_status_t topk_cluster_path(const float *scores, int64_t ld_scores, const int
                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsa::topkc::kSmemBytes);
     });
     DSA_CUDA(attr_err, "cudaFuncSetAttribute(topk_cluster_kernel)");
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)cl, (unsigned)(nq * dsa::kG), 1);
-    cfg.blockDim = dim3(dsa::topkc::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = dsa::topkc::kSmemBytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)cl;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    const dim3 grid((unsigned)cl, (unsigned)(nq * dsa::kG), 1);
     if (cl == 1)
-        DSA_CUDA(cudaLaunchKernelEx(&cfg, dsa::topkc::topk_cluster_kernel<true>, scores, ld_scores, q_pos, k, sel_idx,
-                                    sel_count),
-                 "cudaLaunchKernelEx(topk_cluster_kernel)");
-    else
-        DSA_CUDA(cudaLaunchKernelEx(&cfg, dsa::topkc::topk_cluster_kernel<false>, scores, ld_scores, q_pos, k, sel_idx,
-                                    sel_count),
-                 "cudaLaunchKernelEx(topk_cluster_kernel)");
-    return launched("topk_cluster_kernel");
+        return launch_k("topk_cluster_kernel", dsa::topkc::topk_cluster_kernel<true>, grid, dim3(dsa::topkc::kThreads),
+                        dsa::topkc::kSmemBytes, stream, 1u, scores, ld_scores, q_pos, k, sel_idx, sel_count);
+    return launch_k("topk_cluster_kernel", dsa::topkc::topk_cluster_kernel<false>, grid, dim3(dsa::topkc::kThreads),
+                    dsa::topkc::kSmemBytes, stream, (unsigned)cl, scores, ld_scores, q_pos, k, sel_idx, sel_count);
 }
 
 // Scratch of dsa_topk_regions_noalloc: one static array per GPU that loads the library.
@@ -439,10 +505,9 @@ dsa_status_t dsa_compress_regions(const void *index_k, int64_t row_stride, int64
     dsa_status_t st = device_info(sms);
     if (st != DSA_OK) return st;
     const int grid = (int)std::min<int64_t>(n_regions, (int64_t)sms * 16);
-    dsa::compress_regions_kernel<<<grid, 128, 0, stream>>>(static_cast<const __nv_bfloat16 *>(index_k), row_stride,
-                                                          n_rows, src_row, dst_slot, n_regions, summaries, scales,
-                                                          n_slots);
-    return launched("compress_regions_kernel");
+    return launch_k("compress_regions_kernel", dsa::compress_regions_kernel, dim3(grid), dim3(128), 0, stream, 0,
+                    static_cast<const __nv_bfloat16 *>(index_k), row_stride, n_rows, src_row, dst_slot, n_regions,
+                    summaries, scales, n_slots);
 }
 
 size_t dsa_indexer_workspace_size(int nq, int64_t ld_scores)
@@ -505,8 +570,8 @@ dsa_status_t dsa_indexer_scores(const void *index_q, const float *gate, const in
     });
     DSA_CUDA(attr_err, "cudaFuncSetAttribute(scan_kernel)");
     const int grid = (int)std::min<int64_t>(p.total_units, (int64_t)sms * dsa::idx::kCtasPerSm);
-    dsa::idx::scan_kernel<<<grid, dsa::idx::kThreads, dsa::idx::kSmemBytes, stream>>>(map, p);
-    return launched("scan_kernel");
+    return launch_k("scan_kernel", dsa::idx::scan_kernel, dim3(grid), dim3(dsa::idx::kThreads), dsa::idx::kSmemBytes,
+                    stream, 0, map, p);
 }
 
 size_t dsa_topk_workspace_size(int nq, int64_t ld_scores, int k)

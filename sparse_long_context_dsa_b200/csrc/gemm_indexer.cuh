@@ -80,6 +80,8 @@ __global__ void __launch_bounds__(128) quantize_kernel(const __nv_bfloat16 *__re
                                                        float *__restrict__ qscale, int32_t *__restrict__ q_own,
                                                        int32_t *__restrict__ tile_own, int n_mtiles)
 {
+    pdl_trigger();   // the next kernel may launch; it waits for this one itself
+    pdl_wait();      // the previous kernel's results are visible from here on
     const int gw = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
     if (gw < nq * kHI) {
         const int q = gw / kHI;
@@ -150,6 +152,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     gemm_scores_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                        const Params p)
 {
+    pdl_trigger();   // the next kernel may launch; it waits for this one itself
+    pdl_wait();      // the previous kernel's results are visible from here on
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sb = smem;                                   // summary tile: 2 K columns x [256][128]

@@ -153,6 +153,8 @@ __device__ __forceinline__ void load_query_fragments(const Params &p, int qi, in
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     scan_kernel(const __grid_constant__ CUtensorMap tmap, const Params p)
 {
+    pdl_trigger();   // the next kernel may launch; it waits for this one itself
+    pdl_wait();      // the previous kernel's results are visible from here on
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float *sscale = reinterpret_cast<float *>(smem + kStages * kStageBytes);      // [kStages][4][32]

@@ -100,6 +100,8 @@ __device__ __forceinline__ void find_desc(const uint32_t *hist, int nb, uint32_t
 __global__ void __launch_bounds__(kThreads) hist_kernel(const float *__restrict__ scores, int64_t ld,
                                                         const int32_t *__restrict__ q_pos, int k, Ws ws)
 {
+    pdl_trigger();   // the next kernel may launch; it waits for this one itself
+    pdl_wait();      // the previous kernel's results are visible from here on
     __shared__ uint32_t h[kBins];
     const int row = blockIdx.y;
     const int64_t own = row_own(q_pos, row);
@@ -239,6 +241,8 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const float *__r
                                                                 int32_t *__restrict__ sel_idx,
                                                                 int32_t *__restrict__ sel_count)
 {
+    pdl_trigger();   // the next kernel may launch; it waits for this one itself
+    pdl_wait();      // the previous kernel's results are visible from here on
     extern __shared__ uint32_t dyn[];                 // [kCandStage] uint2, then the bitmap
     uint2 *cstage = reinterpret_cast<uint2 *>(dyn);
     uint32_t *bitmap = dyn + 2 * kCandStage;

@@ -346,6 +346,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     topk_cluster_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ q_pos, int k,
                         int32_t *__restrict__ sel_idx, int32_t *__restrict__ sel_count)
 {
+    pdl_trigger();   // the next kernel may launch; it waits for this one itself
+    pdl_wait();      // the previous kernel's results are visible from here on
     extern __shared__ __align__(16) uint8_t smem_raw[];
     __shared__ uint32_t scan_ws[40];                                         // block scans + select results
     __shared__ uint32_t tot[2];                                              // slice totals (double-buffered)
