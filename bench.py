@@ -314,16 +314,11 @@ def run_ours(args):
         L["step"].run()
     dsa.check_device()
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
+    from sparse_long_context_dsa_b200 import replicas
+    barrier = replicas.barrier
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return replicas.max_over_ranks(x, dev)
 
     # ---- warm-up graph and timed graph(s); each graph holds at most 250 steps
     chunk = min(args.steps, 250)
@@ -407,7 +402,7 @@ def run_ours(args):
     assert torch.equal(e2e_bufs[0]["out"], layers[0]["step"].out.cpu())
 
     hbm, peak_kind = peaks()
-    qps = world * args.steps / (ms / 1e3)
+    qps = replicas.job_throughput(args.steps, world, ms)
     scan_gbs = scan_bytes(own) / (scan_avg_ms / 1e3) / 1e9
     step_gbs = step_bytes(own, TOPK) * args.steps / (ms / 1e3) / 1e9
     line = {
@@ -426,7 +421,7 @@ def run_ours(args):
                      "algorithmic_bytes_per_launch": scan_bytes(own), "avg_launch_us": scan_avg_ms * 1e3,
                      "in_step_us": in_step_avg_ms * 1e3,
                      "traffic": None},
-        "e2e": {"value": world * args.steps / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "e2e": {"value": replicas.job_throughput(args.steps, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": sampler.summary(),
