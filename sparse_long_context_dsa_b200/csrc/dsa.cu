@@ -510,33 +510,12 @@ dsa_status_t dsa_compress_regions(const void *index_k, int64_t row_stride, int64
                     summaries, scales, n_slots);
 }
 
-size_t dsa_indexer_workspace_size(int nq, int64_t ld_scores)
+// The streaming scan of dsa_indexer_scores.
+dsa_status_t scan_path(const void *index_q, const float *gate, const int32_t *q_req, const int32_t *q_pos, int nq,
+                       const uint8_t *summaries, const float *scales, int64_t n_slots, const int64_t *sum_base,
+                       int n_req, float *scores, int64_t ld_scores, uint32_t flags, int sms, dsa_stream_t stream)
 {
-    (void)ld_scores;
-    return gemm_ws_size(nq);
-}
-
-dsa_status_t dsa_indexer_scores(const void *index_q, const float *gate, const int32_t *q_req, const int32_t *q_pos,
-                                int nq, const uint8_t *summaries, const float *scales, int64_t n_slots,
-                                const int64_t *sum_base, int n_req, float *scores, int64_t ld_scores, uint32_t flags,
-                                void *ws, size_t ws_bytes, dsa_stream_t stream)
-{
-    DSA_REQUIRE(nq >= 0, "nq must be >= 0");
-    DSA_REQUIRE((flags & ~DSA_Q_FP8) == 0, "unknown flag");
-    DSA_REQUIRE(ld_scores >= 1 && ld_scores <= (1ll << 26), "ld_scores out of [1, 2^26]");
-    DSA_REQUIRE(n_slots >= 1 && n_slots <= (1ll << 28), "n_slots out of [1, 2^28]");
-    DSA_REQUIRE(n_req >= 1, "n_req must be >= 1");
-    if (nq == 0) return DSA_OK;
-    DSA_REQUIRE(index_q && gate && q_req && q_pos && summaries && scales && sum_base && scores, "NULL pointer");
-    DSA_REQUIRE(aligned(index_q, 16) && aligned(summaries, 16), "index_q and summaries must be 16-byte aligned");
-    int sms = 0;
-    dsa_status_t st = device_info(sms);
-    if (st != DSA_OK) return st;
-
-    if ((flags & DSA_Q_FP8) && n_req == 1 && nq >= kGemmMinQueries && ws && ws_bytes >= gemm_ws_size(nq) &&
-        aligned(ws, 256))
-        return indexer_gemm_path(index_q, gate, q_req, q_pos, nq, summaries, scales, n_slots, sum_base, scores,
-                                 ld_scores, ws, sms, stream);
+    dsa_status_t st;
     CUtensorMap map;
     {
         const cuuint64_t dims[2] = {(cuuint64_t)dsa::kDI, (cuuint64_t)n_slots * dsa::kG};
@@ -572,6 +551,37 @@ dsa_status_t dsa_indexer_scores(const void *index_q, const float *gate, const in
     const int grid = (int)std::min<int64_t>(p.total_units, (int64_t)sms * dsa::idx::kCtasPerSm);
     return launch_k("scan_kernel", dsa::idx::scan_kernel, dim3(grid), dim3(dsa::idx::kThreads), dsa::idx::kSmemBytes,
                     stream, 0, map, p);
+}
+
+size_t dsa_indexer_workspace_size(int nq, int64_t ld_scores)
+{
+    (void)ld_scores;
+    return gemm_ws_size(nq);
+}
+
+dsa_status_t dsa_indexer_scores(const void *index_q, const float *gate, const int32_t *q_req, const int32_t *q_pos,
+                                int nq, const uint8_t *summaries, const float *scales, int64_t n_slots,
+                                const int64_t *sum_base, int n_req, float *scores, int64_t ld_scores, uint32_t flags,
+                                void *ws, size_t ws_bytes, dsa_stream_t stream)
+{
+    DSA_REQUIRE(nq >= 0, "nq must be >= 0");
+    DSA_REQUIRE((flags & ~DSA_Q_FP8) == 0, "unknown flag");
+    DSA_REQUIRE(ld_scores >= 1 && ld_scores <= (1ll << 26), "ld_scores out of [1, 2^26]");
+    DSA_REQUIRE(n_slots >= 1 && n_slots <= (1ll << 28), "n_slots out of [1, 2^28]");
+    DSA_REQUIRE(n_req >= 1, "n_req must be >= 1");
+    if (nq == 0) return DSA_OK;
+    DSA_REQUIRE(index_q && gate && q_req && q_pos && summaries && scales && sum_base && scores, "NULL pointer");
+    DSA_REQUIRE(aligned(index_q, 16) && aligned(summaries, 16), "index_q and summaries must be 16-byte aligned");
+    int sms = 0;
+    dsa_status_t st = device_info(sms);
+    if (st != DSA_OK) return st;
+
+    if ((flags & DSA_Q_FP8) && n_req == 1 && nq >= kGemmMinQueries && ws && ws_bytes >= gemm_ws_size(nq) &&
+        aligned(ws, 256))
+        return indexer_gemm_path(index_q, gate, q_req, q_pos, nq, summaries, scales, n_slots, sum_base, scores,
+                                 ld_scores, ws, sms, stream);
+    return scan_path(index_q, gate, q_req, q_pos, nq, summaries, scales, n_slots, sum_base, n_req, scores, ld_scores,
+                     flags, sms, stream);
 }
 
 size_t dsa_topk_workspace_size(int nq, int64_t ld_scores, int k)

@@ -178,6 +178,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         // ---------------- producer warp: lane 0 issues the TMA loads of the summaries; every
         // lane copies 4 of the stage's 128 fp32 scales into smem asynchronously
         if (lane == 0) prefetch_tensormap(&tmap);
+        const uint64_t pol = l2_evict_first_policy();     // the summaries are read once per query
         int it = 0;
         constexpr int kScalesPerLane = kG * kChunk / 32;          // 4 at 32 regions per stage
         const int sg = (lane * kScalesPerLane) / kChunk, sr = (lane * kScalesPerLane) % kChunk;
@@ -196,8 +197,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 #pragma unroll
                 for (int g = 0; g < kG; ++g) {
                     const int y = (int)(g * p.n_slots + base + r0);
-                    tma_load_2d(st + g * kGroupBytes, &tmap, 0, y, &full[s]);
-                    tma_load_2d(st + g * kGroupBytes + kHalfBytes, &tmap, 128, y, &full[s]);
+                    tma_load_2d_hint(st + g * kGroupBytes, &tmap, 0, y, &full[s], pol);
+                    tma_load_2d_hint(st + g * kGroupBytes + kHalfBytes, &tmap, 128, y, &full[s], pol);
                 }
             }
             // scales: asynchronous 4-byte copies that arrive on the stage's barrier when they

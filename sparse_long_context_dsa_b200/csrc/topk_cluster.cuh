@@ -242,40 +242,61 @@ __device__ __forceinline__ void desc_bin_search(const uint32_t *h, uint32_t m, u
 
 // Exact threshold of the m largest among the block's (key, region) items, each thread holding
 // R of them (item u of a thread counts when valid(u); comp(u) = key << 32 | ~region, all
-// distinct).  Up to three levels of 256-bin key histograms (power-of-two bin widths, the
-// first over [klo, max key], each next one inside the previous level's bin of the m-th
-// largest) narrow the m-th largest down to a key range [*elo, *ehi) holding at most 32 items
-// (or a single key value); those are ranked exactly, pairwise in one warp, else by a radix
-// select over them.  Afterwards an item is selected iff key >= *ehi, or key >= *elo and
-// (comp & *cm) >= *cp: exactly m items.  Needs 1 <= m <= the valid count and every valid key
-// >= klo; returns false (uniformly) when the final range holds more than kDense items.
-// hs: 256 words; list: kDense 8-byte words; sh_kmax, sh_nin: zeroed before the call.
+// distinct, so ties of equal keys go to the lower region).  Levels of 256-bin histograms over
+// the 64-bit composites (power-of-two bin widths: the first over [min, max], each next one
+// inside the previous level's bin of the m-th largest) narrow the m-th largest down to a bin of
+// at most 32 items, which one warp ranks pairwise.  The result is the m-th largest composite T:
+// afterwards an item is selected iff comp >= T (returned as *cp with *cm = all ones, *elo = 0,
+// *ehi = 2^32, the form threshold_selects takes); exactly m items are.  Needs 1 <= m <= the
+// valid count.  hs: 256 words; list: 32 8-byte words; sh_kmax, sh_nin: zeroed before the call
+// (klo and hw are unused: kept for the callers' layout).
 template <int R, typename Valid, typename Comp>
 __device__ bool block_threshold(Valid valid, Comp comp, uint32_t m, uint32_t klo, uint32_t *hs, uint64_t *list,
                                 uint32_t *hw, uint32_t *sh_kmax, uint32_t *sh_nin, uint32_t *res, uint64_t *bc,
                                 uint64_t *elo, uint64_t *ehi, uint64_t *cp, uint64_t *cm)
 {
+    (void)klo;
+    (void)hw;
+    (void)sh_kmax;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    uint32_t kmx = 0u;
-#pragma unroll
+    __shared__ unsigned long long s_min, s_max;
+    uint64_t cmn = ~0ull, cmx = 0ull;
+#pragma unroll 8
     for (int u = 0; u < R; ++u)
-        if (valid(u)) kmx = max(kmx, (uint32_t)(comp(u) >> 32));
+        if (valid(u)) {
+            const uint64_t c = comp(u);
+            cmn = c < cmn ? c : cmn;
+            cmx = c > cmx ? c : cmx;
+        }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) kmx = max(kmx, __shfl_xor_sync(0xffffffffu, kmx, o));
-    if (lane == 0) atomicMax(sh_kmax, kmx);
+    for (int o = 16; o > 0; o >>= 1) {
+        const uint64_t a = __shfl_xor_sync(0xffffffffu, cmn, o), b2 = __shfl_xor_sync(0xffffffffu, cmx, o);
+        cmn = a < cmn ? a : cmn;
+        cmx = b2 > cmx ? b2 : cmx;
+    }
+    if (tid == 0) {
+        s_min = ~0ull;
+        s_max = 0ull;
+    }
     if (tid < 256) hs[tid] = 0u;
     __syncthreads();
-    kmx = *sh_kmax;
-    uint64_t rlo = klo;                                                     // current key range [rlo, rlo + 256 << bsh)
-    int bsh = max(0, 24 - __clz((int)(kmx - klo)));
-    uint32_t m_rem = m, n_in = 0, bin = 0;
-    for (int level = 0; level < 3; ++level) {
-        const uint64_t rhi = rlo + (256ull << bsh);
-#pragma unroll
+    if (lane == 0) {
+        atomicMin(&s_min, (unsigned long long)cmn);
+        atomicMax(&s_max, (unsigned long long)cmx);
+    }
+    __syncthreads();
+    cmn = s_min;
+    cmx = s_max;
+    uint64_t rlo = cmn;
+    int bsh = cmx == cmn ? 0 : max(0, 56 - __clzll((long long)(cmx - cmn)));   // (cmx - cmn) >> bsh < 256
+    uint32_t m_rem = m, bin = 0, n_in = 0;
+    uint64_t width = ~0ull;                                  // extent of the current range [rlo, rlo + width)
+    for (int level = 0; level < 8; ++level) {
+#pragma unroll 8
         for (int u = 0; u < R; ++u) {
             if (!valid(u)) continue;
-            const uint64_t kk = comp(u) >> 32;
-            if (kk >= rlo && kk < rhi) atomicAdd(&hs[(uint32_t)((kk - rlo) >> bsh)], 1u);
+            const uint64_t c = comp(u);
+            if (c >= rlo && c - rlo < width) atomicAdd(&hs[(uint32_t)((c - rlo) >> bsh)], 1u);
         }
         __syncthreads();
         if (warp == 0) desc_bin_search(hs, m_rem, res);
@@ -283,54 +304,33 @@ __device__ bool block_threshold(Valid valid, Comp comp, uint32_t m, uint32_t klo
         bin = res[0];
         m_rem -= res[1];
         n_in = res[2];
-        if (tid < 256) hs[tid] = 0u;                                        // for the next level
+        if (tid < 256) hs[tid] = 0u;
         if (n_in <= 32 || bsh == 0) break;
         rlo += (uint64_t)bin << bsh;
+        width = 1ull << bsh;                                 // the next level stays inside this bin
         bsh = max(0, bsh - 8);
         __syncthreads();
     }
-    const uint64_t blo = rlo + ((uint64_t)bin << bsh), bhi = blo + (1ull << bsh);
-    if (n_in > (uint32_t)kDense) return false;
-#pragma unroll
+    // the bin's members (at most 32: a bin of width 1 holds one composite)
+    const uint64_t blo = rlo + ((uint64_t)bin << bsh);
+#pragma unroll 8
     for (int u = 0; u < R; ++u) {
         if (!valid(u)) continue;
-        const uint64_t kk = comp(u) >> 32;
-        if (kk >= blo && kk < bhi) list[atomicAdd(sh_nin, 1u)] = comp(u);
+        const uint64_t c = comp(u);
+        if (c >= blo && ((c - blo) >> bsh) == 0ull) list[atomicAdd(sh_nin, 1u)] = c;
     }
     __syncthreads();
-    uint64_t p, mk;
-    if (n_in <= 32) {
-        if (warp == 0) {
-            const uint64_t e = lane < (int)n_in ? list[lane] : 0ull;
-            uint32_t gt = 0;
-            for (int j = 0; j < (int)n_in; ++j) gt += __shfl_sync(0xffffffffu, e, j) > e ? 1u : 0u;
-            if (lane < (int)n_in && gt == m_rem - 1) bc[0] = e;
-        }
-        __syncthreads();
-        p = bc[0];
-        mk = ~0ull;
-    } else {
-        constexpr int kLP = kDense / kThreads;
-        uint64_t lv[kLP];
-        uint32_t lvalid = 0;
-        uint64_t lmin = ~0ull, lmax = 0ull;
-#pragma unroll
-        for (int u = 0; u < kLP; ++u) {
-            const uint32_t i = u * kThreads + tid;
-            lv[u] = i < n_in ? list[i] : 0ull;
-            if (i < n_in) {
-                lvalid |= 1u << u;
-                lmin = min(lmin, lv[u]);
-                lmax = max(lmax, lv[u]);
-            }
-        }
-        block_minmax<uint64_t>(lmin, lmax, bc);
-        cta_select_reg<uint64_t, kLP>(lv, lvalid, m_rem, top_differing_bit(lmin, lmax), lmin, hw, hs, res, p, mk);
+    if (warp == 0) {
+        const uint64_t e = lane < (int)n_in ? list[lane] : 0ull;
+        uint32_t gt = 0;
+        for (int j = 0; j < (int)n_in; ++j) gt += __shfl_sync(0xffffffffu, e, j) > e ? 1u : 0u;
+        if (lane < (int)n_in && gt == m_rem - 1) bc[0] = e;
     }
-    *elo = blo;
-    *ehi = bhi;
-    *cp = p;
-    *cm = mk;
+    __syncthreads();
+    *elo = 0ull;
+    *ehi = 1ull << 32;
+    *cp = bc[0];
+    *cm = ~0ull;
     return true;
 }
 

@@ -100,3 +100,16 @@ def test_own_beyond_ld_is_flagged():
     with pytest.raises(dsa.DsaError):
         dsa.check_device()
     assert np.all(cnt.cpu().numpy() == 0) and np.all(idx.cpu().numpy() == -1)
+
+
+@pytest.mark.parametrize("ld", [16000, 16384, 60000, 131071])
+def test_equal_scores_take_the_lowest_regions(ld):
+    # every score of a row equal (one row +0, one row a positive constant, one row two values
+    # in alternating blocks): the exact threshold must narrow through several histogram
+    # levels of the (score, region) composite, on the single-CTA rows (ld <= 16,384) and on
+    # the cluster rows
+    k = 512
+    s = np.zeros((3, G, ld), np.float32)
+    s[1] = 0.75
+    s[2] = np.where((np.arange(ld) // 97) % 2 == 0, 1.5, 1.25).astype(np.float32)
+    check(s, [8 * ld - 1, 8 * ld - 3, 8 * (ld - 5)], k)
