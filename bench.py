@@ -41,6 +41,9 @@ L_CTX = 1 << 20
 TOPK = 512
 N_LAYERS = 4
 KERNELS_PER_STEP = 4      # compress, scan, cluster top-k, clustered attention (split merge inside)
+# DRAM bytes (read + write) of one scan launch on this workload, from one ncu capture of the
+# current scan kernel (dram__bytes_read.sum + dram__bytes_write.sum); None once the kernel changes
+SCAN_TRAFFIC_BYTES = 136_393_216 + 5_188_352
 PREFILL_CTX, PREFILL_NEW = 262144, 2048
 PREFILL_KERNELS = 6       # compress, quantize, GEMM, top-k histogram, top-k select, attention
 
@@ -420,7 +423,7 @@ def run_ours(args):
                      "unit": "GB/s", "frac": scan_gbs / hbm, "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": scan_bytes(own), "avg_launch_us": scan_avg_ms * 1e3,
                      "in_step_us": in_step_avg_ms * 1e3,
-                     "traffic": None},
+                     "traffic": SCAN_TRAFFIC_BYTES},
         "e2e": {"value": replicas.job_throughput(args.steps, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": KERNELS_PER_STEP * args.steps,
