@@ -12,10 +12,11 @@ robin, so consecutive steps never find their inputs in the 126 MB L2.
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload decode_b1_1m|prefill_2k_256k]
 
---workload prefill_2k_256k times the chunked-prefill step instead (2,048 new query tokens
+--workload prefill_2k_256k[_local] times the chunked-prefill step instead (2,048 new query tokens
 on a 262,144-token context: compress the 256 completed regions, FP8 indexer GEMM, top-512
 per query and group, sparse GQA prefill attention) and prints its own line (tokens/s and
-each stage's share; the indexer GEMM's roofline against the FP8 tensor peak).
+each stage's share; the indexer GEMM's roofline against the FP8 tensor peak); _local gives
+the 8 queries of a region one indexer query, so neighbouring queries select the same regions.
 
 --gpus N > 1 (under torchrun): every rank runs an independent replica (requests shard
 across GPUs with no data-path collective, weak scaling); timing is the max over ranks.
@@ -57,7 +58,8 @@ def parse():
     ap.add_argument("--layers", type=int, default=N_LAYERS)
     ap.add_argument("--cpu-queries", type=int, default=3, help="oracle queries timed for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["decode_b1_1m", "prefill_2k_256k"], default="decode_b1_1m")
+    ap.add_argument("--workload", choices=["decode_b1_1m", "prefill_2k_256k", "prefill_2k_256k_local"],
+                    default="decode_b1_1m")
     return ap.parse_args()
 
 
@@ -247,7 +249,8 @@ def record_external(event, stream_handle: int):
 def capture(layers, n_steps, ev_pairs=None, e2e=None):
     """One CUDA graph of n_steps decode steps, layer i % len(layers) at step i.
     ev_pairs: list of (start, end) raw cudaEvent_t recorded (external) around each scan.
-    e2e: per-layer pinned host buffers; copies in/out are captured around each step."""
+    e2e: per-layer pinned host buffers: each step's inputs are copied in from them by a kernel
+    and its output is written into them by the attention kernel."""
     import torch
     from cuda.bindings import runtime as rt
 
@@ -261,15 +264,14 @@ def capture(layers, n_steps, ev_pairs=None, e2e=None):
                 L = layers[i % len(layers)]
                 st = L["step"]
                 if e2e is not None:
-                    st.arena.copy_(e2e[i % len(layers)]["arena"], non_blocking=True)
+                    st.stage(e2e[i % len(layers)]["arena"])      # pinned host -> device, by a kernel
                 pre = post = None
                 if ev_pairs is not None:
                     a, b = ev_pairs[i]
                     pre = lambda a=a: record_external(a, raw)
                     post = lambda b=b: record_external(b, raw)
-                st.run(pre_scan=pre, post_scan=post)
-                if e2e is not None:
-                    e2e[i % len(layers)]["out"].copy_(st.out, non_blocking=True)
+                # e2e: the attention writes the output straight into pinned host memory
+                st.run(pre_scan=pre, post_scan=post, out=None if e2e is None else e2e[i % len(layers)]["out"])
     torch.cuda.current_stream().wait_stream(s)
     return g
 
@@ -469,7 +471,8 @@ def run_prefill(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     dsa.lib()
-    d = W.prefill_chunk(PREFILL_CTX, PREFILL_NEW, seed=1238, device=dev, permute=True)
+    region_local = args.workload == "prefill_2k_256k_local"
+    d = W.prefill_chunk(PREFILL_CTX, PREFILL_NEW, seed=1238, device=dev, permute=True, region_shared_q=region_local)
     n_slots = d["n_slots"]
     S = torch.zeros((4, n_slots, 256), dtype=torch.uint8, device=dev)
     C = torch.zeros((4, n_slots), dtype=torch.float32, device=dev)
@@ -543,7 +546,9 @@ def run_prefill(args):
         "warmup": max(args.warmup, 3), "ms_per_step": ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 indexer, bf16 attention (fp32 accumulate)",
         "data": "synthetic",
-        "config": {"workload": "prefill_2k_256k", "context": PREFILL_CTX, "new_tokens": PREFILL_NEW, "topk": TOPK,
+        "config": {"workload": args.workload, "context": PREFILL_CTX, "new_tokens": PREFILL_NEW, "topk": TOPK,
+                   "queries": "the 8 queries of a region share index_q and gates" if region_local
+                   else "independent N(0,1)",
                    "l2": "flushed (256 MiB write) before every step, outside the timed stages"},
         "stages_ms": {"compress": stage[0] / args.steps, "indexer_gemm": stage[1] / args.steps,
                       "topk": stage[2] / args.steps, "attention": stage[3] / args.steps},
@@ -577,7 +582,7 @@ def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
-    elif args.workload == "prefill_2k_256k":
+    elif args.workload.startswith("prefill_2k_256k"):
         run_prefill(args)
     else:
         run_ours(args)

@@ -171,6 +171,14 @@ dsa_status_t dsa_topk_regions_noalloc(const float *scores, int64_t ld_scores, co
                                       dsa_stream_t stream);
 
 /* ------------------------------------------------------------------------------ */
+/* Byte copy by a kernel, for staging a step's inputs: dst and src are any addresses the
+ * current device can reach (device memory, or pinned host memory, which unified addressing
+ * maps at the same address).  Launched like every call of this library, it joins the
+ * stream's kernel chain without a copy-engine operation in between.  Regions must not
+ * overlap.  bytes == 0 is a no-op. */
+dsa_status_t dsa_copy(void *dst, const void *src, size_t bytes, dsa_stream_t stream);
+
+/* ------------------------------------------------------------------------------ */
 /* A4 sparse GQA attention.  [P1 §DSA ④] exact attention over only the selected regions'
  * real K/V; [P3 §一] the selected regions are gathered from the paged cache through the
  * block_table.  For query q (request b = q_req[q], position p = q_pos[q]) and head h
@@ -188,9 +196,15 @@ dsa_status_t dsa_topk_regions_noalloc(const float *scores, int64_t ld_scores, co
  * A selected region beyond the block table, a page index outside [0, n_pages) or a
  * q_req outside [0, n_req) is skipped and flags DSA_ERR_DEVICE.  An empty T gives
  * out = 0.  decode: one query per request, q_req = identity (nq = n_req = batch).
- * The workspace is needed only when few (query, group) rows must be split across CTAs;
- * dsa_attn_workspace_size() returns 0 otherwise (it depends on the current device's
- * SM count). */
+ * Kernels: rows of one or two decode requests run as one 16-CTA cluster per row with the
+ * splits merged in the kernel; prefill calls of >= 32 queries first try the shared-selection
+ * kernel (8 neighbouring queries of a request stream the union of their selections once,
+ * kept when the union is at most twice the longest selection, [P5]); every other row runs
+ * the per-row kernel (split across CTAs, with a merge kernel, when there are few rows).
+ * The results do not depend on the kernel.  Workspace: dsa_attn_workspace_size(nq, k)
+ * bytes (split partials and one flag per row; it depends on the current device's SM
+ * count), 256-byte aligned, owned by the caller; a smaller one returns DSA_ERR_WORKSPACE
+ * when a kernel needs it. */
 size_t dsa_attn_workspace_size(int nq, int k);
 dsa_status_t dsa_sparse_attn_decode(const void *q, const void *k_cache, const void *v_cache,
                                     int64_t n_pages, const int32_t *block_table, int max_pages,

@@ -28,6 +28,7 @@ constexpr int kWarpRing = kSlots * kPairBytes;          // 24 KiB
 constexpr int kQBytes = 16 * kD * 2;                    // 6 KiB
 constexpr size_t kSmemBytes = 1024 + (size_t)kWarps * kWarpRing + kQBytes + 64;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kSlack = 8.0f;                          // lazy-rescale slack of the running max (log2 units)
 
 struct Params {
     const __nv_bfloat16 *q;
@@ -40,6 +41,7 @@ struct Params {
     float *lse;                // may be null
     float *part_o;             // [rows][n_splits][16][192]   (split mode)
     float *part_ml;            // [rows][n_splits][16][2]
+    uint8_t *row_shared;       // nullable [nq][4]: 1 = the row was served by the shared-selection kernel
     int64_t n_pages;
     int max_pages;
     int n_req;
@@ -72,6 +74,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int split = blockIdx.x;
     const int row = blockIdx.y;            // query * 4 + group
+    if (p.row_shared && p.row_shared[row]) return;
     const int qi = row >> 2, g = row & 3;
     const int b = p.q_req ? p.q_req[qi] : qi;
     const int pos = p.q_pos[qi];
@@ -247,15 +250,19 @@ __global__ void __launch_bounds__(kThreads, 2)
                 s[nt][e] = v;
                 mx[e >> 1] = fmaxf(mx[e >> 1], v);
             }
+        // lazy rescaling: the reference max mrow moves only when a block's max exceeds it by
+        // more than kSlack (log2 units; P stays below 2^kSlack): the same softmax, rarely rescaled
         float alpha[2], mref[2];
+        bool grow_any = false;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
             mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
-            const float mnew = fmaxf(mrow[h], mx[h]);
-            mref[h] = (mnew == -INFINITY) ? 0.0f : mnew;
-            alpha[h] = exp2f(mrow[h] - mref[h]);
-            mrow[h] = mnew;
+            const bool grow = mx[h] > mrow[h] + kSlack;
+            alpha[h] = grow ? exp2f(mrow[h] - mx[h]) : 1.0f;
+            if (grow) mrow[h] = mx[h];
+            grow_any |= grow;
+            mref[h] = (mrow[h] == -INFINITY) ? 0.0f : mrow[h];
         }
         float ps[2] = {0.0f, 0.0f};
 #pragma unroll
@@ -272,12 +279,14 @@ __global__ void __launch_bounds__(kThreads, 2)
             ps[h] += __shfl_xor_sync(0xffffffffu, ps[h], 2);
             lrow[h] = lrow[h] * alpha[h] + ps[h];
         }
+        if (__any_sync(0xffffffffu, grow_any)) {
 #pragma unroll
-        for (int nd = 0; nd < 24; ++nd) {
-            o[nd][0] *= alpha[0];
-            o[nd][1] *= alpha[0];
-            o[nd][2] *= alpha[1];
-            o[nd][3] *= alpha[1];
+            for (int nd = 0; nd < 24; ++nd) {
+                o[nd][0] *= alpha[0];
+                o[nd][1] *= alpha[0];
+                o[nd][2] *= alpha[1];
+                o[nd][3] *= alpha[1];
+            }
         }
         // P (16 x 16 tokens) as the A operand, straight from the S accumulators
         const uint32_t pa0 = pack_bf16x2(s[0][0], s[0][1]);
@@ -406,6 +415,7 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const Params p
     __shared__ float red[2];
     __shared__ float osum[4][kD];
     const int row = blockIdx.x >> 4, hr = blockIdx.x & 15;
+    if (p.row_shared && p.row_shared[row]) return;
     const int qi = row >> 2, g = row & 3;
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int d = tid % kD, sg = tid / kD;

@@ -179,15 +179,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 s[nt][e] = v;
                 mx[e >> 1] = fmaxf(mx[e >> 1], v);
             }
+        // lazy rescaling: the reference max mrow moves only when a block's max exceeds it by
+        // more than kSlack (log2 units; P stays below 2^kSlack): the same softmax, rarely rescaled
         float alpha[2], mref[2];
+        bool grow_any = false;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
             mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
-            const float mnew = fmaxf(mrow[h], mx[h]);
-            mref[h] = (mnew == -INFINITY) ? 0.0f : mnew;
-            alpha[h] = exp2f(mrow[h] - mref[h]);
-            mrow[h] = mnew;
+            const bool grow = mx[h] > mrow[h] + attn::kSlack;
+            alpha[h] = grow ? exp2f(mrow[h] - mx[h]) : 1.0f;
+            if (grow) mrow[h] = mx[h];
+            grow_any |= grow;
+            mref[h] = (mrow[h] == -INFINITY) ? 0.0f : mrow[h];
         }
         float ps[2] = {0.0f, 0.0f};
 #pragma unroll
@@ -204,12 +208,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             ps[h] += __shfl_xor_sync(0xffffffffu, ps[h], 2);
             lrow[h] = lrow[h] * alpha[h] + ps[h];
         }
+        if (__any_sync(0xffffffffu, grow_any)) {
 #pragma unroll
-        for (int nd = 0; nd < 24; ++nd) {
-            o[nd][0] *= alpha[0];
-            o[nd][1] *= alpha[0];
-            o[nd][2] *= alpha[1];
-            o[nd][3] *= alpha[1];
+            for (int nd = 0; nd < 24; ++nd) {
+                o[nd][0] *= alpha[0];
+                o[nd][1] *= alpha[0];
+                o[nd][2] *= alpha[1];
+                o[nd][3] *= alpha[1];
+            }
         }
         const uint32_t pa0 = pack_bf16x2(s[0][0], s[0][1]);
         const uint32_t pa1 = pack_bf16x2(s[0][2], s[0][3]);

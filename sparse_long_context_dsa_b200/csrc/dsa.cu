@@ -10,8 +10,10 @@
 #include "../../include/dsa.h"
 #include "attention.cuh"
 #include "attention_cluster.cuh"
+#include "attention_shared.cuh"
 #include "common.cuh"
 #include "compress.cuh"
+#include "copy.cuh"
 #include "gemm_indexer.cuh"
 #include "indexer.cuh"
 #include "topk.cuh"
@@ -44,6 +46,7 @@ dsa_status_t cuda_fail(cudaError_t e, const char *what)
     } while (0)
 
 constexpr int kGemmMinQueries = 64;   // FP8 prefill chunks at least this long use the GEMM
+constexpr int kSharedMinQueries = 32; // prefill attention calls at least this long share selections
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -248,11 +251,15 @@ dsa_status_t attn_common(const void *q, const void *k_cache, const void *v_cache
     dsa_status_t st = device_info(sms);
     if (st != DSA_OK) return st;
     const bool clustered = k <= dsa::attnc::kMaxK && (int64_t)nq * dsa::kG <= cluster_attn_capacity();
+    // prefill chunks: 8 neighbouring queries per CTA share one stream of their selections' union
+    const bool shared = !clustered && q_req != nullptr && nq >= kSharedMinQueries && k <= dsa::attns::kMaxK &&
+                        (int64_t)max_pages * dsa::kPage / dsa::kRegion <= (int64_t)dsa::attns::kMaxWords * 32;
     const AttnPlan plan = attn_plan(nq, k, sms);
-    if (plan.ws > 0 && !clustered) {
-        if (!ws || ws_bytes < plan.ws || !aligned(ws, 256))
+    const size_t need_ws = plan.ws + (shared ? round_up((size_t)nq * dsa::kG, 256) : 0);
+    if (need_ws > 0 && !clustered) {
+        if (!ws || ws_bytes < need_ws || !aligned(ws, 256))
             return fail(DSA_ERR_WORKSPACE, "attention workspace too small or not 256-byte aligned (need " +
-                                               std::to_string(plan.ws) + " bytes)");
+                                               std::to_string(need_ws) + " bytes)");
     }
     CUtensorMap mk, mv;
     if ((st = kv_map(&mk, k_cache, n_pages)) != DSA_OK) return st;
@@ -281,6 +288,21 @@ dsa_status_t attn_common(const void *q, const void *k_cache, const void *v_cache
     p.scale_log2 = dsa::attn::kLog2e / sqrtf((float)dsa::kD);
 
     if (clustered) return attn_cluster_launch(mk, mv, p, nq, stream);
+    if (shared) {
+        p.row_shared = static_cast<uint8_t *>(ws) + plan.ws;
+        static std::once_flag sh_once;
+        static cudaError_t sh_err = cudaSuccess;
+        std::call_once(sh_once, [] {
+            sh_err = cudaFuncSetAttribute(dsa::attns::sparse_attn_shared_kernel,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsa::attns::kSmemBytes);
+        });
+        DSA_CUDA(sh_err, "cudaFuncSetAttribute(sparse_attn_shared_kernel)");
+        const unsigned blocks = (unsigned)((nq + dsa::attns::kQueries - 1) / dsa::attns::kQueries) * dsa::kG;
+        if ((st = launch_k("sparse_attn_shared_kernel", dsa::attns::sparse_attn_shared_kernel, dim3(blocks),
+                           dim3(dsa::attns::kThreads), dsa::attns::kSmemBytes, stream, 0, mk, mv, p)) != DSA_OK)
+            return st;
+        // then the rows it left to the per-row kernel (the others return at once)
+    }
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
@@ -629,12 +651,26 @@ dsa_status_t dsa_topk_regions_noalloc(const float *scores, int64_t ld_scores, co
     return topk_workspace_path(scores, ld_scores, q_pos, nq, k, sel_idx, sel_count, ws, need, stream);
 }
 
+dsa_status_t dsa_copy(void *dst, const void *src, size_t bytes, dsa_stream_t stream)
+{
+    if (bytes == 0) return DSA_OK;
+    DSA_REQUIRE(dst && src, "NULL pointer");
+    int sms = 0;
+    dsa_status_t st = device_info(sms);
+    if (st != DSA_OK) return st;
+    const size_t per_block = 256 * 16 * 4;                 // about 4 uint4 per thread
+    const unsigned blocks = (unsigned)std::min<size_t>((bytes + per_block - 1) / per_block, (size_t)sms * 4);
+    return launch_k("copy_kernel", dsa::copy_kernel, dim3(std::max(1u, blocks)), dim3(256), 0, stream, 0,
+                    static_cast<uint8_t *>(dst), static_cast<const uint8_t *>(src), bytes);
+}
+
 size_t dsa_attn_workspace_size(int nq, int k)
 {
     if (nq <= 0 || k < 1) return 0;
     int sms = 0;
     if (device_info(sms) != DSA_OK) sms = 148;
-    return attn_plan(nq, k, sms).ws;
+    // split partials, and the per-row flags of the shared-selection prefill kernel
+    return attn_plan(nq, k, sms).ws + round_up((size_t)nq * dsa::kG, 256);
 }
 
 dsa_status_t dsa_sparse_attn_decode(const void *q, const void *k_cache, const void *v_cache, int64_t n_pages,

@@ -49,6 +49,7 @@ _SIG = {
                                         _VP, ctypes.c_size_t, _VP]),
     "dsa_topk_regions_noalloc": (ctypes.c_int, [_F32P, ctypes.c_int64, _I32P, ctypes.c_int, ctypes.c_int, _I32P,
                                                 _I32P, _VP]),
+    "dsa_copy": (ctypes.c_int, [_VP, _VP, ctypes.c_size_t, _VP]),
     "dsa_attn_workspace_size": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int]),
     "dsa_sparse_attn_decode": (ctypes.c_int, [_VP, _VP, _VP, ctypes.c_int64, _I32P, ctypes.c_int, _I32P,
                                               ctypes.c_int, _I32P, _I32P, ctypes.c_int, _VP, _F32P, _VP,
@@ -190,6 +191,21 @@ def topk_regions_noalloc(scores, q_pos, k, sel_idx, sel_count):
     _need(sel_count, torch.int32, (nq, G), "sel_count")
     _check(lib().dsa_topk_regions_noalloc(_p(scores), ld, _p(q_pos), nq, k, _p(sel_idx), _p(sel_count), _stream()))
     return sel_idx, sel_count
+
+
+def copy(dst, src):
+    """dsa_copy: copies src into dst (same byte size) with a kernel on the current stream;
+    either may be a CUDA tensor or a pinned CPU tensor (reached by the GPU directly)."""
+    for t, n in ((dst, "dst"), (src, "src")):
+        if not (t.is_cuda or t.is_pinned()):
+            raise ValueError(f"{n} must be a CUDA tensor or pinned host memory")
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    nbytes = dst.numel() * dst.element_size()
+    if src.numel() * src.element_size() != nbytes:
+        raise ValueError("dst and src differ in size")
+    _check(lib().dsa_copy(_p(dst), _p(src), nbytes, _stream()))
+    return dst
 
 
 def _attn_args(q, k_cache, v_cache, block_table, q_pos, sel_idx, sel_count, out, lse):

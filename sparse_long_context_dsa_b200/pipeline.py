@@ -93,6 +93,11 @@ class DecodeStep:
         if tail is not None:
             self.tail.copy_(tail, non_blocking=True)
 
+    def stage(self, host_arena):
+        """Copies the step's inputs from a pinned host image of `arena` with one library
+        kernel (the GPU reads the pinned memory directly), in the stream's kernel chain."""
+        dsa.copy(self.arena, host_arena)
+
     def set_compress(self, requests, slots):
         """Regions to compress this step: tail block i (rows 8i..8i+7 of `tail`) of each
         listed request goes to pool slot slots[j]."""
@@ -102,10 +107,17 @@ class DecodeStep:
             self.dst_slot[:n].copy_(torch.tensor([int(s) for s in slots], dtype=torch.int64))
         self.n_compress = n
 
-    def run(self, pre_scan=None, post_scan=None):
+    def run(self, pre_scan=None, post_scan=None, out=None):
         """Launches the step on the current stream (capturable).  pre_scan/post_scan are
         optional callables invoked right before/after the indexer-scan launch (the
-        benchmark records timing events there)."""
+        benchmark records timing events there).  out: where the attention writes its
+        output, bf16 [B][64][192], on the device (default `self.out`) or in pinned host
+        memory, which the kernel then writes directly."""
+        if out is None:
+            out = self.out
+        elif tuple(out.shape) != tuple(self.out.shape) or out.dtype != self.out.dtype or not (
+                out.is_cuda or out.is_pinned()):
+            raise ValueError("out must be bf16 [B][64][192], on the device or in pinned host memory")
         L = dsa.lib()
         main = torch.cuda.current_stream()
         p = dsa._p
@@ -129,11 +141,11 @@ class DecodeStep:
                                       p(self.sel_count), p(self.ws_topk), self.ws_topk_n, st))
         dsa._check(L.dsa_sparse_attn_decode(p(self.q), p(self.k_cache), p(self.v_cache), self.k_cache.shape[0],
                                             p(self.block_table), self.block_table.shape[1], p(self.q_pos), self.B,
-                                            p(self.sel_idx), p(self.sel_count), self.k, p(self.out), p(self.lse),
+                                            p(self.sel_idx), p(self.sel_count), self.k, p(out), p(self.lse),
                                             p(self.ws_attn), self.ws_attn_n, st))
         if self.n_compress:
             main.wait_stream(self.side)
-        return self.out
+        return out
 
 
 def compress_all(index_k, lengths, tok_base, sum_base, summaries, scales):

@@ -108,16 +108,23 @@ def complete_regions(lengths, tok_base, sum_base):
     return src, dst
 
 
-def prefill_chunk(ctx_len: int, n_new: int, seed: int, device, permute: bool = True):
+def prefill_chunk(ctx_len: int, n_new: int, seed: int, device, permute: bool = True, region_shared_q: bool = False):
     """One request with ctx_len tokens already cached and n_new new tokens appended in
     one chunk (positions ctx_len .. ctx_len+n_new-1).  index_k/K/V cover all
-    ctx_len+n_new tokens; index_q/gate/Q exist for the n_new queries."""
+    ctx_len+n_new tokens; index_q/gate/Q exist for the n_new queries.
+    region_shared_q: the queries of one region share their indexer query and gates (the
+    locality variant: neighbouring tokens select the same regions)."""
     gen = generator(seed, device)
     total = ctx_len + n_new
     bt, kc, vc = paged_kv([total], gen, device, permute)
     index_k = normal_bf16((total, G, DI), gen, device)
     index_q = normal_bf16((n_new, HI, DI), gen, device)
     gate = uniform_f32((n_new, HI), gen, device)
+    if region_shared_q:
+        first = torch.arange(ctx_len, total, device=device) // REGION * REGION - ctx_len
+        first = first.clamp(min=0)
+        index_q = index_q[first].contiguous()
+        gate = gate[first].contiguous()
     q = normal_bf16((n_new, HQ, D), gen, device)
     q_pos = torch.arange(ctx_len, total, dtype=torch.int32, device=device)
     q_req = torch.zeros(n_new, dtype=torch.int32, device=device)

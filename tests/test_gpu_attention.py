@@ -103,3 +103,45 @@ def test_empty_selection_and_bad_region():
     dsa.sparse_attn_decode(d["q"], d["k_cache"], d["v_cache"], d["block_table"], d["q_pos"], si, sc)
     with pytest.raises(dsa.DsaError):
         dsa.check_device()
+
+
+def test_prefill_queries_of_several_requests_in_one_block():
+    # 40 queries cycling over 3 requests: every block of 8 serves its queries in one pass per
+    # request (the shared-selection kernel); random, unrelated selections (k = 64) mask most of
+    # each union away from each query
+    dev = "cuda"
+    d = W.decode_batch([5000, 3000 + 5, 7000], seed=36, device=dev, permute=True)
+    nq = 40
+    rng = np.random.default_rng(7)
+    lens = [5000, 3005, 7000]
+    q_req = np.arange(nq, dtype=np.int32) % 3
+    q_pos = np.array([rng.integers(8, lens[b]) for b in q_req], np.int32)
+    d["q_pos"] = torch.from_numpy(q_pos).to(dev)
+    d["q"] = W.normal_bf16((nq, 64, 192), W.generator(10, dev), dev)
+    idx, cnt = random_selection(q_pos, 64, seed=8)
+    run(d, idx, cnt, q_req=torch.from_numpy(q_req).to(dev), prefill=True)
+
+
+def test_prefill_shared_block_with_empty_and_overlapping_selections():
+    # 48 queries of one request: neighbours share most of their regions, some rows select
+    # nothing at all, one query's last block is partial
+    dev = "cuda"
+    ctx = 6000
+    d = W.prefill_chunk(ctx, 45, seed=37, device=dev, permute=True)
+    qp = d["q_pos"].cpu().numpy()
+    idx, cnt = random_selection(qp, 128, seed=9)
+    base = idx[0, :, :100].copy()                  # a common core for everyone
+    for i in range(1, len(qp)):
+        idx[i, :, :100] = base
+        idx[i] = np.sort(np.where(idx[i] < 0, 10 ** 9, idx[i]), axis=1)
+        idx[i] = np.where(idx[i] == 10 ** 9, -1, idx[i])
+        for g in range(G):
+            row = np.unique(idx[i, g][idx[i, g] >= 0])
+            idx[i, g] = -1
+            idx[i, g, : len(row)] = row
+            cnt[i, g] = len(row)
+    cnt[5, 2] = 0
+    idx[5, 2] = -1
+    cnt[17] = 0
+    idx[17] = -1
+    run(d, idx, cnt, q_req=d["q_req"], prefill=True)

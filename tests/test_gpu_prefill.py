@@ -115,3 +115,31 @@ def test_full_chunk_2048_queries_on_262144_tokens():
     check_rows(sel.cpu().numpy(), cnt.cpu().numpy(), d["q_pos"].cpu().numpy(), k)
     qi = np.array([0, 1, 7, 8, 511, 1024, 1535, 2040, 2047])
     check_sampled(d, So, Co, scores, sel, cnt, out, lse, qi, k, dsa.Q_FP8)
+
+
+def test_locality_variant_shares_selections():
+    # the 8 queries of a region share index_q: their selections coincide (up to the own region's
+    # causal eligibility), so the shared-selection attention streams one union per block
+    k = 512
+    dev = torch.device("cuda")
+    d = W.prefill_chunk(65536, 256, seed=1240, device=dev, permute=True, region_shared_q=True)
+    n_slots = d["n_slots"]
+    S = torch.zeros((G, n_slots, 256), dtype=torch.uint8, device=dev)
+    C = torch.zeros((G, n_slots), dtype=torch.float32, device=dev)
+    total = 65536 + 256
+    src, dst = W.complete_regions([total], [0], [0])
+    dsa.compress_regions(d["index_k"], torch.tensor(src, dtype=torch.int64, device=dev),
+                         torch.tensor(dst, dtype=torch.int64, device=dev), S, C)
+    ld = total // 8
+    scores = torch.zeros((256, G, ld), dtype=torch.float32, device=dev)
+    dsa.indexer_scores(d["index_q"], d["gate"], d["q_req"], d["q_pos"], S, C, d["sum_base"], scores, dsa.Q_FP8)
+    sel, cnt = dsa.topk_regions(scores, d["q_pos"], k)
+    lse = torch.empty((256, 64), dtype=torch.float32, device=dev)
+    out = dsa.sparse_attn_prefill(d["q"], d["k_cache"], d["v_cache"], d["block_table"], d["q_req"], d["q_pos"],
+                                  sel, cnt, lse=lse)
+    dsa.check_device()
+    s_np = sel.cpu().numpy()
+    assert np.array_equal(s_np[8], s_np[9])                    # same region, same selection
+    So, Co = check_compression(d, S, C)
+    qi = np.array([0, 8, 9, 15, 100, 255])
+    check_sampled(d, So, Co, scores, sel, cnt, out, lse, qi, k, dsa.Q_FP8)
