@@ -18,6 +18,7 @@
 #include "indexer.cuh"
 #include "topk.cuh"
 #include "topk_cluster.cuh"
+#include "topk_rows.cuh"
 
 namespace {
 
@@ -462,6 +463,22 @@ dsa_status_t topk_cluster_path(const float *scores, int64_t ld_scores, const int
                     dsa::topkc::kSmemBytes, stream, (unsigned)cl, scores, ld_scores, q_pos, k, sel_idx, sel_count);
 }
 
+// Many rows of at most 65,536 scores: one CTA per row, no scratch.
+dsa_status_t topk_rows_path(const float *scores, int64_t ld_scores, const int32_t *q_pos, int nq, int k,
+                            int32_t *sel_idx, int32_t *sel_count, dsa_stream_t stream)
+{
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(dsa::topkr::topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)dsa::topkr::kSmemBytes);
+    });
+    DSA_CUDA(attr_err, "cudaFuncSetAttribute(topk_rows_kernel)");
+    return launch_k("topk_rows_kernel", dsa::topkr::topk_rows_kernel, dim3((unsigned)(nq * dsa::kG)),
+                    dim3(dsa::topkr::kThreads), dsa::topkr::kSmemBytes, stream, 0, scores, ld_scores, q_pos, k,
+                    sel_idx, sel_count);
+}
+
 // Scratch of dsa_topk_regions_noalloc: one static array per GPU that loads the library.
 static __device__ __align__(256) uint8_t g_topk_static_scratch[DSA_TOPK_STATIC_SCRATCH_BYTES];
 
@@ -627,6 +644,8 @@ dsa_status_t dsa_topk_regions(const float *scores, int64_t ld_scores, const int3
     const int cl = cluster_size_for(ld_scores);
     if (cl > 0 && (int64_t)rows * cl <= 2 * sms) return topk_cluster_path(scores, ld_scores, q_pos, nq, k, sel_idx,
                                                                            sel_count, cl, stream);
+    if (ld_scores <= dsa::topkr::kMaxLd) return topk_rows_path(scores, ld_scores, q_pos, nq, k, sel_idx, sel_count,
+                                                                stream);
     return topk_workspace_path(scores, ld_scores, q_pos, nq, k, sel_idx, sel_count, ws, ws_bytes, stream);
 }
 

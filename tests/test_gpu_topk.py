@@ -73,12 +73,38 @@ def test_one_million_token_row():
     check(s.astype(np.float32), [8 * 131072 - 1], 512)
 
 
-def test_many_rows_take_the_workspace_path():
-    # more (query, group) rows than the cluster path takes: histogram + select kernels
+def test_many_rows_take_the_per_row_path():
+    # more (query, group) rows than the cluster path takes, rows of at most 65,536 scores:
+    # one CTA per row (group-maxima bound, candidates in smem)
     rng = np.random.default_rng(6)
     nq, ld = 100, 3000
     s = rng.standard_normal((nq, G, ld)).astype(np.float32)
     s[::7] = np.round(s[::7])                     # some tie-heavy rows
+    q_pos = [int(x) for x in rng.integers(0, 8 * ld + 1, nq)]
+    check(s, q_pos, 512)
+
+
+@pytest.mark.parametrize("k", [2, 64, 512, 1024])
+def test_per_row_path_prefill_like_rows(k):
+    # prefill-shaped: 160 rows of 33,024 scores, indexer-like non-negative scores, rows with
+    # all scores equal (the whole-row fallback), rows ending in every region of a chunk
+    rng = np.random.default_rng(k)
+    nq, ld = 40, 33024
+    z = rng.standard_normal((nq, G, 4, ld)).astype(np.float32)
+    s = (np.maximum(z, 0) * rng.uniform(0, 1, (nq, G, 4, 1)).astype(np.float32)).sum(2) / 16
+    s = s.astype(np.float32)
+    s[3] = 0.0
+    s[4] = 0.5
+    q_pos = [8 * ld - 1 - 3 * i for i in range(nq)]
+    check(s, q_pos, k)
+
+
+def test_many_long_rows_take_the_workspace_path():
+    # many rows longer than 65,536 scores: histogram + select kernels with a workspace
+    rng = np.random.default_rng(16)
+    nq, ld = 20, 70000
+    s = rng.standard_normal((nq, G, ld)).astype(np.float32)
+    s[::5] = np.round(s[::5])
     q_pos = [int(x) for x in rng.integers(0, 8 * ld + 1, nq)]
     check(s, q_pos, 512)
 
