@@ -171,6 +171,25 @@ dsa_status_t dsa_topk_regions_noalloc(const float *scores, int64_t ld_scores, co
                                       dsa_stream_t stream);
 
 /* ------------------------------------------------------------------------------ */
+/* A2 + A3 in one call, for decode: the streaming scan of dsa_indexer_scores followed by the
+ * selection of dsa_topk_regions, with the same arguments and exactly their outputs (the
+ * scores in `scores`, the selection in sel_idx/sel_count).  The scan also writes, into the
+ * workspace, the largest score of every chunk of 32 regions, and for few long rows (k <= 512,
+ * rows of up to 131,072 regions, one cluster per row) the selection bounds its threshold
+ * from those maxima and reads only the chunks that can hold a selected region; other calls
+ * select as dsa_topk_regions does.  Compression of filled regions ([P2 §区域压缩CSA]) is not
+ * part of it.  ws: dsa_decode_select_workspace_size(nq, ld_scores, k) bytes, 256-byte
+ * aligned, owned by the caller, free again once the stream has passed the call; a smaller or
+ * unaligned one returns DSA_ERR_WORKSPACE.  Invalid queries flag DSA_ERR_DEVICE as in the
+ * two calls. */
+size_t dsa_decode_select_workspace_size(int nq, int64_t ld_scores, int k);
+dsa_status_t dsa_decode_select(const void *index_q, const float *gate, const int32_t *q_req, const int32_t *q_pos,
+                               int nq, const uint8_t *summaries, const float *scales, int64_t n_slots,
+                               const int64_t *sum_base, int n_req, float *scores, int64_t ld_scores, uint32_t flags,
+                               int k, int32_t *sel_idx, int32_t *sel_count, void *ws, size_t ws_bytes,
+                               dsa_stream_t stream);
+
+/* ------------------------------------------------------------------------------ */
 /* Byte copy by a kernel, for staging a step's inputs: dst and src are any addresses the
  * current device can reach (device memory, or pinned host memory, which unified addressing
  * maps at the same address).  Launched like every call of this library, it joins the

@@ -458,9 +458,11 @@ dsa_status_t topk_cluster_path(const float *scores, int64_t ld_scores, const int
     const dim3 grid((unsigned)cl, (unsigned)(nq * dsa::kG), 1);
     if (cl == 1)
         return launch_k("topk_cluster_kernel", dsa::topkc::topk_cluster_kernel<true>, grid, dim3(dsa::topkc::kThreads),
-                        dsa::topkc::kSmemBytes, stream, 1u, scores, ld_scores, q_pos, k, sel_idx, sel_count);
+                        dsa::topkc::kSmemBytes, stream, 1u, scores, ld_scores, q_pos, k, sel_idx, sel_count,
+                        static_cast<const float *>(nullptr), (int64_t)0);
     return launch_k("topk_cluster_kernel", dsa::topkc::topk_cluster_kernel<false>, grid, dim3(dsa::topkc::kThreads),
-                    dsa::topkc::kSmemBytes, stream, (unsigned)cl, scores, ld_scores, q_pos, k, sel_idx, sel_count);
+                    dsa::topkc::kSmemBytes, stream, (unsigned)cl, scores, ld_scores, q_pos, k, sel_idx, sel_count,
+                    static_cast<const float *>(nullptr), (int64_t)0);
 }
 
 // Many rows of at most 65,536 scores: one CTA per row, no scratch.
@@ -549,10 +551,12 @@ dsa_status_t dsa_compress_regions(const void *index_k, int64_t row_stride, int64
                     summaries, scales, n_slots);
 }
 
-// The streaming scan of dsa_indexer_scores.
+// The streaming scan of dsa_indexer_scores; chunk_max (nullable) receives the largest score of
+// every 32-region chunk, [nq][4][cm_stride].
 dsa_status_t scan_path(const void *index_q, const float *gate, const int32_t *q_req, const int32_t *q_pos, int nq,
                        const uint8_t *summaries, const float *scales, int64_t n_slots, const int64_t *sum_base,
-                       int n_req, float *scores, int64_t ld_scores, uint32_t flags, int sms, dsa_stream_t stream)
+                       int n_req, float *scores, int64_t ld_scores, uint32_t flags, int sms, dsa_stream_t stream,
+                       float *chunk_max = nullptr, int64_t cm_stride = 0)
 {
     dsa_status_t st;
     CUtensorMap map;
@@ -572,6 +576,8 @@ dsa_status_t scan_path(const void *index_q, const float *gate, const int32_t *q_
     p.scales = scales;
     p.sum_base = sum_base;
     p.scores = scores;
+    p.chunk_max = chunk_max;
+    p.cm_stride = cm_stride;
     p.n_slots = n_slots;
     p.ld = ld_scores;
     p.units_per_query = (int)((ld_scores + dsa::idx::kChunk - 1) / dsa::idx::kChunk);
@@ -668,6 +674,65 @@ dsa_status_t dsa_topk_regions_noalloc(const float *scores, int64_t ld_scores, co
     dsa_status_t st = static_scratch(dev, &ws);
     if (st != DSA_OK) return st;
     return topk_workspace_path(scores, ld_scores, q_pos, nq, k, sel_idx, sel_count, ws, need, stream);
+}
+
+// ---- decode selection in one call: the scan writes chunk maxima, the cluster top-k reads them
+namespace {
+int64_t cm_stride_of(int64_t ld) { return ((ld + 31) / 32 + 7) / 8 * 8; }
+}  // namespace
+
+size_t dsa_decode_select_workspace_size(int nq, int64_t ld_scores, int k)
+{
+    if (nq <= 0 || ld_scores < 1) return 0;
+    const size_t cm = round_up((size_t)nq * dsa::kG * (size_t)cm_stride_of(ld_scores) * 4, 256);
+    return cm + dsa_topk_workspace_size(nq, ld_scores, k);
+}
+
+dsa_status_t dsa_decode_select(const void *index_q, const float *gate, const int32_t *q_req, const int32_t *q_pos,
+                               int nq, const uint8_t *summaries, const float *scales, int64_t n_slots,
+                               const int64_t *sum_base, int n_req, float *scores, int64_t ld_scores, uint32_t flags,
+                               int k, int32_t *sel_idx, int32_t *sel_count, void *ws, size_t ws_bytes,
+                               dsa_stream_t stream)
+{
+    DSA_REQUIRE(nq >= 0, "nq must be >= 0");
+    DSA_REQUIRE((flags & ~DSA_Q_FP8) == 0, "unknown flag");
+    DSA_REQUIRE(ld_scores >= 1 && ld_scores <= (1ll << 26), "ld_scores out of [1, 2^26]");
+    DSA_REQUIRE(n_slots >= 1 && n_slots <= (1ll << 28), "n_slots out of [1, 2^28]");
+    DSA_REQUIRE(n_req >= 1, "n_req must be >= 1");
+    DSA_REQUIRE(k >= 1 && k <= DSA_MAX_TOPK, "k out of [1, DSA_MAX_TOPK]");
+    if (nq == 0) return DSA_OK;
+    DSA_REQUIRE(index_q && gate && q_req && q_pos && summaries && scales && sum_base && scores && sel_idx && sel_count,
+                "NULL pointer");
+    DSA_REQUIRE(aligned(index_q, 16) && aligned(summaries, 16), "index_q and summaries must be 16-byte aligned");
+    const size_t need_ws = dsa_decode_select_workspace_size(nq, ld_scores, k);
+    if (!ws || ws_bytes < need_ws || !aligned(ws, 256))
+        return fail(DSA_ERR_WORKSPACE, "decode-select workspace too small or not 256-byte aligned (need " +
+                                           std::to_string(need_ws) + " bytes)");
+    int sms = 0;
+    dsa_status_t st = device_info(sms);
+    if (st != DSA_OK) return st;
+    const int64_t cm_stride = cm_stride_of(ld_scores);
+    float *chunk_max = static_cast<float *>(ws);
+    const size_t cm = round_up((size_t)nq * dsa::kG * (size_t)cm_stride * 4, 256);
+    const int cl = cluster_size_for(ld_scores);
+    const bool maxima = k <= 512 && cl > 1 && (int64_t)nq * dsa::kG * cl <= 2 * sms;
+    if ((st = scan_path(index_q, gate, q_req, q_pos, nq, summaries, scales, n_slots, sum_base, n_req, scores,
+                        ld_scores, flags, sms, stream, maxima ? chunk_max : nullptr, cm_stride)) != DSA_OK)
+        return st;
+    if (!maxima)
+        return dsa_topk_regions(scores, ld_scores, q_pos, nq, k, sel_idx, sel_count, static_cast<uint8_t *>(ws) + cm,
+                                ws_bytes - cm, stream);
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(dsa::topkc::topk_cluster_kernel<false, true>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsa::topkc::kSmemBytes);
+    });
+    DSA_CUDA(attr_err, "cudaFuncSetAttribute(topk_cluster_kernel)");
+    return launch_k("topk_cluster_kernel", dsa::topkc::topk_cluster_kernel<false, true>,
+                    dim3((unsigned)cl, (unsigned)(nq * dsa::kG), 1), dim3(dsa::topkc::kThreads),
+                    dsa::topkc::kSmemBytes, stream, (unsigned)cl, scores, ld_scores, q_pos, k, sel_idx, sel_count,
+                    static_cast<const float *>(chunk_max), cm_stride);
 }
 
 dsa_status_t dsa_copy(void *dst, const void *src, size_t bytes, dsa_stream_t stream)

@@ -61,6 +61,8 @@ struct Params {
     const float *scales;
     const int64_t *sum_base;
     float *scores;
+    float *chunk_max;          // nullable: [nq][4][cm_stride], largest stored score of regions 32c .. 32c+31
+    int64_t cm_stride;
     int64_t n_slots;
     int64_t ld;
     int64_t total_units;
@@ -268,6 +270,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         ++it;
 
         float *out = p.scores + ((int64_t)qi * kG + g) * p.ld;
+        float cmax = -1.0f;                                   // below every score (scores are >= +0)
 #pragma unroll
         for (int m = 0; m < kTiles; ++m) {
             float v0 = z_t * fmaxf((acc[m][0] + acc[m][1]) * sq_t * sc[m][0], 0.0f);
@@ -278,8 +281,18 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             v1 += __shfl_xor_sync(0xffffffffu, v1, 2);
             if (t < 2) {
                 const int64_t r = r0 + 16 * m + 8 * t + n;
-                if (r < own) out[r] = (t == 0 ? v0 : v1) * 0.0625f;
+                const float v = (t == 0 ? v0 : v1) * 0.0625f;
+                if (r < own) {
+                    out[r] = v;
+                    cmax = fmaxf(cmax, v);
+                }
             }
+        }
+        if (p.chunk_max) {                                    // the chunk's largest stored score
+            static_assert(kChunk == 32, "chunk maxima cover 32 regions");
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
+            if (lane == 0) p.chunk_max[((int64_t)qi * kG + g) * p.cm_stride + r0 / kChunk] = cmax;
         }
     }
 }

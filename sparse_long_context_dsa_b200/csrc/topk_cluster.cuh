@@ -340,11 +340,75 @@ __device__ __forceinline__ bool threshold_selects(uint64_t c, uint64_t elo, uint
     return kk >= ehi || (kk >= elo && (c & cm) >= cp);
 }
 
+// Histogram levels over the block's keys (thread item u valid when valid(u)): the range
+// [elo, ehi) holding the m-th largest key, `above` keys >= ehi, n_in keys in the range;
+// stops once n_in <= cap or the range is one value.  Needs m <= the valid count.
+template <int R, typename Valid, typename Key>
+__device__ void key_levels(Valid valid, Key key, uint32_t m, uint32_t cap, uint32_t *hs, uint32_t *sh_min,
+                           uint32_t *sh_max, uint32_t *res, uint64_t &elo, uint64_t &ehi, uint32_t &above,
+                           uint32_t &n_in)
+{
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint32_t kmn = 0xFFFFFFFFu, kmx = 0u;
+#pragma unroll
+    for (int u = 0; u < R; ++u)
+        if (valid(u)) {
+            kmn = min(kmn, key(u));
+            kmx = max(kmx, key(u));
+        }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        kmn = min(kmn, __shfl_xor_sync(0xffffffffu, kmn, o));
+        kmx = max(kmx, __shfl_xor_sync(0xffffffffu, kmx, o));
+    }
+    if (lane == 0) {
+        atomicMin(sh_min, kmn);
+        atomicMax(sh_max, kmx);
+    }
+    if (tid < 256) hs[tid] = 0u;
+    __syncthreads();
+    kmn = *sh_min;
+    kmx = *sh_max;
+    uint64_t rlo = kmn, width = ~0ull;
+    int bsh = max(0, 24 - __clz((int)(kmx - kmn)));
+    uint32_t m_rem = m, bin = 0;
+    above = 0;
+    for (int level = 0; level < 4; ++level) {
+#pragma unroll
+        for (int u = 0; u < R; ++u) {
+            if (!valid(u)) continue;
+            const uint64_t kk = key(u);
+            if (kk >= rlo && kk - rlo < width) atomicAdd(&hs[(uint32_t)((kk - rlo) >> bsh)], 1u);
+        }
+        __syncthreads();
+        if (warp == 0) desc_bin_search(hs, m_rem, res);
+        __syncthreads();
+        bin = res[0];
+        above += res[1];
+        m_rem -= res[1];
+        n_in = res[2];
+        if (tid < 256) hs[tid] = 0u;
+        if (n_in <= cap || bsh == 0) break;
+        rlo += (uint64_t)bin << bsh;
+        width = 1ull << bsh;
+        bsh = max(0, bsh - 8);
+        __syncthreads();
+    }
+    elo = rlo + ((uint64_t)bin << bsh);
+    ehi = elo + (1ull << bsh);
+    __syncthreads();
+}
+
 // kSingle: one CTA per row (launched without a cluster; CL = 1), else a cluster of CL CTAs.
-template <bool kSingle>
+// kMaxima: the indexer scan that wrote the scores also wrote chunk_max[row][c], the largest
+// score of regions 32c .. 32c+31 (row stride cm_stride, a multiple of 4): the cluster then
+// bounds the threshold from those maxima and reads only the chunks that can hold a selected
+// region (the other paths when the maxima tie in bulk).
+template <bool kSingle, bool kMaxima = false>
 __global__ void __launch_bounds__(kThreads, 1)
     topk_cluster_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ q_pos, int k,
-                        int32_t *__restrict__ sel_idx, int32_t *__restrict__ sel_count)
+                        int32_t *__restrict__ sel_idx, int32_t *__restrict__ sel_count,
+                        const float *__restrict__ chunk_max, int64_t cm_stride)
 {
     pdl_trigger();   // the next kernel may launch; it waits for this one itself
     pdl_wait();      // the previous kernel's results are visible from here on
@@ -368,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- loads: this thread's group is the CTA's entries tid, tid+512, ... (coalesced)
     const int p = q_pos[row >> 2];
-    const int64_t part = (ld + CL - 1) / CL;
+    const int64_t part = ((ld + CL - 1) / CL + 31) / 32 * 32;              // whole 32-region chunks
     const int64_t lo = min(ld, (int64_t)rank * part), hi_ld = min(ld, lo + part);
     const float *src = scores + (int64_t)row * ld + lo;
     if (part > kPartMax) {             // the host sizes the cluster so that a part fits
@@ -379,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         return;
     }
     uint32_t *keys = reinterpret_cast<uint32_t *>(smem_raw + kOffKeys);      // [kPadded] staged keys
-    {
+    auto stage_keys = [&]() {
         const int n_ld = (int)(hi_ld - lo);
         float v[kPer];
 #pragma unroll
@@ -392,7 +456,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int i = u * kThreads + tid;
             if (i < n_ld) keys[padded(i)] = score_key(v[u]);
         }
-    }
+    };
+    if constexpr (!kMaxima) stage_keys();
     const bool valid = p >= 0 && (int64_t)(p / kRegion) <= ld;
     const int64_t own = valid ? p / kRegion : 0;
     const int64_t need = valid ? min((int64_t)(k - 1), own) : 0;
@@ -421,7 +486,186 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t *hw = reinterpret_cast<uint32_t *>(smem_raw + kOffHw);
     uint32_t *hs = reinterpret_cast<uint32_t *>(smem_raw + kOffHs);
     int32_t *out = sel_idx + (int64_t)row * k;
-    if constexpr (kSingle) {
+    // after the candidate barrier: the fast-path decision (the same in every CTA from the pushed
+    // counts) and, at rank 0, the exact selection among the gathered candidates, emitted in order
+    uint64_t *slots = reinterpret_cast<uint64_t *>(smem_raw + kOffSlots);
+    auto finish_fast = [&](uint32_t Lk, int lg_slot, uint32_t slot_n) -> bool {
+        bool fast_ok = false;
+        uint32_t total = 0;
+        bool overflow = false;
+        for (int q = 0; q < CL; ++q) {
+            total += cand_cnt[q];
+            overflow |= cand_cnt[q] > slot_n;
+        }
+        fast_ok = !overflow && total >= (uint32_t)need && total <= (uint32_t)kDense;
+        if (fast_ok && rank == 0) {
+            // ---- dense gather in region order: thread t takes entries [t*kDPer, (t+1)*kDPer)
+            uint32_t *first = slice_tot;                                    // first dense entry of each rank
+            if (tid == 0) {
+                uint32_t run = 0;
+                for (int q = 0; q < CL; ++q) {
+                    first[q] = run;
+                    run += cand_cnt[q];
+                }
+            }
+            __syncthreads();
+            uint64_t cv[kDPer];
+            const uint32_t d0 = tid * kDPer;
+            int q = 0;
+            while (q + 1 < CL && d0 >= first[q + 1]) ++q;
+#pragma unroll
+            for (int u = 0; u < kDPer; ++u) {
+                const uint32_t d = d0 + u;
+                while (q + 1 < CL && d >= first[q + 1]) ++q;
+                cv[u] = d < total ? slots[((uint32_t)q << lg_slot) + (d - first[q])] : 0ull;
+            }
+            auto valid_u = [&](int u) { return d0 + (uint32_t)u < total; };
+            auto comp_u = [&](int u) { return cv[u]; };
+            uint64_t elo, ehi, cp, cm;
+            const bool ok = block_threshold<kDPer>(valid_u, comp_u, (uint32_t)need, Lk, hs, dense, hw, &sh_kmax,
+                                                   &sh_nin, scan_ws + 32, mm_ws, &elo, &ehi, &cp, &cm);
+            if (ok) {
+                // ---- ordered emit
+                uint32_t cs = 0;
+#pragma unroll
+                for (int u = 0; u < kDPer; ++u) cs += (valid_u(u) && threshold_selects(cv[u], elo, ehi, cp, cm)) ? 1u : 0u;
+                const uint32_t sincl = block_scan_incl<kThreads>(cs, scan_ws);
+                uint32_t opos = sincl - cs;
+#pragma unroll
+                for (int u = 0; u < kDPer; ++u) {
+                    if (valid_u(u) && threshold_selects(cv[u], elo, ehi, cp, cm)) {
+                        if (opos < (uint32_t)need) out[opos] = (int32_t)(0xFFFFFFFFu - (uint32_t)cv[u]);
+                        ++opos;
+                    }
+                }
+                if (tid == kThreads - 1) {
+                    if (sincl != (uint32_t)need) set_error(kErrTopkInternal);
+                    out[need] = (int32_t)own;                               // own > every eligible region
+                    sel_count[row] = (int32_t)(need + 1);
+                }
+                for (int i = (int)need + 1 + tid; i < k; i += kThreads) out[i] = -1;
+            } else {
+                // more than kDense candidates share one key: cannot happen with total <= kDense
+                if (tid == 0) {
+                    set_error(kErrTopkInternal);
+                    sel_count[row] = 0;
+                }
+            }
+        }
+        return fast_ok;
+    };
+    if constexpr (kMaxima) {
+        bool mfast = false;
+        uint32_t Lk = 0;
+        const int lg_slot = __ffs(kSlots / CL) - 1;                         // CL is a power of 2
+        const uint32_t slot_n = 1u << lg_slot;
+        constexpr int kM = 8;                                                // chunk maxima per thread
+        const int n_ch = (int)((own + 31) / 32);                             // chunks with an eligible region
+        if (!trivial && n_ch >= need && n_ch <= kThreads * kM) {
+            // ---- 1. the row's chunk maxima (thread t: chunks [8t, 8t + 8)) and the bound: the
+            // lower edge L of a range holding the need-th largest maximum and at most 64 maxima
+            uint32_t mk[kM];
+            {
+                float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+                if (tid * kM < n_ch) {
+                    const float4 *cm4 = reinterpret_cast<const float4 *>(chunk_max + (int64_t)row * cm_stride + tid * kM);
+                    a = __ldcg(cm4);
+                    b = __ldcg(cm4 + 1);
+                }
+                const float mv[kM] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int u = 0; u < kM; ++u) mk[u] = tid * kM + u < n_ch ? score_key(mv[u]) : 0u;
+            }
+            auto mvalid = [&](int u) { return tid * kM + u < n_ch; };
+            auto mkey = [&](int u) { return mk[u]; };
+            uint64_t elo, ehi;
+            uint32_t above, n_in;
+            key_levels<kM>(mvalid, mkey, (uint32_t)need, 64u, hs, &sh_kmin, &sh_kmax, scan_ws + 32, elo, ehi, above,
+                           n_in);
+            mfast = n_in <= 64u;                                            // else maxima tie in bulk
+            Lk = (uint32_t)elo;
+            if (mfast) {
+                // ---- 2. this CTA's chunks with maximum >= L, in region order
+                uint32_t *list = reinterpret_cast<uint32_t *>(smem_raw + kOffGmax);   // chunk ids
+                uint32_t take = 0;
+#pragma unroll
+                for (int u = 0; u < kM; ++u) {
+                    const int64_t c = tid * kM + u;
+                    if (mvalid(u) && mk[u] >= Lk && c * 32 >= lo && c * 32 < hi_ld) take |= 1u << u;
+                }
+                const uint32_t nc = __popc(take);
+                const uint32_t cincl = block_scan_incl<kThreads>(nc, scan_ws);
+                const int n_cc = (int)scan_ws[kWarps - 1];
+                {
+                    uint32_t pos = cincl - nc;
+#pragma unroll
+                    for (int u = 0; u < kM; ++u)
+                        if ((take >> u) & 1u) list[pos++] = (uint32_t)(tid * kM + u);
+                }
+                __syncthreads();
+                // ---- 3. their scores (warp per chunk, 16 chunks of a warp in flight), counted per chunk
+                constexpr int kCap = kPadded / 32;                          // chunks that fit the key stage
+                const int nst = min(n_cc, kCap);
+                uint32_t *ccnt = hw;
+                const float *srow = scores + (int64_t)row * ld;
+                const int64_t lim = min(own, hi_ld);                        // eligible regions of this CTA
+                constexpr int kRound = 16;
+                for (int base = warp; base < nst; base += kWarps * kRound) {
+                    float v[kRound];
+#pragma unroll
+                    for (int j = 0; j < kRound; ++j) {
+                        const int i = base + kWarps * j;
+                        const int64_t r = i < nst ? (int64_t)list[i] * 32 + lane : lim;
+                        v[j] = r < lim ? __ldcg(srow + r) : 0.0f;
+                    }
+#pragma unroll
+                    for (int j = 0; j < kRound; ++j) {
+                        const int i = base + kWarps * j;
+                        if (i < nst) {
+                            const int64_t r = (int64_t)list[i] * 32 + lane;
+                            const uint32_t key = r < lim ? score_key(v[j]) : 0u;
+                            keys[i * 32 + lane] = key;
+                            const unsigned m = __ballot_sync(0xffffffffu, key >= Lk && key != 0u);
+                            if (lane == 0) ccnt[i] = __popc(m);
+                        }
+                    }
+                }
+                __syncthreads();
+                // region-order offsets: thread t takes staged chunks [2t, 2t + 2)
+                uint32_t cc0 = 2 * tid < nst ? ccnt[2 * tid] : 0u, cc1 = 2 * tid + 1 < nst ? ccnt[2 * tid + 1] : 0u;
+                const uint32_t oincl = block_scan_incl<kThreads>(cc0 + cc1, scan_ws);
+                const uint32_t cta_total = scan_ws[kWarps - 1];
+                if (2 * tid < nst) ccnt[2 * tid] = oincl - cc0 - cc1;
+                if (2 * tid + 1 < nst) ccnt[2 * tid + 1] = oincl - cc1;
+                __syncthreads();
+                // ---- 4. candidates (key, ~region) into rank 0's slots, counts to every CTA
+                uint64_t *dst = reinterpret_cast<uint64_t *>(cluster.map_shared_rank(slots, 0)) +
+                                ((size_t)rank << lg_slot);
+                const unsigned below = (1u << lane) - 1u;
+                for (int i = warp; i < nst; i += kWarps) {
+                    const uint32_t key = keys[i * 32 + lane];
+                    const bool c = key >= Lk && key != 0u;
+                    const unsigned m = __ballot_sync(0xffffffffu, c);
+                    const uint32_t off = ccnt[i] + __popc(m & below);
+                    if (c && off < slot_n)
+                        dst[off] = ((uint64_t)key << 32) | (uint64_t)(0xFFFFFFFFu - (list[i] * 32 + (uint32_t)lane));
+                }
+                // more candidate chunks than the stage holds: report an overflow (every CTA falls back)
+                const uint32_t reported = n_cc > kCap ? slot_n + 1 : cta_total;
+                if (tid < CL) *cluster.map_shared_rank(&cand_cnt[rank], tid) = reported;
+                if (tid == 0) {
+                    sh_kmax = 0u;
+                    sh_nin = 0u;
+                }
+                cluster.sync();                                             // candidates and counts in place
+                fast_ok = finish_fast(Lk, lg_slot, slot_n);
+            }
+        }
+        if (!fast_ok) {
+            stage_keys();                                                   // the fallback reads every key
+            __syncthreads();
+        }
+    } else if constexpr (kSingle) {
       if (!trivial) {
         // ---- one CTA holds the row: the exact threshold over its keys directly (entry u of
         // a thread is u*512 + tid, as loaded), emitted in region order through a bitmap
@@ -482,7 +726,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else if (!trivial && (int64_t)n_groups >= need) {
         uint32_t *gmax = reinterpret_cast<uint32_t *>(smem_raw + kOffGmax);
-        uint64_t *slots = reinterpret_cast<uint64_t *>(smem_raw + kOffSlots);
         uint32_t key[kPer];
         {
             const uint4 *run = reinterpret_cast<const uint4 *>(keys + padded(tid * kPer));
@@ -559,67 +802,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             sh_nin = 0u;
         }
         cluster.sync();                                                     // candidates and counts in place
-        uint32_t total = 0;
-        bool overflow = false;
-        for (int q = 0; q < CL; ++q) {
-            total += cand_cnt[q];
-            overflow |= cand_cnt[q] > slot_n;
-        }
-        fast_ok = !overflow && total >= (uint32_t)need && total <= (uint32_t)kDense;
-        if (fast_ok && rank == 0) {
-            // ---- dense gather in region order: thread t takes entries [t*kDPer, (t+1)*kDPer)
-            uint32_t *first = slice_tot;                                    // first dense entry of each rank
-            if (tid == 0) {
-                uint32_t run = 0;
-                for (int q = 0; q < CL; ++q) {
-                    first[q] = run;
-                    run += cand_cnt[q];
-                }
-            }
-            __syncthreads();
-            uint64_t cv[kDPer];
-            const uint32_t d0 = tid * kDPer;
-            int q = 0;
-            while (q + 1 < CL && d0 >= first[q + 1]) ++q;
-#pragma unroll
-            for (int u = 0; u < kDPer; ++u) {
-                const uint32_t d = d0 + u;
-                while (q + 1 < CL && d >= first[q + 1]) ++q;
-                cv[u] = d < total ? slots[((uint32_t)q << lg_slot) + (d - first[q])] : 0ull;
-            }
-            auto valid_u = [&](int u) { return d0 + (uint32_t)u < total; };
-            auto comp_u = [&](int u) { return cv[u]; };
-            uint64_t elo, ehi, cp, cm;
-            const bool ok = block_threshold<kDPer>(valid_u, comp_u, (uint32_t)need, Lk, hs, dense, hw, &sh_kmax,
-                                                   &sh_nin, scan_ws + 32, mm_ws, &elo, &ehi, &cp, &cm);
-            if (ok) {
-                // ---- ordered emit
-                uint32_t cs = 0;
-#pragma unroll
-                for (int u = 0; u < kDPer; ++u) cs += (valid_u(u) && threshold_selects(cv[u], elo, ehi, cp, cm)) ? 1u : 0u;
-                const uint32_t sincl = block_scan_incl<kThreads>(cs, scan_ws);
-                uint32_t opos = sincl - cs;
-#pragma unroll
-                for (int u = 0; u < kDPer; ++u) {
-                    if (valid_u(u) && threshold_selects(cv[u], elo, ehi, cp, cm)) {
-                        if (opos < (uint32_t)need) out[opos] = (int32_t)(0xFFFFFFFFu - (uint32_t)cv[u]);
-                        ++opos;
-                    }
-                }
-                if (tid == kThreads - 1) {
-                    if (sincl != (uint32_t)need) set_error(kErrTopkInternal);
-                    out[need] = (int32_t)own;                               // own > every eligible region
-                    sel_count[row] = (int32_t)(need + 1);
-                }
-                for (int i = (int)need + 1 + tid; i < k; i += kThreads) out[i] = -1;
-            } else {
-                // more than kDense candidates share one key: cannot happen with total <= kDense
-                if (tid == 0) {
-                    set_error(kErrTopkInternal);
-                    sel_count[row] = 0;
-                }
-            }
-        }
+        fast_ok = finish_fast(Lk, lg_slot, slot_n);
     }
     if (fast_ok) return;               // nothing reads another CTA's smem after the barrier
 

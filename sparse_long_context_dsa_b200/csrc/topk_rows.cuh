@@ -26,6 +26,7 @@ namespace topkr {
 using topkc::block_scan_incl;
 using topkc::block_threshold;
 using topkc::desc_bin_search;
+using topkc::key_levels;
 using topkc::threshold_selects;
 
 constexpr int kThreads = 512;
@@ -41,65 +42,6 @@ constexpr size_t kOffBitmap = kOffCand + (size_t)kMaxCand * 8;                //
 constexpr size_t kOffList = kOffBitmap + ((size_t)kBitmapWords * 4 + 15) / 16 * 16;   // [32] composites
 constexpr size_t kOffHs = kOffList + 32 * 8;                                  // [256]
 constexpr size_t kSmemBytes = kOffHs + 256 * 4 + 16;
-
-// Histogram levels over the block's keys (thread item u valid when valid(u)): the range
-// [elo, ehi) holding the m-th largest key, `above` keys >= ehi, n_in keys in the range;
-// stops once n_in <= cap or the range is one value.  Needs m <= the valid count.
-template <int R, typename Valid, typename Key>
-__device__ void key_levels(Valid valid, Key key, uint32_t m, uint32_t cap, uint32_t *hs, uint32_t *sh_min,
-                           uint32_t *sh_max, uint32_t *res, uint64_t &elo, uint64_t &ehi, uint32_t &above,
-                           uint32_t &n_in)
-{
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    uint32_t kmn = 0xFFFFFFFFu, kmx = 0u;
-#pragma unroll
-    for (int u = 0; u < R; ++u)
-        if (valid(u)) {
-            kmn = min(kmn, key(u));
-            kmx = max(kmx, key(u));
-        }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        kmn = min(kmn, __shfl_xor_sync(0xffffffffu, kmn, o));
-        kmx = max(kmx, __shfl_xor_sync(0xffffffffu, kmx, o));
-    }
-    if (lane == 0) {
-        atomicMin(sh_min, kmn);
-        atomicMax(sh_max, kmx);
-    }
-    if (tid < 256) hs[tid] = 0u;
-    __syncthreads();
-    kmn = *sh_min;
-    kmx = *sh_max;
-    uint64_t rlo = kmn, width = ~0ull;
-    int bsh = max(0, 24 - __clz((int)(kmx - kmn)));
-    uint32_t m_rem = m, bin = 0;
-    above = 0;
-    for (int level = 0; level < 4; ++level) {
-#pragma unroll
-        for (int u = 0; u < R; ++u) {
-            if (!valid(u)) continue;
-            const uint64_t kk = key(u);
-            if (kk >= rlo && kk - rlo < width) atomicAdd(&hs[(uint32_t)((kk - rlo) >> bsh)], 1u);
-        }
-        __syncthreads();
-        if (warp == 0) desc_bin_search(hs, m_rem, res);
-        __syncthreads();
-        bin = res[0];
-        above += res[1];
-        m_rem -= res[1];
-        n_in = res[2];
-        if (tid < 256) hs[tid] = 0u;
-        if (n_in <= cap || bsh == 0) break;
-        rlo += (uint64_t)bin << bsh;
-        width = 1ull << bsh;
-        bsh = max(0, bsh - 8);
-        __syncthreads();
-    }
-    elo = rlo + ((uint64_t)bin << bsh);
-    ehi = elo + (1ull << bsh);
-    __syncthreads();
-}
 
 __global__ void __launch_bounds__(kThreads, 2)
     topk_rows_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ q_pos, int k,

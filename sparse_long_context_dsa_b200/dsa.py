@@ -49,6 +49,10 @@ _SIG = {
                                         _VP, ctypes.c_size_t, _VP]),
     "dsa_topk_regions_noalloc": (ctypes.c_int, [_F32P, ctypes.c_int64, _I32P, ctypes.c_int, ctypes.c_int, _I32P,
                                                 _I32P, _VP]),
+    "dsa_decode_select_workspace_size": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int64, ctypes.c_int]),
+    "dsa_decode_select": (ctypes.c_int, [_VP, _F32P, _I32P, _I32P, ctypes.c_int, _U8P, _F32P, ctypes.c_int64,
+                                         _I64P, ctypes.c_int, _F32P, ctypes.c_int64, ctypes.c_uint32, ctypes.c_int,
+                                         _I32P, _I32P, _VP, ctypes.c_size_t, _VP]),
     "dsa_copy": (ctypes.c_int, [_VP, _VP, ctypes.c_size_t, _VP]),
     "dsa_attn_workspace_size": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int]),
     "dsa_sparse_attn_decode": (ctypes.c_int, [_VP, _VP, _VP, ctypes.c_int64, _I32P, ctypes.c_int, _I32P,
@@ -156,6 +160,37 @@ def indexer_scores(index_q, gate, q_req, q_pos, summaries, scales, sum_base, sco
     _check(lib().dsa_indexer_scores(_p(index_q), _p(gate), _p(q_req), _p(q_pos), nq, _p(summaries), _p(scales),
                                     n_slots, _p(sum_base), sum_base.numel(), _p(scores), ld, flags, _p(ws),
                                     nbytes, _stream()))
+
+
+def decode_select(index_q, gate, q_req, q_pos, summaries, scales, sum_base, scores, k, flags=0, sel_idx=None,
+                  sel_count=None):
+    """dsa_decode_select: the indexer scores into `scores` [nq][4][ld] and the top-k selection
+    in one call.  Returns (sel_idx, sel_count) as topk_regions does."""
+    nq = index_q.shape[0]
+    _need(index_q, torch.bfloat16, (nq, HI, DI), "index_q")
+    _need(gate, torch.float32, (nq, HI), "gate")
+    _need(q_req, torch.int32, (nq,), "q_req")
+    _need(q_pos, torch.int32, (nq,), "q_pos")
+    _need(summaries, torch.uint8, name="summaries")
+    n_slots = summaries.shape[1]
+    _need(scales, torch.float32, (G, n_slots), "scales")
+    _need(sum_base, torch.int64, name="sum_base")
+    _need(scores, torch.float32, name="scores")
+    if scores.dim() != 3 or scores.shape[0] != nq or scores.shape[1] != G:
+        raise ValueError("scores must be [nq][4][ld]")
+    ld = scores.shape[2]
+    if sel_idx is None:
+        sel_idx = torch.empty((nq, G, k), dtype=torch.int32, device=scores.device)
+    if sel_count is None:
+        sel_count = torch.empty((nq, G), dtype=torch.int32, device=scores.device)
+    _need(sel_idx, torch.int32, (nq, G, k), "sel_idx")
+    _need(sel_count, torch.int32, (nq, G), "sel_count")
+    nbytes = lib().dsa_decode_select_workspace_size(nq, ld, k)
+    ws = _workspace(nbytes, scores.device)
+    _check(lib().dsa_decode_select(_p(index_q), _p(gate), _p(q_req), _p(q_pos), nq, _p(summaries), _p(scales), n_slots,
+                                   _p(sum_base), sum_base.numel(), _p(scores), ld, flags, k, _p(sel_idx),
+                                   _p(sel_count), _p(ws), nbytes, _stream()))
+    return sel_idx, sel_count
 
 
 def topk_regions(scores, q_pos, k, sel_idx=None, sel_count=None):

@@ -2,8 +2,8 @@
 
 A decode step for a batch of requests, one query each, is
     compress the regions that this step completes  (A1, only if any are due)
-    indexer scores over every complete region     (A2)
-    top-k with the own region forced              (A3)
+    indexer scores over every complete region     (A2)  } one call: dsa_decode_select
+    top-k with the own region forced              (A3)  }
     sparse attention over the selected regions    (A4)
 ([P2] Step-5-Preview 如何实现1M长上下文 §区域压缩CSA / §索引器打分).
 
@@ -80,10 +80,12 @@ class DecodeStep:
         L = dsa.lib()
         self.ws_idx_n = L.dsa_indexer_workspace_size(B, self.ld)
         self.ws_topk_n = L.dsa_topk_workspace_size(B, self.ld, self.k)
+        self.ws_sel_n = L.dsa_decode_select_workspace_size(B, self.ld, self.k)
         self.ws_attn_n = L.dsa_attn_workspace_size(B, self.k)
         self.ws_idx = torch.empty(max(1, self.ws_idx_n), dtype=torch.uint8, device=dev)
         self.ws_topk = torch.empty(max(1, self.ws_topk_n), dtype=torch.uint8, device=dev)
         self.ws_attn = torch.empty(max(1, self.ws_attn_n), dtype=torch.uint8, device=dev)
+        self.ws_sel = torch.empty(max(1, self.ws_sel_n), dtype=torch.uint8, device=dev)
 
     def load(self, index_q, gate, q, q_pos, tail=None):
         self.index_q.copy_(index_q, non_blocking=True)
@@ -109,7 +111,7 @@ class DecodeStep:
 
     def run(self, pre_scan=None, post_scan=None, out=None):
         """Launches the step on the current stream (capturable).  pre_scan/post_scan are
-        optional callables invoked right before/after the indexer-scan launch (the
+        optional callables invoked right before/after the scores + selection call (the
         benchmark records timing events there).  out: where the attention writes its
         output, bf16 [B][64][192], on the device (default `self.out`) or in pinned host
         memory, which the kernel then writes directly."""
@@ -131,14 +133,13 @@ class DecodeStep:
         st = dsa._stream()
         if pre_scan is not None:
             pre_scan()
-        dsa._check(L.dsa_indexer_scores(p(self.index_q), p(self.gate), p(self.q_req), p(self.q_pos), self.B,
-                                        p(self.summaries), p(self.scales), self.summaries.shape[1],
-                                        p(self.sum_base), self.sum_base.numel(), p(self.scores), self.ld,
-                                        self.flags, p(self.ws_idx), self.ws_idx_n, st))
+        # scores and selection in one call (the scan's chunk maxima bound the selection)
+        dsa._check(L.dsa_decode_select(p(self.index_q), p(self.gate), p(self.q_req), p(self.q_pos), self.B,
+                                       p(self.summaries), p(self.scales), self.summaries.shape[1], p(self.sum_base),
+                                       self.sum_base.numel(), p(self.scores), self.ld, self.flags, self.k,
+                                       p(self.sel_idx), p(self.sel_count), p(self.ws_sel), self.ws_sel_n, st))
         if post_scan is not None:
             post_scan()
-        dsa._check(L.dsa_topk_regions(p(self.scores), self.ld, p(self.q_pos), self.B, self.k, p(self.sel_idx),
-                                      p(self.sel_count), p(self.ws_topk), self.ws_topk_n, st))
         dsa._check(L.dsa_sparse_attn_decode(p(self.q), p(self.k_cache), p(self.v_cache), self.k_cache.shape[0],
                                             p(self.block_table), self.block_table.shape[1], p(self.q_pos), self.B,
                                             p(self.sel_idx), p(self.sel_count), self.k, p(out), p(self.lse),
