@@ -41,10 +41,10 @@ UNIT = "queries/s"
 L_CTX = 1 << 20
 TOPK = 512
 N_LAYERS = 4
-KERNELS_PER_STEP = 4      # compress, scan, cluster top-k, clustered attention (split merge inside)
+KERNELS_PER_STEP = 4      # compress, scan (+ chunk maxima), cluster top-k, clustered attention
 # DRAM bytes (read + write) of one scan launch on this workload, from one ncu capture of the
 # current scan kernel (dram__bytes_read.sum + dram__bytes_write.sum); None once the kernel changes
-SCAN_TRAFFIC_BYTES = 136_393_216 + 5_188_352
+SCAN_TRAFFIC_BYTES = 136_391_168 + 3_656_960
 PREFILL_CTX, PREFILL_NEW = 262144, 2048
 PREFILL_KERNELS = 6       # compress, quantize, GEMM, top-k histogram, top-k select, attention
 
