@@ -122,9 +122,10 @@ dsa_status_t dsa_compress_regions(const void *index_k, int64_t row_stride, int64
  * Two kernels serve the call.  A call with DSA_Q_FP8 over one request's chunk (n_req == 1,
  * nq >= 64) and a workspace of dsa_indexer_workspace_size(nq, ld) bytes (256-byte
  * aligned, owned by the caller, not kept after the stream reaches the end of the call)
- * runs as a tcgen05 FP8 x FP8 GEMM per group; every other call (decode batches, several
- * requests, bf16 queries, or ws == NULL) runs the streaming scan, which needs no
- * workspace.  Both compute the same scores up to fp32 summation order. */
+ * and 16-byte aligned scales runs as a tcgen05 FP8 x FP8 GEMM per group; every other call
+ * (decode batches, several requests, bf16 queries, ws == NULL or unaligned scales) runs
+ * the streaming scan, which needs no workspace.  Both compute the same scores up to fp32
+ * summation order. */
 size_t dsa_indexer_workspace_size(int nq, int64_t ld_scores);
 dsa_status_t dsa_indexer_scores(const void *index_q, const float *gate, const int32_t *q_req,
                                 const int32_t *q_pos, int nq, const uint8_t *summaries,

@@ -72,10 +72,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint64_t *bars = reinterpret_cast<uint64_t *>(qs + kQBytes);   // [kWarps][kSlots]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int split = blockIdx.x;
-    const int row = blockIdx.y;            // query * 4 + group
+    // block order: split-major, then group, then query, so that the CTAs resident together
+    // gather from one group's (and one split's) share of the cache and reuse it in L2
+    const int rows = p.nq * kG;
+    const int split = (int)blockIdx.x / rows;
+    const int rem = (int)blockIdx.x - split * rows;
+    const int g = rem / p.nq, qi = rem - g * p.nq;
+    const int row = qi * kG + g;           // query * 4 + group
     if (p.row_shared && p.row_shared[row]) return;
-    const int qi = row >> 2, g = row & 3;
     const int b = p.q_req ? p.q_req[qi] : qi;
     const int pos = p.q_pos[qi];
     const int cnt_raw = p.sel_count[row];

@@ -72,8 +72,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     __shared__ int sh_pass_req, sh_max_own, sh_union;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
-    const int g = blockIdx.x & 3;
-    const int q0 = (blockIdx.x >> 2) * kQueries;
+    // group-major block order: the CTAs resident together gather from one group's cache
+    const int n_qblocks = (int)gridDim.x / kG;
+    const int g = (int)blockIdx.x / n_qblocks;
+    const int q0 = ((int)blockIdx.x - g * n_qblocks) * kQueries;
     if (tid == 0) {
         for (int s = 0; s < kSlots; ++s) {
             mbar_init(&full[s], 1);

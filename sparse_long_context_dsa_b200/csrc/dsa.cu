@@ -3,6 +3,7 @@
 // compress.cuh, indexer.cuh, topk.cuh and attention.cuh (one translation unit, so the
 // per-device error word is a single symbol).
 #include <algorithm>
+#include <cstring>
 #include <mutex>
 #include <utility>
 #include <string>
@@ -86,13 +87,14 @@ EncodeTiledFn encode_fn()
 }
 
 dsa_status_t encode(CUtensorMap *map, CUtensorMapDataType dt, int rank, const void *base, const cuuint64_t *dims,
-                    const cuuint64_t *strides, const cuuint32_t *box, CUtensorMapL2promotion l2)
+                    const cuuint64_t *strides, const cuuint32_t *box, CUtensorMapL2promotion l2,
+                    CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
     cuuint32_t estr[5] = {1, 1, 1, 1, 1};
     CUresult r = fn(map, dt, (cuuint32_t)rank, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, l2, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, l2, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (" + std::to_string((int)r) + ")");
     return DSA_OK;
 }
@@ -311,7 +313,7 @@ dsa_status_t attn_common(const void *q, const void *k_cache, const void *v_cache
                                         (int)dsa::attn::kSmemBytes);
     });
     DSA_CUDA(attr_err, "cudaFuncSetAttribute(sparse_attn_kernel)");
-    dim3 grid(plan.n_splits, nq * dsa::kG);
+    dim3 grid((unsigned)(plan.n_splits * nq * dsa::kG));
     if ((st = launch_k("sparse_attn_kernel", dsa::attn::sparse_attn_kernel, grid, dim3(dsa::attn::kThreads),
                        dsa::attn::kSmemBytes, stream, 0, mk, mv, p)) != DSA_OK)
         return st;
@@ -353,21 +355,33 @@ dsa_status_t indexer_gemm_path(const void *index_q, const float *gate, const int
                        qscale, q_own, tile_own, n_mtiles)) != DSA_OK)
         return st;
 
-    CUtensorMap map_a, map_b;
+    CUtensorMap map_q, map_s;
     {
-        const cuuint64_t dims[4] = {(cuuint64_t)dsa::kDI, 4, 4, (cuuint64_t)nq};
-        const cuuint64_t strides[3] = {(cuuint64_t)dsa::kDI, (cuuint64_t)dsa::kDI * 4, (cuuint64_t)dsa::kDI * 16};
-        const cuuint32_t box[4] = {128, 4, 1, (cuuint32_t)dsa::gemm::kQPerTile};
-        if ((st = encode(&map_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, codes, dims, strides, box,
+        // codes [nq][16 heads][256]: a box of 128 bytes of d x one group's 4 heads x 64 queries
+        const cuuint64_t dims[3] = {(cuuint64_t)dsa::kDI, (cuuint64_t)dsa::kHI, (cuuint64_t)nq};
+        const cuuint64_t strides[2] = {(cuuint64_t)dsa::kDI, (cuuint64_t)dsa::kDI * dsa::kHI};
+        const cuuint32_t box[3] = {128, (cuuint32_t)dsa::gemm::kHeads, (cuuint32_t)dsa::gemm::kQPerTile};
+        if ((st = encode(&map_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, codes, dims, strides, box,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B)) != DSA_OK)
             return st;
     }
     {
+        // summaries [4 * n_slots][256]: a box of 128 bytes x 128 regions
         const cuuint64_t dims[2] = {(cuuint64_t)dsa::kDI, (cuuint64_t)n_slots * dsa::kG};
         const cuuint64_t strides[1] = {(cuuint64_t)dsa::kDI};
-        const cuuint32_t box[2] = {128, (cuuint32_t)dsa::gemm::kBN};
-        if ((st = encode(&map_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, summaries, dims, strides, box,
+        const cuuint32_t box[2] = {128, (cuuint32_t)dsa::gemm::kBM};
+        if ((st = encode(&map_s, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, summaries, dims, strides, box,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B)) != DSA_OK)
+            return st;
+    }
+    CUtensorMap map_sc;
+    {
+        // scales [4 * n_slots] fp32 as one line: a block's 128 scales from a 16-byte aligned start
+        const cuuint64_t dims[1] = {(cuuint64_t)n_slots * dsa::kG};
+        const cuuint64_t strides[1] = {(cuuint64_t)n_slots * dsa::kG * 4};   // unused at rank 1
+        const cuuint32_t box[1] = {(cuuint32_t)dsa::gemm::kScaleBox};
+        if ((st = encode(&map_sc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 1, scales, dims, strides, box,
+                         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_SWIZZLE_NONE)) != DSA_OK)
             return st;
     }
     dsa::gemm::Params p{};
@@ -381,13 +395,9 @@ dsa_status_t indexer_gemm_path(const void *index_q, const float *gate, const int
     p.ld = ld;
     p.n_slots = n_slots;
     p.nq = nq;
-    p.n_rblocks = (int)((ld + dsa::gemm::kBN - 1) / dsa::gemm::kBN);
     p.n_mtiles = n_mtiles;
-    int parts = 1;
-    while (4 * p.n_rblocks * parts < 6 * sms && parts < n_mtiles) parts *= 2;
-    p.m_per_unit = (n_mtiles + parts - 1) / parts;
-    p.n_mparts = (n_mtiles + p.m_per_unit - 1) / p.m_per_unit;
-    p.n_units = dsa::kG * p.n_rblocks * p.n_mparts;
+    // persistent grid: at most one CTA per SM (512 TMEM columns, ~225 KiB of smem each)
+    const int64_t blocks_bound = (int64_t)dsa::kG * n_mtiles * ((ld + dsa::gemm::kBM - 1) / dsa::gemm::kBM);
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
@@ -395,8 +405,9 @@ dsa_status_t indexer_gemm_path(const void *index_q, const float *gate, const int
                                         (int)dsa::gemm::kSmemBytes);
     });
     DSA_CUDA(attr_err, "cudaFuncSetAttribute(gemm_scores_kernel)");
-    return launch_k("gemm_scores_kernel", dsa::gemm::gemm_scores_kernel, dim3(std::min(sms, p.n_units)),
-                    dim3(dsa::gemm::kThreads), dsa::gemm::kSmemBytes, stream, 0, map_a, map_b, p);
+    return launch_k("gemm_scores_kernel", dsa::gemm::gemm_scores_kernel,
+                    dim3((unsigned)std::min<int64_t>(sms, std::max<int64_t>(1, blocks_bound))),
+                    dim3(dsa::gemm::kThreads), dsa::gemm::kSmemBytes, stream, 0, map_q, map_s, map_sc, p);
 }
 
 // Workspace path of the top-k: histogram, threshold-bin gather and last-CTA selection
@@ -622,7 +633,7 @@ dsa_status_t dsa_indexer_scores(const void *index_q, const float *gate, const in
     if (st != DSA_OK) return st;
 
     if ((flags & DSA_Q_FP8) && n_req == 1 && nq >= kGemmMinQueries && ws && ws_bytes >= gemm_ws_size(nq) &&
-        aligned(ws, 256))
+        aligned(ws, 256) && aligned(scales, 16))
         return indexer_gemm_path(index_q, gate, q_req, q_pos, nq, summaries, scales, n_slots, sum_base, scores,
                                  ld_scores, ws, sms, stream);
     return scan_path(index_q, gate, q_req, q_pos, nq, summaries, scales, n_slots, sum_base, n_req, scores, ld_scores,

@@ -2,41 +2,57 @@
 // §DSA ③; [P2] Step-5-Preview 如何实现1M长上下文 §索引器打分).
 //
 // For one request's chunk of queries the score is a dense contraction per KV group g:
-//   C_g[(q, h)][r] = sum_d q8[q][h][d] * s8[g][r][d]        (e4m3 x e4m3 -> fp32, K = 256)
-//   score[q][g][r] = scale[g][r] / 16 * sum_{h in g} z[q][h] * sq[q][h] * ReLU(C_g[(q, h)][r])
+//   C[r][(q, h)] = sum_d s8[g][r][d] * q8[q][h][d]        (e4m3 x e4m3 -> fp32, K = 256)
+//   score[q][g][r] = scale[g][r] / 16 * sum_{h in g} z[q][h] * sq[q][h] * ReLU(C[r][(q, h)])
 // with the query quantised per (query, head) to e4m3 with scale sq = absmax/448 (the FP8
-// reading of the method, DSA_Q_FP8).  Layout of the work:
-//  * a work unit is (group g, block of 256 regions, range of 128-row query tiles); the
-//    CTA keeps the unit's 256 x 256 B summary tile in smem (two TMA boxes of 128-byte
-//    columns, 128-byte swizzle) and streams query tiles of 32 queries x 4 heads through a
-//    2-stage TMA ring.  Keeping the summaries resident and streaming the (small) queries
-//    reads the queries ~129 times and the summaries once per query range instead of the
-//    summaries 64 times;
-//  * one thread issues 8 tcgen05.mma kind::f8f6f4 (M = 128, N = 256, K = 32) per tile into
-//    one of two 256-column TMEM accumulators (512 columns: all of TMEM, one CTA per SM);
-//  * four epilogue warps (one per TMEM lane quarter) read 32 columns at a time, apply
-//    ReLU * z * sq per row, sum the 4 heads of a query with a two-step shuffle butterfly
-//    that leaves every lane 8 finished columns, scale by scale[g][r]/16, mask r < own and
-//    store; the accumulator buffer is released to the MMA thread after the last read;
-//  * tiles whose queries all have own <= the block's first region are skipped (causal).
+// reading of the method, DSA_Q_FP8).  Region-major layout of the work:
+//  * a block is 128 regions (the M side: the 128 TMEM lanes) x 64 queries x the group's 4
+//    indexer heads (the N side: 256 columns, column 4q + h); the CTA keeps a 64-query tile
+//    of codes (256 rows x 256 B = 64 KiB, 128-byte swizzle) resident in smem while 128-region
+//    summary blocks (32 KiB) stream through a 4-stage TMA ring;
+//  * one thread issues 8 tcgen05.mma kind::f8f6f4 (M = 128, N = 256, K = 32) per block into
+//    one of two 256-column TMEM accumulators (512 columns, one CTA per SM).  Large-N
+//    instructions matter: the same block cut as 4 heads x (M = 128, N = 64) ran the tensor
+//    pipe at a third of the rate;
+//  * sixteen epilogue warps (four per TMEM lane quarter, one per 16-query quarter) read
+//    their 64 columns, release the buffer, and for each query form sum_h w_h * ReLU(C) in
+//    registers: each thread owns one region, so the head sum stays in the thread, the
+//    region's scale is one register (the block's 128 scales arrive with the summaries by
+//    TMA), and a warp's 32 lanes write one 128-byte line of a query's score row, masked
+//    r < own only on blocks that cross a query's own region;
+//  * the blocks (group, query tile, region block) a tile needs (region blocks that start
+//    before the tile's largest own region) form one sequence split evenly over a persistent
+//    grid.
 #pragma once
+
+#include <climits>
+#include <type_traits>
 
 #include "common.cuh"
 
 namespace dsa {
 namespace gemm {
 
-constexpr int kQPerTile = 32;
-constexpr int kBM = kQPerTile * 4;       // 128 rows: (query, head of the group)
-constexpr int kBN = 256;                 // regions per summary tile
-constexpr int kAStages = 2;
-constexpr int kAHalf = kBM * 128;        // one 128-byte K column of a query tile (16 KiB)
-constexpr int kABytes = 2 * kAHalf;
-constexpr int kBHalf = kBN * 128;        // 32 KiB
-constexpr int kBBytes = 2 * kBHalf;
-constexpr int kThreads = 192;            // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
-constexpr int kTmemCols = 512;           // two 256-column fp32 accumulators
-constexpr size_t kSmemBytes = 1024 + kBBytes + kAStages * kABytes + 4 * kBN * 4 + 256;
+constexpr int kBM = 128;                 // regions per block (M)
+constexpr int kQPerTile = 64;            // queries per tile
+constexpr int kHeads = 4;                // indexer heads of a group
+constexpr int kBN = kQPerTile * kHeads;  // 256 accumulator columns (N)
+constexpr int kQHalf = kBN * 128;        // one 128-byte K column of the query tile (32 KiB)
+constexpr int kQBytes = 2 * kQHalf;      // 64 KiB
+constexpr int kSHalf = kBM * 128;        // one 128-byte K column of a summary block (16 KiB)
+constexpr int kSBytes = 2 * kSHalf;      // 32 KiB
+constexpr int kSStages = 4;
+constexpr int kEpiWarps = 16;
+constexpr int kThreads = 32 * (2 + kEpiWarps);  // warp 0 TMA, warp 1 MMA, warps 2..17 epilogue
+constexpr int kEpiQueries = kQPerTile / 4;      // queries per epilogue warp
+constexpr int kTmemCols = 512;                  // two 256-column fp32 accumulators
+constexpr int kScaleBox = kBM + 4;              // region scales per block, from a 16-byte aligned start
+constexpr int kScaleBytes = kScaleBox * 4;      // 528 bytes loaded per block
+constexpr int kScaleSlot = 640;                 // slot stride: a TMA destination is 128-byte aligned
+constexpr size_t kSmemBytes = 1024 + kQBytes + (size_t)kSStages * (kSBytes + kScaleSlot) +
+                              (size_t)kEpiWarps * kEpiQueries * (16 + 4) + 256;
+static_assert(kSmemBytes <= 232448, "one CTA per SM");
+static_assert(kScaleSlot % 128 == 0 && kScaleSlot >= kScaleBytes, "scale slots");
 constexpr uint32_t kIdesc = umma_idesc_e4m3(kBM, kBN);
 
 struct Params {
@@ -50,11 +66,7 @@ struct Params {
     int64_t ld;
     int64_t n_slots;
     int nq;
-    int n_rblocks;
     int n_mtiles;
-    int m_per_unit;
-    int n_mparts;
-    int n_units;
 };
 
 // The query's own region when the query is valid for this path (request 0, pos >= 0, own
@@ -124,58 +136,96 @@ __global__ void __launch_bounds__(128) quantize_kernel(const __nv_bfloat16 *__re
 }
 
 
-// Work unit u -> (group, region block, query-tile range); a unit is active iff one of its
-// tiles holds a query whose own region lies beyond the block's first region.
-__device__ __forceinline__ void unit_coords(const Params &p, int u, int &g, int &rb, int &t0, int &t1)
+// Region blocks tile t needs: those that start before its largest own region.
+__device__ __forceinline__ int tile_blocks(const Params &p, int t)
 {
-    const int mp = u % p.n_mparts;
-    const int gr = u / p.n_mparts;
-    rb = gr % p.n_rblocks;
-    g = gr / p.n_rblocks;
-    t0 = mp * p.m_per_unit;
-    t1 = min(p.n_mtiles, t0 + p.m_per_unit);
+    const int o = p.tile_own[t];
+    return o > 0 ? (o + kBM - 1) / kBM : 0;
 }
 
-__device__ __forceinline__ bool tile_active(const Params &p, int t, int rb)
+// A position in the sequence of blocks (group g, tile t, region block rb), rb fastest.
+struct Walk {
+    int g, t, rb, nb;
+};
+
+__device__ __forceinline__ int64_t total_blocks(const Params &p)
 {
-    return p.tile_own[t] > rb * kBN;
+    int64_t n = 0;
+    for (int t = 0; t < p.n_mtiles; ++t) n += tile_blocks(p, t);
+    return n * kG;
 }
 
-__device__ __forceinline__ bool unit_active(const Params &p, int t0, int t1, int rb)
+__device__ __forceinline__ void walk_seek(const Params &p, int64_t idx, Walk &w)
 {
-    for (int t = t0; t < t1; ++t)
-        if (tile_active(p, t, rb)) return true;
-    return false;
+    w.g = kG;                                   // past the end unless found
+    for (int g = 0; g < kG; ++g)
+        for (int t = 0; t < p.n_mtiles; ++t) {
+            const int nb = tile_blocks(p, t);
+            if (idx < nb) {
+                w.g = g;
+                w.t = t;
+                w.rb = (int)idx;
+                w.nb = nb;
+                return;
+            }
+            idx -= nb;
+        }
 }
 
+__device__ __forceinline__ void walk_next(const Params &p, Walk &w)
+{
+    if (++w.rb < w.nb) return;
+    w.rb = 0;
+    do {
+        if (++w.t == p.n_mtiles) {
+            w.t = 0;
+            if (++w.g == kG) return;
+        }
+        w.nb = tile_blocks(p, w.t);
+    } while (w.nb == 0);
+}
+
+// This CTA's share [lo, hi) of the block sequence.
+__device__ __forceinline__ void cta_range(const Params &p, int64_t &lo, int64_t &hi)
+{
+    const int64_t total = total_blocks(p);
+    lo = total * blockIdx.x / gridDim.x;
+    hi = total * (blockIdx.x + 1) / gridDim.x;
+}
+
+// 18 warps: 5 share a scheduler's 16K registers, so at most 96 registers per thread
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_scores_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                       const Params p)
+    gemm_scores_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_s,
+                       const __grid_constant__ CUtensorMap map_sc, const Params p)
 {
     pdl_trigger();   // the next kernel may launch; it waits for this one itself
     pdl_wait();      // the previous kernel's results are visible from here on
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sb = smem;                                   // summary tile: 2 K columns x [256][128]
-    uint8_t *sa = smem + kBBytes;                         // query tiles: kAStages x 2 K columns x [128][128]
-    float *sscale_all = reinterpret_cast<float *>(sa + kAStages * kABytes);    // [4 warps][256] scales / 16
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sscale_all + 4 * kBN);
-    uint64_t *b_full = bars + 0, *b_empty = bars + 1;
-    uint64_t *a_full = bars + 2, *a_empty = bars + 4;     // [kAStages]
-    uint64_t *acc_full = bars + 6, *acc_empty = bars + 8; // [2]
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 10);
+    uint8_t *sq = smem;                                   // query tile: 2 K columns x [256 rows (q, h)][128 B]
+    uint8_t *ss = smem + kQBytes;                         // summary blocks: kSStages x 2 K columns x [128][128 B]
+    uint8_t *ssc = ss + kSStages * kSBytes;                                     // [kSStages] scale slots
+    float4 *wsm_all = reinterpret_cast<float4 *>(ssc + kSStages * kScaleSlot);  // [16 warps][8 pairs][2] weights
+    int *own_all = reinterpret_cast<int *>(wsm_all + kEpiWarps * kEpiQueries);  // [16 warps][16 queries]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(own_all + kEpiWarps * kEpiQueries);
+    uint64_t *q_full = bars + 0, *q_empty = bars + 1;
+    uint64_t *s_full = bars + 2, *s_empty = bars + 2 + kSStages;                // [kSStages]
+    uint64_t *acc_full = bars + 2 + 2 * kSStages, *acc_empty = acc_full + 2;    // [2]
+    uint64_t *sc_empty = acc_empty + 2;                                         // [kSStages]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sc_empty + kSStages);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        mbar_init(b_full, 1);
-        mbar_init(b_empty, 1);
-        for (int s = 0; s < kAStages; ++s) {
-            mbar_init(&a_full[s], 1);
-            mbar_init(&a_empty[s], 1);
+        mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
+        for (int s = 0; s < kSStages; ++s) {
+            mbar_init(&s_full[s], 1);
+            mbar_init(&s_empty[s], 1);
+            mbar_init(&sc_empty[s], kEpiWarps);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], 4);
+            mbar_init(&acc_empty[b], kEpiWarps);
         }
         fence_mbar_init();
     }
@@ -185,153 +235,183 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const int64_t base = p.sum_base[0];
+    int64_t lo, hi;
+    cta_range(p, lo, hi);
+    const int64_t n_items = hi - lo;
     bool ok = true;
 
     if (warp == 0) {
-        // ---------------- TMA producer (one lane)
-        if (lane == 0) {
-            prefetch_tensormap(&map_a);
-            prefetch_tensormap(&map_b);
-            int ub = 0, ait = 0;
-            for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-                int g, rb, t0, t1;
-                unit_coords(p, u, g, rb, t0, t1);
-                if (!unit_active(p, t0, t1, rb)) continue;
-                ok = mbar_wait(b_empty, (ub & 1) ^ 1);
-                if (!ok) break;
-                mbar_arrive_expect_tx(b_full, kBBytes);
-                const int y = (int)(g * p.n_slots + base + (int64_t)rb * kBN);
-                tma_load_2d(sb, &map_b, 0, y, b_full);
-                tma_load_2d(sb + kBHalf, &map_b, 128, y, b_full);
-                ++ub;
-                for (int t = t0; t < t1; ++t) {
-                    if (!tile_active(p, t, rb)) continue;
-                    const int s = ait % kAStages;
-                    ok = mbar_wait(&a_empty[s], ((ait / kAStages) & 1) ^ 1);
+        // ---------------- TMA producer (one lane): the query tile when it changes, then the block
+        if (lane == 0 && n_items > 0) {
+            prefetch_tensormap(&map_q);
+            prefetch_tensormap(&map_s);
+            prefetch_tensormap(&map_sc);
+            Walk w;
+            walk_seek(p, lo, w);
+            int cur_g = -1, cur_t = -1, q_loads = 0;
+            for (int64_t it = 0; it < n_items; ++it, walk_next(p, w)) {
+                if (w.g != cur_g || w.t != cur_t) {
+                    ok = mbar_wait_sleep(q_empty, (q_loads & 1) ^ 1);
                     if (!ok) break;
-                    mbar_arrive_expect_tx(&a_full[s], kABytes);
-                    uint8_t *dst = sa + s * kABytes;
-                    tma_load_4d(dst, &map_a, 0, 0, g, t * kQPerTile, &a_full[s]);
-                    tma_load_4d(dst + kAHalf, &map_a, 128, 0, g, t * kQPerTile, &a_full[s]);
-                    ++ait;
+                    mbar_arrive_expect_tx(q_full, kQBytes);
+                    // box: 128 B of d x the group's 4 heads x 64 queries -> rows 4q + h
+                    tma_load_3d(sq, &map_q, 0, w.g * kHeads, w.t * kQPerTile, q_full);
+                    tma_load_3d(sq + kQHalf, &map_q, 128, w.g * kHeads, w.t * kQPerTile, q_full);
+                    ++q_loads;
+                    cur_g = w.g;
+                    cur_t = w.t;
                 }
+                const int s = (int)(it % kSStages);
+                // the slot is free once the MMA has read the summaries and every epilogue
+                // warp its scale
+                ok = mbar_wait_sleep(&s_empty[s], ((int)(it / kSStages) & 1) ^ 1) &&
+                     mbar_wait_sleep(&sc_empty[s], ((int)(it / kSStages) & 1) ^ 1);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&s_full[s], kSBytes + kScaleBytes);
+                const int y = (int)(w.g * p.n_slots + base + (int64_t)w.rb * kBM);
+                uint8_t *dst = ss + s * kSBytes;
+                tma_load_2d(dst, &map_s, 0, y, &s_full[s]);
+                tma_load_2d(dst + kSHalf, &map_s, 128, y, &s_full[s]);
+                // scales y .. y + 127 from the 16-byte aligned element y & ~3 (past the pool: 0)
+                tma_load_1d(ssc + s * kScaleSlot, &map_sc, y & ~3, &s_full[s]);
             }
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer (one lane)
-        if (lane == 0) {
-            int ub = 0, ait = 0, cit = 0;
-            for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-                int g, rb, t0, t1;
-                unit_coords(p, u, g, rb, t0, t1);
-                if (!unit_active(p, t0, t1, rb)) continue;
-                ok = mbar_wait(b_full, ub & 1);
-                if (!ok) break;
-                ++ub;
-                for (int t = t0; t < t1; ++t) {
-                    if (!tile_active(p, t, rb)) continue;
-                    const int s = ait % kAStages, buf = cit & 1;
-                    ok = mbar_wait(&a_full[s], (ait / kAStages) & 1) &&
-                         mbar_wait(&acc_empty[buf], ((cit >> 1) & 1) ^ 1);
+        if (lane == 0 && n_items > 0) {
+            Walk w;
+            walk_seek(p, lo, w);
+            int cur_g = -1, cur_t = -1, q_loads = 0;
+            for (int64_t it = 0; it < n_items; ++it, walk_next(p, w)) {
+                if (w.g != cur_g || w.t != cur_t) {
+                    if (q_loads > 0) umma_commit(q_empty);   // the old query tile is free once its MMAs finish
+                    ok = mbar_wait_sleep(q_full, q_loads & 1);
                     if (!ok) break;
-                    tc_fence_after();
-                    const uint32_t a0 = smem_u32(sa + s * kABytes), b0 = smem_u32(sb);
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t off_a = (kk >> 2) * kAHalf + (kk & 3) * 32;
-                        const uint32_t off_b = (kk >> 2) * kBHalf + (kk & 3) * 32;
-                        umma_e4m3(tmem + buf * kBN, umma_desc_sw128(a0 + off_a), umma_desc_sw128(b0 + off_b), kIdesc,
-                                  kk > 0);
-                    }
-                    umma_commit(&a_empty[s]);        // the query tile may be overwritten
-                    umma_commit(&acc_full[buf]);     // the accumulator is ready
-                    ++ait;
-                    ++cit;
+                    ++q_loads;
+                    cur_g = w.g;
+                    cur_t = w.t;
                 }
+                const int s = (int)(it % kSStages), buf = (int)(it & 1);
+                ok = mbar_wait_sleep(&s_full[s], (int)(it / kSStages) & 1) &&
+                     mbar_wait_sleep(&acc_empty[buf], ((int)(it >> 1) & 1) ^ 1);
                 if (!ok) break;
-                umma_commit(b_empty);                // the summary tile may be overwritten
+                tc_fence_after();
+                // descriptors differ only in the start-address field (16-byte units), which
+                // the constant offsets below never carry out of (smem addresses < 256 KiB)
+                const uint64_t da = umma_desc_sw128(smem_u32(ss + s * kSBytes)), db = umma_desc_sw128(smem_u32(sq));
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off_a = (kk >> 2) * kSHalf + (kk & 3) * 32;
+                    const uint32_t off_b = (kk >> 2) * kQHalf + (kk & 3) * 32;
+                    umma_e4m3(tmem + buf * kBN, da + (off_a >> 4), db + (off_b >> 4), kIdesc, kk > 0);
+                }
+                umma_commit(&s_empty[s]);            // the summary block may be overwritten
+                umma_commit(&acc_full[buf]);         // the accumulator is ready
             }
         }
     } else {
-        // ---------------- epilogue: warps 2..5, TMEM lane quarter sp = warp % 4
-        const int sp = warp & 3;
-        const int qt = sp * 8 + (lane >> 2), h = lane & 3;      // this lane's row: query in tile, head
-        const int cb = 16 * (h & 1) + 8 * ((h >> 1) & 1);        // its 8 finished columns in a chunk
-        float *wscale = sscale_all + (warp - 2) * kBN;
-        int cit = 0;
-        for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-            int g, rb, t0, t1;
-            unit_coords(p, u, g, rb, t0, t1);
-            if (!unit_active(p, t0, t1, rb)) continue;
-            // this unit's 256 region scales / 16, staged by each warp in its own smem slice
-            // (no barrier across the epilogue warps); entries past the pool read as 0
-            {
-                const int64_t s0 = g * p.n_slots + base + (int64_t)rb * kBN;
-                const int64_t lim = (int64_t)kG * p.n_slots;
-#pragma unroll
-                for (int j = 0; j < kBN / 32; ++j) {
-                    const int64_t i = s0 + j * 32 + lane;
-                    wscale[j * 32 + lane] = i < lim ? __ldg(p.scales + i) * 0.0625f : 0.0f;
+        // ---------------- epilogue: warps 2..17.  TMEM lane quarter sp = warp % 4 (the
+        // hardware's lane-access rule): regions 32 sp .. 32 sp + 31 of the block, one per
+        // thread; query quarter qq: queries 16 qq .. 16 qq + 15 of the tile (columns 64 qq ..)
+        const int e = warp - 2, sp = warp & 3, qq = e >> 2;
+        // z * sq / 2 of the 4 heads per query, interleaved by query pair (a, b):
+        // wsm[2 i] = {a h0, b h0, a h1, b h1}, wsm[2 i + 1] = {a h2, b h2, a h3, b h3}
+        float *wsm = reinterpret_cast<float *>(wsm_all + e * kEpiQueries);
+        int *osm = own_all + e * kEpiQueries;             // own region per query (-1: skip)
+        if (n_items > 0) {
+            Walk w;
+            walk_seek(p, lo, w);
+            int cur_g = -1, cur_t = -1, own_min = -1;
+            const int64_t qstride = (int64_t)kG * p.ld;
+            for (int64_t it = 0; it < n_items; ++it, walk_next(p, w)) {
+                if (w.g != cur_g || w.t != cur_t) {           // this warp's 16 queries
+                    __syncwarp();
+                    int o = INT_MAX;
+                    if (lane < kEpiQueries) {
+                        const int q = w.t * kQPerTile + qq * kEpiQueries + lane;
+                        float4 wv = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                        o = -1;
+                        if (q < p.nq) {
+                            const int i = q * kHI + w.g * kHeads;
+                            wv = make_float4(p.gate[i] * p.qscale[i], p.gate[i + 1] * p.qscale[i + 1],
+                                             p.gate[i + 2] * p.qscale[i + 2], p.gate[i + 3] * p.qscale[i + 3]);
+                            o = p.q_own[q];
+                        }
+                        // query lane = 2 i + c of its pair: slots 8 i + 2 h' + c of float4 2 i + h / 2
+                        float *wp = wsm + 8 * (lane >> 1) + (lane & 1);
+                        wp[0] = 0.5f * wv.x;
+                        wp[2] = 0.5f * wv.y;
+                        wp[4] = 0.5f * wv.z;
+                        wp[6] = 0.5f * wv.w;
+                        osm[lane] = o;
+                    }
+                    // blocks ending at or below every query's own region need no mask (a
+                    // query past nq or an invalid one keeps every block masked)
+                    own_min = __reduce_min_sync(0xffffffffu, o);
+                    __syncwarp();
+                    cur_g = w.g;
+                    cur_t = w.t;
                 }
-                __syncwarp();
-            }
-            for (int t = t0; t < t1; ++t) {
-                if (!tile_active(p, t, rb)) continue;
-                const int buf = cit & 1;
-                const int q = t * kQPerTile + qt;
-                const bool qv = q < p.nq;
-                const float w = qv ? p.gate[q * kHI + g * 4 + h] * p.qscale[q * kHI + g * 4 + h] : 0.0f;
-                const int own = qv ? p.q_own[q] : -1;
-                ok = mbar_wait(&acc_full[buf], (cit >> 1) & 1);
+                const int buf = (int)(it & 1), s = (int)(it % kSStages);
+                ok = mbar_wait_sleep(&acc_full[buf], (int)(it >> 1) & 1) &&
+                     mbar_wait_sleep(&s_full[s], (int)(it / kSStages) & 1);   // complete already: makes the scales visible
                 if (!ok) break;
                 tc_fence_after();
-                float *orow = p.scores + ((int64_t)q * kG + g) * p.ld;
-#pragma unroll 1
-                for (int ch = 0; ch < kBN / 32; ++ch) {
-                    float v[32];
-                    tmem_ld32(tmem + ((uint32_t)(32 * sp) << 16) + buf * kBN + ch * 32, v);
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = fmaxf(v[j], 0.0f) * w;
-                    // heads h and h^1: keep 16 columns (h&1 ? 16..31 : 0..15)
-                    float k16[16];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const float send = (h & 1) ? v[j] : v[16 + j];
-                        const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-                        k16[j] = ((h & 1) ? v[16 + j] : v[j]) + recv;
-                    }
-                    // heads {h, h^1} and {h^2, h^3}: keep 8 columns
-                    float k8[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const float send = (h & 2) ? k16[j] : k16[8 + j];
-                        const float recv = __shfl_xor_sync(0xffffffffu, send, 2);
-                        k8[j] = ((h & 2) ? k16[8 + j] : k16[j]) + recv;
-                    }
-                    const int c0 = ch * 32 + cb;
-                    const int64_t r0 = (int64_t)rb * kBN + c0;
-                    if (qv && r0 < own) {
-                        const float4 sa4 = *reinterpret_cast<const float4 *>(wscale + c0);
-                        const float4 sb4 = *reinterpret_cast<const float4 *>(wscale + c0 + 4);
-                        const float sc[8] = {sa4.x, sa4.y, sa4.z, sa4.w, sb4.x, sb4.y, sb4.z, sb4.w};
-                        if (r0 + 8 <= own && (p.ld & 3) == 0) {
-                            *reinterpret_cast<float4 *>(orow + r0) =
-                                make_float4(k8[0] * sc[0], k8[1] * sc[1], k8[2] * sc[2], k8[3] * sc[3]);
-                            *reinterpret_cast<float4 *>(orow + r0 + 4) =
-                                make_float4(k8[4] * sc[4], k8[5] * sc[5], k8[6] * sc[6], k8[7] * sc[7]);
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 8; ++j)
-                                if (r0 + j < own) orow[r0 + j] = k8[j] * sc[j];
-                        }
-                    }
+                float v0[32], v1[32];                             // columns 4q + h of queries 0-7, 8-15
+                {
+                    const uint32_t ta = tmem + ((uint32_t)(32 * sp) << 16) + buf * kBN + qq * 64;
+                    tmem_ld32x2(ta, ta + 32, v0, v1);
                 }
+                const int64_t y = w.g * p.n_slots + base + (int64_t)w.rb * kBM;
+                const float sc =                                  // scale[g][r] / 16
+                    reinterpret_cast<const float *>(ssc + s * kScaleSlot)[(int)(y & 3) + 32 * sp + lane] * 0.0625f;
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&acc_empty[buf]);
-                ++cit;
+                if (lane == 0) {
+                    mbar_arrive(&acc_empty[buf]);              // the MMA may refill this accumulator
+                    mbar_arrive(&sc_empty[s]);                 // and the producer this scale slot
+                }
+                const int r = w.rb * kBM + 32 * sp + lane;     // this thread's region
+                // streaming stores (evict first): the 1 GB of scores must not push the
+                // summaries, re-read by every query tile, out of L2
+                // per query pair (a, b): sum_h w_h / 2 * (v_h + |v_h|) = sum_h w_h ReLU(v_h)
+                // (v + |v| is exact), two queries per packed fma
+                auto emit = [&](auto masked) {
+                    float *dst = p.scores + ((int64_t)(w.t * kQPerTile + qq * kEpiQueries) * kG + w.g) * p.ld + r;
+                    const float2 sc2 = make_float2(sc, sc);
+#pragma unroll
+                    for (int j4 = 0; j4 < 4; ++j4) {
+                        const int4 o4 = reinterpret_cast<const int4 *>(osm)[j4];
+                        const int oj[4] = {o4.x, o4.y, o4.z, o4.w};
+#pragma unroll
+                        for (int u = 0; u < 4; u += 2) {
+                            const int j = 4 * j4 + u;                     // queries j, j + 1
+                            const float4 w01 = reinterpret_cast<const float4 *>(wsm)[j];
+                            const float4 w23 = reinterpret_cast<const float4 *>(wsm)[j + 1];
+                            const float *va = j < 8 ? &v0[4 * j] : &v1[4 * (j - 8)];
+                            const float *vb = va + 4;
+                            float2 acc = fmul2(make_float2(va[0] + fabsf(va[0]), vb[0] + fabsf(vb[0])),
+                                               make_float2(w01.x, w01.y));
+                            acc = ffma2(make_float2(va[1] + fabsf(va[1]), vb[1] + fabsf(vb[1])),
+                                        make_float2(w01.z, w01.w), acc);
+                            acc = ffma2(make_float2(va[2] + fabsf(va[2]), vb[2] + fabsf(vb[2])),
+                                        make_float2(w23.x, w23.y), acc);
+                            acc = ffma2(make_float2(va[3] + fabsf(va[3]), vb[3] + fabsf(vb[3])),
+                                        make_float2(w23.z, w23.w), acc);
+                            acc = fmul2(acc, sc2);
+                            // streaming stores (evict first): the 1 GB of scores must not push
+                            // the summaries, re-read by every query tile, out of L2
+                            if (!decltype(masked)::value || r < oj[u]) __stcs(dst, acc.x);
+                            if (!decltype(masked)::value || r < oj[u + 1]) __stcs(dst + qstride, acc.y);
+                            dst += 2 * qstride;
+                        }
+                    }
+                };
+                if (w.rb * kBM + kBM <= own_min)
+                    emit(std::integral_constant<bool, false>());
+                else
+                    emit(std::integral_constant<bool, true>());
             }
-            __syncwarp();                                   // the slice is rewritten by the next unit
         }
     }
     // every role done (or gave up): release TMEM
