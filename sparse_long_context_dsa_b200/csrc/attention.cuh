@@ -226,22 +226,30 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint32_t kt = smem_u32(ring + slot * kPairBytes);
         const uint32_t vt = kt + 2 * kRegionBytes;
 
-        float s[2][4];
+        // S = Q K^T: even and odd k-steps accumulate separately (four independent mma chains
+        // of 6 instead of two of 12), summed at the end
+        float s[2][4], s2[2][4];
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
             s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.0f;
-            const uint32_t tile = kt + nt * kRegionBytes;
-            const int r = lane & 7;
+            s2[nt][0] = s2[nt][1] = s2[nt][2] = s2[nt][3] = 0.0f;
+        }
 #pragma unroll
-            for (int kp = 0; kp < 6; ++kp) {       // two k-steps (32 dims) per ldmatrix.x4
+        for (int kp = 0; kp < 6; ++kp) {           // two k-steps (32 dims) per ldmatrix.x4
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
                 const int c = kp * 32 + 8 * (lane >> 3);
                 uint32_t b0, b1, b2, b3;
-                ldmatrix_x4(tile + swz(r, c), b0, b1, b2, b3);
+                ldmatrix_x4(kt + nt * kRegionBytes + swz(lane & 7, c), b0, b1, b2, b3);
                 mma_bf16_16816(s[nt], qa[2 * kp][0], qa[2 * kp][1], qa[2 * kp][2], qa[2 * kp][3], b0, b1);
-                mma_bf16_16816(s[nt], qa[2 * kp + 1][0], qa[2 * kp + 1][1], qa[2 * kp + 1][2], qa[2 * kp + 1][3],
+                mma_bf16_16816(s2[nt], qa[2 * kp + 1][0], qa[2 * kp + 1][1], qa[2 * kp + 1][2], qa[2 * kp + 1][3],
                                b2, b3);
             }
         }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) s[nt][e] += s2[nt][e];
         // scale, mask, online softmax (rows gq and gq+8 of this lane)
         float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll

@@ -172,22 +172,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < wpt; ++i)
                 if (w0 + i < words) n += __popc(bitmap[w0 + i]);
             const uint32_t incl = topkc::block_scan_incl<kThreads>(n, scan_ws);
-            uint32_t pos = incl - n;
-            for (int i = 0; i < wpt; ++i) {
-                if (w0 + i >= words) break;
-                uint32_t b = bitmap[w0 + i];
-                while (b) {
-                    const int bit = __ffs(b) - 1;
-                    b &= b - 1;
-                    if (pos < (uint32_t)kMaxUnion) uni[pos] = (w0 + i) * 32 + bit;
-                    ++pos;
+            // stream the union only when it is at most twice the longest selection (the queries
+            // share most regions); otherwise these rows go to the per-row kernel that runs next,
+            // decided before the union is compacted
+            int maxc = 0;
+            for (int w = 0; w < kQueries; ++w)
+                if (sh_req[w] == R) maxc = max(maxc, sh_cnt[w]);
+            const uint32_t total = scan_ws[kThreads / 32 - 1];
+            if (p.row_shared == nullptr || total <= 2u * (uint32_t)maxc) {
+                uint32_t pos = incl - n;
+                for (int i = 0; i < wpt; ++i) {
+                    if (w0 + i >= words) break;
+                    uint32_t b = bitmap[w0 + i];
+                    while (b) {
+                        const int bit = __ffs(b) - 1;
+                        b &= b - 1;
+                        if (pos < (uint32_t)kMaxUnion) uni[pos] = (w0 + i) * 32 + bit;
+                        ++pos;
+                    }
                 }
             }
             if (tid == kThreads - 1) sh_union = (int)min(incl, (uint32_t)kMaxUnion);
         }
         __syncthreads();
-        // stream the union only when it is at most twice the longest selection (the queries share
-        // most regions); otherwise these rows go to the per-row kernel that runs next
         int maxc = 0;
         for (int w = 0; w < kQueries; ++w)
             if (sh_req[w] == R) maxc = max(maxc, sh_cnt[w]);
