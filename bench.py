@@ -46,7 +46,10 @@ KERNELS_PER_STEP = 4      # compress, scan (+ chunk maxima), cluster top-k, clus
 # current scan kernel (dram__bytes_read.sum + dram__bytes_write.sum); None once the kernel changes
 SCAN_TRAFFIC_BYTES = 136_391_168 + 3_656_960
 PREFILL_CTX, PREFILL_NEW = 262144, 2048
-PREFILL_KERNELS = 6       # compress, quantize, GEMM, top-k histogram, top-k select, attention
+PREFILL_KERNELS = 6       # compress, quantize, GEMM, top-k, shared-selection attention, per-row attention
+# DRAM bytes (read + write) of one gemm_scores_kernel launch on the prefill workload, from one
+# ncu capture of the current kernel; None once the kernel changes
+GEMM_TRAFFIC_BYTES = 150_103_808 + 1_020_655_000
 
 
 def parse():
@@ -555,7 +558,7 @@ def run_prefill(args):
         "roofline": {"kernel": "indexer GEMM (quantize + gemm_scores_kernel)", "bound": "tensor",
                      "achieved": f_idx / t_gemm / 1e12, "peak": fp8_peak, "unit": "TFLOP/s",
                      "frac": f_idx / t_gemm / 1e12 / fp8_peak, "peak_kind": kind, "flops_per_launch": f_idx,
-                     "traffic": None},
+                     "traffic": GEMM_TRAFFIC_BYTES},
         "attention": {"flops": f_att, "tflops": f_att / (stage[3] / args.steps * 1e-3) / 1e12,
                       "peak_bf16": tensor_peak(fp8=False)[0]},
         "e2e": {"value": PREFILL_NEW * args.steps / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
