@@ -7,10 +7,11 @@
 // (32 regions x 6 KiB, TMA with the 128-byte swizzle into 16 pair buffers, one mbarrier per
 // pair), so a CTA waits for one memory round trip, not one per pair.  Its 8 warps take two
 // pairs each: S = Q K^T and O += P V on mma.sync m16n8k16 bf16 with fp32 accumulation and an
-// exp2 online softmax, tokens t <= p only.  The warps merge (max, sum, O) in smem; then, after
-// a cluster barrier, CTA r merges head r of the row over the cluster's CTAs through
-// distributed shared memory (O = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c) and writes
-// the bf16 output and the LSE.  No partials in global memory, no second kernel.
+// exp2 online softmax, tokens t <= p only.  The warps merge (max, sum, O) in smem and the
+// CTA pushes head h of its result into CTA h's inbox through distributed shared memory; after
+// one cluster barrier CTA r merges head r of the row from its own inbox (O = sum_c 2^(m_c - M)
+// O_c / sum_c 2^(m_c - M) l_c) and writes the bf16 output and the LSE.  No partials in global
+// memory, no second kernel.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -36,9 +37,10 @@ constexpr int kRow = kD + 8;                   // padded merge row (floats)
 constexpr size_t kPairArea = (size_t)kPairs * kPairBytes;                 // 192 KiB
 constexpr size_t kMergeO = (size_t)kWarps * 16 * kRow * 4;               // per-warp O for the merge
 constexpr size_t kMergeMl = (size_t)kWarps * 16 * 2 * 4;
-constexpr size_t kOffFinal = kMergeO + kMergeMl + 1024;                   // CTA result: O [16][kD], m [16], l [16]
-static_assert(kOffFinal + (16 * kD + 32) * 4 <= kPairArea, "merge buffers fit in the pair area");
-constexpr size_t kSmemBytes = 1024 + kPairArea + kQBytes + 256;
+static_assert(kMergeO + kMergeMl + 16 * kWarps * 4 <= kPairArea, "merge buffers fit in the pair area");
+constexpr int kInRow = kD + 4;                 // inbox row per source CTA: O [kD], m, l, pad
+constexpr size_t kInbox = (size_t)kSplits * kInRow * 4;                  // outside the pair area
+constexpr size_t kSmemBytes = 1024 + kPairArea + kQBytes + 256 + kInbox;
 constexpr int kMaxK = kSplits * kRegionsPerCta;                            // 512
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -51,26 +53,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *qs = smem + kPairArea;
     uint64_t *bars = reinterpret_cast<uint64_t *>(qs + kQBytes);            // [kPairs]
+    float *inbox = reinterpret_cast<float *>(qs + kQBytes + 256);           // [kSplits][kInRow]
     __shared__ int sh_y[kRegionsPerCta], sh_r[kRegionsPerCta], sh_v[kRegionsPerCta];   // per region of the CTA
-    __shared__ float cw[kSplits], cl[kSplits], cstat[2];
 
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
     const int row = blockIdx.y;                                             // query * 4 + group
     const int qi = row >> 2, g = row & 3;
+    // the loads that depend on nothing else go out first: the Q tile (into registers, stored
+    // to smem once the K/V loads are issued) and this warp's selection entries, beside the
+    // selection count
+    const __nv_bfloat16 *qsrc = p.q + ((int64_t)qi * kHQ + g * kHeadsPerGroup) * kD;
+    constexpr int kQChunks = 16 * kD / 8;                                   // 384 16-byte chunks
+    uint4 qv[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int i = tid + u * kThreads;
+        if (i < kQChunks) qv[u] = __ldg(reinterpret_cast<const uint4 *>(qsrc + (i / (kD / 8)) * kD + (i % (kD / 8)) * 8));
+    }
+    auto reg_of = [&](int l) { return (l >> 1) * 16 + 2 * warp + (l & 1); };   // lane l < 4 -> region
+    const int j0 = rank * kRegionsPerCta;
+    int rr_spec = -1;
+    if (lane < 4 && j0 + reg_of(lane) < p.k) rr_spec = p.sel_idx[(int64_t)row * p.k + j0 + reg_of(lane)];
     const int b = p.q_req ? p.q_req[qi] : qi;
     const int pos = p.q_pos[qi];
     const int cnt_raw = p.sel_count[row];
     const int cnt = min(max(cnt_raw, 0), p.k);
     if (cnt != cnt_raw && rank == 0 && tid == 0) set_error(kErrAttnIndex);
-    const int j0 = rank * kRegionsPerCta;
     const int nr = max(0, min(kRegionsPerCta, cnt - j0));                   // regions of this CTA
     const bool bad_req = (b < 0 || b >= p.n_req || pos < 0);
     // Warp w owns pairs w and w + 8 (regions 2w, 2w+1, 2w+16, 2w+17 of the CTA): it sets up
     // their barriers, resolves their coordinates (sel_idx -> block_table, lanes 0..3) and
     // issues their TMA loads itself, so the 8 warps issue in parallel.
-    auto reg_of = [&](int l) { return (l >> 1) * 16 + 2 * warp + (l & 1); };   // lane l < 4 -> region
     if (lane < 2) mbar_init(&bars[warp + 8 * lane], 1);
     fence_mbar_init();
     __syncwarp();
@@ -78,7 +93,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int j = reg_of(lane);
         int y = 0, r = -1, v = 0;
         if (!bad_req && j < nr) {
-            const int rr = p.sel_idx[(int64_t)row * p.k + j0 + j];
+            const int rr = rr_spec;
             if (rr < 0 || rr / 8 >= p.max_pages) {
                 set_error(kErrAttnIndex);
             } else {
@@ -119,11 +134,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_3d(dst + (2 + half) * kRegionBytes, &tmap_v, 0, 0, sh_y[j], &bars[pr]);
         }
     }
-    // Q tile [16 heads][192] into smem with the K/V tiles' swizzled layout: 384 16-byte chunks
-    const __nv_bfloat16 *qsrc = p.q + ((int64_t)qi * kHQ + g * kHeadsPerGroup) * kD;
-    for (int i = tid; i < 16 * kD / 8; i += kThreads) {
-        const uint4 qv = __ldg(reinterpret_cast<const uint4 *>(qsrc + (i / (kD / 8)) * kD + (i % (kD / 8)) * 8));
-        *reinterpret_cast<uint4 *>(qs + swz(i / (kD / 8), (i % (kD / 8)) * 8)) = qv;
+    // Q tile [16 heads][192] into smem with the K/V tiles' swizzled layout
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int i = tid + u * kThreads;
+        if (i < kQChunks) *reinterpret_cast<uint4 *>(qs + swz(i / (kD / 8), (i % (kD / 8)) * 8)) = qv[u];
     }
     __syncthreads();
 
@@ -243,8 +258,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     float *red_o = reinterpret_cast<float *>(smem);                          // [8][16][kRow]
     float *red_ml = red_o + kWarps * 16 * kRow;                              // [8][16][2]
-    float *fin_o = reinterpret_cast<float *>(smem + kOffFinal);              // [16][kD]
-    float *fin_m = fin_o + 16 * kD, *fin_l = fin_m + 16;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const int hr = gq + 8 * h;
@@ -259,6 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
     float *wts = red_ml + kWarps * 16 * 2;                                   // [16][8]
+    // this CTA's (m, l) of head hr and its O row go to CTA hr's inbox row `rank`
     if (tid < 16) {
         const int hr = tid;
         float M = -INFINITY;
@@ -272,8 +286,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             wts[hr * kWarps + w] = wt;
             L += wt * red_ml[(w * 16 + hr) * 2 + 1];
         }
-        fin_m[hr] = M;
-        fin_l[hr] = L;
+        float *dst = cluster.map_shared_rank(inbox, hr) + rank * kInRow + kD;
+        dst[0] = M;
+        dst[1] = L;
     }
     __syncthreads();
     for (int e = tid; e < 16 * kD / 4; e += kThreads) {
@@ -288,50 +303,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             acc.z += wt * v.z;
             acc.w += wt * v.w;
         }
-        *reinterpret_cast<float4 *>(fin_o + hr * kD + d) = acc;
+        *reinterpret_cast<float4 *>(cluster.map_shared_rank(inbox, hr) + rank * kInRow + d) = acc;
     }
-    cluster.sync();                                                          // every CTA's result in place
-
-    // ---- CTA `rank` merges head `rank` of the row over the cluster
-    const int hr = rank;
-    if (tid < kSplits) {
-        cw[tid] = cluster.map_shared_rank(fin_m, tid)[hr];
-        cl[tid] = cluster.map_shared_rank(fin_l, tid)[hr];
-    }
-    __syncthreads();
-    if (tid == 0) {
-        float M = -INFINITY;
-        for (int c = 0; c < kSplits; ++c) M = fmaxf(M, cw[c]);
-        const float Mref = (M == -INFINITY) ? 0.0f : M;
-        float L = 0.0f;
-        for (int c = 0; c < kSplits; ++c) {
-            const float wt = exp2f(cw[c] - Mref);
-            L += wt * cl[c];
-            cw[c] = wt;
-        }
-        cstat[0] = M;
-        cstat[1] = L;
-    }
-    __syncthreads();
-    float acc = 0.0f;
-    if (tid < kD) {
-        float v[kSplits];
-#pragma unroll
-        for (int c = 0; c < kSplits; ++c) v[c] = cluster.map_shared_rank(fin_o, c)[hr * kD + tid];
-#pragma unroll
-        for (int c = 0; c < kSplits; ++c) acc += cw[c] * v[c];
-    }
-    // every remote read is done: let the other CTAs go while this one writes
+    // every CTA's rows are in the inboxes; afterwards no CTA touches another's smem
     asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+
+    // ---- CTA `rank` merges head `rank` of the row from its inbox
+    const int hr = rank;
     if (tid < kD) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < kSplits; ++c) M = fmaxf(M, inbox[c * kInRow + kD]);
+        const float Mref = (M == -INFINITY) ? 0.0f : M;
+        float L = 0.0f, acc = 0.0f;
+#pragma unroll
+        for (int c = 0; c < kSplits; ++c) {
+            const float wt = exp2f(inbox[c * kInRow + kD] - Mref);
+            L += wt * inbox[c * kInRow + kD + 1];
+            acc += wt * inbox[c * kInRow + tid];
+        }
         const int d = tid;
-        const float L = cstat[1];
         const int head = g * kHeadsPerGroup + hr;
         p.out[((int64_t)qi * kHQ + head) * kD + d] = __float2bfloat16_rn(L > 0.0f ? acc / L : 0.0f);
-        if (p.lse && d == 0)
-            p.lse[(int64_t)qi * kHQ + head] = (L > 0.0f) ? (cstat[0] + log2f(L)) * 0.69314718055994531f : -INFINITY;
+        if (p.lse && d == 0) p.lse[(int64_t)qi * kHQ + head] = (L > 0.0f) ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
     }
-    asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");   // no CTA leaves while others read it
 }
 
 }  // namespace attnc

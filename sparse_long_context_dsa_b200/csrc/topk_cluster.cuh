@@ -429,6 +429,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = blockIdx.y;
     const int tid = threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
+    // kMaxima: this thread's 8 chunk maxima go out with the query position (entries past the
+    // row's eligible chunks are masked once the position is known)
+    float4 cm_a = make_float4(0.f, 0.f, 0.f, 0.f), cm_b = cm_a;
+    if constexpr (kMaxima) {
+        if ((int64_t)tid * 8 + 8 <= cm_stride) {
+            const float4 *cm4 = reinterpret_cast<const float4 *>(chunk_max + (int64_t)row * cm_stride + tid * 8);
+            cm_a = __ldcg(cm4);
+            cm_b = __ldcg(cm4 + 1);
+        }
+    }
 
     // ---- loads: this thread's group is the CTA's entries tid, tid+512, ... (coalesced)
     const int p = q_pos[row >> 2];
@@ -566,13 +576,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // lower edge L of a range holding the need-th largest maximum and at most 64 maxima
             uint32_t mk[kM];
             {
-                float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
-                if (tid * kM < n_ch) {
-                    const float4 *cm4 = reinterpret_cast<const float4 *>(chunk_max + (int64_t)row * cm_stride + tid * kM);
-                    a = __ldcg(cm4);
-                    b = __ldcg(cm4 + 1);
-                }
-                const float mv[kM] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+                static_assert(kM == 8, "two float4 of chunk maxima per thread");
+                const float mv[kM] = {cm_a.x, cm_a.y, cm_a.z, cm_a.w, cm_b.x, cm_b.y, cm_b.z, cm_b.w};
 #pragma unroll
                 for (int u = 0; u < kM; ++u) mk[u] = tid * kM + u < n_ch ? score_key(mv[u]) : 0u;
             }
