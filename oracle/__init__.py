@@ -11,6 +11,7 @@ Functions mirror the library's C-ABI calls:
   indexer_scores     A2  16-head indexer score        sum_h z_h ReLU(q_h . s)/16
   topk_regions       A3  own region + top-(k-1)       ties -> lower index
   sparse_attention   A4  exact GQA over the selection softmax(q K^T / sqrt(192)) V
+  window_attention       the window layers: the same over the last `window` tokens
 plus the number-format helpers the pins use (bf16 and OCP E4M3 codecs).
 """
 from __future__ import annotations
@@ -81,6 +82,11 @@ def lib():
                 _P(ctypes.c_int32), ctypes.c_int, _P(ctypes.c_int32), _P(ctypes.c_int32),
                 ctypes.c_int, _P(ctypes.c_int32), _P(ctypes.c_int32), ctypes.c_int,
                 _P(ctypes.c_uint16), _P(ctypes.c_float), _P(ctypes.c_double)]
+            L.oracle_window_attention.restype = None
+            L.oracle_window_attention.argtypes = [
+                _P(ctypes.c_uint16), _P(ctypes.c_uint16), _P(ctypes.c_uint16),
+                _P(ctypes.c_int32), ctypes.c_int, _P(ctypes.c_int32), _P(ctypes.c_int32),
+                ctypes.c_int, ctypes.c_int, _P(ctypes.c_uint16), _P(ctypes.c_float), _P(ctypes.c_double)]
             L.oracle_set_threads.restype = None
             L.oracle_set_threads.argtypes = [ctypes.c_int]
             L.oracle_get_threads.restype = ctypes.c_int
@@ -246,6 +252,47 @@ def sparse_attention(q_bits, k_cache_bits, v_cache_bits, block_table, q_req, q_p
         _ptr(bt, ctypes.c_int32), max_pages, _ptr(qr, ctypes.c_int32), _ptr(qp, ctypes.c_int32),
         nq, _ptr(si, ctypes.c_int32), _ptr(sc, ctypes.c_int32), k, _ptr(out, ctypes.c_uint16),
         _ptr(lse, ctypes.c_float), _ptr(o64, ctypes.c_double) if want_f64 else None)
+    if want_f64:
+        return out, lse, o64
+    return out, lse
+
+
+def window_attention(q_bits, k_cache_bits, v_cache_bits, block_table, q_req, q_pos, window=512,
+                     want_f64=False):
+    """Sliding-window GQA of the window layers ([P1] §滑窗注意力; [P2] §第一招: the last 512
+    tokens, kept in a ring buffer): query i attends tokens max(0, p - window + 1) .. p of its
+    request through the block table.  q uint16 [nq][64][192]; caches uint16
+    [pages][4][64][192]; block_table int32 [B][max_pages].  Returns (out bf16 bits
+    [nq][64][192], lse float32 [nq][64][, out float64])."""
+    q = _arr(q_bits, np.uint16)
+    kc = _arr(k_cache_bits, np.uint16)
+    vc = _arr(v_cache_bits, np.uint16)
+    bt = _arr(np.asarray(block_table, np.int32), np.int32)
+    qr = _arr(np.asarray(q_req, np.int32), np.int32)
+    qp = _arr(np.asarray(q_pos, np.int32), np.int32)
+    if window < 1:
+        raise ValueError("window must be >= 1")
+    nq = int(q.shape[0])
+    max_pages = int(bt.shape[1])
+    n_pages = int(kc.shape[0])
+    for i in range(nq):
+        p = int(qp[i])
+        if p < 0:
+            continue
+        lo = max(0, p - window + 1)
+        if p // PAGE >= max_pages:
+            raise ValueError("window token beyond the block table")
+        pages = bt[qr[i], lo // PAGE: p // PAGE + 1]
+        if pages.min() < 0 or pages.max() >= n_pages:
+            raise ValueError("page index out of range")
+    out = np.empty((nq, HQ, D), np.uint16)
+    lse = np.empty((nq, HQ), np.float32)
+    o64 = np.empty((nq, HQ, D), np.float64) if want_f64 else None
+    lib().oracle_window_attention(
+        _ptr(q, ctypes.c_uint16), _ptr(kc, ctypes.c_uint16), _ptr(vc, ctypes.c_uint16),
+        _ptr(bt, ctypes.c_int32), max_pages, _ptr(qr, ctypes.c_int32), _ptr(qp, ctypes.c_int32),
+        nq, int(window), _ptr(out, ctypes.c_uint16), _ptr(lse, ctypes.c_float),
+        _ptr(o64, ctypes.c_double) if want_f64 else None)
     if want_f64:
         return out, lse, o64
     return out, lse

@@ -16,6 +16,7 @@
  *   A2 indexer score         [P1 §DSA ③], [P2 §索引器打分]
  *   A3 top-k region select   [P2 §索引器打分], [P2 §第二招 sparse_config table]
  *   A4 sparse GQA attention  [P1 §DSA ④], [P2 §索引器打分], [P3 §一]
+ *   sliding-window attention of the window layers [P1 §滑窗注意力], [P2 §第一招]
  * The pages leave the arithmetic open; the fixed reading is:
  *   summary = mean of the 8 tokens' bf16 index_k, e4m3 with one fp32 absmax/448 scale;
  *   score(r,g) = sum_{h in group g} z_h * ReLU(q_h . s_{r,g}) / 16, heads 4g..4g+3;
@@ -357,6 +358,69 @@ void oracle_sparse_attention(const uint16_t *q, const uint16_t *k_cache, const u
             double den = 0.0;
             for (int i = 0; i < ntok; ++i) { lg[i] = exp(lg[i] - mx); den += lg[i]; }
             for (int i = 0; i < ntok; ++i) {
+                double w = lg[i] / den;
+                for (int d = 0; d < OR_D; ++d) o[d] += w * oracle_bf16_to_f64(v_cache[rows[i] + d]);
+            }
+            l = mx + log(den);
+        }
+        uint16_t *ov = out + ((int64_t)qi * OR_HQ + h) * OR_D;
+        for (int d = 0; d < OR_D; ++d) ov[d] = oracle_f64_to_bf16(o[d]);
+        if (out_f64) for (int d = 0; d < OR_D; ++d) out_f64[((int64_t)qi * OR_HQ + h) * OR_D + d] = o[d];
+        if (lse) lse[(int64_t)qi * OR_HQ + h] = (float)l;
+        free(rows);
+        free(lg);
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* sliding-window attention (the 69 window layers)                      */
+/* ------------------------------------------------------------------ */
+
+/* Same cache layout as oracle_sparse_attention.  Query qi (request q_req, position p)
+ * attends, for head h in group g = h/16, every token of the window
+ *   T = { t : max(0, p - window + 1) <= t <= p },
+ * the window's tokens read through the block table (a ring buffer is a block table
+ * that maps the request's pages cyclically onto a few physical pages).
+ *   o_h = sum_t softmax_t(q_h . k_t / sqrt(192)) v_t,  lse_h = log sum_t exp(...)
+ * in double; out rounded once to bf16, lse to fp32.  [P1 §滑窗注意力]: the window layers
+ * read only the most recent 512 tokens; [P2 §第一招]: sliding_window 512, a ring buffer
+ * that keeps each request's last 512 tokens, attention inside the window. */
+void oracle_window_attention(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                             const int32_t *block_table, int max_pages,
+                             const int32_t *q_req, const int32_t *q_pos, int nq, int window,
+                             uint16_t *out, float *lse, double *out_f64)
+{
+    const double inv_sqrt_d = 1.0 / sqrt((double)OR_D);
+#pragma omp parallel for schedule(dynamic)
+    for (int qh = 0; qh < nq * OR_HQ; ++qh) {
+        int qi = qh / OR_HQ, h = qh % OR_HQ, g = h / (OR_HQ / OR_G);
+        int b = q_req[qi], p = q_pos[qi];
+        int64_t lo = (int64_t)p - window + 1;
+        if (lo < 0) lo = 0;
+        int n = p >= 0 ? (int)(p - lo + 1) : 0;
+        const uint16_t *qv = q + ((int64_t)qi * OR_HQ + h) * OR_D;
+        double qd[OR_D];
+        for (int d = 0; d < OR_D; ++d) qd[d] = oracle_bf16_to_f64(qv[d]);
+        int64_t *rows = (int64_t *)malloc(sizeof(int64_t) * (size_t)(n + 1));
+        double *lg = (double *)malloc(sizeof(double) * (size_t)(n + 1));
+        for (int i = 0; i < n; ++i) {
+            int64_t t = lo + i;
+            int64_t page = block_table[(int64_t)b * max_pages + t / OR_PAGE];
+            int64_t row = ((page * OR_G + g) * OR_PAGE + t % OR_PAGE) * OR_D;
+            double dot = 0.0;
+            for (int d = 0; d < OR_D; ++d) dot += qd[d] * oracle_bf16_to_f64(k_cache[row + d]);
+            rows[i] = row;
+            lg[i] = dot * inv_sqrt_d;
+        }
+        double o[OR_D];
+        for (int d = 0; d < OR_D; ++d) o[d] = 0.0;
+        double l = -INFINITY;
+        if (n > 0) {
+            double mx = lg[0];
+            for (int i = 1; i < n; ++i) if (lg[i] > mx) mx = lg[i];
+            double den = 0.0;
+            for (int i = 0; i < n; ++i) { lg[i] = exp(lg[i] - mx); den += lg[i]; }
+            for (int i = 0; i < n; ++i) {
                 double w = lg[i] / den;
                 for (int d = 0; d < OR_D; ++d) o[d] += w * oracle_bf16_to_f64(v_cache[rows[i] + d]);
             }
