@@ -61,8 +61,8 @@ def parse():
     ap.add_argument("--layers", type=int, default=N_LAYERS)
     ap.add_argument("--cpu-queries", type=int, default=3, help="oracle queries timed for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["decode_b1_1m", "prefill_2k_256k", "prefill_2k_256k_local"],
-                    default="decode_b1_1m")
+    ap.add_argument("--workload", choices=["decode_b1_1m", "prefill_2k_256k", "prefill_2k_256k_local",
+                                           "swa_decode_b8"], default="decode_b1_1m")
     return ap.parse_args()
 
 
@@ -569,6 +569,142 @@ def run_prefill(args):
     print(json.dumps(line), flush=True)
 
 
+SWA_BATCH, SWA_LAYERS, SWA_WINDOW, SWA_RING = 8, 69, 512, 8
+
+
+def swa_bytes_per_query() -> int:
+    """Algorithmic bytes of one window-layer decode query: the window's K and V (512 tokens
+    x 4 groups x 192 x 2 B each), Q and O (64 x 192 x 2 B each), the new token's K and V read
+    and written into the ring (4 x 192 x 2 B each, twice)."""
+    kv = SWA_WINDOW * 4 * 192 * 2 * 2
+    qo = 2 * 64 * 192 * 2
+    new = 2 * 2 * 4 * 192 * 2
+    return kv + qo + new
+
+
+def run_swa(args):
+    """Decode of the window layers ([P1] §滑窗注意力: 69 of 92 layers attend the last 512
+    tokens from a ring buffer): a step is one layer for a batch of 8 requests at ~1M
+    positions, the new tokens appended to each request's ring and attended over their last
+    512 tokens; steps rotate through 69 layers' rings (868 MB, larger than L2)."""
+    import numpy as np
+    import torch
+    from sparse_long_context_dsa_b200 import dsa, pipeline
+
+    import torch.distributed as dist
+    from sparse_long_context_dsa_b200 import replicas
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dsa.lib()
+    g = torch.Generator(device=dev)
+    g.manual_seed(1240 + rank)
+    max_pages = (L_CTX + 64) // 64 + 1
+    bt = pipeline.ring_block_table(SWA_BATCH, max_pages, SWA_RING, dev)
+    layers = []
+    for _ in range(SWA_LAYERS):
+        kr = torch.randn((SWA_BATCH * SWA_RING, 4, 64, 192), generator=g, device=dev).to(torch.bfloat16)
+        vr = torch.randn(kr.shape, generator=g, device=dev).to(torch.bfloat16)
+        st = pipeline.WindowDecodeStep(kr, vr, bt, SWA_WINDOW)
+        st.load(torch.randn((SWA_BATCH, 64, 192), generator=g, device=dev).to(torch.bfloat16),
+                torch.randn((SWA_BATCH, 4, 192), generator=g, device=dev).to(torch.bfloat16),
+                torch.randn((SWA_BATCH, 4, 192), generator=g, device=dev).to(torch.bfloat16),
+                torch.full((SWA_BATCH,), L_CTX - 1, dtype=torch.int32, device=dev))
+        layers.append(st)
+    for i in range(max(args.warmup, 3)):
+        layers[i % SWA_LAYERS].run()
+    torch.cuda.synchronize()
+    dsa.check_device()
+
+    def graph(n):
+        gr = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(gr, stream=s):
+                for i in range(n):
+                    layers[i % SWA_LAYERS].run()
+        torch.cuda.current_stream().wait_stream(s)
+        return gr
+
+    n = args.steps
+    gr = graph(n)
+    gr.replay()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    replicas.barrier()
+    with sampler:
+        torch.cuda.synchronize()
+        t0.record()
+        gr.replay()
+        t1.record()
+        torch.cuda.synchronize()
+    dsa.check_device()
+    ms = replicas.max_over_ranks(t0.elapsed_time(t1), dev)
+    step_us = ms * 1e3 / n
+    bytes_step = SWA_BATCH * swa_bytes_per_query()
+    peak, kind = peaks()
+    achieved = bytes_step / (step_us * 1e-6) / 1e9
+    # e2e: per step the inputs from pinned host memory and the output back, through the calls
+    host = [dict(q=st.q.cpu().pin_memory(), k=st.new_k.cpu().pin_memory(), v=st.new_v.cpu().pin_memory(),
+                 pos=st.q_pos.cpu().pin_memory()) for st in layers[:4]]
+    out_host = torch.empty((SWA_BATCH, 64, 192), dtype=torch.bfloat16).pin_memory()
+    n_e2e = min(n, 400)
+    torch.cuda.synchronize()
+    t0.record()
+    for i in range(n_e2e):
+        st, h = layers[i % SWA_LAYERS], host[i % 4]
+        st.load(h["q"], h["k"], h["v"], h["pos"])
+        st.run()
+        out_host.copy_(st.out, non_blocking=True)
+    t1.record()
+    torch.cuda.synchronize()
+    e2e_ms = replicas.max_over_ranks(t0.elapsed_time(t1), dev)
+    h2d = sum(t.numel() * t.element_size() for t in host[0].values())
+    d2h = out_host.numel() * out_host.element_size()
+    line = {
+        "metric": "window-layer decode queries/s (8 requests at 1M context, 512-token ring)",
+        "value": world * SWA_BATCH * n / (ms / 1e3), "unit": "queries/s", "n_gpus": world, "steps": n,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms / n, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 (fp32 softmax and accumulate)", "data": "synthetic",
+        "config": {"workload": "swa_decode_b8", "batch": SWA_BATCH, "position": L_CTX - 1, "window": SWA_WINDOW,
+                   "ring_pages": SWA_RING, "layers": SWA_LAYERS,
+                   "l2": "69 layers' rings rotate (868 MB > L2)"},
+        "roofline": {"kernel": "window step (kv_append + sparse_attn_kernel + combine_kernel)", "bound": "hbm",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_kind": kind, "bytes_per_step": bytes_step, "traffic": None},
+        "e2e": {"value": world * SWA_BATCH * n_e2e / (e2e_ms / 1e3), "unit": "queries/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 3 * n,
+        "clocks": sampler.summary(),
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        import oracle
+        st = layers[0]
+        kc, vc, btc = (st.k_ring.cpu().contiguous().view(torch.int16).numpy().view(np.uint16),
+                       st.v_ring.cpu().contiguous().view(torch.int16).numpy().view(np.uint16), bt.cpu().numpy())
+        qb = st.q.cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+        qp = st.q_pos.cpu().numpy()
+        reps = 40
+        c0 = time.perf_counter()
+        for _ in range(reps):
+            oracle.window_attention(qb, kc, vc, btc, np.arange(SWA_BATCH), qp, SWA_WINDOW)
+        dt = time.perf_counter() - c0
+        line["cpu_baseline"] = {"value": reps * SWA_BATCH / dt, "unit": "queries/s", "cores": oracle.get_threads(),
+                                "kind": "oracle", "sample": f"{reps} x 8 window queries on one layer's rings"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del gr
+    if world > 1:
+        dist.destroy_process_group()
+
+
 def tensor_peak(fp8: bool):
     """Dense tensor peak in TFLOP/s: the measured cuBLAS bf16 burst figure (x2 for e4m3,
     the nominal fp8/bf16 ratio of the part), else the fallback."""
@@ -587,6 +723,8 @@ def main():
         run_reference(args)
     elif args.workload.startswith("prefill_2k_256k"):
         run_prefill(args)
+    elif args.workload == "swa_decode_b8":
+        run_swa(args)
     else:
         run_ours(args)
 

@@ -13,6 +13,9 @@
  *   dsa_topk_regions         A3  own region + top-(k-1), ties -> lower index [P2 §索引器打分]
  *   dsa_sparse_attn_decode   A4  exact GQA over the selected regions         [P1 §DSA ④][P3 §一]
  *   dsa_sparse_attn_prefill  A4  the same for a chunk of prefill queries     [P3 §一 sparse_attention_prefill]
+ * and, for the window layers beside the DSA layers:
+ *   dsa_kv_append            new tokens' K/V into their page slots (a ring with a cyclic table)
+ *   dsa_window_attn          GQA over each query's last `window` tokens      [P1 §滑窗注意力][P2 §第一招]
  *
  * Conventions (every call):
  *   - Pointers are DEVICE pointers unless stated otherwise, owned by the caller.  The
@@ -237,6 +240,38 @@ dsa_status_t dsa_sparse_attn_prefill(const void *q, const void *k_cache, const v
                                      const int32_t *sel_idx, const int32_t *sel_count, int k,
                                      void *out, float *lse, void *ws, size_t ws_bytes,
                                      dsa_stream_t stream);
+
+/* ------------------------------------------------------------------------------ */
+/* The window layers.  [P1 §滑窗注意力] 69 of the 92 layers read only the most recent 512
+ * tokens; [P2 §第一招] their cache is a ring buffer keeping each request's last 512 tokens
+ * (a new token overwrites the slot of the token 512 before it) and decode attends inside
+ * the window.  A ring is a paged cache whose block table maps a request's virtual pages
+ * cyclically onto a few physical pages: with 8 pages of 64 tokens (block_table[b][v] =
+ * ring page (v mod 8) of b) token t lands on the slot of token t - 512.
+ *
+ * dsa_kv_append: writes token i's K and V rows (new_k, new_v bf16 [n][4][192]) to row
+ * q_pos[i] % 64 of page block_table[b*max_pages + q_pos[i]/64], b = q_req[i] (q_req NULL:
+ * b = i).  Caches as for dsa_sparse_attn_decode.  A position beyond the block table or a
+ * page outside [0, n_pages) is skipped and flags DSA_ERR_DEVICE.  Tokens of one call must
+ * not share a slot.
+ *
+ * dsa_window_attn: for query q (request b = q_req[q], or q when q_req is NULL; position
+ * p = q_pos[q]) and head h (group g = h/16), T = { t : max(0, p - window + 1) <= t <= p },
+ * read through the block table:
+ *   out[q][h] = sum_{t in T} softmax_t(q[q][h] . K_t / sqrt(192)) V_t   (bf16, fp32 math)
+ *   lse[q][h] = ln sum_{t in T} exp(q[q][h] . K_t / sqrt(192))          (NULL: not written)
+ * The caller keeps every token of the window in the cache (a ring of at least `window`
+ * tokens).  1 <= window <= 2^20.  Runs on the per-row attention kernel (split across CTAs,
+ * with a merge kernel, when there are few rows); workspace dsa_window_attn_workspace_size(
+ * nq, window) bytes, 256-byte aligned (0: none needed).  Errors as for the sparse calls. */
+dsa_status_t dsa_kv_append(void *k_cache, void *v_cache, int64_t n_pages, const int32_t *block_table,
+                           int max_pages, int n_req, const int32_t *q_req, const int32_t *q_pos, int n,
+                           const void *new_k, const void *new_v, dsa_stream_t stream);
+size_t dsa_window_attn_workspace_size(int nq, int window);
+dsa_status_t dsa_window_attn(const void *q, const void *k_cache, const void *v_cache, int64_t n_pages,
+                             const int32_t *block_table, int max_pages, int n_req, const int32_t *q_req,
+                             const int32_t *q_pos, int nq, int window, void *out, float *lse, void *ws,
+                             size_t ws_bytes, dsa_stream_t stream);
 
 #ifdef __cplusplus
 }

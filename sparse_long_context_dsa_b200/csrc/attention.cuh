@@ -42,6 +42,7 @@ struct Params {
     float *part_o;             // [rows][n_splits][16][192]   (split mode)
     float *part_ml;            // [rows][n_splits][16][2]
     uint8_t *row_shared;       // nullable [nq][4]: 1 = the row was served by the shared-selection kernel
+    int window;                // 0: the selection (sel_idx, sel_count); > 0: the last `window` tokens
     int64_t n_pages;
     int max_pages;
     int n_req;
@@ -58,6 +59,25 @@ __device__ __forceinline__ uint32_t swz(int row, int col)
 {
     const int blk = col >> 6, c16 = (col & 63) >> 3, line = row * 3 + blk;
     return (uint32_t)(line * 128 + ((c16 ^ (line & 7)) << 4) + (col & 7) * 2);
+}
+
+// The rows' regions: the selection, or (window mode) the regions holding tokens
+// max(0, pos - window + 1) .. pos, whose first token is the window's lower bound.
+__device__ __forceinline__ int window_lo(const Params &p, int pos)
+{
+    return p.window > 0 ? max(0, pos - p.window + 1) : 0;
+}
+
+__device__ __forceinline__ int row_count(const Params &p, int row, int pos, bool &bad)
+{
+    if (p.window > 0) {
+        bad = false;
+        return pos < 0 ? 0 : (pos >> 3) - (window_lo(p, pos) >> 3) + 1;   // <= p.k (host-checked)
+    }
+    const int raw = p.sel_count[row];
+    const int c = min(max(raw, 0), p.k);     // never index past the row of sel_idx
+    bad = c != raw;
+    return c;
 }
 
 __global__ void __launch_bounds__(kThreads, 2)
@@ -82,9 +102,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (p.row_shared && p.row_shared[row]) return;
     const int b = p.q_req ? p.q_req[qi] : qi;
     const int pos = p.q_pos[qi];
-    const int cnt_raw = p.sel_count[row];
-    const int cnt = min(max(cnt_raw, 0), p.k);   // never index past the row of sel_idx
-    if (cnt != cnt_raw && split == 0 && threadIdx.x == 0) set_error(kErrAttnIndex);
+    bool bad_cnt;
+    const int cnt = row_count(p, row, pos, bad_cnt);
+    if (bad_cnt && split == 0 && threadIdx.x == 0) set_error(kErrAttnIndex);
+    const int t_lo = window_lo(p, pos);         // tokens below it are masked (window mode)
     const int j0 = split * p.rps;
     const int nr = min(p.rps, cnt - j0);   // regions of this CTA
     if (nr <= 0 && p.n_splits > 1) return; // combine_kernel ignores empty splits
@@ -94,7 +115,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int n_pairs = (max(nr, 0) + 1) >> 1;
     uint8_t *ring = smem + warp * kWarpRing;
     uint64_t *wbar = bars + warp * kSlots;
-    const int32_t *sel = p.sel_idx + (int64_t)row * p.k + j0;
+    const int32_t *sel = p.window > 0 ? nullptr : p.sel_idx + (int64_t)row * p.k + j0;
 
     // This warp handles pairs warp, warp + 4, ...; its local region q (pair q/2, half q%2)
     // is region j = 2*(warp + 4*(q/2)) + q%2 of the CTA.  Lanes resolve the coordinates of
@@ -113,7 +134,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         c_v = 0;
         c_r = -1;
         if (!bad_req && j < nr) {
-            const int r = sel[j];
+            const int r = sel ? sel[j] : (t_lo >> 3) + j0 + j;
             if (r < 0 || r / 8 >= p.max_pages) {
                 set_error(kErrAttnIndex);
             } else {
@@ -257,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int tok = 8 * rr[nt] + 2 * t + (e & 1);
-                const bool ok = rv[nt] && tok <= pos;
+                const bool ok = rv[nt] && tok <= pos && tok >= t_lo;
                 const float v = ok ? s[nt][e] * p.scale_log2 : -INFINITY;
                 s[nt][e] = v;
                 mx[e >> 1] = fmaxf(mx[e >> 1], v);
@@ -431,7 +452,8 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const Params p
     const int qi = row >> 2, g = row & 3;
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int d = tid % kD, sg = tid / kD;
-    const int cnt = min(max(p.sel_count[row], 0), p.k);
+    bool bad_cnt;
+    const int cnt = row_count(p, row, p.q_pos[qi], bad_cnt);
     const int ns = min(p.n_splits, (cnt + p.rps - 1) / p.rps);   // <= kD (host-checked)
     const int64_t pbase = (int64_t)row * p.n_splits * 16 + hr;
     float m = -INFINITY, l = 0.0f;

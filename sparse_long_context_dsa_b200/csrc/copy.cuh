@@ -26,4 +26,43 @@ __global__ void __launch_bounds__(256) copy_kernel(uint8_t *__restrict__ dst, co
     for (size_t i = done + tid; i < bytes; i += nt) dst[i] = src[i];
 }
 
+// New tokens' K and V rows written into their page slots: token i (request q_req[i], or i
+// when q_req is null, position q_pos[i]) goes to page block_table[b][pos / 64], row pos % 64,
+// all 4 groups.  With a block table that maps a request's pages cyclically onto a few physical
+// pages this is the window layers' ring buffer: a token overwrites the one `ring` tokens
+// before it ([P2] Step-5-Preview 如何实现1M长上下文 §第一招: the write goes to a fixed set of
+// slots by a modulo of the position).  One CTA per token; threads 0..95 copy K, 128..223 V.
+__global__ void __launch_bounds__(256) kv_append_kernel(__nv_bfloat16 *__restrict__ k_cache,
+                                                        __nv_bfloat16 *__restrict__ v_cache, int64_t n_pages,
+                                                        const int32_t *__restrict__ block_table, int max_pages,
+                                                        const int32_t *__restrict__ q_req, int n_req,
+                                                        const int32_t *__restrict__ q_pos, int n,
+                                                        const __nv_bfloat16 *__restrict__ new_k,
+                                                        const __nv_bfloat16 *__restrict__ new_v)
+{
+    pdl_trigger();   // the next kernel may launch; it waits for this one itself
+    pdl_wait();      // the previous kernel's results are visible from here on
+    const int i = blockIdx.x;
+    if (i >= n) return;
+    const int b = q_req ? q_req[i] : i;
+    const int pos = q_pos[i];
+    if (b < 0 || b >= n_req || pos < 0 || pos / kPage >= max_pages) {
+        if (threadIdx.x == 0) set_error(kErrAttnIndex);
+        return;
+    }
+    const int64_t page = block_table[(int64_t)b * max_pages + pos / kPage];
+    if (page < 0 || page >= n_pages) {
+        if (threadIdx.x == 0) set_error(kErrAttnIndex);
+        return;
+    }
+    constexpr int kChunks = kD / 8;                          // 16-byte chunks of a 192-wide row
+    const int t = threadIdx.x & 127, which = threadIdx.x >> 7;
+    if (t < kG * kChunks) {
+        const int g = t / kChunks, c = t % kChunks;
+        const __nv_bfloat16 *src = (which ? new_v : new_k) + ((int64_t)i * kG + g) * kD + c * 8;
+        __nv_bfloat16 *dst = (which ? v_cache : k_cache) + ((page * kG + g) * kPage + pos % kPage) * kD + c * 8;
+        *reinterpret_cast<uint4 *>(dst) = __ldg(reinterpret_cast<const uint4 *>(src));
+    }
+}
+
 }  // namespace dsa

@@ -236,26 +236,34 @@ dsa_status_t attn_cluster_launch(const CUtensorMap &mk, const CUtensorMap &mv, c
                     dsa::attnc::kSmemBytes, stream, (unsigned)dsa::attnc::kSplits, mk, mv, p);
 }
 
+// Regions a window of `window` tokens can touch: its first token may sit anywhere in a region.
+int window_regions(int window) { return window / dsa::kRegion + 2; }
+
+// window == 0: attention over the selection (sel_idx, sel_count, k); window > 0: over each
+// query's last `window` tokens (k = window_regions(window), no selection).
 dsa_status_t attn_common(const void *q, const void *k_cache, const void *v_cache, int64_t n_pages,
                          const int32_t *block_table, int max_pages, const int32_t *q_req, int n_req,
                          const int32_t *q_pos, int nq, const int32_t *sel_idx, const int32_t *sel_count, int k,
-                         void *out, float *lse, void *ws, size_t ws_bytes, dsa_stream_t stream)
+                         void *out, float *lse, void *ws, size_t ws_bytes, dsa_stream_t stream, int window = 0)
 {
     DSA_REQUIRE(nq >= 0, "nq must be >= 0");
-    DSA_REQUIRE(k >= 1 && k <= DSA_MAX_TOPK, "k out of [1, DSA_MAX_TOPK]");
+    DSA_REQUIRE(window > 0 || (k >= 1 && k <= DSA_MAX_TOPK), "k out of [1, DSA_MAX_TOPK]");
     DSA_REQUIRE(n_pages >= 1 && n_pages <= (INT32_MAX / (dsa::kG * dsa::kPage)), "n_pages out of range");
     DSA_REQUIRE(max_pages >= 1, "max_pages must be >= 1");
     DSA_REQUIRE(n_req >= 1, "n_req must be >= 1");
     if (nq == 0) return DSA_OK;
-    DSA_REQUIRE(q && k_cache && v_cache && block_table && q_pos && sel_idx && sel_count && out, "NULL pointer");
+    DSA_REQUIRE(q && k_cache && v_cache && block_table && q_pos && out, "NULL pointer");
+    DSA_REQUIRE(window > 0 || (sel_idx && sel_count), "NULL pointer");
     DSA_REQUIRE(aligned(q, 16) && aligned(k_cache, 16) && aligned(v_cache, 16) && aligned(out, 4),
                 "q, k_cache, v_cache must be 16-byte aligned, out 4-byte aligned");
     int sms = 0;
     dsa_status_t st = device_info(sms);
     if (st != DSA_OK) return st;
-    const bool clustered = k <= dsa::attnc::kMaxK && (int64_t)nq * dsa::kG <= cluster_attn_capacity();
+    const bool clustered =
+        window == 0 && k <= dsa::attnc::kMaxK && (int64_t)nq * dsa::kG <= cluster_attn_capacity();
     // prefill chunks: 8 neighbouring queries per CTA share one stream of their selections' union
-    const bool shared = !clustered && q_req != nullptr && nq >= kSharedMinQueries && k <= dsa::attns::kMaxK &&
+    const bool shared = window == 0 && !clustered && q_req != nullptr && nq >= kSharedMinQueries &&
+                        k <= dsa::attns::kMaxK &&
                         (int64_t)max_pages * dsa::kPage / dsa::kRegion <= (int64_t)dsa::attns::kMaxWords * 32;
     const AttnPlan plan = attn_plan(nq, k, sms);
     const size_t need_ws = plan.ws + (shared ? round_up((size_t)nq * dsa::kG, 256) : 0);
@@ -288,6 +296,7 @@ dsa_status_t attn_common(const void *q, const void *k_cache, const void *v_cache
     p.k = k;
     p.rps = plan.rps;
     p.n_splits = plan.n_splits;
+    p.window = window;
     p.scale_log2 = dsa::attn::kLog2e / sqrtf((float)dsa::kD);
 
     if (clustered) return attn_cluster_launch(mk, mv, p, nq, stream);
@@ -775,6 +784,42 @@ dsa_status_t dsa_sparse_attn_decode(const void *q, const void *k_cache, const vo
 {
     return attn_common(q, k_cache, v_cache, n_pages, block_table, max_pages, nullptr, batch, q_pos, batch, sel_idx,
                        sel_count, k, out, lse, ws, ws_bytes, stream);
+}
+
+size_t dsa_window_attn_workspace_size(int nq, int window)
+{
+    if (nq <= 0 || window < 1) return 0;
+    int sms = 0;
+    if (device_info(sms) != DSA_OK) sms = 148;
+    return attn_plan(nq, window_regions(window), sms).ws;
+}
+
+dsa_status_t dsa_window_attn(const void *q, const void *k_cache, const void *v_cache, int64_t n_pages,
+                             const int32_t *block_table, int max_pages, int n_req, const int32_t *q_req,
+                             const int32_t *q_pos, int nq, int window, void *out, float *lse, void *ws,
+                             size_t ws_bytes, dsa_stream_t stream)
+{
+    DSA_REQUIRE(window >= 1 && window <= (1 << 20), "window out of [1, 2^20]");
+    return attn_common(q, k_cache, v_cache, n_pages, block_table, max_pages, q_req, q_req ? n_req : nq, q_pos, nq,
+                       nullptr, nullptr, window_regions(window), out, lse, ws, ws_bytes, stream, window);
+}
+
+dsa_status_t dsa_kv_append(void *k_cache, void *v_cache, int64_t n_pages, const int32_t *block_table, int max_pages,
+                           int n_req, const int32_t *q_req, const int32_t *q_pos, int n, const void *new_k,
+                           const void *new_v, dsa_stream_t stream)
+{
+    DSA_REQUIRE(n >= 0, "n must be >= 0");
+    DSA_REQUIRE(n_pages >= 1 && n_pages <= (INT32_MAX / (dsa::kG * dsa::kPage)), "n_pages out of range");
+    DSA_REQUIRE(max_pages >= 1, "max_pages must be >= 1");
+    if (n == 0) return DSA_OK;
+    DSA_REQUIRE(k_cache && v_cache && block_table && q_pos && new_k && new_v, "NULL pointer");
+    DSA_REQUIRE(q_req == nullptr || n_req >= 1, "n_req must be >= 1");
+    DSA_REQUIRE(aligned(k_cache, 16) && aligned(v_cache, 16) && aligned(new_k, 16) && aligned(new_v, 16),
+                "caches and new rows must be 16-byte aligned");
+    return launch_k("kv_append_kernel", dsa::kv_append_kernel, dim3((unsigned)n), dim3(256), 0, stream, 0,
+                    static_cast<__nv_bfloat16 *>(k_cache), static_cast<__nv_bfloat16 *>(v_cache), n_pages,
+                    block_table, max_pages, q_req, q_req ? n_req : n, q_pos, n,
+                    static_cast<const __nv_bfloat16 *>(new_k), static_cast<const __nv_bfloat16 *>(new_v));
 }
 
 dsa_status_t dsa_sparse_attn_prefill(const void *q, const void *k_cache, const void *v_cache, int64_t n_pages,

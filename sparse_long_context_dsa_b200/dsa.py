@@ -61,6 +61,11 @@ _SIG = {
     "dsa_sparse_attn_prefill": (ctypes.c_int, [_VP, _VP, _VP, ctypes.c_int64, _I32P, ctypes.c_int, ctypes.c_int,
                                                _I32P, _I32P, ctypes.c_int, _I32P, _I32P, ctypes.c_int, _VP, _F32P,
                                                _VP, ctypes.c_size_t, _VP]),
+    "dsa_kv_append": (ctypes.c_int, [_VP, _VP, ctypes.c_int64, _I32P, ctypes.c_int, ctypes.c_int, _I32P, _I32P,
+                                     ctypes.c_int, _VP, _VP, _VP]),
+    "dsa_window_attn_workspace_size": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int]),
+    "dsa_window_attn": (ctypes.c_int, [_VP, _VP, _VP, ctypes.c_int64, _I32P, ctypes.c_int, ctypes.c_int, _I32P,
+                                       _I32P, ctypes.c_int, ctypes.c_int, _VP, _F32P, _VP, ctypes.c_size_t, _VP]),
 }
 
 
@@ -284,4 +289,50 @@ def sparse_attn_prefill(q, k_cache, v_cache, block_table, q_req, q_pos, sel_idx,
                                          block_table.shape[1], block_table.shape[0], _p(q_req), _p(q_pos), nq,
                                          _p(sel_idx), _p(sel_count), k, _p(out), _p(lse), _p(ws), nbytes,
                                          _stream()))
+    return out
+
+
+def _cache_args(k_cache, v_cache, block_table):
+    _need(k_cache, torch.bfloat16, name="k_cache")
+    if k_cache.dim() != 4 or tuple(k_cache.shape[1:]) != (G, PAGE, D):
+        raise ValueError("k_cache must be [n_pages][4][64][192]")
+    _need(v_cache, torch.bfloat16, tuple(k_cache.shape), "v_cache")
+    _need(block_table, torch.int32, name="block_table")
+    if block_table.dim() != 2:
+        raise ValueError("block_table must be [n_req][max_pages]")
+
+
+def kv_append(k_cache, v_cache, block_table, q_pos, new_k, new_v, q_req=None):
+    """Writes token i's K and V rows (new_k, new_v bf16 [n][4][192]) to the slot of position
+    q_pos[i] of request q_req[i] (or i).  With a cyclic block table: the window ring buffer."""
+    _cache_args(k_cache, v_cache, block_table)
+    n = q_pos.shape[0]
+    _need(q_pos, torch.int32, (n,), "q_pos")
+    _need(new_k, torch.bfloat16, (n, G, D), "new_k")
+    _need(new_v, torch.bfloat16, (n, G, D), "new_v")
+    if q_req is not None:
+        _need(q_req, torch.int32, (n,), "q_req")
+    _check(lib().dsa_kv_append(_p(k_cache), _p(v_cache), k_cache.shape[0], _p(block_table), block_table.shape[1],
+                               block_table.shape[0], _p(q_req), _p(q_pos), n, _p(new_k), _p(new_v), _stream()))
+
+
+def window_attn(q, k_cache, v_cache, block_table, q_pos, window=512, q_req=None, out=None, lse=None):
+    """GQA of each query over its last `window` tokens (positions max(0, p-window+1) .. p of
+    request q_req[i], or i), read through the block table.  Returns out bf16 [nq][64][192]."""
+    nq = q.shape[0]
+    _need(q, torch.bfloat16, (nq, HQ, D), "q")
+    _cache_args(k_cache, v_cache, block_table)
+    _need(q_pos, torch.int32, (nq,), "q_pos")
+    if q_req is not None:
+        _need(q_req, torch.int32, (nq,), "q_req")
+    if out is None:
+        out = torch.empty((nq, HQ, D), dtype=torch.bfloat16, device=q.device)
+    _need(out, torch.bfloat16, (nq, HQ, D), "out")
+    if lse is not None:
+        _need(lse, torch.float32, (nq, HQ), "lse")
+    nbytes = lib().dsa_window_attn_workspace_size(nq, window)
+    ws = _workspace(nbytes, q.device)
+    _check(lib().dsa_window_attn(_p(q), _p(k_cache), _p(v_cache), k_cache.shape[0], _p(block_table),
+                                 block_table.shape[1], block_table.shape[0], _p(q_req), _p(q_pos), nq, int(window),
+                                 _p(out), _p(lse), _p(ws), nbytes, _stream()))
     return out

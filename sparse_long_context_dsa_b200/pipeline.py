@@ -198,3 +198,50 @@ class StreamingDecode:
         out = self.step.run()
         self.lengths = [L + 1 for L in self.lengths]
         return out, due
+
+
+def ring_block_table(batch: int, max_pages: int, ring_pages: int = 8, device="cuda") -> torch.Tensor:
+    """Block table of per-request rings: request b's virtual page v maps to physical page
+    b * ring_pages + v % ring_pages, so with 64-token pages a ring of 8 pages holds the last
+    512 tokens and token t overwrites the slot of token t - 512 ([P2] Step-5-Preview
+    如何实现1M长上下文 §第一招: the window layers' ring buffer)."""
+    b = torch.arange(batch, dtype=torch.int32)[:, None]
+    v = torch.arange(max_pages, dtype=torch.int32)[None, :]
+    return (b * ring_pages + v % ring_pages).to(device)
+
+
+class WindowDecodeStep:
+    """One decode step of a window layer for a batch of requests, one token each: the new
+    token's K/V into the request's ring (dsa_kv_append), then GQA over its last `window`
+    tokens (dsa_window_attn).  Buffers are allocated once (capturable in a CUDA graph).
+
+    k_ring/v_ring: bf16 [B * ring_pages][4][64][192]; block_table: ring_block_table(...).
+    Per-step inputs: q bf16 [B][64][192], new_k/new_v bf16 [B][4][192], q_pos int32 [B]."""
+
+    def __init__(self, k_ring, v_ring, block_table, window: int = 512):
+        dev = k_ring.device
+        self.B = block_table.shape[0]
+        self.k_ring, self.v_ring, self.block_table, self.window = k_ring, v_ring, block_table, window
+        self.q = torch.zeros((self.B, HQ, D), dtype=torch.bfloat16, device=dev)
+        self.new_k = torch.zeros((self.B, G, D), dtype=torch.bfloat16, device=dev)
+        self.new_v = torch.zeros_like(self.new_k)
+        self.q_pos = torch.zeros((self.B,), dtype=torch.int32, device=dev)
+        self.out = torch.empty((self.B, HQ, D), dtype=torch.bfloat16, device=dev)
+        L = dsa.lib()
+        self.ws_n = L.dsa_window_attn_workspace_size(self.B, window)
+        self.ws = torch.empty(max(1, self.ws_n), dtype=torch.uint8, device=dev)
+
+    def load(self, q, new_k, new_v, q_pos):
+        self.q.copy_(q, non_blocking=True)
+        self.new_k.copy_(new_k, non_blocking=True)
+        self.new_v.copy_(new_v, non_blocking=True)
+        self.q_pos.copy_(q_pos, non_blocking=True)
+
+    def run(self):
+        L, p, st = dsa.lib(), dsa._p, dsa._stream()
+        kr, bt = self.k_ring, self.block_table
+        dsa._check(L.dsa_kv_append(p(kr), p(self.v_ring), kr.shape[0], p(bt), bt.shape[1], self.B, None,
+                                   p(self.q_pos), self.B, p(self.new_k), p(self.new_v), st))
+        dsa._check(L.dsa_window_attn(p(self.q), p(kr), p(self.v_ring), kr.shape[0], p(bt), bt.shape[1], self.B,
+                                     None, p(self.q_pos), self.B, self.window, p(self.out), None, p(self.ws),
+                                     self.ws_n, st))
