@@ -356,8 +356,8 @@ dsa_status_t indexer_gemm_path(const void *index_q, const float *gate, const int
                                                  round_up((size_t)nq * dsa::kHI * 4, 256));
     int32_t *tile_own = reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(q_own) + round_up((size_t)nq * 4, 256));
     const int n_mtiles = (nq + dsa::gemm::kQPerTile - 1) / dsa::gemm::kQPerTile;
-    const int qblocks = (nq * dsa::kHI + 3) / 4;
-    const int grid_q = std::max(qblocks, (n_mtiles + 127) / 128);
+    const int qblocks = (nq * dsa::kHI + 3) / 4;            // 4 warps per block: (q, h) pairs, then tiles
+    const int grid_q = std::max(qblocks, (n_mtiles + 3) / 4);
     dsa_status_t st;
     if ((st = launch_k("gemm quantize_kernel", dsa::gemm::quantize_kernel, dim3(grid_q), dim3(128), 0, stream, 0,
                        static_cast<const __nv_bfloat16 *>(index_q), q_req, q_pos, sum_base, ld, n_slots, nq, codes,

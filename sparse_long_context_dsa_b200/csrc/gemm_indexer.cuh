@@ -83,7 +83,7 @@ __device__ __forceinline__ int valid_own(const int32_t *q_req, const int32_t *q_
 
 // Per (query, head): sq = absmax/448 (IEEE division), codes = e4m3(x / sq), all 0 when the
 // head is zero.  One warp per (q, h).  Also the validated own region of every query
-// (-1 and an error for an invalid one) and the largest own region of every 32-query tile.
+// (-1 and an error for an invalid one) and the largest own region of every query tile.
 __global__ void __launch_bounds__(128) quantize_kernel(const __nv_bfloat16 *__restrict__ index_q,
                                                        const int32_t *__restrict__ q_req,
                                                        const int32_t *__restrict__ q_pos,
@@ -124,14 +124,16 @@ __global__ void __launch_bounds__(128) quantize_kernel(const __nv_bfloat16 *__re
             make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
         if (lane == 0) qscale[gw] = sq;
     }
-    const int t = blockIdx.x * blockDim.x + threadIdx.x;
-    if (t < n_mtiles) {
+    // the largest own region of every 64-query tile: warp gw takes tile gw (2 queries a lane)
+    if (gw < n_mtiles) {
         int m = -1;
-        for (int i = 0; i < kQPerTile; ++i) {
-            const int q = t * kQPerTile + i;
+#pragma unroll
+        for (int i = lane; i < kQPerTile; i += 32) {
+            const int q = gw * kQPerTile + i;
             if (q < nq) m = max(m, valid_own(q_req, q_pos, sum_base, ld, n_slots, q));
         }
-        tile_own[t] = m;
+        m = __reduce_max_sync(0xffffffffu, m);
+        if (lane == 0) tile_own[gw] = m;
     }
 }
 
