@@ -49,7 +49,7 @@ PREFILL_CTX, PREFILL_NEW = 262144, 2048
 PREFILL_KERNELS = 6       # compress, quantize, GEMM, top-k, shared-selection attention, per-row attention
 # DRAM bytes (read + write) of one gemm_scores_kernel launch on the prefill workload, from one
 # ncu capture of the current kernel; None once the kernel changes
-GEMM_TRAFFIC_BYTES = 150_103_808 + 1_020_655_000
+GEMM_TRAFFIC_BYTES = 139_658_240 + 1_020_275_000
 
 
 def parse():

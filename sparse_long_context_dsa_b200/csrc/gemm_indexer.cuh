@@ -14,8 +14,8 @@
 //    one of two 256-column TMEM accumulators (512 columns, one CTA per SM).  Large-N
 //    instructions matter: the same block cut as 4 heads x (M = 128, N = 64) ran the tensor
 //    pipe at a third of the rate;
-//  * sixteen epilogue warps (four per TMEM lane quarter, one per 16-query quarter) read
-//    their 64 columns, release the buffer, and for each query form sum_h w_h * ReLU(C) in
+//  * eight epilogue warps (two per TMEM lane quarter, one per 32-query half) read their
+//    128 columns, release the buffer, and for each query form sum_h w_h * ReLU(C) in
 //    registers: each thread owns one region, so the head sum stays in the thread, the
 //    region's scale is one register (the block's 128 scales arrive with the summaries by
 //    TMA), and a warp's 32 lanes write one 128-byte line of a query's score row, masked
@@ -42,9 +42,11 @@ constexpr int kQBytes = 2 * kQHalf;      // 64 KiB
 constexpr int kSHalf = kBM * 128;        // one 128-byte K column of a summary block (16 KiB)
 constexpr int kSBytes = 2 * kSHalf;      // 32 KiB
 constexpr int kSStages = 4;
-constexpr int kEpiWarps = 16;
-constexpr int kThreads = 32 * (2 + kEpiWarps);  // warp 0 TMA, warp 1 MMA, warps 2..17 epilogue
-constexpr int kEpiQueries = kQPerTile / 4;      // queries per epilogue warp
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 32 * (2 + kEpiWarps);  // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
+constexpr int kEpiQueries = kQPerTile * 4 / kEpiWarps;   // queries per epilogue warp (32)
+constexpr int kEpiChunks = kEpiQueries / 8;                // 32-column TMEM loads per warp and block
+static_assert(kEpiChunks % 2 == 0, "column loads go in pairs");
 constexpr int kTmemCols = 512;                  // two 256-column fp32 accumulators
 constexpr int kScaleBox = kBM + 4;              // region scales per block, from a 16-byte aligned start
 constexpr int kScaleBytes = kScaleBox * 4;      // 528 bytes loaded per block
@@ -195,7 +197,7 @@ __device__ __forceinline__ void cta_range(const Params &p, int64_t &lo, int64_t 
     hi = total * (blockIdx.x + 1) / gridDim.x;
 }
 
-// 18 warps: 5 share a scheduler's 16K registers, so at most 96 registers per thread
+// 10 warps: 3 share a scheduler's 16K registers, so at most 168 registers per thread
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_scores_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_s,
                        const __grid_constant__ CUtensorMap map_sc, const Params p)
@@ -207,8 +209,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *sq = smem;                                   // query tile: 2 K columns x [256 rows (q, h)][128 B]
     uint8_t *ss = smem + kQBytes;                         // summary blocks: kSStages x 2 K columns x [128][128 B]
     uint8_t *ssc = ss + kSStages * kSBytes;                                     // [kSStages] scale slots
-    float4 *wsm_all = reinterpret_cast<float4 *>(ssc + kSStages * kScaleSlot);  // [16 warps][8 pairs][2] weights
-    int *own_all = reinterpret_cast<int *>(wsm_all + kEpiWarps * kEpiQueries);  // [16 warps][16 queries]
+    float4 *wsm_all = reinterpret_cast<float4 *>(ssc + kSStages * kScaleSlot);  // [warps][pairs][2] weights
+    int *own_all = reinterpret_cast<int *>(wsm_all + kEpiWarps * kEpiQueries);  // [warps][queries]
     uint64_t *bars = reinterpret_cast<uint64_t *>(own_all + kEpiWarps * kEpiQueries);
     uint64_t *q_full = bars + 0, *q_empty = bars + 1;
     uint64_t *s_full = bars + 2, *s_empty = bars + 2 + kSStages;                // [kSStages]
@@ -312,9 +314,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else {
-        // ---------------- epilogue: warps 2..17.  TMEM lane quarter sp = warp % 4 (the
+        // ---------------- epilogue: warps 2..9.  TMEM lane quarter sp = warp % 4 (the
         // hardware's lane-access rule): regions 32 sp .. 32 sp + 31 of the block, one per
-        // thread; query quarter qq: queries 16 qq .. 16 qq + 15 of the tile (columns 64 qq ..)
+        // thread; query half qq: queries 32 qq .. 32 qq + 31 of the tile (columns 128 qq ..)
         const int e = warp - 2, sp = warp & 3, qq = e >> 2;
         // z * sq / 2 of the 4 heads per query, interleaved by query pair (a, b):
         // wsm[2 i] = {a h0, b h0, a h1, b h1}, wsm[2 i + 1] = {a h2, b h2, a h3, b h3}
@@ -359,10 +361,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                      mbar_wait_sleep(&s_full[s], (int)(it / kSStages) & 1);   // complete already: makes the scales visible
                 if (!ok) break;
                 tc_fence_after();
-                float v0[32], v1[32];                             // columns 4q + h of queries 0-7, 8-15
+                float v[kEpiChunks][32];                          // columns 4q + h of the warp's queries
                 {
-                    const uint32_t ta = tmem + ((uint32_t)(32 * sp) << 16) + buf * kBN + qq * 64;
-                    tmem_ld32x2(ta, ta + 32, v0, v1);
+                    const uint32_t ta = tmem + ((uint32_t)(32 * sp) << 16) + buf * kBN + qq * (kEpiQueries * 4);
+#pragma unroll
+                    for (int c = 0; c < kEpiChunks; c += 2) tmem_ld32x2(ta + 32 * c, ta + 32 * (c + 1), v[c], v[c + 1]);
                 }
                 const int64_t y = w.g * p.n_slots + base + (int64_t)w.rb * kBM;
                 const float sc =                                  // scale[g][r] / 16
@@ -382,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     float *dst = p.scores + ((int64_t)(w.t * kQPerTile + qq * kEpiQueries) * kG + w.g) * p.ld + r;
                     const float2 sc2 = make_float2(sc, sc);
 #pragma unroll
-                    for (int j4 = 0; j4 < 4; ++j4) {
+                    for (int j4 = 0; j4 < kEpiQueries / 4; ++j4) {
                         const int4 o4 = reinterpret_cast<const int4 *>(osm)[j4];
                         const int oj[4] = {o4.x, o4.y, o4.z, o4.w};
 #pragma unroll
@@ -390,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const int j = 4 * j4 + u;                     // queries j, j + 1
                             const float4 w01 = reinterpret_cast<const float4 *>(wsm)[j];
                             const float4 w23 = reinterpret_cast<const float4 *>(wsm)[j + 1];
-                            const float *va = j < 8 ? &v0[4 * j] : &v1[4 * (j - 8)];
+                            const float *va = &v[j / 8][4 * (j % 8)];
                             const float *vb = va + 4;
                             float2 acc = fmul2(make_float2(va[0] + fabsf(va[0]), vb[0] + fabsf(vb[0])),
                                                make_float2(w01.x, w01.y));
