@@ -12,6 +12,7 @@ Functions mirror the library's C-ABI calls:
   topk_regions       A3  own region + top-(k-1)       ties -> lower index
   sparse_attention   A4  exact GQA over the selection softmax(q K^T / sqrt(192)) V
   window_attention       the window layers: the same over the last `window` tokens
+  indexer_frontend       hidden state -> index_q, index_k (RMSNorm, partial RoPE), gates
 plus the number-format helpers the pins use (bf16 and OCP E4M3 codecs).
 """
 from __future__ import annotations
@@ -87,6 +88,11 @@ def lib():
                 _P(ctypes.c_uint16), _P(ctypes.c_uint16), _P(ctypes.c_uint16),
                 _P(ctypes.c_int32), ctypes.c_int, _P(ctypes.c_int32), _P(ctypes.c_int32),
                 ctypes.c_int, ctypes.c_int, _P(ctypes.c_uint16), _P(ctypes.c_float), _P(ctypes.c_double)]
+            L.oracle_indexer_frontend.restype = None
+            L.oracle_indexer_frontend.argtypes = [
+                _P(ctypes.c_uint16), _P(ctypes.c_uint16), _P(ctypes.c_uint16), _P(ctypes.c_uint16),
+                _P(ctypes.c_int32), ctypes.c_int, ctypes.c_int, _P(ctypes.c_uint16), _P(ctypes.c_uint16),
+                _P(ctypes.c_float)]
             L.oracle_set_threads.restype = None
             L.oracle_set_threads.argtypes = [ctypes.c_int]
             L.oracle_get_threads.restype = ctypes.c_int
@@ -296,3 +302,29 @@ def window_attention(q_bits, k_cache_bits, v_cache_bits, block_table, q_req, q_p
     if want_f64:
         return out, lse, o64
     return out, lse
+
+
+FRONTEND_ROWS = HI * DI + G * DI + HI          # 5,136 projection rows: q heads, k groups, gates
+
+
+def indexer_frontend(hidden_bits, w_bits, gamma_q_bits, gamma_k_bits, pos):
+    """Indexer front end ([P2] §索引器打分: index_q / index_k / index_z projected from the
+    hidden state, normalised, RoPE on part of the dimensions).  hidden uint16 (bf16 bits)
+    [T][hid]; w uint16 [5136][hid] (rows: 16 x 256 q, 4 x 256 k, 16 gates); gamma_q/gamma_k
+    uint16 [256]; pos int32 [T].  Returns (index_q bf16 bits [T][16][256], index_k bf16 bits
+    [T][4][256], z float32 [T][16])."""
+    h = _arr(hidden_bits, np.uint16)
+    w = _arr(w_bits, np.uint16)
+    gq = _arr(gamma_q_bits, np.uint16)
+    gk = _arr(gamma_k_bits, np.uint16)
+    p = _arr(np.asarray(pos, np.int32), np.int32)
+    T, hid = int(h.shape[0]), int(h.shape[1])
+    if w.shape != (FRONTEND_ROWS, hid) or gq.shape != (DI,) or gk.shape != (DI,) or p.shape != (T,):
+        raise ValueError("shapes: hidden [T][hid], w [5136][hid], gammas [256], pos [T]")
+    iq = np.empty((T, HI, DI), np.uint16)
+    ik = np.empty((T, G, DI), np.uint16)
+    z = np.empty((T, HI), np.float32)
+    lib().oracle_indexer_frontend(_ptr(h, ctypes.c_uint16), _ptr(w, ctypes.c_uint16), _ptr(gq, ctypes.c_uint16),
+                                  _ptr(gk, ctypes.c_uint16), _ptr(p, ctypes.c_int32), T, hid,
+                                  _ptr(iq, ctypes.c_uint16), _ptr(ik, ctypes.c_uint16), _ptr(z, ctypes.c_float))
+    return iq, ik, z

@@ -17,6 +17,7 @@
  *   A3 top-k region select   [P2 §索引器打分], [P2 §第二招 sparse_config table]
  *   A4 sparse GQA attention  [P1 §DSA ④], [P2 §索引器打分], [P3 §一]
  *   sliding-window attention of the window layers [P1 §滑窗注意力], [P2 §第一招]
+ *   indexer front end (projections, norm, partial RoPE, gates) [P2 §索引器打分]
  * The pages leave the arithmetic open; the fixed reading is:
  *   summary = mean of the 8 tokens' bf16 index_k, e4m3 with one fp32 absmax/448 scale;
  *   score(r,g) = sum_{h in group g} z_h * ReLU(q_h . s_{r,g}) / 16, heads 4g..4g+3;
@@ -432,6 +433,62 @@ void oracle_window_attention(const uint16_t *q, const uint16_t *k_cache, const u
         if (lse) lse[(int64_t)qi * OR_HQ + h] = (float)l;
         free(rows);
         free(lg);
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* indexer front end: hidden state -> index_q, index_k, z               */
+/* ------------------------------------------------------------------ */
+
+/* [P2 §索引器打分]: the indexer projects the hidden state to index_q / index_k / index_z,
+ * then normalises and applies RoPE to part of the dimensions.  The pages give no constants;
+ * the fixed reading, per token t at position pos[t] with hidden row h (bf16 [hid]):
+ *   a_j   = sum_i W[j][i] h[i]                          (W bf16 [16*256 + 4*256 + 16][hid];
+ *                                                         rows: q heads, k groups, gates)
+ *   for each 256-d head vector x (16 q heads, 4 k groups, weights gamma_q / gamma_k [256]):
+ *     y_d = x_d / sqrt(mean_d(x_d^2) + 1e-6) * gamma[d]                     (RMSNorm)
+ *     for i < 32, theta = pos * 10000^(-2i/64):                            (RoPE on d < 64)
+ *       y'_i      = y_i cos(theta) - y_{i+32} sin(theta)
+ *       y'_{i+32} = y_{i+32} cos(theta) + y_i sin(theta)
+ *   z_h = 1 / (1 + exp(-a_{gate h}))                                        (sigmoid gates)
+ * in double; index_q/index_k rounded once to bf16, z to fp32. */
+void oracle_indexer_frontend(const uint16_t *hidden, const uint16_t *w, const uint16_t *gamma_q,
+                             const uint16_t *gamma_k, const int32_t *pos, int n_tok, int hid,
+                             uint16_t *index_q, uint16_t *index_k, float *z)
+{
+    const int n_out = OR_HI * OR_DI + OR_G * OR_DI + OR_HI;
+#pragma omp parallel for schedule(dynamic)
+    for (int t = 0; t < n_tok; ++t) {
+        double *a = (double *)malloc(sizeof(double) * (size_t)n_out);
+        const uint16_t *h = hidden + (int64_t)t * hid;
+        for (int j = 0; j < n_out; ++j) {
+            const uint16_t *wr = w + (int64_t)j * hid;
+            double s = 0.0;
+            for (int i = 0; i < hid; ++i) s += oracle_bf16_to_f64(wr[i]) * oracle_bf16_to_f64(h[i]);
+            a[j] = s;
+        }
+        for (int v = 0; v < OR_HI + OR_G; ++v) {
+            const double *x = a + (int64_t)v * OR_DI;
+            const uint16_t *gm = v < OR_HI ? gamma_q : gamma_k;
+            double ms = 0.0;
+            for (int d = 0; d < OR_DI; ++d) ms += x[d] * x[d];
+            const double inv = 1.0 / sqrt(ms / OR_DI + 1e-6);
+            double y[OR_DI];
+            for (int d = 0; d < OR_DI; ++d) y[d] = x[d] * inv * oracle_bf16_to_f64(gm[d]);
+            for (int i = 0; i < 32; ++i) {
+                const double th = (double)pos[t] * pow(10000.0, -2.0 * i / 64.0);
+                const double c = cos(th), sn = sin(th);
+                const double u0 = y[i], u1 = y[i + 32];
+                y[i] = u0 * c - u1 * sn;
+                y[i + 32] = u1 * c + u0 * sn;
+            }
+            uint16_t *dst = v < OR_HI ? index_q + ((int64_t)t * OR_HI + v) * OR_DI
+                                      : index_k + ((int64_t)t * OR_G + (v - OR_HI)) * OR_DI;
+            for (int d = 0; d < OR_DI; ++d) dst[d] = oracle_f64_to_bf16(y[d]);
+        }
+        for (int hh = 0; hh < OR_HI; ++hh)
+            z[(int64_t)t * OR_HI + hh] = (float)(1.0 / (1.0 + exp(-a[(OR_HI + OR_G) * OR_DI + hh])));
+        free(a);
     }
 }
 
