@@ -62,7 +62,7 @@ def parse():
     ap.add_argument("--cpu-queries", type=int, default=3, help="oracle queries timed for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", choices=["decode_b1_1m", "prefill_2k_256k", "prefill_2k_256k_local",
-                                           "swa_decode_b8"], default="decode_b1_1m")
+                                           "swa_decode_b8", "frontend_2k"], default="decode_b1_1m")
     return ap.parse_args()
 
 
@@ -705,6 +705,101 @@ def run_swa(args):
         dist.destroy_process_group()
 
 
+FE_TOKENS, FE_HID = 2048, 6144
+
+
+def run_frontend(args):
+    """The indexer front end for a 2,048-token prefill chunk ([P2] §索引器打分: index_q /
+    index_k / index_z projected from the hidden state, normalised, partially rotated): one
+    dsa_indexer_frontend call per step, hidden size 6,144 (a reading: the pages give none),
+    synthetic weights; L2 flushed before every step (the weights, 63 MB, would stay in it)."""
+    import numpy as np
+    import torch
+    from sparse_long_context_dsa_b200 import dsa
+
+    rank, world, local = dist_env()
+    if world > 1:
+        raise SystemExit("--workload frontend_2k runs on one GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dsa.lib()
+    g = torch.Generator(device=dev)
+    g.manual_seed(1241)
+    T, hid = FE_TOKENS, FE_HID
+    hidden = torch.randn((T, hid), generator=g, device=dev).to(torch.bfloat16)
+    w = (torch.randn((dsa.FRONTEND_ROWS, hid), generator=g, device=dev) / hid ** 0.5).to(torch.bfloat16)
+    gq = (1.0 + 0.1 * torch.randn(256, generator=g, device=dev)).to(torch.bfloat16)
+    gk = (1.0 + 0.1 * torch.randn(256, generator=g, device=dev)).to(torch.bfloat16)
+    pos = (262144 + torch.arange(T, device=dev)).to(torch.int32)
+    iq = torch.empty((T, 16, 256), dtype=torch.bfloat16, device=dev)
+    ik = torch.empty((T, 4, 256), dtype=torch.bfloat16, device=dev)
+    z = torch.empty((T, 16), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(max(args.warmup, 3)):
+        dsa.indexer_frontend(hidden, w, gq, gk, pos, iq, ik, z)
+    torch.cuda.synchronize()
+    dsa.check_device()
+    n = min(args.steps, 50)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    sampler = ClockSampler(local)
+    with sampler:
+        for a, b in evs:
+            flush.zero_()
+            a.record()
+            dsa.indexer_frontend(hidden, w, gq, gk, pos, iq, ik, z)
+            b.record()
+        torch.cuda.synchronize()
+    dsa.check_device()
+    ms = sum(a.elapsed_time(b) for a, b in evs) / n
+    flops = 2.0 * T * hid * dsa.FRONTEND_ROWS
+    peak, kind = tensor_peak(fp8=False)
+    achieved = flops / (ms * 1e-3) / 1e12
+    # e2e: hidden states from pinned host memory, the three outputs back
+    h_host = hidden.cpu().pin_memory()
+    oq, ok_, oz = (torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (iq, ik, z))
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = min(n, 10)
+    torch.cuda.synchronize()
+    t0.record()
+    for _ in range(n_e2e):
+        hidden.copy_(h_host, non_blocking=True)
+        dsa.indexer_frontend(hidden, w, gq, gk, pos, iq, ik, z)
+        oq.copy_(iq, non_blocking=True)
+        ok_.copy_(ik, non_blocking=True)
+        oz.copy_(z, non_blocking=True)
+    t1.record()
+    torch.cuda.synchronize()
+    e2e_ms = t0.elapsed_time(t1) / n_e2e
+    line = {
+        "metric": "indexer front-end tokens/s (hidden 6,144 -> index_q, index_k, gates)", "value": T / (ms * 1e-3),
+        "unit": "tokens/s", "n_gpus": 1, "steps": n, "warmup": max(args.warmup, 3), "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 (fp32 accumulate)",
+        "data": "synthetic",
+        "config": {"workload": "frontend_2k", "tokens": T, "hidden": hid, "rows": dsa.FRONTEND_ROWS,
+                   "l2": "flushed (256 MiB write) before every step"},
+        "roofline": {"kernel": "frontend_kernel (tcgen05 bf16 GEMM + RMSNorm/RoPE/sigmoid epilogue)",
+                     "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "peak_kind": kind, "flops_per_launch": flops, "traffic": None},
+        "e2e": {"value": T / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h_host.numel() * 2,
+                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in (oq, ok_, oz))},
+        "gpu_launches": n,
+        "clocks": sampler.summary(),
+    }
+    if not args.no_cpu_baseline:
+        import oracle
+        rows = np.arange(8)
+        hb = hidden[rows].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+        wb = w.cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+        gqb = gq.cpu().view(torch.int16).numpy().view(np.uint16)
+        gkb = gk.cpu().view(torch.int16).numpy().view(np.uint16)
+        c0 = time.perf_counter()
+        oracle.indexer_frontend(hb, wb, gqb, gkb, pos.cpu().numpy()[rows])
+        dt = time.perf_counter() - c0
+        line["cpu_baseline"] = {"value": len(rows) / dt, "unit": "tokens/s", "cores": oracle.get_threads(),
+                                "kind": "oracle", "sample": f"{len(rows)} tokens of the chunk"}
+    print(json.dumps(line), flush=True)
+
+
 def tensor_peak(fp8: bool):
     """Dense tensor peak in TFLOP/s: the measured cuBLAS bf16 burst figure (x2 for e4m3,
     the nominal fp8/bf16 ratio of the part), else the fallback."""
@@ -725,6 +820,8 @@ def main():
         run_prefill(args)
     elif args.workload == "swa_decode_b8":
         run_swa(args)
+    elif args.workload == "frontend_2k":
+        run_frontend(args)
     else:
         run_ours(args)
 

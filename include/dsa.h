@@ -16,6 +16,8 @@
  * and, for the window layers beside the DSA layers:
  *   dsa_kv_append            new tokens' K/V into their page slots (a ring with a cyclic table)
  *   dsa_window_attn          GQA over each query's last `window` tokens      [P1 §滑窗注意力][P2 §第一招]
+ * and the indexer's front end, upstream of A1/A2:
+ *   dsa_indexer_frontend     hidden state -> index_q, index_k, gates        [P2 §索引器打分]
  *
  * Conventions (every call):
  *   - Pointers are DEVICE pointers unless stated otherwise, owned by the caller.  The
@@ -272,6 +274,26 @@ dsa_status_t dsa_window_attn(const void *q, const void *k_cache, const void *v_c
                              const int32_t *block_table, int max_pages, int n_req, const int32_t *q_req,
                              const int32_t *q_pos, int nq, int window, void *out, float *lse, void *ws,
                              size_t ws_bytes, dsa_stream_t stream);
+
+/* ------------------------------------------------------------------------------ */
+/* Indexer front end.  [P2 §索引器打分] the indexer projects the hidden state to index_q /
+ * index_k / index_z, then normalises and applies RoPE to part of the dimensions.  The pages
+ * give no constants; this library's reading, per token t at position pos[t]:
+ *   a = W h_t                                  (W bf16 [5136][hid], fp32 accumulation; rows
+ *                                               0..4095: 16 q heads x 256, 4096..5119: 4 k
+ *                                               groups x 256, 5120..5135: 16 gates)
+ *   each 256-d head vector x (q heads with gamma_q, k groups with gamma_k, bf16 [256]):
+ *     y = x / sqrt(mean(x^2) + 1e-6) * gamma                                 (RMSNorm)
+ *     dims 0..63 rotated in pairs (i, i + 32) by pos * 10000^(-i/32)         (partial RoPE)
+ *   z_h = sigmoid(a_gate h)
+ * hidden  bf16 [n_tok][hid] (hid a multiple of 8), pos int32 [n_tok]
+ * index_q bf16 [n_tok][16][256], index_k bf16 [n_tok][4][256], z fp32 [n_tok][16]
+ * (the layouts dsa_indexer_scores and dsa_compress_regions read).  All device pointers
+ * 16-byte aligned except gamma_q, gamma_k and pos.  Runs as one tcgen05 bf16 GEMM with the
+ * norm, rotation and gates in its epilogue; no workspace. */
+dsa_status_t dsa_indexer_frontend(const void *hidden, int hid, int n_tok, const void *w, const void *gamma_q,
+                                  const void *gamma_k, const int32_t *pos, void *index_q, void *index_k, float *z,
+                                  dsa_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -15,6 +15,7 @@
 #include "common.cuh"
 #include "compress.cuh"
 #include "copy.cuh"
+#include "frontend.cuh"
 #include "gemm_indexer.cuh"
 #include "indexer.cuh"
 #include "topk.cuh"
@@ -784,6 +785,58 @@ dsa_status_t dsa_sparse_attn_decode(const void *q, const void *k_cache, const vo
 {
     return attn_common(q, k_cache, v_cache, n_pages, block_table, max_pages, nullptr, batch, q_pos, batch, sel_idx,
                        sel_count, k, out, lse, ws, ws_bytes, stream);
+}
+
+dsa_status_t dsa_indexer_frontend(const void *hidden, int hid, int n_tok, const void *w, const void *gamma_q,
+                                  const void *gamma_k, const int32_t *pos, void *index_q, void *index_k, float *z,
+                                  dsa_stream_t stream)
+{
+    DSA_REQUIRE(n_tok >= 0, "n_tok must be >= 0");
+    DSA_REQUIRE(hid >= 8 && hid % 8 == 0 && hid <= (1 << 20), "hid must be a multiple of 8 in [8, 2^20]");
+    if (n_tok == 0) return DSA_OK;
+    DSA_REQUIRE(hidden && w && gamma_q && gamma_k && pos && index_q && index_k && z, "NULL pointer");
+    DSA_REQUIRE(aligned(hidden, 16) && aligned(w, 16) && aligned(index_q, 16) && aligned(index_k, 16) &&
+                    aligned(z, 16),
+                "hidden, w, index_q, index_k and z must be 16-byte aligned");
+    int sms = 0;
+    dsa_status_t st = device_info(sms);
+    if (st != DSA_OK) return st;
+    CUtensorMap map_h, map_w;
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)hid, (cuuint64_t)n_tok};
+        const cuuint64_t strides[1] = {(cuuint64_t)hid * 2};
+        const cuuint32_t box[2] = {(cuuint32_t)dsa::fe::kBK, (cuuint32_t)dsa::fe::kBM};
+        if ((st = encode(&map_h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, hidden, dims, strides, box,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B)) != DSA_OK)
+            return st;
+    }
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)hid, (cuuint64_t)dsa::fe::kRows};
+        const cuuint64_t strides[1] = {(cuuint64_t)hid * 2};
+        const cuuint32_t box[2] = {(cuuint32_t)dsa::fe::kBK, (cuuint32_t)dsa::fe::kBN};
+        if ((st = encode(&map_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w, dims, strides, box,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B)) != DSA_OK)
+            return st;
+    }
+    dsa::fe::Params p{};
+    p.gamma_q = static_cast<const __nv_bfloat16 *>(gamma_q);
+    p.gamma_k = static_cast<const __nv_bfloat16 *>(gamma_k);
+    p.pos = pos;
+    p.index_q = static_cast<__nv_bfloat16 *>(index_q);
+    p.index_k = static_cast<__nv_bfloat16 *>(index_k);
+    p.z = z;
+    p.n_tok = n_tok;
+    p.n_k = (hid + dsa::fe::kBK - 1) / dsa::fe::kBK;
+    p.n_units = (n_tok + dsa::fe::kBM - 1) / dsa::fe::kBM * dsa::fe::kUnitsPerTile;
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(dsa::fe::frontend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)dsa::fe::kSmemBytes);
+    });
+    DSA_CUDA(attr_err, "cudaFuncSetAttribute(frontend_kernel)");
+    return launch_k("frontend_kernel", dsa::fe::frontend_kernel, dim3((unsigned)std::min(sms, p.n_units)),
+                    dim3(dsa::fe::kThreads), dsa::fe::kSmemBytes, stream, 0, map_h, map_w, p);
 }
 
 size_t dsa_window_attn_workspace_size(int nq, int window)

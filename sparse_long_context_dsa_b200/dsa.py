@@ -64,6 +64,8 @@ _SIG = {
     "dsa_kv_append": (ctypes.c_int, [_VP, _VP, ctypes.c_int64, _I32P, ctypes.c_int, ctypes.c_int, _I32P, _I32P,
                                      ctypes.c_int, _VP, _VP, _VP]),
     "dsa_window_attn_workspace_size": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int]),
+    "dsa_indexer_frontend": (ctypes.c_int, [_VP, ctypes.c_int, ctypes.c_int, _VP, _VP, _VP, _I32P, _VP, _VP, _F32P,
+                                            _VP]),
     "dsa_window_attn": (ctypes.c_int, [_VP, _VP, _VP, ctypes.c_int64, _I32P, ctypes.c_int, ctypes.c_int, _I32P,
                                        _I32P, ctypes.c_int, ctypes.c_int, _VP, _F32P, _VP, ctypes.c_size_t, _VP]),
 }
@@ -336,3 +338,31 @@ def window_attn(q, k_cache, v_cache, block_table, q_pos, window=512, q_req=None,
                                  block_table.shape[1], block_table.shape[0], _p(q_req), _p(q_pos), nq, int(window),
                                  _p(out), _p(lse), _p(ws), nbytes, _stream()))
     return out
+
+
+FRONTEND_ROWS = HI * DI + G * DI + HI      # weight rows: 16 q heads x 256, 4 k groups x 256, 16 gates
+
+
+def indexer_frontend(hidden, w, gamma_q, gamma_k, pos, index_q=None, index_k=None, z=None):
+    """Hidden states bf16 [T][hid] -> (index_q bf16 [T][16][256], index_k bf16 [T][4][256],
+    z fp32 [T][16]): projection by w bf16 [5136][hid], per-head RMSNorm with gamma_q / gamma_k,
+    partial RoPE at positions pos int32 [T], sigmoid gates."""
+    T, hid = hidden.shape
+    _need(hidden, torch.bfloat16, (T, hid), "hidden")
+    _need(w, torch.bfloat16, (FRONTEND_ROWS, hid), "w")
+    _need(gamma_q, torch.bfloat16, (DI,), "gamma_q")
+    _need(gamma_k, torch.bfloat16, (DI,), "gamma_k")
+    _need(pos, torch.int32, (T,), "pos")
+    dev = hidden.device
+    if index_q is None:
+        index_q = torch.empty((T, HI, DI), dtype=torch.bfloat16, device=dev)
+    if index_k is None:
+        index_k = torch.empty((T, G, DI), dtype=torch.bfloat16, device=dev)
+    if z is None:
+        z = torch.empty((T, HI), dtype=torch.float32, device=dev)
+    _need(index_q, torch.bfloat16, (T, HI, DI), "index_q")
+    _need(index_k, torch.bfloat16, (T, G, DI), "index_k")
+    _need(z, torch.float32, (T, HI), "z")
+    _check(lib().dsa_indexer_frontend(_p(hidden), hid, T, _p(w), _p(gamma_q), _p(gamma_k), _p(pos), _p(index_q),
+                                      _p(index_k), _p(z), _stream()))
+    return index_q, index_k, z
