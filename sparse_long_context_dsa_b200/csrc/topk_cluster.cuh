@@ -253,7 +253,7 @@ __device__ __forceinline__ void desc_bin_search(const uint32_t *h, uint32_t m, u
 template <int R, typename Valid, typename Comp>
 __device__ bool block_threshold(Valid valid, Comp comp, uint32_t m, uint32_t klo, uint32_t *hs, uint64_t *list,
                                 uint32_t *hw, uint32_t *sh_kmax, uint32_t *sh_nin, uint32_t *res, uint64_t *bc,
-                                uint64_t *elo, uint64_t *ehi, uint64_t *cp, uint64_t *cm)
+                                uint64_t *elo, uint64_t *ehi, uint64_t *cp, uint64_t *cm, int r_used = R)
 {
     (void)klo;
     (void)hw;
@@ -262,7 +262,7 @@ __device__ bool block_threshold(Valid valid, Comp comp, uint32_t m, uint32_t klo
     __shared__ unsigned long long s_min, s_max;
     uint64_t cmn = ~0ull, cmx = 0ull;
 #pragma unroll 8
-    for (int u = 0; u < R; ++u)
+    for (int u = 0; u < R && u < r_used; ++u)
         if (valid(u)) {
             const uint64_t c = comp(u);
             cmn = c < cmn ? c : cmn;
@@ -293,7 +293,7 @@ __device__ bool block_threshold(Valid valid, Comp comp, uint32_t m, uint32_t klo
     uint64_t width = ~0ull;                                  // extent of the current range [rlo, rlo + width)
     for (int level = 0; level < 8; ++level) {
 #pragma unroll 8
-        for (int u = 0; u < R; ++u) {
+        for (int u = 0; u < R && u < r_used; ++u) {
             if (!valid(u)) continue;
             const uint64_t c = comp(u);
             if (c >= rlo && c - rlo < width) atomicAdd(&hs[(uint32_t)((c - rlo) >> bsh)], 1u);
@@ -314,7 +314,7 @@ __device__ bool block_threshold(Valid valid, Comp comp, uint32_t m, uint32_t klo
     // the bin's members (at most 32: a bin of width 1 holds one composite)
     const uint64_t blo = rlo + ((uint64_t)bin << bsh);
 #pragma unroll 8
-    for (int u = 0; u < R; ++u) {
+    for (int u = 0; u < R && u < r_used; ++u) {
         if (!valid(u)) continue;
         const uint64_t c = comp(u);
         if (c >= blo && ((c - blo) >> bsh) == 0ull) list[atomicAdd(sh_nin, 1u)] = c;

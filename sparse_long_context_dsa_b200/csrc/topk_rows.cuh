@@ -144,12 +144,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         constexpr int R = kMaxCand / kThreads;          // 20
         auto cvalid = [&](int u) { return (uint32_t)(u * kThreads + tid) < n_cand; };
         auto ccomp = [&](int u) { return cand[u * kThreads + tid]; };
+        const int r_used = (int)((n_cand + kThreads - 1) / kThreads);
         block_threshold<R>(cvalid, ccomp, (uint32_t)need, lo_key, hs, list, nullptr, &sh_max, &sh_nin, scan_ws + 32,
-                           bc, &elo2, &ehi2, &cp, &cm);
+                           bc, &elo2, &ehi2, &cp, &cm, r_used);
         for (int i = tid; i < words; i += kThreads) bitmap[i] = 0u;
         __syncthreads();
 #pragma unroll 4
-        for (int u = 0; u < R; ++u)
+        for (int u = 0; u < r_used; ++u)
             if (cvalid(u) && threshold_selects(ccomp(u), elo2, ehi2, cp, cm)) {
                 const uint32_t r = 0xFFFFFFFFu - (uint32_t)ccomp(u);
                 atomicOr(&bitmap[r >> 5], 1u << (r & 31));
@@ -163,7 +164,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             return ((uint64_t)score_key(__ldcg(src + i)) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)i);
         };
         block_threshold<R>(rvalid, rcomp, (uint32_t)need, 0u, hs, list, nullptr, &sh_max, &sh_nin, scan_ws + 32, bc,
-                           &elo2, &ehi2, &cp, &cm);
+                           &elo2, &ehi2, &cp, &cm, (n + kThreads - 1) / kThreads);
         for (int i = tid; i < words; i += kThreads) bitmap[i] = 0u;
         __syncthreads();
 #pragma unroll 4
