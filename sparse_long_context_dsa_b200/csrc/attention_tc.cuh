@@ -1,0 +1,467 @@
+// A4 sparse GQA attention for prefill blocks whose queries share their selections, on the
+// tcgen05 tensor cores ([P1] kwkr.cn/news/601179 §DSA ④; [P5] Stepfun … Step 5 Preview:
+// neighbouring queries reuse one selection).
+//
+// A CTA takes 8 consecutive queries of one request and one KV group: 128 rows (query, head) of
+// one attention tile.  The union of their selections is built in smem as in the mma.sync
+// shared-selection kernel (a region bitmap, compacted in region order) together with each
+// union region's 8-bit membership (which queries selected it).  The union streams in tiles of
+// 8 regions (64 tokens), flash-attention style:
+//  * a TMA warp loads each region's K and V (8 tokens x 192: three 8 x 64 boxes, 128-byte
+//    swizzle, laid out [block][8 rows][128 B] so that 8-token atoms sit 3 KiB apart) into a
+//    2-stage ring; a region that is invalid or past the union is loaded from rows past the
+//    cache, which fill zeros;
+//  * one thread issues S = Q K^T (M = 128, N = 64, K = 192: 12 tcgen05.mma.kind::f16) into
+//    one of two 64-column TMEM buffers, and O += P V (M = 128, N = 192, K = 64: 4 MMAs, V as
+//    an MN-major operand) into a 192-column TMEM accumulator; S of tile i+1 runs while the
+//    softmax of tile i does;
+//  * four softmax warps (one row per thread, the TMEM lane) mask the tile (the region must
+//    be the row's query's, the token at or before its position), keep the online softmax in
+//    exp2 with lazy rescaling (the reference max moves only past a slack of 2^8; O is
+//    rescaled in TMEM then), write P as bf16 into smem (the A operand of P V), and at the end
+//    write O / l and the LSE.
+// Blocks spanning several requests, with an invalid query, or whose union exceeds twice the
+// longest selection are flagged in row_shared and left to the per-row kernel that runs next.
+#pragma once
+
+#include <climits>
+
+#include "attention.cuh"
+#include "topk_cluster.cuh"
+
+namespace dsa {
+namespace attntc {
+
+using attn::Params;
+
+constexpr int kQueries = 8;                          // queries per CTA: 8 x 16 heads = 128 rows
+constexpr int kThreads = 256;                        // warp 0 TMA, warp 1 MMA, warps 4..7 softmax
+constexpr int kMaxK = 512;                           // selection length per query
+constexpr int kMaxUnion = 2 * kMaxK;                 // a longer union is not shared
+constexpr int kMaxWords = 8192;                      // bitmap words: regions < 262,144
+constexpr int kTileRegions = 8;                      // regions per tile: 64 tokens
+constexpr int kRegionBox = 3 * 8 * 128;              // one region of K or V: [3 blocks][8 rows][128 B]
+constexpr int kTileBytes = kTileRegions * kRegionBox;        // 24 KiB
+constexpr int kStages = 2;
+// smem layout (bytes, after 1024-byte alignment)
+constexpr size_t kOffQ = 0;                                          // Q: [3 blocks][128 rows][128 B]
+constexpr size_t kOffKV = kOffQ + 3 * 128 * 128;                     // kStages x (K tile, V tile)
+constexpr size_t kOffP = kOffKV + (size_t)kStages * 2 * kTileBytes;  // P: 2 x [128 rows][128 B]
+constexpr size_t kOffUni = kOffP + 2 * 128 * 128;                    // [kMaxUnion] region ids
+constexpr size_t kOffRow = kOffUni + (size_t)kMaxUnion * 4;          // [kMaxUnion] cache rows (TMA y)
+constexpr size_t kOffMask = kOffRow + (size_t)kMaxUnion * 4;         // [kMaxUnion / 4] membership bytes
+constexpr size_t kOffBars = kOffMask + (size_t)kMaxUnion;
+constexpr size_t kSmemBytes = 1024 + kOffBars + 256;
+// set-up scratch, overlaid on the K/V ring (used before the first load)
+constexpr size_t kOffBitmap = kOffKV;                                // [kMaxWords]
+constexpr size_t kOffSel = kOffBitmap + (size_t)kMaxWords * 4;       // [8][kMaxK]
+static_assert(kOffSel + (size_t)kQueries * kMaxK * 4 <= kOffP, "set-up scratch fits the ring");
+static_assert(kSmemBytes <= 232448, "one CTA per SM");
+constexpr int kTmemCols = 512;                                       // S: 2 x 64 columns, O: 192 at 256
+constexpr int kOCol = 256;
+
+// Shared-memory descriptor, 128-byte swizzle, with explicit leading / stride byte offsets.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t smem_addr, uint32_t lbo, uint32_t sbo)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1u << 46;                               // descriptor version (sm_100)
+    d |= (uint64_t)2u << 61;                               // layout: 128-byte swizzle
+    return d;
+}
+
+// kind::f16 instruction descriptor: BF16 x BF16 -> F32; b_mn: B operand MN-major.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn)
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         bool accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
+        : "memory");
+}
+
+// 32 consecutive fp32 columns of this warp's 32 TMEM lanes written from registers.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        ::"r"(taddr), "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]),
+          "f"(v[8]), "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15]),
+          "f"(v[16]), "f"(v[17]), "f"(v[18]), "f"(v[19]), "f"(v[20]), "f"(v[21]), "f"(v[22]), "f"(v[23]),
+          "f"(v[24]), "f"(v[25]), "f"(v[26]), "f"(v[27]), "f"(v[28]), "f"(v[29]), "f"(v[30]), "f"(v[31])
+        : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// byte offset of 16-byte chunk c of row r in a [rows][128 B] tile with the 128-byte swizzle
+__device__ __forceinline__ uint32_t sw128_off(int r, int c)
+{
+    return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
+}
+
+// tmap_k / tmap_v: 2-D views [n_pages * 4 * 64 rows][192] of the caches, box 64 x 8 rows
+// (one 64-wide column block of a region), 128-byte swizzle.  kv_rows: the views' row count
+// (a load there reads zeros).
+__global__ void __launch_bounds__(kThreads, 1)
+    sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+                          const Params p, int kv_rows)
+{
+    pdl_trigger();   // the next kernel may launch; it waits for this one itself
+    pdl_wait();      // the previous kernel's results are visible from here on
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *qs = smem + kOffQ;
+    uint8_t *kvs = smem + kOffKV;
+    uint8_t *pst = smem + kOffP;
+    int32_t *uni = reinterpret_cast<int32_t *>(smem + kOffUni);
+    int32_t *urow = reinterpret_cast<int32_t *>(smem + kOffRow);
+    uint32_t *umask = reinterpret_cast<uint32_t *>(smem + kOffMask);
+    uint32_t *bitmap = reinterpret_cast<uint32_t *>(smem + kOffBitmap);
+    int32_t *sels = reinterpret_cast<int32_t *>(smem + kOffSel);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBars);
+    uint64_t *kv_full = bars, *kv_empty = bars + 2, *s_full = bars + 4, *s_empty = bars + 6;
+    uint64_t *p_full = bars + 8, *p_free = bars + 10, *o_done = bars + 12;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 13);
+    __shared__ uint32_t scan_ws[40];
+    __shared__ int sh_req[kQueries], sh_pos[kQueries], sh_cnt[kQueries], sh_own[kQueries];
+    __shared__ int sh_U;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+    // group-major block order: the CTAs resident together gather from one group's cache
+    const int n_qblocks = (int)gridDim.x / kG;
+    const int g = (int)blockIdx.x / n_qblocks;
+    const int q0 = ((int)blockIdx.x - g * n_qblocks) * kQueries;
+
+    // ---- the block's queries: request, position, own region, selection count
+    if (tid < kQueries) {
+        const int q = q0 + tid;
+        int req = -1, pos = -1, c = 0;
+        if (q < p.nq) {
+            const int b = p.q_req ? p.q_req[q] : q;
+            pos = p.q_pos[q];
+            const int craw = p.sel_count[(int64_t)q * kG + g];
+            c = min(max(craw, 0), p.k);
+            if (c != craw) set_error(kErrAttnIndex);
+            if (b < 0 || b >= p.n_req || pos < 0) set_error(kErrAttnIndex);
+            else req = b;
+        }
+        sh_req[tid] = req;
+        sh_pos[tid] = pos;
+        sh_own[tid] = pos >= 0 ? pos / kRegion : -1;
+        sh_cnt[tid] = req >= 0 ? c : 0;
+    }
+    __syncthreads();
+    // served here: every query of the block valid and of one request, and a small union
+    int R = -1, maxc = 0, max_own = -1;
+    bool share = true;
+    for (int w = 0; w < kQueries; ++w) {
+        if (q0 + w >= p.nq) continue;
+        if (sh_req[w] < 0 || (R >= 0 && sh_req[w] != R)) share = false;
+        R = sh_req[w];
+        maxc = max(maxc, sh_cnt[w]);
+        max_own = max(max_own, sh_own[w]);
+    }
+    share = share && R >= 0 && maxc > 0;
+    const int words = share ? min(kMaxWords, (max_own + 1 + 31) / 32) : 0;
+    if (share) {
+        // ---- the union of the selections (region bitmap), each query's entries kept
+        for (int i = tid; i < words; i += kThreads) bitmap[i] = 0u;
+        __syncthreads();
+        if (warp < kQueries && q0 + warp < p.nq) {
+            const int c = sh_cnt[warp];
+            const int32_t *src = p.sel_idx + ((int64_t)(q0 + warp) * kG + g) * p.k;
+            for (int i = lane; i < c; i += 32) {
+                int r = src[i];
+                if (r < 0 || r > sh_own[warp] || r / 8 >= p.max_pages || (r >> 5) >= words) {
+                    set_error(kErrAttnIndex);
+                    r = -1;
+                }
+                sels[warp * kMaxK + i] = r;
+                if (r >= 0) atomicOr(&bitmap[r >> 5], 1u << (r & 31));
+            }
+        }
+        __syncthreads();
+        const int wpt = (words + kThreads - 1) / kThreads;
+        const int w0 = tid * wpt;
+        uint32_t n = 0;
+        for (int i = 0; i < wpt; ++i)
+            if (w0 + i < words) n += __popc(bitmap[w0 + i]);
+        const uint32_t incl = topkc::block_scan_incl<kThreads>(n, scan_ws);
+        const uint32_t total = scan_ws[kThreads / 32 - 1];
+        share = total > 0 && total <= 2u * (uint32_t)maxc && total <= (uint32_t)kMaxUnion;
+        if (share) {
+            uint32_t pos = incl - n;
+            for (int i = 0; i < wpt; ++i) {
+                if (w0 + i >= words) break;
+                uint32_t b = bitmap[w0 + i];
+                while (b) {
+                    const int bit = __ffs(b) - 1;
+                    b &= b - 1;
+                    uni[pos++] = (w0 + i) * 32 + bit;
+                }
+            }
+        }
+        if (tid == 0) sh_U = (int)total;
+        __syncthreads();
+    }
+    if (p.row_shared && tid < kQueries && q0 + tid < p.nq) p.row_shared[(int64_t)(q0 + tid) * kG + g] = share ? 1 : 0;
+    if (!share) return;                                   // block-uniform: the per-row kernel serves it
+    const int U = sh_U;
+    // ---- each union region's first cache row (through the block table, all at once; a bad
+    // page reads zeros), and membership: bit 8 (u % 4) + w of word u / 4 when query w selected
+    // union region u
+    for (int u = tid; u < U; u += kThreads) {
+        const int r = uni[u];
+        const int64_t page = p.block_table[(int64_t)R * p.max_pages + r / 8];
+        int y = kv_rows;
+        if (page >= 0 && page < p.n_pages) y = (int)((page * kG + g) * kPage + (r % 8) * kRegion);
+        else set_error(kErrAttnIndex);
+        urow[u] = y;
+    }
+    for (int i = tid; i < (U + 3) / 4; i += kThreads) umask[i] = 0u;
+    __syncthreads();
+    if (warp < kQueries && q0 + warp < p.nq) {
+        const int c = sh_cnt[warp];
+        for (int i = lane; i < c; i += 32) {
+            const int r = sels[warp * kMaxK + i];
+            if (r < 0) continue;
+            int lo = 0, hi = U - 1;                         // uni is ascending and holds r
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (uni[mid] < r) lo = mid + 1;
+                else hi = mid;
+            }
+            atomicOr(&umask[lo >> 2], 1u << ((lo & 3) * 8 + warp));
+        }
+    }
+    // ---- Q tile: row (query qq, head h) = 16 qq + h, K-major in 3 swizzled 64-wide blocks
+    for (int i = tid; i < 128 * (kD / 8); i += kThreads) {
+        const int r = i / (kD / 8), c16 = i % (kD / 8);
+        const int q = q0 + (r >> 4);
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (q < p.nq)
+            v = __ldg(reinterpret_cast<const uint4 *>(p.q + ((int64_t)q * kHQ + g * kHeadsPerGroup + (r & 15)) * kD +
+                                                      c16 * 8));
+        *reinterpret_cast<uint4 *>(qs + (c16 >> 3) * (128 * 128) + sw128_off(r, c16 & 7)) = v;
+    }
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&s_full[b], 1);
+            mbar_init(&s_empty[b], 4);
+            mbar_init(&p_full[b], 4);
+            mbar_init(&p_free[b], 1);
+        }
+        mbar_init(o_done, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
+    fence_proxy_async();                                  // Q and the reused scratch, for the async proxy
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int n_tiles = (U + kTileRegions - 1) / kTileRegions;
+    bool ok = true;
+
+    if (warp == 0) {
+        // ---------------- TMA producer (one lane): K and V of 8 union regions per tile
+        if (lane == 0) {
+            prefetch_tensormap(&tmap_k);
+            prefetch_tensormap(&tmap_v);
+            for (int i = 0; i < n_tiles && ok; ++i) {
+                const int s = i % kStages;
+                ok = mbar_wait_sleep(&kv_empty[s], ((i / kStages) & 1) ^ 1);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&kv_full[s], 2 * kTileBytes);
+                uint8_t *kd = kvs + s * 2 * kTileBytes, *vd = kd + kTileBytes;
+                for (int jr = 0; jr < kTileRegions; ++jr) {
+                    const int u = i * kTileRegions + jr;
+                    const int y = u < U ? urow[u] : kv_rows;    // past the union: zeros
+#pragma unroll
+                    for (int blk = 0; blk < 3; ++blk) {
+                        tma_load_2d(kd + jr * kRegionBox + blk * 1024, &tmap_k, blk * 64, y, &kv_full[s]);
+                        tma_load_2d(vd + jr * kRegionBox + blk * 1024, &tmap_v, blk * 64, y, &kv_full[s]);
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer (one lane): S(i), then O += P(i-1) V(i-1)
+        if (lane == 0) {
+            constexpr uint32_t kIdS = idesc_bf16(128, 64, false), kIdO = idesc_bf16(128, kD, true);
+            const uint32_t qa = smem_u32(qs);
+            auto issue_pv = [&](int j) {
+                const int s = j % kStages, pb = j & 1;
+                ok = ok && mbar_wait_sleep(&p_full[pb], (j >> 1) & 1);
+                if (!ok) return;
+                tc_fence_after();
+                const uint32_t pa = smem_u32(pst + pb * (128 * 128));
+                const uint32_t vb = smem_u32(kvs + s * 2 * kTileBytes + kTileBytes);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)                  // 16 tokens (two regions) per instruction
+                    mma_bf16(tmem + kOCol, desc_sw128(pa + kk * 32, 16, 1024),
+                             desc_sw128(vb + kk * 2 * kRegionBox, 1024, kRegionBox), kIdO, j > 0 || kk > 0);
+                umma_commit(&p_free[pb]);                       // P(j) read
+                umma_commit(&kv_empty[s]);                      // K(j) and V(j) read
+                umma_commit(o_done);                            // O holds the tiles up to j
+            };
+            for (int i = 0; i < n_tiles && ok; ++i) {
+                const int s = i % kStages, sb = i & 1;
+                ok = mbar_wait_sleep(&kv_full[s], (i / kStages) & 1) &&
+                     mbar_wait_sleep(&s_empty[sb], ((i >> 1) & 1) ^ 1);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t kb = smem_u32(kvs + s * 2 * kTileBytes);
+#pragma unroll
+                for (int blk = 0; blk < 3; ++blk)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)              // 16 dims per instruction
+                        mma_bf16(tmem + sb * 64, desc_sw128(qa + blk * (128 * 128) + kk * 32, 16, 1024),
+                                 desc_sw128(kb + blk * 1024 + kk * 32, 16, kRegionBox), kIdS, blk > 0 || kk > 0);
+                umma_commit(&s_full[sb]);
+                if (i > 0) issue_pv(i - 1);
+            }
+            if (ok && n_tiles > 0) issue_pv(n_tiles - 1);
+        }
+    } else if (warp >= 4) {
+        // ---------------- softmax warps 4..7: TMEM lane quarter warp % 4, row r = query, head
+        const int r = (warp & 3) * 32 + lane;
+        const int qq = r >> 4, h = r & 15;
+        const int q = q0 + qq;
+        const bool qv = q < p.nq;
+        const int pos = qv ? sh_pos[qq] : -1;
+        const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        float mrow = -INFINITY, lrow = 0.0f;
+        for (int i = 0; i < n_tiles && ok; ++i) {
+            const int sb = i & 1;
+            ok = __all_sync(0xffffffffu, mbar_wait_sleep(&s_full[sb], (i >> 1) & 1));
+            if (!ok) break;
+            tc_fence_after();
+            float sv[64];
+            {
+                float a[32], b[32];
+                tmem_ld32x2(trow + sb * 64, trow + sb * 64 + 32, a, b);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    sv[j] = a[j];
+                    sv[32 + j] = b[j];
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_empty[sb]);       // the MMA may write S(i + 2) here
+            // mask: a union region this row's query selected, tokens at or before its position
+            float mx = -INFINITY;
+#pragma unroll
+            for (int jr = 0; jr < kTileRegions; ++jr) {
+                const int u = i * kTileRegions + jr;
+                const bool member = u < U && ((umask[u >> 2] >> ((u & 3) * 8 + qq)) & 1u);
+                const int t0 = member ? uni[u] * kRegion : INT_MAX;
+#pragma unroll
+                for (int e = 0; e < kRegion; ++e) {
+                    const bool keep = member && t0 + e <= pos;
+                    const float v = keep ? sv[jr * kRegion + e] * p.scale_log2 : -INFINITY;
+                    sv[jr * kRegion + e] = v;
+                    mx = fmaxf(mx, v);
+                }
+            }
+            // lazy rescaling: the reference max moves only when the tile's max exceeds it by more
+            // than the slack (P stays below 2^slack): the same softmax, rarely rescaled
+            const bool grow = mx > mrow + attn::kSlack;
+            float alpha = 1.0f;
+            if (grow) {
+                alpha = exp2f(mrow - mx);
+                mrow = mx;
+            }
+            const float mref = (mrow == -INFINITY) ? 0.0f : mrow;
+            float ps = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 64; ++j) {
+                const float pv = exp2f(sv[j] - mref);
+                sv[j] = pv;
+                ps += pv;
+            }
+            lrow = lrow * alpha + ps;
+            if (__any_sync(0xffffffffu, grow && i > 0)) {
+                // O holds the tiles before i once their P V has completed: scale it in TMEM
+                ok = __all_sync(0xffffffffu, mbar_wait_sleep(o_done, (i - 1) & 1));
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int c = 0; c < kD / 32; ++c) {
+                    float o[32];
+                    tmem_ld32(trow + kOCol + 32 * c, o);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) o[j] *= alpha;
+                    tmem_st32(trow + kOCol + 32 * c, o);
+                }
+                tc_fence_before();
+            }
+            // P(i) as bf16 into the A-operand tile of P V (row r, 128-byte swizzle)
+            ok = __all_sync(0xffffffffu, mbar_wait_sleep(&p_free[sb], ((i >> 1) & 1) ^ 1));
+            if (!ok) break;
+            uint8_t *pr = pst + sb * (128 * 128);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint4 w;
+                w.x = pack_bf16x2(sv[8 * c + 0], sv[8 * c + 1]);
+                w.y = pack_bf16x2(sv[8 * c + 2], sv[8 * c + 3]);
+                w.z = pack_bf16x2(sv[8 * c + 4], sv[8 * c + 5]);
+                w.w = pack_bf16x2(sv[8 * c + 6], sv[8 * c + 7]);
+                *reinterpret_cast<uint4 *>(pr + sw128_off(r, c)) = w;
+            }
+            fence_proxy_async();                               // generic writes -> the MMA's reads
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[sb]);
+        }
+        // ---- output: O / l (bf16) and the LSE, once the last P V has completed
+        if (ok && n_tiles > 0) ok = __all_sync(0xffffffffu, mbar_wait_sleep(o_done, (n_tiles - 1) & 1));
+        if (ok) {
+            tc_fence_after();
+            const float inv = lrow > 0.0f ? 1.0f / lrow : 0.0f;
+            __nv_bfloat16 *dst = p.out + ((int64_t)q * kHQ + g * kHeadsPerGroup + h) * kD;
+#pragma unroll 1
+            for (int c = 0; c < kD / 32; ++c) {
+                float o[32];
+                tmem_ld32(trow + kOCol + 32 * c, o);
+                if (qv) {
+#pragma unroll
+                    for (int k8 = 0; k8 < 4; ++k8) {
+                        uint4 w;
+                        w.x = pack_bf16x2(o[8 * k8 + 0] * inv, o[8 * k8 + 1] * inv);
+                        w.y = pack_bf16x2(o[8 * k8 + 2] * inv, o[8 * k8 + 3] * inv);
+                        w.z = pack_bf16x2(o[8 * k8 + 4] * inv, o[8 * k8 + 5] * inv);
+                        w.w = pack_bf16x2(o[8 * k8 + 6] * inv, o[8 * k8 + 7] * inv);
+                        reinterpret_cast<uint4 *>(dst + 32 * c)[k8] = w;
+                    }
+                }
+            }
+            if (qv && p.lse)
+                p.lse[(int64_t)q * kHQ + g * kHeadsPerGroup + h] =
+                    lrow > 0.0f ? (mrow + log2f(lrow)) * 0.69314718055994531f : -INFINITY;
+        }
+    }
+    // every role done (or gave up): release TMEM
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_free(tmem, kTmemCols);
+}
+
+}  // namespace attntc
+}  // namespace dsa

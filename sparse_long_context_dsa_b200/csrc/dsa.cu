@@ -12,6 +12,7 @@
 #include "attention.cuh"
 #include "attention_cluster.cuh"
 #include "attention_shared.cuh"
+#include "attention_tc.cuh"
 #include "common.cuh"
 #include "compress.cuh"
 #include "copy.cuh"
@@ -145,6 +146,16 @@ dsa_status_t kv_map(CUtensorMap *m, const void *cache, int64_t n_pages)
     const cuuint64_t strides[2] = {128, (cuuint64_t)dsa::kD * 2};
     const cuuint32_t box[3] = {64, 3, (cuuint32_t)dsa::kRegion};
     return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, cache, dims, strides, box, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+}
+
+// 2-D view [n_pages * 4 * 64 rows][192] of a K/V cache: one 64-wide column block of 8 rows
+// per box (the tcgen05 shared-selection attention's operand tiles).
+dsa_status_t kv_map_rows(CUtensorMap *m, const void *cache, int64_t n_pages)
+{
+    const cuuint64_t dims[2] = {(cuuint64_t)dsa::kD, (cuuint64_t)n_pages * dsa::kG * dsa::kPage};
+    const cuuint64_t strides[1] = {(cuuint64_t)dsa::kD * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)dsa::kRegion};
+    return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, cache, dims, strides, box, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 }
 
 struct TopkLayout {
@@ -302,17 +313,22 @@ dsa_status_t attn_common(const void *q, const void *k_cache, const void *v_cache
 
     if (clustered) return attn_cluster_launch(mk, mv, p, nq, stream);
     if (shared) {
+        // 8 neighbouring queries of one request with a small union: tcgen05 tiles of 128 rows
         p.row_shared = static_cast<uint8_t *>(ws) + plan.ws;
         static std::once_flag sh_once;
         static cudaError_t sh_err = cudaSuccess;
         std::call_once(sh_once, [] {
-            sh_err = cudaFuncSetAttribute(dsa::attns::sparse_attn_shared_kernel,
-                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsa::attns::kSmemBytes);
+            sh_err = cudaFuncSetAttribute(dsa::attntc::sparse_attn_tc_kernel,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsa::attntc::kSmemBytes);
         });
-        DSA_CUDA(sh_err, "cudaFuncSetAttribute(sparse_attn_shared_kernel)");
-        const unsigned blocks = (unsigned)((nq + dsa::attns::kQueries - 1) / dsa::attns::kQueries) * dsa::kG;
-        if ((st = launch_k("sparse_attn_shared_kernel", dsa::attns::sparse_attn_shared_kernel, dim3(blocks),
-                           dim3(dsa::attns::kThreads), dsa::attns::kSmemBytes, stream, 0, mk, mv, p)) != DSA_OK)
+        DSA_CUDA(sh_err, "cudaFuncSetAttribute(sparse_attn_tc_kernel)");
+        CUtensorMap rk, rv;
+        if ((st = kv_map_rows(&rk, k_cache, n_pages)) != DSA_OK) return st;
+        if ((st = kv_map_rows(&rv, v_cache, n_pages)) != DSA_OK) return st;
+        const unsigned blocks = (unsigned)((nq + dsa::attntc::kQueries - 1) / dsa::attntc::kQueries) * dsa::kG;
+        if ((st = launch_k("sparse_attn_tc_kernel", dsa::attntc::sparse_attn_tc_kernel, dim3(blocks),
+                           dim3(dsa::attntc::kThreads), dsa::attntc::kSmemBytes, stream, 0, rk, rv, p,
+                           (int)(n_pages * dsa::kG * dsa::kPage))) != DSA_OK)
             return st;
         // then the rows it left to the per-row kernel (the others return at once)
     }
