@@ -7,19 +7,20 @@
 // shared-selection kernel (a region bitmap, compacted in region order) together with each
 // union region's 8-bit membership (which queries selected it).  The union streams in tiles of
 // 8 regions (64 tokens), flash-attention style:
-//  * a TMA warp loads each region's K and V (8 tokens x 192: three 8 x 64 boxes, 128-byte
-//    swizzle, laid out [block][8 rows][128 B] so that 8-token atoms sit 3 KiB apart) into a
-//    2-stage ring; a region that is invalid or past the union is loaded from rows past the
+//  * two TMA warps load each region's K (one warp) and V (the other) as three 8 x 64 boxes
+//    (128-byte swizzle, laid out [block][8 rows][128 B] so that 8-token atoms sit 3 KiB
+//    apart) into separate 3-stage rings: a K stage frees as soon as S has read it, a V stage
+//    once P V has; a region that is invalid or past the union is loaded from rows past the
 //    cache, which fill zeros;
 //  * one thread issues S = Q K^T (M = 128, N = 64, K = 192: 12 tcgen05.mma.kind::f16) into
-//    one of two 64-column TMEM buffers, and O += P V (M = 128, N = 192, K = 64: 4 MMAs, V as
-//    an MN-major operand) into a 192-column TMEM accumulator; S of tile i+1 runs while the
-//    softmax of tile i does;
+//    one of two 64-column TMEM buffers, and O += P V (M = 128, N = 192, K = 64: 4 MMAs with
+//    P read from TMEM and V an MN-major smem operand) into a 192-column TMEM accumulator;
+//    S of tile i+1 runs while the softmax of tile i does;
 //  * four softmax warps (one row per thread, the TMEM lane) mask the tile (the region must
 //    be the row's query's, the token at or before its position), keep the online softmax in
 //    exp2 with lazy rescaling (the reference max moves only past a slack of 2^8; O is
-//    rescaled in TMEM then), write P as bf16 into smem (the A operand of P V), and at the end
-//    write O / l and the LSE.
+//    rescaled in TMEM then), write P as packed bf16 into TMEM (two tokens per column, the
+//    A operand of P V), and at the end write O / l and the LSE.
 // Blocks spanning several requests, with an invalid query, or whose union exceeds twice the
 // longest selection are flagged in row_shared and left to the per-row kernel that runs next.
 #pragma once
@@ -35,29 +36,31 @@ namespace attntc {
 using attn::Params;
 
 constexpr int kQueries = 8;                          // queries per CTA: 8 x 16 heads = 128 rows
-constexpr int kThreads = 256;                        // warp 0 TMA, warp 1 MMA, warps 4..7 softmax
+constexpr int kThreads = 256;                        // warp 0 K loads, 1 MMA, 2 V loads, 4..7 softmax
 constexpr int kMaxK = 512;                           // selection length per query
 constexpr int kMaxUnion = 2 * kMaxK;                 // a longer union is not shared
 constexpr int kMaxWords = 8192;                      // bitmap words: regions < 262,144
 constexpr int kTileRegions = 8;                      // regions per tile: 64 tokens
 constexpr int kRegionBox = 3 * 8 * 128;              // one region of K or V: [3 blocks][8 rows][128 B]
-constexpr int kTileBytes = kTileRegions * kRegionBox;        // 24 KiB
-constexpr int kStages = 2;
+constexpr int kTileBytes = kTileRegions * kRegionBox;        // 24 KiB: K or V of one tile
+constexpr int kStages = 3;                                   // per ring (K and V)
 // smem layout (bytes, after 1024-byte alignment)
 constexpr size_t kOffQ = 0;                                          // Q: [3 blocks][128 rows][128 B]
-constexpr size_t kOffKV = kOffQ + 3 * 128 * 128;                     // kStages x (K tile, V tile)
-constexpr size_t kOffP = kOffKV + (size_t)kStages * 2 * kTileBytes;  // P: 2 x [128 rows][128 B]
-constexpr size_t kOffUni = kOffP + 2 * 128 * 128;                    // [kMaxUnion] region ids
+constexpr size_t kOffK = kOffQ + 3 * 128 * 128;                      // kStages K tiles
+constexpr size_t kOffV = kOffK + (size_t)kStages * kTileBytes;       // kStages V tiles
+constexpr size_t kOffUni = kOffV + (size_t)kStages * kTileBytes;     // [kMaxUnion] region ids
 constexpr size_t kOffRow = kOffUni + (size_t)kMaxUnion * 4;          // [kMaxUnion] cache rows (TMA y)
 constexpr size_t kOffMask = kOffRow + (size_t)kMaxUnion * 4;         // [kMaxUnion / 4] membership bytes
 constexpr size_t kOffBars = kOffMask + (size_t)kMaxUnion;
 constexpr size_t kSmemBytes = 1024 + kOffBars + 256;
-// set-up scratch, overlaid on the K/V ring (used before the first load)
-constexpr size_t kOffBitmap = kOffKV;                                // [kMaxWords]
+// set-up scratch, overlaid on the K/V rings (used before the first load)
+constexpr size_t kOffBitmap = kOffK;                                 // [kMaxWords]
 constexpr size_t kOffSel = kOffBitmap + (size_t)kMaxWords * 4;       // [8][kMaxK]
-static_assert(kOffSel + (size_t)kQueries * kMaxK * 4 <= kOffP, "set-up scratch fits the ring");
+static_assert(kOffSel + (size_t)kQueries * kMaxK * 4 <= kOffUni, "set-up scratch fits the rings");
 static_assert(kSmemBytes <= 232448, "one CTA per SM");
-constexpr int kTmemCols = 512;                                       // S: 2 x 64 columns, O: 192 at 256
+// TMEM columns: S at 0 and 64, P (64 bf16 tokens in 32 columns) at 128 and 160, O at 256
+constexpr int kTmemCols = 512;
+constexpr int kPCol = 128;
 constexpr int kOCol = 256;
 
 // Shared-memory descriptor, 128-byte swizzle, with explicit leading / stride byte offsets.
@@ -88,6 +91,27 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
         ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
         : "memory");
+}
+
+// The same with A read from TMEM (M lanes, two 16-bit K elements per 32-bit column, the
+// lower K element in the lower half).
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            bool accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
+        : "memory");
+}
+
+// hardware base-2 exponential (ex2.approx, flush-to-zero); ex2(-inf) = +0
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 // 32 consecutive fp32 columns of this warp's 32 TMEM lanes written from registers.
@@ -122,17 +146,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *qs = smem + kOffQ;
-    uint8_t *kvs = smem + kOffKV;
-    uint8_t *pst = smem + kOffP;
+    uint8_t *ks = smem + kOffK;
+    uint8_t *vs = smem + kOffV;
     int32_t *uni = reinterpret_cast<int32_t *>(smem + kOffUni);
     int32_t *urow = reinterpret_cast<int32_t *>(smem + kOffRow);
     uint32_t *umask = reinterpret_cast<uint32_t *>(smem + kOffMask);
     uint32_t *bitmap = reinterpret_cast<uint32_t *>(smem + kOffBitmap);
     int32_t *sels = reinterpret_cast<int32_t *>(smem + kOffSel);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBars);
-    uint64_t *kv_full = bars, *kv_empty = bars + 2, *s_full = bars + 4, *s_empty = bars + 6;
-    uint64_t *p_full = bars + 8, *p_free = bars + 10, *o_done = bars + 12;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 13);
+    uint64_t *k_full = bars, *k_empty = bars + kStages, *v_full = bars + 2 * kStages, *v_empty = bars + 3 * kStages;
+    uint64_t *s_full = bars + 4 * kStages, *s_empty = s_full + 2, *p_full = s_full + 4, *p_free = s_full + 6;
+    uint64_t *o_done = s_full + 8;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_done + 1);
+    static_assert((4 * kStages + 9) * 8 + 4 <= 256, "barriers fit their slot");
     __shared__ uint32_t scan_ws[40];
     __shared__ int sh_req[kQueries], sh_pos[kQueries], sh_cnt[kQueries], sh_own[kQueries];
     __shared__ int sh_U;
@@ -257,8 +283,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&kv_full[s], 1);
-            mbar_init(&kv_empty[s], 1);
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&s_full[b], 1);
@@ -278,26 +306,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n_tiles = (U + kTileRegions - 1) / kTileRegions;
     bool ok = true;
 
-    if (warp == 0) {
-        // ---------------- TMA producer (one lane): K and V of 8 union regions per tile
-        if (lane == 0) {
-            prefetch_tensormap(&tmap_k);
-            prefetch_tensormap(&tmap_v);
-            for (int i = 0; i < n_tiles && ok; ++i) {
-                const int s = i % kStages;
-                ok = mbar_wait_sleep(&kv_empty[s], ((i / kStages) & 1) ^ 1);
-                if (!ok) break;
-                mbar_arrive_expect_tx(&kv_full[s], 2 * kTileBytes);
-                uint8_t *kd = kvs + s * 2 * kTileBytes, *vd = kd + kTileBytes;
-                for (int jr = 0; jr < kTileRegions; ++jr) {
-                    const int u = i * kTileRegions + jr;
-                    const int y = u < U ? urow[u] : kv_rows;    // past the union: zeros
+    if (warp == 0 || warp == 2) {
+        // ---------------- TMA producers: warp 0 loads K, warp 2 loads V; lane j < 8 issues
+        // region j of each tile (three 8 x 64 boxes)
+        const bool is_k = warp == 0;
+        const CUtensorMap *map = is_k ? &tmap_k : &tmap_v;
+        uint8_t *ring = is_k ? ks : vs;
+        uint64_t *full = is_k ? k_full : v_full, *empty = is_k ? k_empty : v_empty;
+        if (lane == 0) prefetch_tensormap(map);
+        for (int i = 0; i < n_tiles && ok; ++i) {
+            const int s = i % kStages;
+            int got = 1;
+            if (lane == 0) {
+                got = mbar_wait_sleep(&empty[s], ((i / kStages) & 1) ^ 1) ? 1 : 0;
+                if (got) mbar_arrive_expect_tx(&full[s], kTileBytes);
+            }
+            ok = __shfl_sync(0xffffffffu, got, 0) != 0;
+            if (!ok) break;
+            if (lane < kTileRegions) {
+                const int u = i * kTileRegions + lane;
+                const int y = u < U ? urow[u] : kv_rows;        // past the union: zeros
+                uint8_t *dst = ring + s * kTileBytes + lane * kRegionBox;
 #pragma unroll
-                    for (int blk = 0; blk < 3; ++blk) {
-                        tma_load_2d(kd + jr * kRegionBox + blk * 1024, &tmap_k, blk * 64, y, &kv_full[s]);
-                        tma_load_2d(vd + jr * kRegionBox + blk * 1024, &tmap_v, blk * 64, y, &kv_full[s]);
-                    }
-                }
+                for (int blk = 0; blk < 3; ++blk) tma_load_2d(dst + blk * 1024, map, blk * 64, y, &full[s]);
             }
         }
     } else if (warp == 1) {
@@ -307,26 +338,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t qa = smem_u32(qs);
             auto issue_pv = [&](int j) {
                 const int s = j % kStages, pb = j & 1;
-                ok = ok && mbar_wait_sleep(&p_full[pb], (j >> 1) & 1);
+                ok = ok && mbar_wait_sleep(&p_full[pb], (j >> 1) & 1) &&
+                     mbar_wait_sleep(&v_full[s], (j / kStages) & 1);
                 if (!ok) return;
                 tc_fence_after();
-                const uint32_t pa = smem_u32(pst + pb * (128 * 128));
-                const uint32_t vb = smem_u32(kvs + s * 2 * kTileBytes + kTileBytes);
+                const uint32_t vb = smem_u32(vs + s * kTileBytes);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)                  // 16 tokens (two regions) per instruction
-                    mma_bf16(tmem + kOCol, desc_sw128(pa + kk * 32, 16, 1024),
-                             desc_sw128(vb + kk * 2 * kRegionBox, 1024, kRegionBox), kIdO, j > 0 || kk > 0);
+                    mma_bf16_ts(tmem + kOCol, tmem + kPCol + pb * 32 + kk * 8,
+                                desc_sw128(vb + kk * 2 * kRegionBox, 1024, kRegionBox), kIdO, j > 0 || kk > 0);
                 umma_commit(&p_free[pb]);                       // P(j) read
-                umma_commit(&kv_empty[s]);                      // K(j) and V(j) read
+                umma_commit(&v_empty[s]);                       // V(j) read
                 umma_commit(o_done);                            // O holds the tiles up to j
             };
             for (int i = 0; i < n_tiles && ok; ++i) {
                 const int s = i % kStages, sb = i & 1;
-                ok = mbar_wait_sleep(&kv_full[s], (i / kStages) & 1) &&
+                ok = mbar_wait_sleep(&k_full[s], (i / kStages) & 1) &&
                      mbar_wait_sleep(&s_empty[sb], ((i >> 1) & 1) ^ 1);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t kb = smem_u32(kvs + s * 2 * kTileBytes);
+                const uint32_t kb = smem_u32(ks + s * kTileBytes);
 #pragma unroll
                 for (int blk = 0; blk < 3; ++blk)
 #pragma unroll
@@ -334,6 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_bf16(tmem + sb * 64, desc_sw128(qa + blk * (128 * 128) + kk * 32, 16, 1024),
                                  desc_sw128(kb + blk * 1024 + kk * 32, 16, kRegionBox), kIdS, blk > 0 || kk > 0);
                 umma_commit(&s_full[sb]);
+                umma_commit(&k_empty[s]);                       // K(i) read
                 if (i > 0) issue_pv(i - 1);
             }
             if (ok && n_tiles > 0) issue_pv(n_tiles - 1);
@@ -346,6 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool qv = q < p.nq;
         const int pos = qv ? sh_pos[qq] : -1;
         const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        const float sc = p.scale_log2;
         float mrow = -INFINITY, lrow = 0.0f;
         for (int i = 0; i < n_tiles && ok; ++i) {
             const int sb = i & 1;
@@ -366,37 +399,40 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&s_empty[sb]);       // the MMA may write S(i + 2) here
             // mask: a union region this row's query selected, tokens at or before its position
-            float mx = -INFINITY;
+            // (token e of a region is kept when e <= lim)
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
             for (int jr = 0; jr < kTileRegions; ++jr) {
                 const int u = i * kTileRegions + jr;
                 const bool member = u < U && ((umask[u >> 2] >> ((u & 3) * 8 + qq)) & 1u);
-                const int t0 = member ? uni[u] * kRegion : INT_MAX;
+                const int lim = member ? pos - uni[u] * kRegion : -1;
 #pragma unroll
                 for (int e = 0; e < kRegion; ++e) {
-                    const bool keep = member && t0 + e <= pos;
-                    const float v = keep ? sv[jr * kRegion + e] * p.scale_log2 : -INFINITY;
+                    const float v = e <= lim ? sv[jr * kRegion + e] : -INFINITY;
                     sv[jr * kRegion + e] = v;
-                    mx = fmaxf(mx, v);
+                    m4[e & 3] = fmaxf(m4[e & 3], v);
                 }
             }
+            const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sc;   // sc > 0
             // lazy rescaling: the reference max moves only when the tile's max exceeds it by more
             // than the slack (P stays below 2^slack): the same softmax, rarely rescaled
             const bool grow = mx > mrow + attn::kSlack;
             float alpha = 1.0f;
             if (grow) {
-                alpha = exp2f(mrow - mx);
+                alpha = ex2(mrow - mx);
                 mrow = mx;
             }
-            const float mref = (mrow == -INFINITY) ? 0.0f : mrow;
-            float ps = 0.0f;
+            const float nref = (mrow == -INFINITY) ? 0.0f : -mrow;
+            float s4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            float pk[32];                                   // P(i): bf16 pairs (tokens 2c, 2c + 1)
 #pragma unroll
-            for (int j = 0; j < 64; ++j) {
-                const float pv = exp2f(sv[j] - mref);
-                sv[j] = pv;
-                ps += pv;
+            for (int c = 0; c < 32; ++c) {
+                const float p0 = ex2(fmaf(sv[2 * c], sc, nref));
+                const float p1 = ex2(fmaf(sv[2 * c + 1], sc, nref));
+                s4[c & 3] += p0 + p1;
+                pk[c] = __uint_as_float(pack_bf16x2(p0, p1));
             }
-            lrow = lrow * alpha + ps;
+            lrow = lrow * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
             if (__any_sync(0xffffffffu, grow && i > 0)) {
                 // O holds the tiles before i once their P V has completed: scale it in TMEM
                 ok = __all_sync(0xffffffffu, mbar_wait_sleep(o_done, (i - 1) & 1));
@@ -410,22 +446,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int j = 0; j < 32; ++j) o[j] *= alpha;
                     tmem_st32(trow + kOCol + 32 * c, o);
                 }
-                tc_fence_before();
             }
-            // P(i) as bf16 into the A-operand tile of P V (row r, 128-byte swizzle)
+            // P(i) into its TMEM buffer once P V has read the tile two back from it
             ok = __all_sync(0xffffffffu, mbar_wait_sleep(&p_free[sb], ((i >> 1) & 1) ^ 1));
             if (!ok) break;
-            uint8_t *pr = pst + sb * (128 * 128);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint4 w;
-                w.x = pack_bf16x2(sv[8 * c + 0], sv[8 * c + 1]);
-                w.y = pack_bf16x2(sv[8 * c + 2], sv[8 * c + 3]);
-                w.z = pack_bf16x2(sv[8 * c + 4], sv[8 * c + 5]);
-                w.w = pack_bf16x2(sv[8 * c + 6], sv[8 * c + 7]);
-                *reinterpret_cast<uint4 *>(pr + sw128_off(r, c)) = w;
-            }
-            fence_proxy_async();                               // generic writes -> the MMA's reads
+            tc_fence_after();
+            tmem_st32(trow + kPCol + sb * 32, pk);
+            tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[sb]);
         }
