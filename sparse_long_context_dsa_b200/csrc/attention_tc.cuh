@@ -9,18 +9,21 @@
 // 8 regions (64 tokens), flash-attention style:
 //  * two TMA warps load each region's K (one warp) and V (the other) as three 8 x 64 boxes
 //    (128-byte swizzle, laid out [block][8 rows][128 B] so that 8-token atoms sit 3 KiB
-//    apart) into separate 3-stage rings: a K stage frees as soon as S has read it, a V stage
+//    apart) into separate 4-stage rings: a K stage frees as soon as S has read it, a V stage
 //    once P V has; a region that is invalid or past the union is loaded from rows past the
 //    cache, which fill zeros;
-//  * one thread issues S = Q K^T (M = 128, N = 64, K = 192: 12 tcgen05.mma.kind::f16) into
-//    one of two 64-column TMEM buffers, and O += P V (M = 128, N = 192, K = 64: 4 MMAs with
+//  * one thread issues S = Q K^T (M = 128, N = 64, K = 192: 12 tcgen05.mma.kind::f16, Q
+//    read from TMEM where the softmax warps put it at the start) into one of two 64-column
+//    TMEM buffers, and O += P V (M = 128, N = 192, K = 64: 4 MMAs with
 //    P read from TMEM and V an MN-major smem operand) into a 192-column TMEM accumulator;
 //    S of tile i+1 runs while the softmax of tile i does;
-//  * four softmax warps (one row per thread, the TMEM lane) mask the tile (the region must
-//    be the row's query's, the token at or before its position), keep the online softmax in
-//    exp2 with lazy rescaling (the reference max moves only past a slack of 2^8; O is
-//    rescaled in TMEM then), write P as packed bf16 into TMEM (two tokens per column, the
-//    A operand of P V), and at the end write O / l and the LSE.
+//  * eight softmax warps, two per row (one row per thread, the TMEM lane; one warp takes the
+//    tile's first 32 tokens, the other the last 32, and the two agree on the row's running
+//    max through smem each tile), mask the tile (the region must be the row's query's, the
+//    token at or before its position), keep the online softmax in exp2 with lazy rescaling
+//    (the reference max moves only past a slack of 2^8; O is rescaled in TMEM then), write P
+//    as packed bf16 into TMEM (two tokens per column, the A operand of P V), and at the end
+//    write O / l and the LSE.
 // Blocks spanning several requests, with an invalid query, or whose union exceeds twice the
 // longest selection are flagged in row_shared and left to the per-row kernel that runs next.
 #pragma once
@@ -36,44 +39,36 @@ namespace attntc {
 using attn::Params;
 
 constexpr int kQueries = 8;                          // queries per CTA: 8 x 16 heads = 128 rows
-constexpr int kThreads = 256;                        // warp 0 K loads, 1 MMA, 2 V loads, 4..7 softmax
+constexpr int kThreads = 384;                        // warp 0 K loads, 1 MMA, 2 V loads, 4..11 softmax
 constexpr int kMaxK = 512;                           // selection length per query
 constexpr int kMaxUnion = 2 * kMaxK;                 // a longer union is not shared
 constexpr int kMaxWords = 8192;                      // bitmap words: regions < 262,144
 constexpr int kTileRegions = 8;                      // regions per tile: 64 tokens
 constexpr int kRegionBox = 3 * 8 * 128;              // one region of K or V: [3 blocks][8 rows][128 B]
 constexpr int kTileBytes = kTileRegions * kRegionBox;        // 24 KiB: K or V of one tile
-constexpr int kStages = 3;                                   // per ring (K and V)
+constexpr int kStages = 4;                                   // per ring (K and V)
 // smem layout (bytes, after 1024-byte alignment)
-constexpr size_t kOffQ = 0;                                          // Q: [3 blocks][128 rows][128 B]
-constexpr size_t kOffK = kOffQ + 3 * 128 * 128;                      // kStages K tiles
+constexpr size_t kOffK = 0;                                          // kStages K tiles
 constexpr size_t kOffV = kOffK + (size_t)kStages * kTileBytes;       // kStages V tiles
 constexpr size_t kOffUni = kOffV + (size_t)kStages * kTileBytes;     // [kMaxUnion] region ids
 constexpr size_t kOffRow = kOffUni + (size_t)kMaxUnion * 4;          // [kMaxUnion] cache rows (TMA y)
 constexpr size_t kOffMask = kOffRow + (size_t)kMaxUnion * 4;         // [kMaxUnion / 4] membership bytes
-constexpr size_t kOffBars = kOffMask + (size_t)kMaxUnion;
-constexpr size_t kSmemBytes = 1024 + kOffBars + 256;
+constexpr size_t kOffXch = kOffMask + (size_t)kMaxUnion;             // [2 buffers][2 halves][128 rows] f32
+constexpr size_t kOffBars = kOffXch + 2 * 2 * 128 * 4;
+constexpr size_t kSmemBytes = 1024 + kOffBars + 512;
 // set-up scratch, overlaid on the K/V rings (used before the first load)
 constexpr size_t kOffBitmap = kOffK;                                 // [kMaxWords]
 constexpr size_t kOffSel = kOffBitmap + (size_t)kMaxWords * 4;       // [8][kMaxK]
-static_assert(kOffSel + (size_t)kQueries * kMaxK * 4 <= kOffUni, "set-up scratch fits the rings");
+constexpr size_t kOffRank = kOffSel + (size_t)kQueries * kMaxK * 4;  // [kMaxWords] union rank of each word's first bit
+static_assert(kOffRank + (size_t)kMaxWords * 4 <= kOffUni, "set-up scratch fits the rings");
 static_assert(kSmemBytes <= 232448, "one CTA per SM");
-// TMEM columns: S at 0 and 64, P (64 bf16 tokens in 32 columns) at 128 and 160, O at 256
+// TMEM columns: S at 0 and 64; Q (192 bf16 dims, two per column) at 128; P (64 bf16 tokens
+// in 32 columns) at 224 and 256; O at 288
 constexpr int kTmemCols = 512;
-constexpr int kPCol = 128;
-constexpr int kOCol = 256;
-
-// Shared-memory descriptor, 128-byte swizzle, with explicit leading / stride byte offsets.
-__device__ __forceinline__ uint64_t desc_sw128(uint32_t smem_addr, uint32_t lbo, uint32_t sbo)
-{
-    uint64_t d = 0;
-    d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
-    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-    d |= (uint64_t)1u << 46;                               // descriptor version (sm_100)
-    d |= (uint64_t)2u << 61;                               // layout: 128-byte swizzle
-    return d;
-}
+constexpr int kQCol = 128;
+constexpr int kPCol = 224;
+constexpr int kOCol = 288;
+static_assert(kOCol + kD <= kTmemCols, "TMEM map fits");
 
 // kind::f16 instruction descriptor: BF16 x BF16 -> F32; b_mn: B operand MN-major.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn)
@@ -82,28 +77,29 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn)
            ((uint32_t)(M >> 4) << 24);
 }
 
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                         bool accumulate)
+// Shared-memory matrix descriptor (128-byte swizzle) in two 32-bit halves: lo = start
+// address >> 4 | LBO >> 4 << 16 (the start address of a later tile is lo + byte offset / 16,
+// no carry below 256 KiB), hi = SBO >> 4 | version (sm_100) | layout.
+__device__ __forceinline__ uint32_t desc_lo(uint32_t smem_addr, uint32_t lbo)
 {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
-        : "memory");
+    return ((smem_addr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
 }
+__host__ __device__ constexpr uint32_t desc_hi(uint32_t sbo) { return ((sbo >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29); }
 
-// The same with A read from TMEM (M lanes, two 16-bit K elements per 32-bit column, the
-// lower K element in the lower half).
-__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                            bool accumulate)
+// tcgen05.mma kind::f16 with A from TMEM and B from smem (descriptor halves), the accumulate
+// flag an immediate: the issuing thread spends a handful of instructions per MMA.
+template <bool kAccumulate>
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi, uint32_t idesc)
 {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
-        : "memory");
+    const uint64_t b = ((uint64_t)b_hi << 32) | b_lo;
+    if constexpr (kAccumulate)
+        asm volatile("tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, 1;" ::"r"(d_tmem), "r"(a_tmem), "l"(b),
+                     "r"(idesc)
+                     : "memory");
+    else
+        asm volatile("tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, 0;" ::"r"(d_tmem), "r"(a_tmem), "l"(b),
+                     "r"(idesc)
+                     : "memory");
 }
 
 // hardware base-2 exponential (ex2.approx, flush-to-zero); ex2(-inf) = +0
@@ -128,10 +124,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32])
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// byte offset of 16-byte chunk c of row r in a [rows][128 B] tile with the 128-byte swizzle
-__device__ __forceinline__ uint32_t sw128_off(int r, int c)
+// 16 consecutive 32-bit columns of this warp's 32 TMEM lanes written from registers.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16])
 {
-    return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+        ::"r"(taddr), "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]),
+          "f"(v[8]), "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15])
+        : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // tmap_k / tmap_v: 2-D views [n_pages * 4 * 64 rows][192] of the caches, box 64 x 8 rows
@@ -145,7 +146,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     pdl_wait();      // the previous kernel's results are visible from here on
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *qs = smem + kOffQ;
     uint8_t *ks = smem + kOffK;
     uint8_t *vs = smem + kOffV;
     int32_t *uni = reinterpret_cast<int32_t *>(smem + kOffUni);
@@ -153,21 +153,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t *umask = reinterpret_cast<uint32_t *>(smem + kOffMask);
     uint32_t *bitmap = reinterpret_cast<uint32_t *>(smem + kOffBitmap);
     int32_t *sels = reinterpret_cast<int32_t *>(smem + kOffSel);
+    uint32_t *rank = reinterpret_cast<uint32_t *>(smem + kOffRank);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBars);
     uint64_t *k_full = bars, *k_empty = bars + kStages, *v_full = bars + 2 * kStages, *v_empty = bars + 3 * kStages;
     uint64_t *s_full = bars + 4 * kStages, *s_empty = s_full + 2, *p_full = s_full + 4, *p_free = s_full + 6;
+    // o_done[j & 1] completes when P V of tile j has (and with it every earlier MMA): two
+    // barriers, since P V runs two tiles behind S and a waiter must be at most one phase behind
     uint64_t *o_done = s_full + 8;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_done + 1);
-    static_assert((4 * kStages + 9) * 8 + 4 <= 256, "barriers fit their slot");
+    uint64_t *x_full = o_done + 2;                        // [4 quarters][2 buffers]
+    uint64_t *q_ready = x_full + 8;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(q_ready + 1);
+    static_assert((4 * kStages + 19) * 8 + 4 <= 512, "barriers fit their slot");
+    float *xch = reinterpret_cast<float *>(smem + kOffXch);
     __shared__ uint32_t scan_ws[40];
     __shared__ int sh_req[kQueries], sh_pos[kQueries], sh_cnt[kQueries], sh_own[kQueries];
     __shared__ int sh_U;
+    __shared__ uint32_t sh_whole[kMaxUnion / kTileRegions / 32];   // bit i: tile i needs no mask
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
     // group-major block order: the CTAs resident together gather from one group's cache
     const int n_qblocks = (int)gridDim.x / kG;
     const int g = (int)blockIdx.x / n_qblocks;
     const int q0 = ((int)blockIdx.x - g * n_qblocks) * kQueries;
+    // softmax threads (warps 4..11) fetch their Q row half now; it goes to TMEM after set-up
+    uint4 qreg[12];
+    if (warp >= 4) {
+        const int r = (warp & 3) * 32 + lane, q = q0 + (r >> 4);
+        const uint4 *src = reinterpret_cast<const uint4 *>(
+            p.q + ((int64_t)q * kHQ + g * kHeadsPerGroup + (r & 15)) * kD + ((warp - 4) >> 2) * 96);
+#pragma unroll
+        for (int k = 0; k < 12; ++k) qreg[k] = q < p.nq ? __ldg(src + k) : make_uint4(0u, 0u, 0u, 0u);
+    }
 
     // ---- the block's queries: request, position, own region, selection count
     if (tid < kQueries) {
@@ -207,8 +223,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (warp < kQueries && q0 + warp < p.nq) {
             const int c = sh_cnt[warp];
             const int32_t *src = p.sel_idx + ((int64_t)(q0 + warp) * kG + g) * p.k;
-            for (int i = lane; i < c; i += 32) {
-                int r = src[i];
+            int rv[kMaxK / 32];                             // all loads in flight at once
+#pragma unroll
+            for (int k = 0; k < kMaxK / 32; ++k) rv[k] = lane + 32 * k < c ? __ldg(src + lane + 32 * k) : -1;
+#pragma unroll
+            for (int k = 0; k < kMaxK / 32; ++k) {
+                const int i = lane + 32 * k;
+                if (i >= c) break;
+                int r = rv[k];
                 if (r < 0 || r > sh_own[warp] || r / 8 >= p.max_pages || (r >> 5) >= words) {
                     set_error(kErrAttnIndex);
                     r = -1;
@@ -230,6 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t pos = incl - n;
             for (int i = 0; i < wpt; ++i) {
                 if (w0 + i >= words) break;
+                rank[w0 + i] = pos;
                 uint32_t b = bitmap[w0 + i];
                 while (b) {
                     const int bit = __ffs(b) - 1;
@@ -244,16 +267,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (p.row_shared && tid < kQueries && q0 + tid < p.nq) p.row_shared[(int64_t)(q0 + tid) * kG + g] = share ? 1 : 0;
     if (!share) return;                                   // block-uniform: the per-row kernel serves it
     const int U = sh_U;
-    // ---- each union region's first cache row (through the block table, all at once; a bad
-    // page reads zeros), and membership: bit 8 (u % 4) + w of word u / 4 when query w selected
-    // union region u
-    for (int u = tid; u < U; u += kThreads) {
-        const int r = uni[u];
-        const int64_t page = p.block_table[(int64_t)R * p.max_pages + r / 8];
-        int y = kv_rows;
-        if (page >= 0 && page < p.n_pages) y = (int)((page * kG + g) * kPage + (r % 8) * kRegion);
-        else set_error(kErrAttnIndex);
-        urow[u] = y;
+    // ---- each union region's first cache row (through the block table, all lookups in flight
+    // at once; a bad page reads zeros), and membership: bit 8 (u % 4) + w of word u / 4 when
+    // query w selected union region u, whose union rank comes from the bitmap
+    static_assert(3 * kThreads >= kMaxUnion, "three block-table lookups per thread");
+    {
+        int64_t page[3];
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+            const int u = tid + k * kThreads;
+            page[k] = u < U ? __ldg(p.block_table + (int64_t)R * p.max_pages + uni[u] / 8) : 0;
+        }
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+            const int u = tid + k * kThreads;
+            if (u >= U) break;
+            int y = kv_rows;
+            if (page[k] >= 0 && page[k] < p.n_pages)
+                y = (int)((page[k] * kG + g) * kPage + (uni[u] % 8) * kRegion);
+            else
+                set_error(kErrAttnIndex);
+            urow[u] = y;
+        }
     }
     for (int i = tid; i < (U + 3) / 4; i += kThreads) umask[i] = 0u;
     __syncthreads();
@@ -262,24 +297,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = lane; i < c; i += 32) {
             const int r = sels[warp * kMaxK + i];
             if (r < 0) continue;
-            int lo = 0, hi = U - 1;                         // uni is ascending and holds r
-            while (lo < hi) {
-                const int mid = (lo + hi) >> 1;
-                if (uni[mid] < r) lo = mid + 1;
-                else hi = mid;
-            }
-            atomicOr(&umask[lo >> 2], 1u << ((lo & 3) * 8 + warp));
+            const uint32_t b = bitmap[r >> 5];
+            const int u = (int)(rank[r >> 5] + __popc(b & ((1u << (r & 31)) - 1u)));
+            atomicOr(&umask[u >> 2], 1u << ((u & 3) * 8 + warp));
         }
     }
-    // ---- Q tile: row (query qq, head h) = 16 qq + h, K-major in 3 swizzled 64-wide blocks
-    for (int i = tid; i < 128 * (kD / 8); i += kThreads) {
-        const int r = i / (kD / 8), c16 = i % (kD / 8);
-        const int q = q0 + (r >> 4);
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (q < p.nq)
-            v = __ldg(reinterpret_cast<const uint4 *>(p.q + ((int64_t)q * kHQ + g * kHeadsPerGroup + (r & 15)) * kD +
-                                                      c16 * 8));
-        *reinterpret_cast<uint4 *>(qs + (c16 >> 3) * (128 * 128) + sw128_off(r, c16 & 7)) = v;
+    __syncthreads();
+    // ---- tiles that need no mask: all 8 regions in the union, selected by every query of the
+    // block, and wholly at or before the earliest position
+    if (warp < kMaxUnion / kTileRegions / 32) {
+        uint32_t qmask = 0u;
+        int min_pos = INT_MAX;
+        for (int w = 0; w < kQueries; ++w)
+            if (q0 + w < p.nq) {
+                qmask |= 1u << w;
+                min_pos = min(min_pos, sh_pos[w]);
+            }
+        const int t = warp * 32 + lane;
+        bool whole = (t + 1) * kTileRegions <= U;
+        for (int jr = 0; jr < kTileRegions && whole; ++jr) {
+            const int u = t * kTileRegions + jr;
+            whole = ((umask[u >> 2] >> ((u & 3) * 8)) & qmask) == qmask && uni[u] * kRegion + kRegion - 1 <= min_pos;
+        }
+        const uint32_t bits = __ballot_sync(0xffffffffu, whole);
+        if (lane == 0) sh_whole[warp] = bits;
     }
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -290,15 +331,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&s_full[b], 1);
-            mbar_init(&s_empty[b], 4);
-            mbar_init(&p_full[b], 4);
+            mbar_init(&s_empty[b], 8);
+            mbar_init(&p_full[b], 8);
             mbar_init(&p_free[b], 1);
         }
-        mbar_init(o_done, 1);
+        mbar_init(&o_done[0], 1);
+        mbar_init(&o_done[1], 1);
+        for (int b = 0; b < 8; ++b) mbar_init(&x_full[b], 2);
+        mbar_init(q_ready, 8);
         fence_mbar_init();
     }
     if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
-    fence_proxy_async();                                  // Q and the reused scratch, for the async proxy
+    fence_proxy_async();                                  // the reused scratch, for the async proxy
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -332,90 +376,133 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else if (warp == 1) {
-        // ---------------- MMA issuer (one lane): S(i), then O += P(i-1) V(i-1)
+        // ---------------- MMA issuer (one lane): S(i), then O += P(i-2) V(i-2): S runs two tiles
+        // ahead, so that the tensor pipe has S(i) queued while the softmax of tile i-1 runs
         if (lane == 0) {
             constexpr uint32_t kIdS = idesc_bf16(128, 64, false), kIdO = idesc_bf16(128, kD, true);
-            const uint32_t qa = smem_u32(qs);
+            // K: K-major, 8-token atoms 3 KiB apart; V: MN-major, 64-dim blocks 1 KiB apart
+            const uint32_t k_lo0 = desc_lo(smem_u32(ks), 16), v_lo0 = desc_lo(smem_u32(vs), 1024);
+            constexpr uint32_t kHi = desc_hi(kRegionBox);
+            ok = mbar_wait(q_ready, 0);                   // Q in TMEM
             auto issue_pv = [&](int j) {
                 const int s = j % kStages, pb = j & 1;
-                ok = ok && mbar_wait_sleep(&p_full[pb], (j >> 1) & 1) &&
-                     mbar_wait_sleep(&v_full[s], (j / kStages) & 1);
+                ok = ok && mbar_wait(&p_full[pb], (j >> 1) & 1) &&
+                     mbar_wait(&v_full[s], (j / kStages) & 1);
                 if (!ok) return;
                 tc_fence_after();
-                const uint32_t vb = smem_u32(vs + s * kTileBytes);
+                const uint32_t vlo = v_lo0 + (uint32_t)s * (kTileBytes >> 4);
+                const uint32_t pa = tmem + kPCol + pb * 32;
+                // 16 tokens (two regions) per instruction
+                if (j > 0) mma_ts<true>(tmem + kOCol, pa, vlo, kHi, kIdO);
+                else mma_ts<false>(tmem + kOCol, pa, vlo, kHi, kIdO);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)                  // 16 tokens (two regions) per instruction
-                    mma_bf16_ts(tmem + kOCol, tmem + kPCol + pb * 32 + kk * 8,
-                                desc_sw128(vb + kk * 2 * kRegionBox, 1024, kRegionBox), kIdO, j > 0 || kk > 0);
+                for (int kk = 1; kk < 4; ++kk)
+                    mma_ts<true>(tmem + kOCol, pa + kk * 8, vlo + kk * (2 * kRegionBox >> 4), kHi, kIdO);
                 umma_commit(&p_free[pb]);                       // P(j) read
                 umma_commit(&v_empty[s]);                       // V(j) read
-                umma_commit(o_done);                            // O holds the tiles up to j
+                umma_commit(&o_done[j & 1]);                    // O holds the tiles up to j
             };
-            for (int i = 0; i < n_tiles && ok; ++i) {
+            for (int i = 0; i < n_tiles + 2 && ok; ++i) {
+                if (i >= n_tiles) {                             // the last two P V
+                    if (i >= 2) issue_pv(i - 2);
+                    continue;
+                }
                 const int s = i % kStages, sb = i & 1;
-                ok = mbar_wait_sleep(&k_full[s], (i / kStages) & 1) &&
-                     mbar_wait_sleep(&s_empty[sb], ((i >> 1) & 1) ^ 1);
+                ok = mbar_wait(&k_full[s], (i / kStages) & 1) &&
+                     mbar_wait(&s_empty[sb], ((i >> 1) & 1) ^ 1);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t kb = smem_u32(ks + s * kTileBytes);
+                const uint32_t klo = k_lo0 + (uint32_t)s * (kTileBytes >> 4), sd = tmem + sb * 64;
+                // 16 dims per instruction, Q from TMEM
+                mma_ts<false>(sd, tmem + kQCol, klo, kHi, kIdS);
 #pragma unroll
-                for (int blk = 0; blk < 3; ++blk)
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)              // 16 dims per instruction
-                        mma_bf16(tmem + sb * 64, desc_sw128(qa + blk * (128 * 128) + kk * 32, 16, 1024),
-                                 desc_sw128(kb + blk * 1024 + kk * 32, 16, kRegionBox), kIdS, blk > 0 || kk > 0);
+                for (int kk = 1; kk < kD / 16; ++kk)
+                    mma_ts<true>(sd, tmem + kQCol + kk * 8, klo + (((kk >> 2) * 1024 + (kk & 3) * 32) >> 4), kHi, kIdS);
                 umma_commit(&s_full[sb]);
                 umma_commit(&k_empty[s]);                       // K(i) read
-                if (i > 0) issue_pv(i - 1);
+                if (i >= 2) issue_pv(i - 2);
             }
-            if (ok && n_tiles > 0) issue_pv(n_tiles - 1);
         }
     } else if (warp >= 4) {
-        // ---------------- softmax warps 4..7: TMEM lane quarter warp % 4, row r = query, head
-        const int r = (warp & 3) * 32 + lane;
+        // ---------------- softmax warps 4..11: TMEM lane quarter warp % 4 (row r = query, head),
+        // column half (warps 4..7 the tile's first 32 tokens, 8..11 the last 32).  The two warps
+        // of a row agree on its running max through xch (one mbarrier per quarter and buffer);
+        // each keeps the sum of its own columns.
+        const int quarter = warp & 3, half = (warp - 4) >> 2;
+        const int r = quarter * 32 + lane;
         const int qq = r >> 4, h = r & 15;
         const int q = q0 + qq;
         const bool qv = q < p.nq;
         const int pos = qv ? sh_pos[qq] : -1;
-        const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
         const float sc = p.scale_log2;
+        const float2 sc2 = make_float2(sc, sc), one2 = make_float2(1.0f, 1.0f);
+        {
+            // Q: this warp's half of row r (96 dims, two per column) into TMEM, A of S = Q K^T
+#pragma unroll
+            for (int j = 0; j < 3; ++j) {
+                float qc[16];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint4 v = qreg[4 * j + k];
+                    qc[4 * k + 0] = __uint_as_float(v.x);
+                    qc[4 * k + 1] = __uint_as_float(v.y);
+                    qc[4 * k + 2] = __uint_as_float(v.z);
+                    qc[4 * k + 3] = __uint_as_float(v.w);
+                }
+                tmem_st16(trow + kQCol + half * 48 + 16 * j, qc);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(q_ready);
+        }
         float mrow = -INFINITY, lrow = 0.0f;
+        uint32_t whole_bits = 0u;
+        auto exchange = [&](int i, float mine) -> float {    // the partner warp's value for row r
+            const int b = i & 1;
+            xch[(b * 2 + half) * 128 + r] = mine;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&x_full[quarter * 2 + b]);
+            ok = __all_sync(0xffffffffu, mbar_wait(&x_full[quarter * 2 + b], (i >> 1) & 1));
+            return ok ? xch[(b * 2 + (half ^ 1)) * 128 + r] : 0.0f;
+        };
         for (int i = 0; i < n_tiles && ok; ++i) {
             const int sb = i & 1;
-            ok = __all_sync(0xffffffffu, mbar_wait_sleep(&s_full[sb], (i >> 1) & 1));
+            ok = __all_sync(0xffffffffu, mbar_wait(&s_full[sb], (i >> 1) & 1));
             if (!ok) break;
             tc_fence_after();
-            float sv[64];
-            {
-                float a[32], b[32];
-                tmem_ld32x2(trow + sb * 64, trow + sb * 64 + 32, a, b);
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    sv[j] = a[j];
-                    sv[32 + j] = b[j];
-                }
-            }
+            float sv[32];
+            tmem_ld32(trow + sb * 64 + half * 32, sv);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s_empty[sb]);       // the MMA may write S(i + 2) here
             // mask: a union region this row's query selected, tokens at or before its position
-            // (token e of a region is kept when e <= lim)
+            // (token e of a region is kept when e <= lim); most tiles need none
+            if ((i & 31) == 0) whole_bits = sh_whole[i >> 5];
             float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            if ((whole_bits >> (i & 31)) & 1u) {               // block-uniform
 #pragma unroll
-            for (int jr = 0; jr < kTileRegions; ++jr) {
-                const int u = i * kTileRegions + jr;
-                const bool member = u < U && ((umask[u >> 2] >> ((u & 3) * 8 + qq)) & 1u);
-                const int lim = member ? pos - uni[u] * kRegion : -1;
+                for (int j = 0; j < 32; ++j) m4[j & 3] = fmaxf(m4[j & 3], sv[j]);
+            } else {
+                int lim[4];
 #pragma unroll
-                for (int e = 0; e < kRegion; ++e) {
-                    const float v = e <= lim ? sv[jr * kRegion + e] : -INFINITY;
-                    sv[jr * kRegion + e] = v;
-                    m4[e & 3] = fmaxf(m4[e & 3], v);
+                for (int jr = 0; jr < 4; ++jr) {
+                    const int u = i * kTileRegions + half * 4 + jr;
+                    const bool member = u < U && ((umask[u >> 2] >> ((u & 3) * 8 + qq)) & 1u);
+                    lim[jr] = member ? pos - uni[u] * kRegion : -1;
+                }
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    sv[j] = (j & 7) <= lim[j >> 3] ? sv[j] : -INFINITY;
+                    m4[j & 3] = fmaxf(m4[j & 3], sv[j]);
                 }
             }
-            const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sc;   // sc > 0
+            const float mine = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sc;   // sc > 0
+            const float mx = fmaxf(mine, exchange(i, mine));
+            if (!ok) break;
             // lazy rescaling: the reference max moves only when the tile's max exceeds it by more
-            // than the slack (P stays below 2^slack): the same softmax, rarely rescaled
+            // than the slack (P stays below 2^slack): the same softmax, rarely rescaled.  Both
+            // warps of a row take the same decision from the same values.
             const bool grow = mx > mrow + attn::kSlack;
             float alpha = 1.0f;
             if (grow) {
@@ -423,49 +510,56 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mrow = mx;
             }
             const float nref = (mrow == -INFINITY) ? 0.0f : -mrow;
-            float s4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-            float pk[32];                                   // P(i): bf16 pairs (tokens 2c, 2c + 1)
+            const float2 nref2 = make_float2(nref, nref);
+            float2 s2a = make_float2(0.0f, 0.0f), s2b = s2a;
+            float pk[16];                                   // P(i): bf16 pairs (tokens 2c, 2c + 1)
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const float p0 = ex2(fmaf(sv[2 * c], sc, nref));
-                const float p1 = ex2(fmaf(sv[2 * c + 1], sc, nref));
-                s4[c & 3] += p0 + p1;
-                pk[c] = __uint_as_float(pack_bf16x2(p0, p1));
+            for (int c = 0; c < 16; ++c) {
+                const float2 t = ffma2(make_float2(sv[2 * c], sv[2 * c + 1]), sc2, nref2);
+                const float2 e = make_float2(ex2(t.x), ex2(t.y));
+                if (c & 1) s2b = ffma2(e, one2, s2b);
+                else s2a = ffma2(e, one2, s2a);
+                pk[c] = __uint_as_float(pack_bf16x2(e.x, e.y));
             }
-            lrow = lrow * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+            lrow = lrow * alpha + ((s2a.x + s2a.y) + (s2b.x + s2b.y));
             if (__any_sync(0xffffffffu, grow && i > 0)) {
-                // O holds the tiles before i once their P V has completed: scale it in TMEM
-                ok = __all_sync(0xffffffffu, mbar_wait_sleep(o_done, (i - 1) & 1));
+                // O holds the tiles before i once their P V has completed: scale this warp's
+                // 96 columns of it in TMEM
+                ok = __all_sync(0xffffffffu, mbar_wait_sleep(&o_done[(i - 1) & 1], ((i - 1) >> 1) & 1));
                 if (!ok) break;
                 tc_fence_after();
 #pragma unroll 1
-                for (int c = 0; c < kD / 32; ++c) {
+                for (int c = 0; c < 3; ++c) {
                     float o[32];
-                    tmem_ld32(trow + kOCol + 32 * c, o);
+                    const uint32_t ta = trow + kOCol + half * 96 + 32 * c;
+                    tmem_ld32(ta, o);
 #pragma unroll
                     for (int j = 0; j < 32; ++j) o[j] *= alpha;
-                    tmem_st32(trow + kOCol + 32 * c, o);
+                    tmem_st32(ta, o);
                 }
             }
             // P(i) into its TMEM buffer once P V has read the tile two back from it
             ok = __all_sync(0xffffffffu, mbar_wait_sleep(&p_free[sb], ((i >> 1) & 1) ^ 1));
             if (!ok) break;
             tc_fence_after();
-            tmem_st32(trow + kPCol + sb * 32, pk);
+            tmem_st16(trow + kPCol + sb * 32 + half * 16, pk);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[sb]);
         }
-        // ---- output: O / l (bf16) and the LSE, once the last P V has completed
-        if (ok && n_tiles > 0) ok = __all_sync(0xffffffffu, mbar_wait_sleep(o_done, (n_tiles - 1) & 1));
+        // ---- output: O / l (bf16, this warp's 96 columns) and the LSE, once the last P V has
+        // completed; l is the sum of both halves'
+        if (ok) lrow += exchange(n_tiles, lrow);
+        if (ok && n_tiles > 0)
+            ok = __all_sync(0xffffffffu, mbar_wait_sleep(&o_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1));
         if (ok) {
             tc_fence_after();
             const float inv = lrow > 0.0f ? 1.0f / lrow : 0.0f;
-            __nv_bfloat16 *dst = p.out + ((int64_t)q * kHQ + g * kHeadsPerGroup + h) * kD;
+            __nv_bfloat16 *dst = p.out + ((int64_t)q * kHQ + g * kHeadsPerGroup + h) * kD + half * 96;
 #pragma unroll 1
-            for (int c = 0; c < kD / 32; ++c) {
+            for (int c = 0; c < 3; ++c) {
                 float o[32];
-                tmem_ld32(trow + kOCol + 32 * c, o);
+                tmem_ld32(trow + kOCol + half * 96 + 32 * c, o);
                 if (qv) {
 #pragma unroll
                     for (int k8 = 0; k8 < 4; ++k8) {
@@ -478,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            if (qv && p.lse)
+            if (qv && p.lse && half == 0)
                 p.lse[(int64_t)q * kHQ + g * kHeadsPerGroup + h] =
                     lrow > 0.0f ? (mrow + log2f(lrow)) * 0.69314718055994531f : -INFINITY;
         }

@@ -11,7 +11,6 @@
 #include "../../include/dsa.h"
 #include "attention.cuh"
 #include "attention_cluster.cuh"
-#include "attention_shared.cuh"
 #include "attention_tc.cuh"
 #include "common.cuh"
 #include "compress.cuh"
@@ -275,8 +274,8 @@ dsa_status_t attn_common(const void *q, const void *k_cache, const void *v_cache
         window == 0 && k <= dsa::attnc::kMaxK && (int64_t)nq * dsa::kG <= cluster_attn_capacity();
     // prefill chunks: 8 neighbouring queries per CTA share one stream of their selections' union
     const bool shared = window == 0 && !clustered && q_req != nullptr && nq >= kSharedMinQueries &&
-                        k <= dsa::attns::kMaxK &&
-                        (int64_t)max_pages * dsa::kPage / dsa::kRegion <= (int64_t)dsa::attns::kMaxWords * 32;
+                        k <= dsa::attntc::kMaxK &&
+                        (int64_t)max_pages * dsa::kPage / dsa::kRegion <= (int64_t)dsa::attntc::kMaxWords * 32;
     const AttnPlan plan = attn_plan(nq, k, sms);
     const size_t need_ws = plan.ws + (shared ? round_up((size_t)nq * dsa::kG, 256) : 0);
     if (need_ws > 0 && !clustered) {
