@@ -84,6 +84,17 @@ def test_many_rows_take_the_per_row_path():
     check(s, q_pos, 512)
 
 
+def test_per_row_path_unaligned_rows():
+    # rows that do not start on 16-byte boundaries (ld not a multiple of 4) are loaded
+    # directly instead of streamed through the smem ring; same selection either way
+    rng = np.random.default_rng(11)
+    nq, ld = 100, 3001
+    s = rng.standard_normal((nq, G, ld)).astype(np.float32)
+    s[::5] = np.round(s[::5] * 2) / 2             # tie-heavy rows
+    q_pos = [int(x) for x in rng.integers(0, 8 * ld + 1, nq)]
+    check(s, q_pos, 512)
+
+
 @pytest.mark.parametrize("k", [2, 64, 512, 1024])
 def test_per_row_path_prefill_like_rows(k):
     # prefill-shaped: 160 rows of 33,024 scores, indexer-like non-negative scores, rows with
