@@ -2,9 +2,10 @@
 // up to 65,536 scores), one CTA per (query, group) row, no global scratch ([P2] Step-5-Preview
 // 如何实现1M长上下文 §索引器打分: a radix-style top-k keeps the best regions and always includes
 // the query's own region).
-//  1. one pass over the row: thread t reads entries t, t+512, ... (coalesced) and keeps the
-//     maximum of each of its 4 strided groups (entry t + 512j joins group j % 4): 2,048 group
-//     maxima per row;
+//  1. one pass over the row: thread t of 256 reads entries t, t+256, ... (coalesced) and keeps
+//     the maximum of each of its 8 strided groups (entry t + 256j joins group j % 8): 2,048
+//     group maxima per row.  Five CTAs share an SM, so one row's threshold and emit overlap
+//     the other rows' streaming;
 //  2. 256-bin histogram levels over the group maxima narrow the need-th largest maximum to a
 //     range [elo, ehi) holding at most 64 maxima (or one value).  At least need groups have a
 //     maximum >= elo, so at least need scores are >= elo; the scores >= elo all lie in those
@@ -29,11 +30,11 @@ using topkc::desc_bin_search;
 using topkc::key_levels;
 using topkc::threshold_selects;
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kGroupsPerThread = 4;
+constexpr int kGroupsPerThread = 8;
 constexpr int kMaxLd = 65536;                       // scores per row
-constexpr int kMaxCand = 10240;                     // >= (511 + 64) groups x 16 entries
+constexpr int kMaxCand = 4096;                      // candidates kept in smem (more: the whole-row path)
 constexpr int kBitmapWords = kMaxLd / 32 + 1;
 constexpr int kBatch = 16;                          // loads in flight per thread
 // smem (bytes)
@@ -42,8 +43,9 @@ constexpr size_t kOffBitmap = kOffCand + (size_t)kMaxCand * 8;                //
 constexpr size_t kOffList = kOffBitmap + ((size_t)kBitmapWords * 4 + 15) / 16 * 16;   // [32] composites
 constexpr size_t kOffHs = kOffList + 32 * 8;                                  // [256]
 constexpr size_t kSmemBytes = kOffHs + 256 * 4 + 16;
+static_assert(5 * kSmemBytes <= 227 * 1024, "five CTAs per SM");
 
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 5)
     topk_rows_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ q_pos, int k,
                      int32_t *__restrict__ sel_idx, int32_t *__restrict__ sel_count)
 {
@@ -87,7 +89,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int n = (int)own;                             // eligible entries 0 .. own-1
     const float *src = scores + (int64_t)row * ld;
     // ---- 1. group maxima (0: a group with no eligible entry)
-    uint32_t gm[kGroupsPerThread] = {0u, 0u, 0u, 0u};
+    uint32_t gm[kGroupsPerThread] = {};
     for (int base = 0; base < n; base += kThreads * kBatch) {
         float v[kBatch];
 #pragma unroll
@@ -141,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int words = (int)((own + 1 + 31) / 32);
     if (n_cand <= (uint32_t)kMaxCand) {
         // ---- 4. the exact threshold over the candidates (read from smem on demand)
-        constexpr int R = kMaxCand / kThreads;          // 20
+        constexpr int R = kMaxCand / kThreads;          // 16
         auto cvalid = [&](int u) { return (uint32_t)(u * kThreads + tid) < n_cand; };
         auto ccomp = [&](int u) { return cand[u * kThreads + tid]; };
         const int r_used = (int)((n_cand + kThreads - 1) / kThreads);
@@ -157,7 +159,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
     } else {
         // equal scores in bulk: the same threshold over the whole row, read in every level
-        constexpr int R = kMaxLd / kThreads;            // 128
+        constexpr int R = kMaxLd / kThreads;            // 256
         auto rvalid = [&](int u) { return u * kThreads + tid < n; };
         auto rcomp = [&](int u) {
             const int i = u * kThreads + tid;
