@@ -572,7 +572,43 @@ def run_prefill(args):
         "gpu_launches": PREFILL_KERNELS * args.steps,
         "clocks": sampler.summary(),
     }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = prefill_oracle_time(d, n_queries=32, time_cap_s=30.0)
     print(json.dumps(line), flush=True)
+
+
+def prefill_oracle_time(d, n_queries: int, time_cap_s: float):
+    """The oracle on the host over a bounded sample of the same chunk: the chunk's 256 new
+    regions compressed, then per query (the chunk's first ones, up to n_queries or the time
+    cap) the scores over every region, the top-512 and the attention.  The summaries of the
+    cached context come from the oracle itself (untimed)."""
+    import numpy as np
+    import torch
+    import oracle
+
+    def bits(t):
+        return t.cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    index_k = bits(d["index_k"])
+    kc, vc = bits(d["k_cache"]), bits(d["v_cache"])
+    index_q, q = bits(d["index_q"]), bits(d["q"])
+    gate, qp = d["gate"].cpu().numpy(), d["q_pos"].cpu().numpy()
+    bt = d["block_table"].cpu().numpy()
+    first, last = PREFILL_CTX // 8, (PREFILL_CTX + PREFILL_NEW) // 8
+    S, C = oracle.compress_regions(index_k, [8 * r for r in range(first)], list(range(first)), last)
+    t0 = time.perf_counter()
+    oracle.compress_regions(index_k, [8 * r for r in range(first, last)], list(range(first, last)), last, S, C)
+    done = 0
+    while done < n_queries and time.perf_counter() - t0 < time_cap_s:
+        i = done
+        sc = oracle.indexer_scores(index_q[i:i + 1], gate[i:i + 1], [0], qp[i:i + 1], S, C, [0], ld=last)
+        idx, cnt = oracle.topk_regions(np.nan_to_num(sc), qp[i:i + 1], TOPK)
+        oracle.sparse_attention(q[i:i + 1], kc, vc, bt, [0], qp[i:i + 1], idx, cnt)
+        done += 1
+    dt = time.perf_counter() - t0
+    return {"value": done / dt, "unit": "tokens/s", "cores": oracle.get_threads(), "kind": "oracle",
+            "sample": f"the chunk's 256 new regions compressed and {done} of its queries scored, selected and "
+                      f"attended ({dt:.1f} s)"}
 
 
 SWA_BATCH, SWA_LAYERS, SWA_WINDOW, SWA_RING = 8, 69, 512, 8
