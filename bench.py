@@ -573,7 +573,7 @@ def run_prefill(args):
         "clocks": sampler.summary(),
     }
     if not args.no_cpu_baseline:
-        line["cpu_baseline"] = prefill_oracle_time(d, n_queries=32, time_cap_s=30.0)
+        line["cpu_baseline"] = prefill_oracle_time(d, n_queries=128, time_cap_s=30.0)
     print(json.dumps(line), flush=True)
 
 

@@ -145,3 +145,32 @@ def test_prefill_shared_block_with_empty_and_overlapping_selections():
     cnt[17] = 0
     idx[17] = -1
     run(d, idx, cnt, q_req=d["q_req"], prefill=True)
+
+
+def test_prefill_shared_block_running_max_grows():
+    # 48 queries in six blocks of 8 (one region each), every block sharing one selection of
+    # 200 regions; the K rows of region r are scaled by 1 + r / 16, so along the union (in
+    # region order) each row's running max climbs past the lazy-rescale slack again and again
+    # and the shared kernel rescales O in TMEM several times per row
+    dev = "cuda"
+    ctx = 6000
+    d = W.prefill_chunk(ctx, 48, seed=41, device=dev, permute=True)
+    bt = d["block_table"][0]
+    n_log = (ctx + 48 + 63) // 64
+    rows = torch.arange(n_log * 64, device=dev) // 8                 # region of each logical row
+    scale = (1.0 + rows.float() / 16).view(n_log, 1, 64, 1)
+    kc = d["k_cache"].float()
+    kc[bt[:n_log].long()] *= scale
+    d["k_cache"] = kc.to(torch.bfloat16)
+    qp = d["q_pos"].cpu().numpy()
+    rng = np.random.default_rng(12)
+    k = 256
+    idx = np.full((48, G, k), -1, np.int32)
+    cnt = np.zeros((48, G), np.int32)
+    for b in range(6):
+        own = int(qp[8 * b]) // 8
+        for g in range(G):
+            sel = np.sort(np.concatenate([rng.choice(own, 199, replace=False), [own]])).astype(np.int32)
+            idx[8 * b: 8 * b + 8, g, :200] = sel
+            cnt[8 * b: 8 * b + 8, g] = 200
+    run(d, idx, cnt, q_req=d["q_req"], prefill=True)
