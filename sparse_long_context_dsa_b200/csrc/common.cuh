@@ -317,34 +317,6 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b)
     return d;
 }
 
-// TMA tensor store (shared -> global) of a 3-D box with an L2 cache policy, in this
-// thread's bulk async-group; the generic-proxy writes to the box must be fenced first
-// (fence_proxy_async by the writing threads).
-__device__ __forceinline__ void tma_store_3d_hint(const CUtensorMap *map, const void *smem_src, int x, int y, int z,
-                                                  uint64_t policy)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3, %4}], [%1], %5;"
-        ::"l"(map), "r"(smem_u32(smem_src)), "r"(x), "r"(y), "r"(z), "l"(policy)
-        : "memory");
-}
-
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-
-// This thread's bulk stores have finished reading shared memory (the source may be rewritten).
-__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-
-// This thread's bulk stores are complete (their writes performed).
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-
-__device__ __forceinline__ void tma_load_4d(void *smem_dst, const CUtensorMap *map, int x, int y, int z, int w,
-                                            uint64_t *bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];"
-        ::"r"(smem_u32(smem_dst)), "l"(map), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
-        : "memory");
-}
 
 // ------------------------------------------------------------------ ldmatrix / mma
 
