@@ -88,22 +88,29 @@ __global__ void __launch_bounds__(kThreads, 5)
     }
     const int n = (int)own;                             // eligible entries 0 .. own-1
     const float *src = scores + (int64_t)row * ld;
-    // ---- 1. group maxima (0: a group with no eligible entry)
-    uint32_t gm[kGroupsPerThread] = {};
+    // ---- 1. group maxima (0: a group with no eligible entry).  The maximum is taken over the
+    // floats (entries past the row as -inf) and turned into a key once per group: fmaxf skips
+    // a NaN and may return -0 for +0, so a group's key can only fall short of its largest
+    // entry's, which lowers the bound below and keeps the candidates a superset of the
+    // selection.  Group j of thread t first holds entry j * kThreads + t (kBatch is a multiple
+    // of kGroupsPerThread).
+    static_assert(kBatch % kGroupsPerThread == 0, "group j's first entry is j * kThreads + t");
+    float gf[kGroupsPerThread];
+#pragma unroll
+    for (int j = 0; j < kGroupsPerThread; ++j) gf[j] = -INFINITY;
     for (int base = 0; base < n; base += kThreads * kBatch) {
         float v[kBatch];
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
             const int i = base + u * kThreads + tid;
-            v[u] = i < n ? __ldcg(src + i) : 0.0f;
+            v[u] = i < n ? __ldcg(src + i) : -INFINITY;
         }
 #pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-            const int i = base + u * kThreads + tid;
-            const int j = (base / kThreads + u) & (kGroupsPerThread - 1);
-            if (i < n) gm[j] = max(gm[j], score_key(v[u]));
-        }
+        for (int u = 0; u < kBatch; ++u) gf[u & (kGroupsPerThread - 1)] = fmaxf(gf[u & (kGroupsPerThread - 1)], v[u]);
     }
+    uint32_t gm[kGroupsPerThread];
+#pragma unroll
+    for (int j = 0; j < kGroupsPerThread; ++j) gm[j] = j * kThreads + tid < n ? score_key(gf[j]) : 0u;
     __syncthreads();                                    // shared counters initialised
     // ---- 2. the bound: a range [elo, ehi) of group maxima holding the need-th largest
     auto gvalid = [&](int u) { return gm[u] != 0u; };
