@@ -120,7 +120,11 @@ __global__ void __launch_bounds__(kThreads, 5)
     key_levels<kGroupsPerThread>(gvalid, gkey, (uint32_t)need, 64u, hs, &sh_min, &sh_max, scan_ws + 32, elo, ehi,
                                  above, n_in);
     const uint32_t lo_key = (uint32_t)elo;
-    // ---- 3. candidates: scores >= elo, compacted (warp-aggregated slots)
+    // ---- 3. candidates: scores >= elo, compacted (warp-aggregated slots).  The test runs on
+    // floats against lo_f, the float whose key is lo_key: !(v < lo_f) holds for every entry of
+    // key >= lo_key, and also for NaN and for the other zero, so the candidates are again a
+    // superset; their exact keys are formed only for the candidates
+    const float lo_f = __uint_as_float((lo_key & 0x80000000u) ? (lo_key & 0x7FFFFFFFu) : ~lo_key);
     const unsigned below = (1u << lane) - 1u;
     for (int base = 0; base < n; base += kThreads * kBatch) {
         float v[kBatch];
@@ -132,10 +136,10 @@ __global__ void __launch_bounds__(kThreads, 5)
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
             const int i = base + u * kThreads + tid;
-            const uint32_t key = score_key(v[u]);
-            const bool c = i < n && key >= lo_key;
+            const bool c = i < n && !(v[u] < lo_f);
             const unsigned m = __ballot_sync(0xffffffffu, c);
             if (m == 0u) continue;
+            const uint32_t key = score_key(v[u]);
             uint32_t slot0 = 0;
             if (lane == 0) slot0 = atomicAdd(&sh_ncand, (uint32_t)__popc(m));
             slot0 = __shfl_sync(0xffffffffu, slot0, 0);
