@@ -162,8 +162,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *o_done = s_full + 8;
     uint64_t *x_full = o_done + 2;                        // [4 quarters][2 buffers]
     uint64_t *q_ready = x_full + 8;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(q_ready + 1);
-    static_assert((4 * kStages + 19) * 8 + 4 <= 512, "barriers fit their slot");
+    uint64_t *mma_drain = q_ready + 1;                    // the MMA issuer's last commit
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_drain + 1);
+    static_assert((4 * kStages + 20) * 8 + 4 <= 512, "barriers fit their slot");
     float *xch = reinterpret_cast<float *>(smem + kOffXch);
     __shared__ uint32_t scan_ws[40];
     __shared__ int sh_req[kQueries], sh_pos[kQueries], sh_cnt[kQueries], sh_own[kQueries];
@@ -339,6 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&o_done[1], 1);
         for (int b = 0; b < 8; ++b) mbar_init(&x_full[b], 2);
         mbar_init(q_ready, 8);
+        mbar_init(mma_drain, 1);
         fence_mbar_init();
     }
     if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
@@ -358,6 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t *ring = is_k ? ks : vs;
         uint64_t *full = is_k ? k_full : v_full, *empty = is_k ? k_empty : v_empty;
         if (lane == 0) prefetch_tensormap(map);
+        int issued = 0;                                   // tiles whose loads went out
         for (int i = 0; i < n_tiles && ok; ++i) {
             const int s = i % kStages;
             int got = 1;
@@ -374,7 +377,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int blk = 0; blk < 3; ++blk) tma_load_2d(dst + blk * 1024, map, blk * 64, y, &full[s]);
             }
+            issued = i + 1;
         }
+        // drain: none of this warp's loads is in flight when the CTA exits, after a wait that
+        // gave up as well (the last phase issued into every stage; complete already otherwise)
+        __syncwarp();
+        if (lane == 0)
+            for (int s = 0; s < kStages && s < issued; ++s) {
+                const int last = issued - 1 - (issued - 1 - s) % kStages;
+                mbar_wait(&full[s], (last / kStages) & 1);
+            }
     } else if (warp == 1) {
         // ---------------- MMA issuer (one lane): S(i), then O += P(i-2) V(i-2): S runs two tiles
         // ahead, so that the tensor pipe has S(i) queued while the softmax of tile i-1 runs
@@ -422,6 +434,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 umma_commit(&k_empty[s]);                       // K(i) read
                 if (i >= 2) issue_pv(i - 2);
             }
+            // drain: no MMA of this CTA is in flight when TMEM is released, after a wait that
+            // gave up as well
+            umma_commit(mma_drain);
+            mbar_wait(mma_drain, 0);
         }
     } else if (warp >= 4) {
         // ---------------- softmax warps 4..11: TMEM lane quarter warp % 4 (row r = query, head),

@@ -81,7 +81,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(inv_freq + 32);
     uint64_t *full = bars, *empty = bars + kStages;                           // [kStages]
     uint64_t *acc_full = bars + 2 * kStages, *acc_empty = acc_full + 2;      // [2]
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
+    uint64_t *mma_drain = acc_empty + 2;                                     // the MMA issuer's last commit
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_drain + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -93,6 +94,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&acc_full[b], 1);
             mbar_init(&acc_empty[b], 4);
         }
+        mbar_init(mma_drain, 1);
         fence_mbar_init();
     }
     for (int i = threadIdx.x; i < kDI; i += kThreads) {
@@ -112,7 +114,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             prefetch_tensormap(&map_h);
             prefetch_tensormap(&map_w);
-            int it = 0;
+            int it = 0, issued = 0;                           // issued: stages whose loads went out
             for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
                 const int m = u / kUnitsPerTile, n = u % kUnitsPerTile;
                 for (int kk = 0; kk < p.n_k; ++kk, ++it) {
@@ -123,7 +125,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t *dst = smem + s * kStageBytes;
                     tma_load_2d(dst, &map_h, kk * kBK, m * kBM, &full[s]);
                     tma_load_2d(dst + kABytes, &map_w, kk * kBK, n * kBN, &full[s]);
+                    issued = it + 1;
                 }
+            }
+            // drain: none of these loads is in flight when the CTA exits, after a wait that gave
+            // up as well (the last phase issued into every stage; complete already otherwise)
+            for (int s = 0; s < kStages && s < issued; ++s) {
+                const int last = issued - 1 - (issued - 1 - s) % kStages;
+                mbar_wait(&full[s], (last / kStages) & 1);
             }
         }
     } else if (warp == 1) {
@@ -151,6 +160,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 umma_commit(&acc_full[buf]);                      // the unit's accumulator is ready
             }
+            // drain: no MMA of this CTA is in flight when TMEM is released
+            umma_commit(mma_drain);
+            mbar_wait(mma_drain, 0);
         }
     } else {
         // ---------------- epilogue: warps 2..5; TMEM lane quarter sp = warp % 4 (the hardware's

@@ -216,7 +216,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *s_full = bars + 2, *s_empty = bars + 2 + kSStages;                // [kSStages]
     uint64_t *acc_full = bars + 2 + 2 * kSStages, *acc_empty = acc_full + 2;    // [2]
     uint64_t *sc_empty = acc_empty + 2;                                         // [kSStages]
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sc_empty + kSStages);
+    uint64_t *mma_drain = sc_empty + kSStages;                                  // the MMA issuer's last commit
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_drain + 1);
+    static_assert((2 + 3 * kSStages + 4 + 1) * 8 + 4 <= 256, "barriers fit their slot");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -231,6 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&acc_full[b], 1);
             mbar_init(&acc_empty[b], kEpiWarps);
         }
+        mbar_init(mma_drain, 1);
         fence_mbar_init();
     }
     if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
@@ -253,6 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             Walk w;
             walk_seek(p, lo, w);
             int cur_g = -1, cur_t = -1, q_loads = 0;
+            int64_t issued = 0;                                   // blocks whose loads went out
             for (int64_t it = 0; it < n_items; ++it, walk_next(p, w)) {
                 if (w.g != cur_g || w.t != cur_t) {
                     ok = mbar_wait_sleep(q_empty, (q_loads & 1) ^ 1);
@@ -278,6 +282,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tma_load_2d(dst + kSHalf, &map_s, 128, y, &s_full[s]);
                 // scales y .. y + 127 from the 16-byte aligned element y & ~3 (past the pool: 0)
                 tma_load_1d(ssc + s * kScaleSlot, &map_sc, y & ~3, &s_full[s]);
+                issued = it + 1;
+            }
+            // drain: none of these loads is in flight when the CTA exits, after a wait that gave
+            // up as well (the last phases issued; complete already otherwise)
+            if (q_loads > 0) mbar_wait(q_full, (q_loads - 1) & 1);
+            for (int s = 0; s < kSStages && s < issued; ++s) {
+                const int64_t last = issued - 1 - (issued - 1 - s) % kSStages;
+                mbar_wait(&s_full[s], (int)(last / kSStages) & 1);
             }
         }
     } else if (warp == 1) {
@@ -312,6 +324,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 umma_commit(&s_empty[s]);            // the summary block may be overwritten
                 umma_commit(&acc_full[buf]);         // the accumulator is ready
             }
+            // drain: no MMA of this CTA is in flight when TMEM is released
+            umma_commit(mma_drain);
+            mbar_wait(mma_drain, 0);
         }
     } else {
         // ---------------- epilogue: warps 2..9.  TMEM lane quarter sp = warp % 4 (the
