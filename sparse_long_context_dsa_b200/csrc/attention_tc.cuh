@@ -3,10 +3,12 @@
 // neighbouring queries reuse one selection).
 //
 // A CTA takes 8 consecutive queries of one request and one KV group: 128 rows (query, head) of
-// one attention tile.  The union of their selections is built in smem as in the mma.sync
-// shared-selection kernel (a region bitmap, compacted in region order) together with each
-// union region's 8-bit membership (which queries selected it).  The union streams in tiles of
-// 8 regions (64 tokens), flash-attention style:
+// one attention tile.  The union of their selections is built in smem (a region bitmap,
+// compacted in region order; the running count per bitmap word gives each selected region its
+// union position) together with each union region's 8-bit membership (which queries selected
+// it) and one bit per tile that needs no mask (every query selected all its regions, all at or
+// before the earliest position).  The union streams in tiles of 8 regions (64 tokens),
+// flash-attention style:
 //  * two TMA warps load each region's K (one warp) and V (the other) as three 8 x 64 boxes
 //    (128-byte swizzle, laid out [block][8 rows][128 B] so that 8-token atoms sit 3 KiB
 //    apart) into separate 4-stage rings: a K stage frees as soon as S has read it, a V stage
@@ -16,7 +18,7 @@
 //    read from TMEM where the softmax warps put it at the start) into one of two 64-column
 //    TMEM buffers, and O += P V (M = 128, N = 192, K = 64: 4 MMAs with
 //    P read from TMEM and V an MN-major smem operand) into a 192-column TMEM accumulator;
-//    S of tile i+1 runs while the softmax of tile i does;
+//    S runs two tiles ahead of P V, so the tensor pipe has S queued while a softmax runs;
 //  * eight softmax warps, two per row (one row per thread, the TMEM lane; one warp takes the
 //    tile's first 32 tokens, the other the last 32, and the two agree on the row's running
 //    max through smem each tile), mask the tile (the region must be the row's query's, the
@@ -24,6 +26,8 @@
 //    (the reference max moves only past a slack of 2^8; O is rescaled in TMEM then), write P
 //    as packed bf16 into TMEM (two tokens per column, the A operand of P V), and at the end
 //    write O / l and the LSE.
+// Every wait is bounded; after the loops the producers wait for their last loads and the MMA
+// issuer for a final commit, so nothing is in flight when TMEM is released.
 // Blocks spanning several requests, with an invalid query, or whose union exceeds twice the
 // longest selection are flagged in row_shared and left to the per-row kernel that runs next.
 #pragma once
