@@ -54,11 +54,15 @@ def run_pipeline(d, k):
     return out, lse, o64, idx, cnt
 
 
-@pytest.mark.parametrize("L,permute", [(200, False), (517, True), (1024, True)])
+@pytest.mark.parametrize("L,permute", [(200, False), (517, True), (1024, True), (4096, True)])
 def test_dense_equivalence_when_k_covers_every_region(L, permute):
     d = W.decode_batch([L], seed=100 + L, device="cpu", permute=permute)
     out, lse, o64, idx, cnt = run_pipeline(d, k=512)
-    assert cnt[0, 0] == (L - 1) // 8 + 1
+    assert np.all(cnt[0] == (L - 1) // 8 + 1)
+    if L == 4096:
+        # the boundary: k = 512 equals the region count R = L / 8, so every region is selected
+        assert np.all(cnt[0] == 512) and L // 8 == 512
+        assert np.array_equal(idx[0], np.tile(np.arange(512, dtype=idx.dtype), (G, 1)))
     ref, ref_lse = dense_reference(d["q"][0], d["k_cache"], d["v_cache"], d["block_table"][0], L - 1)
     np.testing.assert_allclose(o64[0], ref, rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(lse[0], ref_lse, rtol=1e-6)

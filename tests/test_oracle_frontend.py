@@ -8,12 +8,16 @@ rotated in rotate-half pairs (i, i + 32) by pos * 10000^(-2i/64), and the gates 
 z = sigmoid(W_z h).
 
 Pins: the projection and norm at position 0 against numpy's float64 matmul (a library routine
-the oracle does not use); the unrotated dimensions identical at every position; every rotated
+the oracle does not use); the rotation angle itself on hand-built one-hot head vectors (the
+pair (i, i + 32) must come out as the plane rotation by pos * 10000^(-2i/64), evaluated here
+with numpy's cos/sin, for i = 0, 1, 31 at positions 1, 1000 and 2^20 - 1, so a wrong frequency
+table, base or pair map fails); the unrotated dimensions identical at every position; every rotated
 pair keeping its norm; the score-relevant dot product over the rotated dimensions depending on
 the positions only through their difference; RMSNorm's invariance to scaling the hidden state;
 zero gate weights giving z = 1/2 and negated ones 1 - z.
 """
 import numpy as np
+import pytest
 
 import oracle
 
@@ -124,3 +128,35 @@ def test_gates_are_sigmoids():
     wn[(HI + G) * DI:] ^= np.uint16(0x8000)                     # negate the gate rows
     _, _, zn = oracle.indexer_frontend(h, wn, gq, gk, np.zeros(T, np.int32))
     np.testing.assert_allclose(zn, 1.0 - z, rtol=1e-6, atol=1e-7)
+
+
+def one_hot_case(dim, val=16.0, hid=8):
+    """Hidden state e_0 and weights whose only non-zero entry puts `val` at `dim` of every
+    q head and k group: each pre-norm head vector is val * e_dim (mean square val^2 / 256,
+    so with val = 16 the RMSNorm leaves it at 16 up to eps, and gamma = 1)."""
+    h = np.zeros((1, hid), np.uint16)
+    h[0, 0] = to_bits(1.0)
+    w = np.zeros((ROWS, hid), np.uint16)
+    for v in range(HI + G):
+        w[v * DI + dim, 0] = to_bits(val)
+    ones = to_bits(np.ones(DI))
+    return h, w, ones, ones
+
+
+@pytest.mark.parametrize("i", [0, 1, 31])
+@pytest.mark.parametrize("p", [1, 1000, (1 << 20) - 1])
+def test_rotation_angle_by_hand(i, p):
+    # RoPE on the first 64 dims in rotate-half pairs (i, i + 32), angle p * 10000^(-2i/64)
+    # ([P2] §索引器打分 names RoPE on part of the dims; the frequency table is the reading).
+    th = p * 10000.0 ** (-2.0 * i / 64.0)
+    c, s = np.cos(th), np.sin(th)
+    mag = 16.0 / np.sqrt(1.0 + 1e-6)                           # the RMSNorm's eps, exactly
+    for dim, exp_i, exp_j in ((i, mag * c, mag * s), (i + 32, -mag * s, mag * c)):
+        h, w, gq, gk = one_hot_case(dim)
+        iq, ik, _ = oracle.indexer_frontend(h, w, gq, gk, np.array([p], np.int32))
+        for out in (f64(iq[0]), f64(ik[0])):                    # every q head and k group
+            want = np.zeros(DI)
+            want[i], want[i + 32] = exp_i, exp_j
+            # one bf16 rounding of each output (8 significant bits): half an ulp, <= 2^-8 relative
+            tol = np.abs(want) * 2.0 ** -8 + 1e-30
+            assert np.all(np.abs(out - want[None, :]) <= tol[None, :]), (dim, p, out[0, [i, i + 32]], want[[i, i + 32]])
