@@ -57,12 +57,13 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--repeats", type=int, default=5, help="timed passes of --steps steps; the median is reported")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--layers", type=int, default=N_LAYERS)
     ap.add_argument("--cpu-queries", type=int, default=32, help="oracle queries timed for cpu_baseline (30 s cap)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", choices=["decode_b1_1m", "prefill_2k_256k", "prefill_2k_256k_local",
-                                           "swa_decode_b8", "frontend_2k"], default="decode_b1_1m")
+                                           "swa_decode_b8", "frontend_2k", "fp8_peak"], default="decode_b1_1m")
     return ap.parse_args()
 
 
@@ -246,41 +247,28 @@ def build_layers(n_layers, seed0, device):
     return layers
 
 
-def record_external(event, stream_handle: int):
-    """cudaEventRecordWithFlags(..., External): inside a stream capture this becomes an
-    event-record node, so each replay timestamps the event."""
-    from cuda.bindings import runtime as rt
-    err = rt.cudaEventRecordWithFlags(event, rt.cudaStream_t(stream_handle), int(rt.cudaEventRecordExternal))[0]
-    if err != rt.cudaError_t.cudaSuccess:
-        raise RuntimeError(f"cudaEventRecordWithFlags failed: {err}")
-
-
-def capture(layers, n_steps, ev_pairs=None, e2e=None):
+def capture(layers, n_steps, e2e=None, attn_only=False):
     """One CUDA graph of n_steps decode steps, layer i % len(layers) at step i.
-    ev_pairs: list of (start, end) raw cudaEvent_t recorded (external) around each scan.
     e2e: per-layer pinned host buffers: each step's inputs are copied in from them by a kernel
-    and its output is written into them by the attention kernel."""
+    and its output is written into them by the attention kernel.
+    attn_only: only each step's attention (over the selection already in place)."""
     import torch
-    from cuda.bindings import runtime as rt
 
     g = torch.cuda.CUDAGraph()
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
         with torch.cuda.graph(g, stream=s):
-            raw = torch.cuda.current_stream().cuda_stream
             for i in range(n_steps):
                 L = layers[i % len(layers)]
                 st = L["step"]
+                if attn_only:
+                    st.run_attention()
+                    continue
                 if e2e is not None:
                     st.stage(e2e[i % len(layers)]["arena"])      # pinned host -> device, by a kernel
-                pre = post = None
-                if ev_pairs is not None:
-                    a, b = ev_pairs[i]
-                    pre = lambda a=a: record_external(a, raw)
-                    post = lambda b=b: record_external(b, raw)
                 # e2e: the attention writes the output straight into pinned host memory
-                st.run(pre_scan=pre, post_scan=post, out=None if e2e is None else e2e[i % len(layers)]["out"])
+                st.run(out=None if e2e is None else e2e[i % len(layers)]["out"])
     torch.cuda.current_stream().wait_stream(s)
     return g
 
@@ -310,8 +298,6 @@ def capture_scans(layers, n_steps):
 def run_ours(args):
     import torch
     import torch.distributed as dist
-    from cuda.bindings import runtime as rt
-
     rank, world, local = dist_env()
     if world > 1:
         import datetime
@@ -337,34 +323,42 @@ def run_ours(args):
     # ---- warm-up graph and timed graph(s); each graph holds at most 250 steps
     chunk = min(args.steps, 250)
     n_full, rem = divmod(args.steps, chunk)
-    evs = [(rt.cudaEventCreate()[1], rt.cudaEventCreate()[1]) for _ in range(chunk)]
     g_warm = capture(layers, max(args.warmup, 3))
     g_main = capture(layers, chunk)
     g_tail = capture(layers, rem) if rem else None
-    # the same steps with event-record nodes around every scan: a second timed pass gives the
-    # scan's launch duration (the nodes cost a few microseconds a step, so they stay out of
-    # the headline pass)
-    g_ev = capture(layers, chunk, ev_pairs=evs)
-    for _ in range(2):
-        g_warm.replay()
+    g_warm.replay()
+    # every graph the timed region replays runs once untimed first (a graph's first replay
+    # uploads it and pays one-time costs)
+    g_main.replay()
+    if g_tail is not None:
+        g_tail.replay()
+    g_warm.replay()
     dsa.check_device()
     torch.cuda.synchronize()
 
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(local)
-    barrier()
-    torch.cuda.synchronize()
-    with sampler:
-        start.record()
+    def timed(graphs_once):
+        """One timed pass of exactly K steps: barrier + synchronize on both sides, CUDA
+        events on the replaying stream; the slowest rank's milliseconds."""
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        a.record()
+        graphs_once()
+        b.record()
+        torch.cuda.synchronize()
+        barrier()
+        return max_over_ranks(a.elapsed_time(b))
+
+    def main_pass():
         for _ in range(n_full):
             g_main.replay()
         if g_tail is not None:
             g_tail.replay()
-        end.record()
-        torch.cuda.synchronize()
-    barrier()
-    ms = start.elapsed_time(end)
-    ms = max_over_ranks(ms)
+
+    sampler = ClockSampler(local)
+    with sampler:
+        passes = [timed(main_pass) for _ in range(args.repeats)]
+    ms = statistics.median(passes)
     # the scan's launch duration: the same scans (layer round robin) back to back in one graph,
     # CUDA events around it on its stream
     g_scan = capture_scans(layers, chunk)
@@ -372,19 +366,27 @@ def run_ours(args):
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     scan_ms = []
-    for _ in range(n_full):
+    for _ in range(max(n_full, 3)):
         e0.record()
         g_scan.replay()
         e1.record()
         torch.cuda.synchronize()
         scan_ms.append(e0.elapsed_time(e1) / chunk)
-    scan_avg_ms = max_over_ranks(sum(scan_ms) / len(scan_ms))
-    # the same steps with event-record nodes around every scan (their cost, a few microseconds
-    # a step, stays out of the headline pass): the scan's duration inside the step, reported
-    g_ev.replay()
+    scan_avg_ms = max_over_ranks(statistics.median(scan_ms))
+    # the attention alone (over the selections the steps left in place), back to back in one
+    # graph: with the scan alone it splits the step's time (the selection takes the rest)
+    g_sa = capture(layers, chunk, attn_only=True)
+    g_sa.replay()
     torch.cuda.synchronize()
-    in_step_ms = [rt.cudaEventElapsedTime(a, b)[1] for a, b in evs]
-    in_step_avg_ms = max_over_ranks(sum(in_step_ms) / len(in_step_ms))
+    sa_ms = []
+    for _ in range(3):
+        e0.record()
+        g_sa.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        sa_ms.append(e0.elapsed_time(e1) / chunk)
+    sa_avg_ms = max_over_ranks(statistics.median(sa_ms))
+    del g_sa
     dsa.check_device()
 
     # ---- e2e: host (pinned) inputs in, result out, every step
@@ -398,19 +400,17 @@ def run_ours(args):
     g_e2e = capture(layers, chunk, e2e=e2e_bufs)
     g_e2e_tail = capture(layers, rem, e2e=e2e_bufs) if rem else None
     g_e2e.replay()
-    torch.cuda.synchronize()
-    barrier()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record()
-    for _ in range(n_full):
-        g_e2e.replay()
     if g_e2e_tail is not None:
         g_e2e_tail.replay()
-    t1.record()
     torch.cuda.synchronize()
-    barrier()
-    e2e_ms = max_over_ranks(t0.elapsed_time(t1))
+
+    def e2e_pass():
+        for _ in range(n_full):
+            g_e2e.replay()
+        if g_e2e_tail is not None:
+            g_e2e_tail.replay()
+
+    e2e_ms = statistics.median([timed(e2e_pass) for _ in range(args.repeats)])
     dsa.check_device()
     # e2e results must equal the device-resident results (same inputs)
     assert torch.equal(e2e_bufs[0]["out"], layers[0]["step"].out.cpu())
@@ -428,12 +428,15 @@ def run_ours(args):
                    "l2": f"inputs larger than L2: {args.layers} layer caches of "
                          f"{scan_bytes(own) / 1e6:.0f} MB summaries + 3 GiB K/V used round robin",
                    "graph": "each step captured in a CUDA graph; kernels chained by programmatic dependent launch",
+                   "timing": f"median of {args.repeats} timed passes of {args.steps} steps (every graph replayed "
+                             "once untimed first)",
                    "scan_timing": "graph of the step's scans back to back, CUDA events around it"},
+        "passes_ms": passes,
         "step_hbm_gbs": step_gbs,
         "roofline": {"kernel": "indexer scan (scan_kernel)", "bound": "hbm", "achieved": scan_gbs, "peak": hbm,
                      "unit": "GB/s", "frac": scan_gbs / hbm, "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": scan_bytes(own), "avg_launch_us": scan_avg_ms * 1e3,
-                     "in_step_us": in_step_avg_ms * 1e3,
+                     "step_us": ms * 1e3 / args.steps, "attn_alone_us": sa_avg_ms * 1e3,
                      "traffic": SCAN_TRAFFIC_BYTES},
         "e2e": {"value": replicas.job_throughput(args.steps, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
@@ -842,6 +845,56 @@ def run_frontend(args):
     print(json.dumps(line), flush=True)
 
 
+def run_fp8_peak(args):
+    """The dense e4m3 tensor peak of this GPU, measured the way the bf16 figure is: a cuBLAS
+    e4m3 x e4m3 GEMM (torch._scaled_mm, 8192^3, bf16 output, 2 * 8192^3 FLOP) as a burst
+    (the best of 10 single launches, CUDA events) and sustained (back to back for 4 s)."""
+    import torch
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    n = 8192
+    g = torch.Generator(device=dev)
+    g.manual_seed(1242)
+    a = torch.randn((n, n), generator=g, device=dev).to(torch.float8_e4m3fn)
+    b = torch.randn((n, n), generator=g, device=dev).to(torch.float8_e4m3fn).t()   # column-major
+    one = torch.ones((), dtype=torch.float32, device=dev)
+    out = torch.empty((n, n), dtype=torch.bfloat16, device=dev)
+
+    def mm():
+        torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16, out=out)
+
+    for _ in range(5):
+        mm()
+    torch.cuda.synchronize()
+    flop = 2.0 * n ** 3
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    burst = []
+    for _ in range(10):
+        e0.record()
+        mm()
+        e1.record()
+        torch.cuda.synchronize()
+        burst.append(flop / (e0.elapsed_time(e1) * 1e-3) / 1e12)
+    sampler = ClockSampler(0)
+    with sampler:
+        reps, t0 = 0, time.perf_counter()
+        e0.record()
+        while time.perf_counter() - t0 < 4.0:
+            for _ in range(20):
+                mm()
+            reps += 20
+            torch.cuda.synchronize()
+        e1.record()
+        torch.cuda.synchronize()
+    sustained = flop * reps / (e0.elapsed_time(e1) * 1e-3) / 1e12
+    line = {"metric": "dense e4m3 GEMM TFLOP/s (torch._scaled_mm 8192^3, bf16 out)", "value": max(burst),
+            "unit": "TFLOP/s", "n_gpus": 1, "burst_tflops": max(burst), "sustained_tflops": sustained,
+            "sustained_launches": reps, "higher_is_better": True, "dtype": "e4m3", "data": "synthetic",
+            "config": {"workload": "fp8_peak", "m": n, "n": n, "k": n}, "clocks": sampler.summary()}
+    print(json.dumps(line), flush=True)
+
+
 def tensor_peak(fp8: bool):
     """Dense tensor peak in TFLOP/s: the measured cuBLAS bf16 burst figure (x2 for e4m3,
     the nominal fp8/bf16 ratio of the part), else the fallback."""
@@ -864,6 +917,8 @@ def main():
         run_swa(args)
     elif args.workload == "frontend_2k":
         run_frontend(args)
+    elif args.workload == "fp8_peak":
+        run_fp8_peak(args)
     else:
         run_ours(args)
 

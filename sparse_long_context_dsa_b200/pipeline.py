@@ -109,12 +109,10 @@ class DecodeStep:
             self.dst_slot[:n].copy_(torch.tensor([int(s) for s in slots], dtype=torch.int64))
         self.n_compress = n
 
-    def run(self, pre_scan=None, post_scan=None, out=None):
-        """Launches the step on the current stream (capturable).  pre_scan/post_scan are
-        optional callables invoked right before/after the scores + selection call (the
-        benchmark records timing events there).  out: where the attention writes its
-        output, bf16 [B][64][192], on the device (default `self.out`) or in pinned host
-        memory, which the kernel then writes directly."""
+    def run(self, out=None):
+        """Launches the step on the current stream (capturable).  out: where the attention
+        writes its output, bf16 [B][64][192], on the device (default `self.out`) or in pinned
+        host memory, which the kernel then writes directly."""
         if out is None:
             out = self.out
         elif tuple(out.shape) != tuple(self.out.shape) or out.dtype != self.out.dtype or not (
@@ -131,21 +129,24 @@ class DecodeStep:
                                                   self.n_compress, p(self.summaries), p(self.scales),
                                                   self.summaries.shape[1], dsa._stream()))
         st = dsa._stream()
-        if pre_scan is not None:
-            pre_scan()
         # scores and selection in one call (the scan's chunk maxima bound the selection)
         dsa._check(L.dsa_decode_select(p(self.index_q), p(self.gate), p(self.q_req), p(self.q_pos), self.B,
                                        p(self.summaries), p(self.scales), self.summaries.shape[1], p(self.sum_base),
                                        self.sum_base.numel(), p(self.scores), self.ld, self.flags, self.k,
                                        p(self.sel_idx), p(self.sel_count), p(self.ws_sel), self.ws_sel_n, st))
-        if post_scan is not None:
-            post_scan()
+        self.run_attention(out)
+        if self.n_compress:
+            main.wait_stream(self.side)
+        return out
+
+    def run_attention(self, out=None):
+        """The step's attention alone, over the selection in sel_idx / sel_count."""
+        L, p, st = dsa.lib(), dsa._p, dsa._stream()
+        out = self.out if out is None else out
         dsa._check(L.dsa_sparse_attn_decode(p(self.q), p(self.k_cache), p(self.v_cache), self.k_cache.shape[0],
                                             p(self.block_table), self.block_table.shape[1], p(self.q_pos), self.B,
                                             p(self.sel_idx), p(self.sel_count), self.k, p(out), p(self.lse),
                                             p(self.ws_attn), self.ws_attn_n, st))
-        if self.n_compress:
-            main.wait_stream(self.side)
         return out
 
 
