@@ -20,7 +20,11 @@
  *   dsa_indexer_frontend     hidden state -> index_q, index_k, gates        [P2 §索引器打分]
  *
  * Conventions (every call):
- *   - Pointers are DEVICE pointers unless stated otherwise, owned by the caller.  The
+ *   - Pointers are DEVICE pointers unless stated otherwise, owned by the caller.  Every
+ *     pointer argument is checked on the host (cudaPointerGetAttributes) before anything is
+ *     launched: device memory of another GPU, and pageable host memory on a GPU that cannot
+ *     read pageable memory, return DSA_ERR_INVALID_ARG (a kernel touching them would fault).
+ *     Pinned or registered host memory and managed memory are accepted.  The
  *     library never allocates device memory; scratch comes from a caller-provided
  *     workspace `ws` of at least the size the matching *_workspace_size() returns,
  *     aligned to 256 bytes.  Workspace contents need not be initialised and are
@@ -294,6 +298,17 @@ dsa_status_t dsa_window_attn(const void *q, const void *k_cache, const void *v_c
 dsa_status_t dsa_indexer_frontend(const void *hidden, int hid, int n_tok, const void *w, const void *gamma_q,
                                   const void *gamma_k, const int32_t *pos, void *index_q, void *index_k, float *z,
                                   dsa_stream_t stream);
+
+/* ------------------------------------------------------------------------------ */
+/* Self-test of the failure detection (no counterpart in the pages).  Every mbarrier wait in
+ * this library's kernels is bounded (2^31 SM cycles, about a second); a wait that runs out
+ * sets the timeout bit of the per-device error word and lets its kernel return, so a stuck
+ * pipeline becomes DSA_ERR_DEVICE from dsa_check_device() instead of a hung GPU.  This call
+ * launches one small kernel whose barrier nothing ever completes, with the bound set to
+ * limit_cycles (1 <= limit_cycles <= 2^31) for that kernel only: it returns after about that
+ * many cycles and leaves the timeout bit set (dsa_check_device reports it and clears it).  The
+ * kernel issues no copy or MMA and holds no tensor memory; other kernels keep their bound. */
+dsa_status_t dsa_selftest_wait_timeout(int64_t limit_cycles, dsa_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -79,15 +79,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, unsigned parity)
     return ok != 0;
 }
 
+// Bound of every mbarrier wait in the library's kernels, in SM cycles (~1 s at 1.9 GHz).
+constexpr long long kWaitLimitCycles = 1ll << 31;
+
 // Waits for the phase of `bar` with the given parity to complete.  The wait is bounded
-// (about 2^31 SM cycles, ~1 s); on timeout the error word is set and false returned,
-// so a logic error can never hang the GPU.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, unsigned parity)
+// (`limit` SM cycles); on timeout the error word is set and false returned, so a logic
+// error can never hang the GPU.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, unsigned parity, long long limit = kWaitLimitCycles)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const long long start = clock64();
     while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - start > (1ll << 31)) {
+        if (clock64() - start > limit) {
             set_error(kErrWaitTimeout);
             return false;
         }
@@ -111,12 +114,12 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, unsigned pari
     return ok != 0;
 }
 
-__device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, unsigned parity)
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, unsigned parity, long long limit = kWaitLimitCycles)
 {
     if (mbar_try_wait_sleep(bar, parity)) return true;
     const long long start = clock64();
     while (!mbar_try_wait_sleep(bar, parity)) {
-        if (clock64() - start > (1ll << 31)) {
+        if (clock64() - start > limit) {
             set_error(kErrWaitTimeout);
             return false;
         }

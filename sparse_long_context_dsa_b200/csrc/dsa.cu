@@ -4,6 +4,7 @@
 // per-device error word is a single symbol).
 #include <algorithm>
 #include <cstring>
+#include <initializer_list>
 #include <mutex>
 #include <utility>
 #include <string>
@@ -18,6 +19,7 @@
 #include "frontend.cuh"
 #include "gemm_indexer.cuh"
 #include "indexer.cuh"
+#include "selftest.cuh"
 #include "topk.cuh"
 #include "topk_cluster.cuh"
 #include "topk_rows.cuh"
@@ -46,6 +48,51 @@ dsa_status_t cuda_fail(cudaError_t e, const char *what)
     do {                                                        \
         cudaError_t e_ = (call);                                \
         if (e_ != cudaSuccess) return cuda_fail(e_, (what));    \
+    } while (0)
+
+// Every pointer argument must be memory the current device can dereference: device memory
+// of this device, managed memory, or pinned / registered host memory.  Pageable host memory
+// is refused (a kernel touching it would fault) unless the device reads pageable memory
+// coherently (cudaDevAttrPageableMemoryAccess).  Checked on the host before any launch.
+struct Ptr {
+    const void *p;
+    const char *name;
+};
+
+dsa_status_t check_reachable(std::initializer_list<Ptr> ptrs)
+{
+    int dev = 0;
+    DSA_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+    int pageable = -1;
+    for (const Ptr &x : ptrs) {
+        if (!x.p) continue;                       // NULL is each call's own business
+        cudaPointerAttributes a;
+        const cudaError_t e = cudaPointerGetAttributes(&a, x.p);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return cuda_fail(e, (std::string("cudaPointerGetAttributes(") + x.name + ")").c_str());
+        }
+        if (a.type == cudaMemoryTypeDevice && a.device != dev)
+            return fail(DSA_ERR_INVALID_ARG, std::string(x.name) + " is device memory of GPU " +
+                                                 std::to_string(a.device) + ", the call runs on GPU " +
+                                                 std::to_string(dev));
+        if (a.type != cudaMemoryTypeUnregistered) continue;
+        if (pageable < 0) {
+            DSA_CUDA(cudaDeviceGetAttribute(&pageable, cudaDevAttrPageableMemoryAccess, dev),
+                     "cudaDeviceGetAttribute(PageableMemoryAccess)");
+        }
+        if (!pageable)
+            return fail(DSA_ERR_INVALID_ARG, std::string(x.name) +
+                                                 " is pageable host memory, which this GPU cannot read: pass device "
+                                                 "memory or pinned host memory (cudaHostAlloc / cudaHostRegister)");
+    }
+    return DSA_OK;
+}
+
+#define DSA_REACHABLE(...)                                      \
+    do {                                                        \
+        dsa_status_t r_ = check_reachable({__VA_ARGS__});       \
+        if (r_ != DSA_OK) return r_;                            \
     } while (0)
 
 constexpr int kGemmMinQueries = 64;   // FP8 prefill chunks at least this long use the GEMM
@@ -267,6 +314,9 @@ dsa_status_t attn_common(const void *q, const void *k_cache, const void *v_cache
     DSA_REQUIRE(window > 0 || (sel_idx && sel_count), "NULL pointer");
     DSA_REQUIRE(aligned(q, 16) && aligned(k_cache, 16) && aligned(v_cache, 16) && aligned(out, 4),
                 "q, k_cache, v_cache must be 16-byte aligned, out 4-byte aligned");
+    DSA_REACHABLE({q, "q"}, {k_cache, "k_cache"}, {v_cache, "v_cache"}, {block_table, "block_table"},
+                  {q_req, "q_req"}, {q_pos, "q_pos"}, {sel_idx, "sel_idx"}, {sel_count, "sel_count"}, {out, "out"},
+                  {lse, "lse"}, {ws, "ws"});
     int sms = 0;
     dsa_status_t st = device_info(sms);
     if (st != DSA_OK) return st;
@@ -578,6 +628,8 @@ dsa_status_t dsa_compress_regions(const void *index_k, int64_t row_stride, int64
     DSA_REQUIRE(row_stride >= dsa::kG * dsa::kDI && row_stride % 8 == 0, "row_stride must be >= 1024 and a multiple of 8");
     DSA_REQUIRE(n_rows >= dsa::kRegion && n_slots >= 1, "n_rows >= 8 and n_slots >= 1 required");
     DSA_REQUIRE(aligned(index_k, 16) && aligned(summaries, 8) && aligned(scales, 4), "misaligned pointer");
+    DSA_REACHABLE({index_k, "index_k"}, {src_row, "src_row"}, {dst_slot, "dst_slot"}, {summaries, "summaries"},
+                  {scales, "scales"});
     int sms = 0;
     dsa_status_t st = device_info(sms);
     if (st != DSA_OK) return st;
@@ -653,6 +705,8 @@ dsa_status_t dsa_indexer_scores(const void *index_q, const float *gate, const in
     if (nq == 0) return DSA_OK;
     DSA_REQUIRE(index_q && gate && q_req && q_pos && summaries && scales && sum_base && scores, "NULL pointer");
     DSA_REQUIRE(aligned(index_q, 16) && aligned(summaries, 16), "index_q and summaries must be 16-byte aligned");
+    DSA_REACHABLE({index_q, "index_q"}, {gate, "gate"}, {q_req, "q_req"}, {q_pos, "q_pos"}, {summaries, "summaries"},
+                  {scales, "scales"}, {sum_base, "sum_base"}, {scores, "scores"}, {ws, "ws"});
     int sms = 0;
     dsa_status_t st = device_info(sms);
     if (st != DSA_OK) return st;
@@ -679,6 +733,7 @@ dsa_status_t dsa_topk_regions(const float *scores, int64_t ld_scores, const int3
     DSA_REQUIRE(ld_scores >= 1 && ld_scores < dsa::topk::kMaxRegions, "ld_scores out of [1, 2^20)");
     if (nq == 0) return DSA_OK;
     DSA_REQUIRE(scores && q_pos && sel_idx && sel_count, "NULL pointer");
+    DSA_REACHABLE({scores, "scores"}, {q_pos, "q_pos"}, {sel_idx, "sel_idx"}, {sel_count, "sel_count"}, {ws, "ws"});
     int sms = 0;
     dsa_status_t st = device_info(sms);
     if (st != DSA_OK) return st;
@@ -698,6 +753,8 @@ dsa_status_t dsa_topk_regions_noalloc(const float *scores, int64_t ld_scores, co
     DSA_REQUIRE(k >= 1 && k <= DSA_MAX_TOPK, "k out of [1, DSA_MAX_TOPK]");
     DSA_REQUIRE(ld_scores >= 1 && ld_scores < dsa::topk::kMaxRegions, "ld_scores out of [1, 2^20)");
     if (nq == 0) return DSA_OK;
+    DSA_REQUIRE(scores && q_pos && sel_idx && sel_count, "NULL pointer");
+    DSA_REACHABLE({scores, "scores"}, {q_pos, "q_pos"}, {sel_idx, "sel_idx"}, {sel_count, "sel_count"});
     const size_t need = topk_layout(nq, ld_scores, k).total;
     if (need > DSA_TOPK_STATIC_SCRATCH_BYTES)
         return fail(DSA_ERR_UNSUPPORTED, "dsa_topk_regions_noalloc: this call needs " + std::to_string(need) +
@@ -740,6 +797,9 @@ dsa_status_t dsa_decode_select(const void *index_q, const float *gate, const int
     DSA_REQUIRE(index_q && gate && q_req && q_pos && summaries && scales && sum_base && scores && sel_idx && sel_count,
                 "NULL pointer");
     DSA_REQUIRE(aligned(index_q, 16) && aligned(summaries, 16), "index_q and summaries must be 16-byte aligned");
+    DSA_REACHABLE({index_q, "index_q"}, {gate, "gate"}, {q_req, "q_req"}, {q_pos, "q_pos"}, {summaries, "summaries"},
+                  {scales, "scales"}, {sum_base, "sum_base"}, {scores, "scores"}, {sel_idx, "sel_idx"},
+                  {sel_count, "sel_count"}, {ws, "ws"});
     const size_t need_ws = dsa_decode_select_workspace_size(nq, ld_scores, k);
     if (!ws || ws_bytes < need_ws || !aligned(ws, 256))
         return fail(DSA_ERR_WORKSPACE, "decode-select workspace too small or not 256-byte aligned (need " +
@@ -775,6 +835,7 @@ dsa_status_t dsa_copy(void *dst, const void *src, size_t bytes, dsa_stream_t str
 {
     if (bytes == 0) return DSA_OK;
     DSA_REQUIRE(dst && src, "NULL pointer");
+    DSA_REACHABLE({dst, "dst"}, {src, "src"});
     int sms = 0;
     dsa_status_t st = device_info(sms);
     if (st != DSA_OK) return st;
@@ -813,6 +874,8 @@ dsa_status_t dsa_indexer_frontend(const void *hidden, int hid, int n_tok, const 
     DSA_REQUIRE(aligned(hidden, 16) && aligned(w, 16) && aligned(index_q, 16) && aligned(index_k, 16) &&
                     aligned(z, 16),
                 "hidden, w, index_q, index_k and z must be 16-byte aligned");
+    DSA_REACHABLE({hidden, "hidden"}, {w, "w"}, {gamma_q, "gamma_q"}, {gamma_k, "gamma_k"}, {pos, "pos"},
+                  {index_q, "index_q"}, {index_k, "index_k"}, {z, "z"});
     int sms = 0;
     dsa_status_t st = device_info(sms);
     if (st != DSA_OK) return st;
@@ -884,6 +947,8 @@ dsa_status_t dsa_kv_append(void *k_cache, void *v_cache, int64_t n_pages, const 
     DSA_REQUIRE(q_req == nullptr || n_req >= 1, "n_req must be >= 1");
     DSA_REQUIRE(aligned(k_cache, 16) && aligned(v_cache, 16) && aligned(new_k, 16) && aligned(new_v, 16),
                 "caches and new rows must be 16-byte aligned");
+    DSA_REACHABLE({k_cache, "k_cache"}, {v_cache, "v_cache"}, {block_table, "block_table"}, {q_req, "q_req"},
+                  {q_pos, "q_pos"}, {new_k, "new_k"}, {new_v, "new_v"});
     return launch_k("kv_append_kernel", dsa::kv_append_kernel, dim3((unsigned)n), dim3(256), 0, stream, 0,
                     static_cast<__nv_bfloat16 *>(k_cache), static_cast<__nv_bfloat16 *>(v_cache), n_pages,
                     block_table, max_pages, q_req, q_req ? n_req : n, q_pos, n,
@@ -898,6 +963,17 @@ dsa_status_t dsa_sparse_attn_prefill(const void *q, const void *k_cache, const v
     DSA_REQUIRE(q_req != nullptr || nq == 0, "q_req must not be NULL");
     return attn_common(q, k_cache, v_cache, n_pages, block_table, max_pages, q_req, n_req, q_pos, nq, sel_idx,
                        sel_count, k, out, lse, ws, ws_bytes, stream);
+}
+
+dsa_status_t dsa_selftest_wait_timeout(int64_t limit_cycles, dsa_stream_t stream)
+{
+    DSA_REQUIRE(limit_cycles >= 1 && limit_cycles <= dsa::kWaitLimitCycles,
+                "limit_cycles out of [1, 2^31]");
+    int sms = 0;
+    dsa_status_t st = device_info(sms);
+    if (st != DSA_OK) return st;
+    return launch_k("wait_timeout_kernel", dsa::wait_timeout_kernel, dim3(1), dim3(64), 0, stream, 0,
+                    (long long)limit_cycles);
 }
 
 }  // extern "C"

@@ -54,6 +54,7 @@ _SIG = {
                                          _I64P, ctypes.c_int, _F32P, ctypes.c_int64, ctypes.c_uint32, ctypes.c_int,
                                          _I32P, _I32P, _VP, ctypes.c_size_t, _VP]),
     "dsa_copy": (ctypes.c_int, [_VP, _VP, ctypes.c_size_t, _VP]),
+    "dsa_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_int64, _VP]),
     "dsa_attn_workspace_size": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int]),
     "dsa_sparse_attn_decode": (ctypes.c_int, [_VP, _VP, _VP, ctypes.c_int64, _I32P, ctypes.c_int, _I32P,
                                               ctypes.c_int, _I32P, _I32P, ctypes.c_int, _VP, _F32P, _VP,
@@ -233,6 +234,12 @@ def topk_regions_noalloc(scores, q_pos, k, sel_idx, sel_count):
     _need(sel_count, torch.int32, (nq, G), "sel_count")
     _check(lib().dsa_topk_regions_noalloc(_p(scores), ld, _p(q_pos), nq, k, _p(sel_idx), _p(sel_count), _stream()))
     return sel_idx, sel_count
+
+
+def selftest_wait_timeout(limit_cycles: int):
+    """dsa_selftest_wait_timeout: one kernel whose mbarrier wait nothing completes gives up
+    after limit_cycles and sets the timeout bit (read it with check_device)."""
+    _check(lib().dsa_selftest_wait_timeout(int(limit_cycles), _stream()))
 
 
 def copy(dst, src):

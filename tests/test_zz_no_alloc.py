@@ -6,12 +6,14 @@ For them the library keeps the top-k scratch in one static per-GPU array.  This 
 last so that a failure here leaves every other result already reported; it must pass
 both alone in a fresh process and after the other tests.  The selection is integer work,
 so the two entry points must agree exactly, on two calls in a row (the static array keeps
-the first call's contents, which the second call must not depend on).
+the first call's contents, which the second call must not depend on), and both must equal
+the CPU oracle's selection on the same scores.
 """
 import numpy as np
 import pytest
 import torch
 
+import oracle
 from sparse_long_context_dsa_b200 import dsa
 
 pytestmark = pytest.mark.gpu
@@ -36,7 +38,12 @@ def regular_and_static(scores, q_pos, k):
     return a_idx.cpu(), a_cnt.cpu(), b_idx.cpu(), b_cnt.cpu()
 
 
-def test_two_calls_in_a_row_match_the_workspace_entry_point():
+def oracle_selection(scores, q_pos, k):
+    idx, cnt = oracle.topk_regions(scores.cpu().numpy(), q_pos.cpu().numpy(), k)
+    return torch.from_numpy(np.ascontiguousarray(idx)), torch.from_numpy(np.ascontiguousarray(cnt))
+
+
+def test_two_calls_in_a_row_match_the_workspace_entry_point_and_the_oracle():
     # call 1: a 1M-token decode row set (4 groups x 131,071 regions); call 2: a batch of
     # shorter rows with heavy ties, which would expose stale candidates or counters
     s1 = indexer_like_scores(1, 1, 131071)
@@ -44,11 +51,15 @@ def test_two_calls_in_a_row_match_the_workspace_entry_point():
     a, ac, b, bc = regular_and_static(s1, p1, 512)
     assert torch.equal(ac, bc) and torch.equal(a, b)
     assert int(bc.min()) == 512
+    oi, oc = oracle_selection(s1, p1, 512)
+    assert torch.equal(bc, oc) and torch.equal(b, oi)
 
     s2 = torch.randint(0, 3, (3, G, 20000), device="cuda").float()
     p2 = torch.tensor([8 * 20000, 8 * 9000 + 5, 8 * 300], dtype=torch.int32, device="cuda")
     a, ac, b, bc = regular_and_static(s2, p2, 512)
     assert torch.equal(ac, bc) and torch.equal(a, b)
+    oi, oc = oracle_selection(s2, p2, 512)
+    assert torch.equal(bc, oc) and torch.equal(b, oi)
 
 
 def test_oversized_call_is_rejected_with_a_clear_error():
