@@ -895,16 +895,23 @@ def run_fp8_peak(args):
     print(json.dumps(line), flush=True)
 
 
+# Dense e4m3 GEMM peak of this machine's B200s, burst (cuBLAS e4m3 8192^3 through
+# torch._scaled_mm: `python bench.py --workload fp8_peak`; sustained under the power cap: 2,643)
+FP8_PEAK_TFLOPS = 3093.0
+
+
 def tensor_peak(fp8: bool):
-    """Dense tensor peak in TFLOP/s: the measured cuBLAS bf16 burst figure (x2 for e4m3,
-    the nominal fp8/bf16 ratio of the part), else the fallback."""
+    """Dense tensor peak in TFLOP/s: e4m3 the measured burst GEMM figure above; bf16 the
+    measured cuBLAS burst figure of MEASURED_PEAKS.json, else the fallback."""
+    if fp8:
+        return FP8_PEAK_TFLOPS, "measured e4m3 (cuBLAS 8192^3 burst, bench.py --workload fp8_peak)"
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             v, kind = float(json.load(f)["bf16_tflops"]), "measured bf16"
     except Exception:
         v, kind = 1590.0, "fallback bf16"
-    return (2 * v, kind + " x 2 (nominal e4m3/bf16 ratio)") if fp8 else (v, kind)
+    return v, kind
 
 
 def main():
