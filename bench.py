@@ -58,6 +58,11 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--repeats", type=int, default=5, help="timed passes of --steps steps; the median is reported")
+    ap.add_argument("--shard", choices=["replicas", "groups"], default="replicas",
+                    help="replicas: independent requests per GPU; groups: KV-group shards of one request")
+    ap.add_argument("--tp", type=int, default=0,
+                    help="--shard groups: GPUs per request (1, 2 or 4; default min(world, 4)); on fewer GPUs "
+                         "than tp the run times one shard of a tp-way split")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--layers", type=int, default=N_LAYERS)
     ap.add_argument("--cpu-queries", type=int, default=32, help="oracle queries timed for cpu_baseline (30 s cap)")
@@ -222,7 +227,9 @@ def run_reference(args):
 
 # ------------------------------------------------------------------ GPU arm
 
-def build_layers(n_layers, seed0, device):
+def build_layers(n_layers, seed0, device, g0=0, ng=4):
+    """n_layers independent 1M-token layer caches; with ng < 4 only the summaries and K/V of
+    groups g0 .. g0 + ng - 1 are kept (one GPU of a KV-group-sharded decode)."""
     import torch
     from sparse_long_context_dsa_b200 import pipeline
     from sparse_long_context_dsa_b200 import workloads as W
@@ -236,10 +243,14 @@ def build_layers(n_layers, seed0, device):
         pipeline.compress_all(d["index_k"], [L_CTX - 1], [0], d["sum_base"], S, C)
         tail = d["index_k"][L_CTX - 8:].clone()            # the region this step completes
         del d["index_k"]
+        if ng < 4:
+            S, C = S[g0:g0 + ng].contiguous(), C[g0:g0 + ng].contiguous()
+            d["k_cache"] = d["k_cache"][:, g0:g0 + ng].contiguous()
+            d["v_cache"] = d["v_cache"][:, g0:g0 + ng].contiguous()
         torch.cuda.empty_cache()
         own = (L_CTX - 1) // 8
         step = pipeline.DecodeStep(S, C, d["sum_base"], d["block_table"], d["k_cache"], d["v_cache"], ld=own,
-                                   k=TOPK, tail_tokens=8)
+                                   k=TOPK, tail_tokens=8, g0=g0)
         step.load(d["index_q"], d["gate"], d["q"], d["q_pos"], tail)
         step.set_compress([0], [own])
         layers.append(dict(step=step, inputs=d))
@@ -293,6 +304,96 @@ def capture_scans(layers, n_steps):
                                                  p(st.ws_idx), st.ws_idx_n, dsa._stream()))
     torch.cuda.current_stream().wait_stream(s)
     return g
+
+
+def run_groups(args):
+    """Decode at 1M context with KV-group shards ([P2] §索引器打分: the 4 groups split cleanly):
+    tp GPUs share each request, GPU i holding groups 4i/tp .. 4(i+1)/tp - 1 of its summaries and
+    K/V; a step is that shard's compress / score / select / attend (one CUDA graph per layer)
+    followed by an NCCL all-gather of the 16*ng output heads of every shard (world / tp
+    replicas of tp shards).  On fewer GPUs than tp, a run times one shard's step alone (the
+    per-GPU compute of a tp-way split, no gather)."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    from sparse_long_context_dsa_b200 import dsa, replicas
+
+    rank, world, local = dist_env()
+    tp = args.tp or min(world, 4)
+    lone = world < tp                          # one shard of a tp-way split, timed alone
+    if lone and world != 1:
+        raise SystemExit("--tp larger than the number of GPUs runs on one GPU only")
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dsa.lib()
+    replica, g0, ng = replicas.group_plan(0 if lone else rank, tp if lone else world, tp)
+    grp = replicas.tp_group(world, tp) if (tp > 1 and not lone) else None
+    layers = build_layers(args.layers, seed0=1237 + 7919 * replica, device=dev, g0=g0, ng=ng)
+    for L in layers:
+        L["step"].run()
+    dsa.check_device()
+    graphs = []
+    for L in layers:                           # one graph per layer's step (compute only)
+        graphs.append(capture([L], 1))
+        graphs[-1].replay()
+    torch.cuda.synchronize()
+    gather = grp is not None
+
+    def one_pass():
+        for i in range(args.steps):
+            j = i % len(layers)
+            graphs[j].replay()
+            if gather:
+                replicas.gather_heads(layers[j]["step"].out, grp, tp)
+
+    for i in range(max(args.warmup, 3)):
+        graphs[i % len(graphs)].replay()
+        if gather:
+            replicas.gather_heads(layers[i % len(layers)]["step"].out, grp, tp)
+    torch.cuda.synchronize()
+
+    def timed():
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        replicas.barrier()
+        torch.cuda.synchronize()
+        a.record()
+        one_pass()
+        b.record()
+        torch.cuda.synchronize()
+        replicas.barrier()
+        return replicas.max_over_ranks(a.elapsed_time(b), dev)
+
+    sampler = ClockSampler(local)
+    with sampler:
+        passes = [timed() for _ in range(args.repeats)]
+    ms = statistics.median(passes)
+    dsa.check_device()
+    n_rep = 1 if lone else world // tp
+    qps = n_rep * args.steps / (ms / 1e3)
+    own = (L_CTX - 1) // 8
+    shard_bytes = step_bytes(own, TOPK) * ng // 4
+    line = {
+        "metric": METRIC, "value": qps, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "strong" if tp > 1 and n_rep == 1 else "weak", "vs_baseline": None,
+        "dtype": "e4m3+bf16 (fp32 accumulate)", "data": "synthetic",
+        "config": {"workload": "decode_b1_1m", "context": L_CTX, "topk": TOPK, "parallelism": f"groups tp{tp}",
+                   "shard": {"g0": g0, "groups": ng, "replicas": n_rep},
+                   "gather": "NCCL all-gather of the 16*ng output heads per step" if gather else
+                   ("none: one shard of a %d-way split timed alone" % tp if lone else "none (tp = 1)"),
+                   "layer_caches": args.layers, "l2": "inputs larger than L2 (layer caches round robin)",
+                   "timing": f"median of {args.repeats} timed passes of {args.steps} steps"},
+        "shard_hbm_gbs": shard_bytes * args.steps / (ms / 1e3) / 1e9,
+        "passes_ms": passes, "gpu_launches": KERNELS_PER_STEP * args.steps, "clocks": sampler.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del graphs
+    if world > 1:
+        dist.destroy_process_group()
 
 
 def run_ours(args):
@@ -926,6 +1027,8 @@ def main():
         run_frontend(args)
     elif args.workload == "fp8_peak":
         run_fp8_peak(args)
+    elif args.shard == "groups":
+        run_groups(args)
     else:
         run_ours(args)
 

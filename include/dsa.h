@@ -300,6 +300,46 @@ dsa_status_t dsa_indexer_frontend(const void *hidden, int hid, int n_tok, const 
                                   dsa_stream_t stream);
 
 /* ------------------------------------------------------------------------------ */
+/* KV-group-sharded decode.  [P2 §索引器打分] the indexer's regions and heads map one to one
+ * onto the 4 KV groups (num_provider_groups 4), and every step of the method is per group:
+ * summaries, scores, selection and attention of group g touch only group g's data and its
+ * heads (indexer heads 4g..4g+3, query heads 16g..16g+15).  A GPU that holds the groups
+ * g0 .. g0+ng-1 (ng = 1, 2 or 4, g0 + ng <= 4; e.g. two GPUs with groups {0,1} and {2,3})
+ * runs these calls on its own shard and produces exactly the rows of the 4-group calls for
+ * its groups; the 16*ng heads of output per query are then gathered across GPUs by the
+ * caller (one all-gather of 16 x 192 bf16 per group and query).  Layouts of a shard:
+ *   summaries e4m3 [ng][n_slots][256], scales fp32 [ng][n_slots]   (local group gl = g - g0)
+ *   k_cache / v_cache bf16 [n_pages][ng][64][192]
+ *   scores fp32 [nq][ng][ld_scores], sel_idx int32 [nq][ng][k], sel_count int32 [nq][ng]
+ *   out bf16 [nq][16*ng][192] (head 16*gl + i is query head 16*(g0+gl) + i), lse fp32 [nq][16*ng]
+ * index_k, index_q, gate and q keep their full layouts; each call reads its groups' part.
+ *
+ * dsa_compress_regions_groups: dsa_compress_regions for groups g0..g0+ng-1 of index_k (row
+ *   stride >= (g0+ng)*256) into the shard's pool.
+ * dsa_decode_select_groups: dsa_decode_select for the shard; the workspace of
+ *   dsa_decode_select_workspace_size(nq, ld_scores, k) bytes suffices.
+ * dsa_sparse_attn_decode_groups: dsa_sparse_attn_decode for the shard; workspace
+ *   dsa_attn_groups_workspace_size(nq, k, ng) bytes (0: none needed).
+ * A group range outside these limits returns DSA_ERR_INVALID_ARG; all else as the 4-group
+ * calls. */
+dsa_status_t dsa_compress_regions_groups(const void *index_k, int64_t row_stride, int64_t n_rows,
+                                         const int64_t *src_row, const int64_t *dst_slot, int n_regions,
+                                         int g0, int ng, uint8_t *summaries, float *scales, int64_t n_slots,
+                                         dsa_stream_t stream);
+dsa_status_t dsa_decode_select_groups(const void *index_q, const float *gate, const int32_t *q_req,
+                                      const int32_t *q_pos, int nq, int g0, int ng, const uint8_t *summaries,
+                                      const float *scales, int64_t n_slots, const int64_t *sum_base,
+                                      int n_req, float *scores, int64_t ld_scores, uint32_t flags, int k,
+                                      int32_t *sel_idx, int32_t *sel_count, void *ws, size_t ws_bytes,
+                                      dsa_stream_t stream);
+size_t dsa_attn_groups_workspace_size(int nq, int k, int ng);
+dsa_status_t dsa_sparse_attn_decode_groups(const void *q, const void *k_cache, const void *v_cache,
+                                           int64_t n_pages, const int32_t *block_table, int max_pages,
+                                           const int32_t *q_pos, int batch, int g0, int ng,
+                                           const int32_t *sel_idx, const int32_t *sel_count, int k, void *out,
+                                           float *lse, void *ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* ------------------------------------------------------------------------------ */
 /* Self-test of the failure detection (no counterpart in the pages).  Every mbarrier wait in
  * this library's kernels is bounded (2^31 SM cycles, about a second); a wait that runs out
  * sets the timeout bit of the per-device error word and lets its kernel return, so a stuck

@@ -51,7 +51,24 @@ struct Params {
     int rps;                   // regions per split
     int n_splits;
     float scale_log2;          // log2(e) / sqrt(192)
+    // KV groups held by this call: groups g0 .. g0 + 2^gshift - 1 (all four: g0 = 0, gshift = 2).
+    // Rows are (query, local group gl); K/V caches hold only these groups ([pages][ng][64][192]),
+    // q is the full [nq][64][192] and out / lse hold the local groups' heads ([nq][16 ng][192]).
+    int gshift;
+    int g0;
 };
+
+// Index of head hr of local group gl of query qi in out / lse ([nq][16 << gshift]).
+__device__ __forceinline__ int64_t out_head(const Params &p, int qi, int gl, int hr)
+{
+    return ((int64_t)qi << (p.gshift + 4)) + gl * kHeadsPerGroup + hr;
+}
+
+// First Q head of local group gl of query qi in the full q [nq][64][192].
+__device__ __forceinline__ int64_t q_head(const Params &p, int qi, int gl)
+{
+    return (int64_t)qi * kHQ + (p.g0 + gl) * kHeadsPerGroup;
+}
 
 // byte offset of element (row, col) in a [rows][3][64] bf16 tile written by TMA with the
 // 128-byte swizzle: 16-byte chunk index XOR (128-byte line index & 7)
@@ -94,11 +111,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // block order: split-major, then group, then query, so that the CTAs resident together
     // gather from one group's (and one split's) share of the cache and reuse it in L2
-    const int rows = p.nq * kG;
+    const int rows = p.nq << p.gshift;
     const int split = (int)blockIdx.x / rows;
     const int rem = (int)blockIdx.x - split * rows;
-    const int g = rem / p.nq, qi = rem - g * p.nq;
-    const int row = qi * kG + g;           // query * 4 + group
+    const int g = rem / p.nq, qi = rem - g * p.nq;      // g: local group
+    const int row = (qi << p.gshift) + g;  // query * groups + local group
     if (p.row_shared && p.row_shared[row]) return;
     const int b = p.q_req ? p.q_req[qi] : qi;
     const int pos = p.q_pos[qi];
@@ -142,7 +159,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 if (page < 0 || page >= p.n_pages) {
                     set_error(kErrAttnIndex);
                 } else {
-                    c_y = (int)((page * kG + g) * kPage + (r % 8) * kRegion);
+                    c_y = (int)(((page << p.gshift) + g) * kPage + (r % 8) * kRegion);
                     c_r = r;
                     c_v = 1;
                 }
@@ -191,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     if (my_pairs > 0) refill(0);
     // Q tile [16 heads][192] into smem with the same swizzled layout as the K/V tiles
-    const __nv_bfloat16 *qsrc = p.q + ((int64_t)qi * kHQ + g * kHeadsPerGroup) * kD;
+    const __nv_bfloat16 *qsrc = p.q + q_head(p, qi, g) * kD;
     static_assert(16 * kD / 8 == 3 * kThreads, "Q tile: three 16-byte chunks per thread");
     uint4 qv[3];
 #pragma unroll
@@ -401,14 +418,13 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             const float L = hw[64 + hr];
             const float inv = (L > 0.0f) ? 1.0f / L : 0.0f;
-            const int head = g * kHeadsPerGroup + hr;
-            *reinterpret_cast<__nv_bfloat162 *>(p.out + ((int64_t)qi * kHQ + head) * kD + d) =
+            *reinterpret_cast<__nv_bfloat162 *>(p.out + out_head(p, qi, g, hr) * kD + d) =
                 __floats2bfloat162_rn(a * inv, c * inv);
         }
         if (p.lse && threadIdx.x < 16) {
             const int hr = threadIdx.x;
             const float L = hw[64 + hr], M = hw[80 + hr];
-            p.lse[(int64_t)qi * kHQ + g * kHeadsPerGroup + hr] =
+            p.lse[out_head(p, qi, g, hr)] =
                 (L > 0.0f) ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
         }
     } else {
@@ -449,7 +465,7 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const Params p
     __shared__ float osum[4][kD];
     const int row = blockIdx.x >> 4, hr = blockIdx.x & 15;
     if (p.row_shared && p.row_shared[row]) return;
-    const int qi = row >> 2, g = row & 3;
+    const int qi = row >> p.gshift, g = row & ((1 << p.gshift) - 1);
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int d = tid % kD, sg = tid / kD;
     bool bad_cnt;
@@ -500,10 +516,10 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const Params p
     __syncthreads();
     if (sg == 0) {
         const float o = (osum[0][d] + osum[1][d]) + (osum[2][d] + osum[3][d]);
-        const int head = g * kHeadsPerGroup + hr;
-        p.out[((int64_t)qi * kHQ + head) * kD + d] = __float2bfloat16_rn(L > 0.0f ? o / L : 0.0f);
+        const int64_t head = out_head(p, qi, g, hr);
+        p.out[head * kD + d] = __float2bfloat16_rn(L > 0.0f ? o / L : 0.0f);
         if (p.lse && d == 0)
-            p.lse[(int64_t)qi * kHQ + head] = (L > 0.0f) ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+            p.lse[head] = (L > 0.0f) ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
     }
 }
 

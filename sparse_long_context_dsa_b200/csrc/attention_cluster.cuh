@@ -59,12 +59,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
-    const int row = blockIdx.y;                                             // query * 4 + group
-    const int qi = row >> 2, g = row & 3;
+    const int row = blockIdx.y;                                             // query * groups + local group
+    const int qi = row >> p.gshift, g = row & ((1 << p.gshift) - 1);
     // the loads that depend on nothing else go out first: the Q tile (into registers, stored
     // to smem once the K/V loads are issued) and this warp's selection entries, beside the
     // selection count
-    const __nv_bfloat16 *qsrc = p.q + ((int64_t)qi * kHQ + g * kHeadsPerGroup) * kD;
+    const __nv_bfloat16 *qsrc = p.q + attn::q_head(p, qi, g) * kD;
     constexpr int kQChunks = 16 * kD / 8;                                   // 384 16-byte chunks
     uint4 qv[2];
 #pragma unroll
@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (page < 0 || page >= p.n_pages) {
                     set_error(kErrAttnIndex);
                 } else {
-                    y = (int)((page * kG + g) * kPage + (rr % 8) * kRegion);
+                    y = (int)(((page << p.gshift) + g) * kPage + (rr % 8) * kRegion);
                     r = rr;
                     v = 1;
                 }
@@ -324,9 +324,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             acc += wt * inbox[c * kInRow + tid];
         }
         const int d = tid;
-        const int head = g * kHeadsPerGroup + hr;
-        p.out[((int64_t)qi * kHQ + head) * kD + d] = __float2bfloat16_rn(L > 0.0f ? acc / L : 0.0f);
-        if (p.lse && d == 0) p.lse[(int64_t)qi * kHQ + head] = (L > 0.0f) ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+        const int64_t head = attn::out_head(p, qi, g, hr);
+        p.out[head * kD + d] = __float2bfloat16_rn(L > 0.0f ? acc / L : 0.0f);
+        if (p.lse && d == 0) p.lse[head] = (L > 0.0f) ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
     }
 }
 

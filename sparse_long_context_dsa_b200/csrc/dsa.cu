@@ -95,6 +95,14 @@ dsa_status_t check_reachable(std::initializer_list<Ptr> ptrs)
         if (r_ != DSA_OK) return r_;                            \
     } while (0)
 
+// A KV group range: 1, 2 or 4 consecutive groups starting at g0.
+dsa_status_t group_range_args(int g0, int ng)
+{
+    DSA_REQUIRE(ng == 1 || ng == 2 || ng == 4, "ng must be 1, 2 or 4");
+    DSA_REQUIRE(g0 >= 0 && g0 + ng <= dsa::kG, "groups g0 .. g0 + ng - 1 must lie in 0 .. 3");
+    return DSA_OK;
+}
+
 constexpr int kGemmMinQueries = 64;   // FP8 prefill chunks at least this long use the GEMM
 constexpr int kSharedMinQueries = 32; // prefill attention calls at least this long share selections
 
@@ -185,10 +193,11 @@ dsa_status_t launch_k(const char *what, void (*kern)(KArgs...), dim3 grid, dim3 
     return launched(what);
 }
 
-// K/V cache viewed as [rows = n_pages*4*64][3][64] bf16: one region = box {64, 3, 8}.
-dsa_status_t kv_map(CUtensorMap *m, const void *cache, int64_t n_pages)
+// K/V cache viewed as [rows = n_pages*ng*64][3][64] bf16 (ng KV groups per page, 4 unless
+// the call holds a group range): one region = box {64, 3, 8}.
+dsa_status_t kv_map(CUtensorMap *m, const void *cache, int64_t n_pages, int ng = dsa::kG)
 {
-    const cuuint64_t dims[3] = {64, 3, (cuuint64_t)n_pages * dsa::kG * dsa::kPage};
+    const cuuint64_t dims[3] = {64, 3, (cuuint64_t)n_pages * ng * dsa::kPage};
     const cuuint64_t strides[2] = {128, (cuuint64_t)dsa::kD * 2};
     const cuuint32_t box[3] = {64, 3, (cuuint32_t)dsa::kRegion};
     return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, cache, dims, strides, box, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
@@ -208,9 +217,9 @@ struct TopkLayout {
     size_t hist, ctr, sure, cand, total;
 };
 
-TopkLayout topk_layout(int nq, int64_t ld, int k)
+TopkLayout topk_layout(int nq, int64_t ld, int k, int ng = dsa::kG)
 {
-    const size_t rows = (size_t)nq * dsa::kG;
+    const size_t rows = (size_t)nq * ng;
     TopkLayout L;
     L.hist = 0;
     L.ctr = round_up(rows * dsa::topk::kBins * 4, 256);
@@ -226,7 +235,10 @@ struct AttnPlan {
     size_t ws;
 };
 
-AttnPlan attn_plan(int nq, int k, int sm_count)
+// The split is decided on all four groups' rows, also for a call that holds fewer groups,
+// so a group shard runs exactly the splits of the 4-group call (and its rows come out bit
+// for bit the same); the workspace counts the call's own rows (nq * ng).
+AttnPlan attn_plan(int nq, int k, int sm_count, int ng = dsa::kG)
 {
     AttnPlan a;
     const int rows = nq * dsa::kG;
@@ -243,7 +255,7 @@ AttnPlan attn_plan(int nq, int k, int sm_count)
         while ((k + rps - 1) / rps > dsa::kD) rps += 2;
         a.rps = rps;
         a.n_splits = (k + a.rps - 1) / a.rps;
-        const size_t n = (size_t)rows * a.n_splits * 16;
+        const size_t n = (size_t)nq * ng * a.n_splits * 16;
         a.ws = round_up(n * dsa::kD * 4, 256) + round_up(n * 2 * 4, 256);
     }
     return a;
@@ -290,7 +302,7 @@ dsa_status_t attn_cluster_launch(const CUtensorMap &mk, const CUtensorMap &mv, c
                                  dsa_stream_t stream)
 {
     return launch_k("sparse_attn_cluster_kernel", dsa::attnc::sparse_attn_cluster_kernel,
-                    dim3(dsa::attnc::kSplits, (unsigned)(nq * dsa::kG)), dim3(dsa::attnc::kThreads),
+                    dim3(dsa::attnc::kSplits, (unsigned)(nq * ((int)1 << p.gshift))), dim3(dsa::attnc::kThreads),
                     dsa::attnc::kSmemBytes, stream, (unsigned)dsa::attnc::kSplits, mk, mv, p);
 }
 
@@ -302,7 +314,8 @@ int window_regions(int window) { return window / dsa::kRegion + 2; }
 dsa_status_t attn_common(const void *q, const void *k_cache, const void *v_cache, int64_t n_pages,
                          const int32_t *block_table, int max_pages, const int32_t *q_req, int n_req,
                          const int32_t *q_pos, int nq, const int32_t *sel_idx, const int32_t *sel_count, int k,
-                         void *out, float *lse, void *ws, size_t ws_bytes, dsa_stream_t stream, int window = 0)
+                         void *out, float *lse, void *ws, size_t ws_bytes, dsa_stream_t stream, int window = 0,
+                         int g0 = 0, int ng = dsa::kG)
 {
     DSA_REQUIRE(nq >= 0, "nq must be >= 0");
     DSA_REQUIRE(window > 0 || (k >= 1 && k <= DSA_MAX_TOPK), "k out of [1, DSA_MAX_TOPK]");
@@ -320,13 +333,15 @@ dsa_status_t attn_common(const void *q, const void *k_cache, const void *v_cache
     int sms = 0;
     dsa_status_t st = device_info(sms);
     if (st != DSA_OK) return st;
+    // (decided on all four groups' rows, as the split above: a group shard runs the kernels
+    // of the 4-group call)
     const bool clustered =
         window == 0 && k <= dsa::attnc::kMaxK && (int64_t)nq * dsa::kG <= cluster_attn_capacity();
     // prefill chunks: 8 neighbouring queries per CTA share one stream of their selections' union
-    const bool shared = window == 0 && !clustered && q_req != nullptr && nq >= kSharedMinQueries &&
+    const bool shared = window == 0 && !clustered && ng == dsa::kG && q_req != nullptr && nq >= kSharedMinQueries &&
                         k <= dsa::attntc::kMaxK &&
                         (int64_t)max_pages * dsa::kPage / dsa::kRegion <= (int64_t)dsa::attntc::kMaxWords * 32;
-    const AttnPlan plan = attn_plan(nq, k, sms);
+    const AttnPlan plan = attn_plan(nq, k, sms, ng);
     const size_t need_ws = plan.ws + (shared ? round_up((size_t)nq * dsa::kG, 256) : 0);
     if (need_ws > 0 && !clustered) {
         if (!ws || ws_bytes < need_ws || !aligned(ws, 256))
@@ -334,8 +349,8 @@ dsa_status_t attn_common(const void *q, const void *k_cache, const void *v_cache
                                                std::to_string(need_ws) + " bytes)");
     }
     CUtensorMap mk, mv;
-    if ((st = kv_map(&mk, k_cache, n_pages)) != DSA_OK) return st;
-    if ((st = kv_map(&mv, v_cache, n_pages)) != DSA_OK) return st;
+    if ((st = kv_map(&mk, k_cache, n_pages, ng)) != DSA_OK) return st;
+    if ((st = kv_map(&mv, v_cache, n_pages, ng)) != DSA_OK) return st;
 
     dsa::attn::Params p{};
     p.q = static_cast<const __nv_bfloat16 *>(q);
@@ -346,7 +361,7 @@ dsa_status_t attn_common(const void *q, const void *k_cache, const void *v_cache
     p.sel_count = sel_count;
     p.out = static_cast<__nv_bfloat16 *>(out);
     p.lse = lse;
-    const size_t n = (size_t)nq * dsa::kG * plan.n_splits * 16;
+    const size_t n = (size_t)nq * ng * plan.n_splits * 16;
     p.part_o = plan.ws ? static_cast<float *>(ws) : nullptr;
     p.part_ml = plan.ws ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + round_up(n * dsa::kD * 4, 256))
                         : nullptr;
@@ -359,6 +374,8 @@ dsa_status_t attn_common(const void *q, const void *k_cache, const void *v_cache
     p.n_splits = plan.n_splits;
     p.window = window;
     p.scale_log2 = dsa::attn::kLog2e / sqrtf((float)dsa::kD);
+    p.gshift = ng == 4 ? 2 : ng == 2 ? 1 : 0;
+    p.g0 = g0;
 
     if (clustered) return attn_cluster_launch(mk, mv, p, nq, stream);
     if (shared) {
@@ -388,12 +405,12 @@ dsa_status_t attn_common(const void *q, const void *k_cache, const void *v_cache
                                         (int)dsa::attn::kSmemBytes);
     });
     DSA_CUDA(attr_err, "cudaFuncSetAttribute(sparse_attn_kernel)");
-    dim3 grid((unsigned)(plan.n_splits * nq * dsa::kG));
+    dim3 grid((unsigned)(plan.n_splits * nq * ng));
     if ((st = launch_k("sparse_attn_kernel", dsa::attn::sparse_attn_kernel, grid, dim3(dsa::attn::kThreads),
                        dsa::attn::kSmemBytes, stream, 0, mk, mv, p)) != DSA_OK)
         return st;
     if (plan.n_splits > 1) {
-        if ((st = launch_k("combine_kernel", dsa::attn::combine_kernel, dim3(nq * dsa::kG * 16),
+        if ((st = launch_k("combine_kernel", dsa::attn::combine_kernel, dim3(nq * ng * 16),
                            dim3(dsa::attn::kCombineThreads), 0, stream, 0, p)) != DSA_OK)
             return st;
     }
@@ -487,10 +504,13 @@ dsa_status_t indexer_gemm_path(const void *index_q, const float *gate, const int
 
 // Workspace path of the top-k: histogram, threshold-bin gather and last-CTA selection
 // (scales to many rows; scratch from the caller's workspace).
+int gshift_of(int ng) { return ng == 4 ? 2 : ng == 2 ? 1 : 0; }
+
 dsa_status_t topk_workspace_path(const float *scores, int64_t ld_scores, const int32_t *q_pos, int nq, int k,
-                                 int32_t *sel_idx, int32_t *sel_count, void *ws, size_t ws_bytes, dsa_stream_t stream)
+                                 int32_t *sel_idx, int32_t *sel_count, void *ws, size_t ws_bytes, dsa_stream_t stream,
+                                 int ng = dsa::kG)
 {
-    const TopkLayout L = topk_layout(nq, ld_scores, k);
+    const TopkLayout L = topk_layout(nq, ld_scores, k, ng);
     if (!ws || ws_bytes < L.total || reinterpret_cast<uintptr_t>(ws) % 256 != 0)
         return fail(DSA_ERR_WORKSPACE, "top-k workspace too small or not 256-byte aligned (need " +
                                            std::to_string(L.total) + " bytes)");
@@ -500,8 +520,9 @@ dsa_status_t topk_workspace_path(const float *scores, int64_t ld_scores, const i
     tw.ctr = reinterpret_cast<uint32_t *>(w + L.ctr);
     tw.sure = reinterpret_cast<int32_t *>(w + L.sure);
     tw.cand = reinterpret_cast<uint2 *>(w + L.cand);
+    tw.gshift = gshift_of(ng);
     DSA_CUDA(cudaMemsetAsync(w, 0, L.sure, stream), "cudaMemsetAsync(top-k histograms)");
-    const int rows = nq * dsa::kG;
+    const int rows = nq * ng;
     const dim3 grid((unsigned)((ld_scores + dsa::topk::kChunk - 1) / dsa::topk::kChunk), (unsigned)rows);
     dsa_status_t st;
     if ((st = launch_k("topk hist_kernel", dsa::topk::hist_kernel, grid, dim3(dsa::topk::kThreads), 0, stream, 0,
@@ -529,7 +550,7 @@ int cluster_size_for(int64_t ld)
 }
 
 dsa_status_t topk_cluster_path(const float *scores, int64_t ld_scores, const int32_t *q_pos, int nq, int k,
-                               int32_t *sel_idx, int32_t *sel_count, int cl, dsa_stream_t stream)
+                               int32_t *sel_idx, int32_t *sel_count, int cl, dsa_stream_t stream, int ng = dsa::kG)
 {
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
@@ -541,19 +562,19 @@ dsa_status_t topk_cluster_path(const float *scores, int64_t ld_scores, const int
                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsa::topkc::kSmemBytes);
     });
     DSA_CUDA(attr_err, "cudaFuncSetAttribute(topk_cluster_kernel)");
-    const dim3 grid((unsigned)cl, (unsigned)(nq * dsa::kG), 1);
+    const dim3 grid((unsigned)cl, (unsigned)(nq * ng), 1);
     if (cl == 1)
         return launch_k("topk_cluster_kernel", dsa::topkc::topk_cluster_kernel<true>, grid, dim3(dsa::topkc::kThreads),
                         dsa::topkc::kSmemBytes, stream, 1u, scores, ld_scores, q_pos, k, sel_idx, sel_count,
-                        static_cast<const float *>(nullptr), (int64_t)0);
+                        static_cast<const float *>(nullptr), (int64_t)0, gshift_of(ng));
     return launch_k("topk_cluster_kernel", dsa::topkc::topk_cluster_kernel<false>, grid, dim3(dsa::topkc::kThreads),
                     dsa::topkc::kSmemBytes, stream, (unsigned)cl, scores, ld_scores, q_pos, k, sel_idx, sel_count,
-                    static_cast<const float *>(nullptr), (int64_t)0);
+                    static_cast<const float *>(nullptr), (int64_t)0, gshift_of(ng));
 }
 
 // Many rows of at most 65,536 scores: one CTA per row, no scratch.
 dsa_status_t topk_rows_path(const float *scores, int64_t ld_scores, const int32_t *q_pos, int nq, int k,
-                            int32_t *sel_idx, int32_t *sel_count, dsa_stream_t stream)
+                            int32_t *sel_idx, int32_t *sel_count, dsa_stream_t stream, int ng = dsa::kG)
 {
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
@@ -562,9 +583,26 @@ dsa_status_t topk_rows_path(const float *scores, int64_t ld_scores, const int32_
                                         (int)dsa::topkr::kSmemBytes);
     });
     DSA_CUDA(attr_err, "cudaFuncSetAttribute(topk_rows_kernel)");
-    return launch_k("topk_rows_kernel", dsa::topkr::topk_rows_kernel, dim3((unsigned)(nq * dsa::kG)),
+    return launch_k("topk_rows_kernel", dsa::topkr::topk_rows_kernel, dim3((unsigned)(nq * ng)),
                     dim3(dsa::topkr::kThreads), dsa::topkr::kSmemBytes, stream, 0, scores, ld_scores, q_pos, k,
-                    sel_idx, sel_count);
+                    sel_idx, sel_count, gshift_of(ng));
+}
+
+// The top-k of nq queries x ng group rows: few long rows on clusters, many rows of up to
+// 65,536 scores one CTA each, longer many-row calls through the workspace.
+dsa_status_t topk_dispatch(const float *scores, int64_t ld_scores, const int32_t *q_pos, int nq, int k,
+                           int32_t *sel_idx, int32_t *sel_count, void *ws, size_t ws_bytes, dsa_stream_t stream, int ng)
+{
+    int sms = 0;
+    dsa_status_t st = device_info(sms);
+    if (st != DSA_OK) return st;
+    const int rows = nq * ng;
+    const int cl = cluster_size_for(ld_scores);
+    if (cl > 0 && (int64_t)rows * cl <= 2 * sms)
+        return topk_cluster_path(scores, ld_scores, q_pos, nq, k, sel_idx, sel_count, cl, stream, ng);
+    if (ld_scores <= dsa::topkr::kMaxLd)
+        return topk_rows_path(scores, ld_scores, q_pos, nq, k, sel_idx, sel_count, stream, ng);
+    return topk_workspace_path(scores, ld_scores, q_pos, nq, k, sel_idx, sel_count, ws, ws_bytes, stream, ng);
 }
 
 // Scratch of dsa_topk_regions_noalloc: one static array per GPU that loads the library.
@@ -618,14 +656,16 @@ dsa_status_t dsa_check_device(dsa_stream_t stream)
     return fail(DSA_ERR_DEVICE, msg);
 }
 
-dsa_status_t dsa_compress_regions(const void *index_k, int64_t row_stride, int64_t n_rows, const int64_t *src_row,
-                                  const int64_t *dst_slot, int n_regions, uint8_t *summaries, float *scales,
-                                  int64_t n_slots, dsa_stream_t stream)
+namespace {
+dsa_status_t compress_impl(const void *index_k, int64_t row_stride, int64_t n_rows, const int64_t *src_row,
+                           const int64_t *dst_slot, int n_regions, uint8_t *summaries, float *scales, int64_t n_slots,
+                           dsa_stream_t stream, int g0, int ng)
 {
     DSA_REQUIRE(n_regions >= 0, "n_regions must be >= 0");
     if (n_regions == 0) return DSA_OK;
     DSA_REQUIRE(index_k && src_row && dst_slot && summaries && scales, "NULL pointer");
-    DSA_REQUIRE(row_stride >= dsa::kG * dsa::kDI && row_stride % 8 == 0, "row_stride must be >= 1024 and a multiple of 8");
+    DSA_REQUIRE(row_stride >= (int64_t)(g0 + ng) * dsa::kDI && row_stride % 8 == 0,
+                "row_stride must cover the groups' 256-element vectors and be a multiple of 8");
     DSA_REQUIRE(n_rows >= dsa::kRegion && n_slots >= 1, "n_rows >= 8 and n_slots >= 1 required");
     DSA_REQUIRE(aligned(index_k, 16) && aligned(summaries, 8) && aligned(scales, 4), "misaligned pointer");
     DSA_REACHABLE({index_k, "index_k"}, {src_row, "src_row"}, {dst_slot, "dst_slot"}, {summaries, "summaries"},
@@ -634,9 +674,30 @@ dsa_status_t dsa_compress_regions(const void *index_k, int64_t row_stride, int64
     dsa_status_t st = device_info(sms);
     if (st != DSA_OK) return st;
     const int grid = (int)std::min<int64_t>(n_regions, (int64_t)sms * 16);
-    return launch_k("compress_regions_kernel", dsa::compress_regions_kernel, dim3(grid), dim3(128), 0, stream, 0,
-                    static_cast<const __nv_bfloat16 *>(index_k), row_stride, n_rows, src_row, dst_slot, n_regions,
-                    summaries, scales, n_slots);
+    // one warp per group: warp gl compresses group g0 + gl into pool row gl
+    return launch_k("compress_regions_kernel", dsa::compress_regions_kernel, dim3(grid), dim3(32 * ng), 0, stream, 0,
+                    static_cast<const __nv_bfloat16 *>(index_k) + (size_t)g0 * dsa::kDI, row_stride, n_rows, src_row,
+                    dst_slot, n_regions, summaries, scales, n_slots);
+}
+}  // namespace
+
+dsa_status_t dsa_compress_regions(const void *index_k, int64_t row_stride, int64_t n_rows, const int64_t *src_row,
+                                  const int64_t *dst_slot, int n_regions, uint8_t *summaries, float *scales,
+                                  int64_t n_slots, dsa_stream_t stream)
+{
+    return compress_impl(index_k, row_stride, n_rows, src_row, dst_slot, n_regions, summaries, scales, n_slots, stream,
+                         0, dsa::kG);
+}
+
+dsa_status_t dsa_compress_regions_groups(const void *index_k, int64_t row_stride, int64_t n_rows,
+                                         const int64_t *src_row, const int64_t *dst_slot, int n_regions, int g0,
+                                         int ng, uint8_t *summaries, float *scales, int64_t n_slots,
+                                         dsa_stream_t stream)
+{
+    dsa_status_t st = group_range_args(g0, ng);
+    if (st != DSA_OK) return st;
+    return compress_impl(index_k, row_stride, n_rows, src_row, dst_slot, n_regions, summaries, scales, n_slots, stream,
+                         g0, ng);
 }
 
 // The streaming scan of dsa_indexer_scores; chunk_max (nullable) receives the largest score of
@@ -644,12 +705,12 @@ dsa_status_t dsa_compress_regions(const void *index_k, int64_t row_stride, int64
 dsa_status_t scan_path(const void *index_q, const float *gate, const int32_t *q_req, const int32_t *q_pos, int nq,
                        const uint8_t *summaries, const float *scales, int64_t n_slots, const int64_t *sum_base,
                        int n_req, float *scores, int64_t ld_scores, uint32_t flags, int sms, dsa_stream_t stream,
-                       float *chunk_max = nullptr, int64_t cm_stride = 0)
+                       float *chunk_max = nullptr, int64_t cm_stride = 0, int g0 = 0, int ng = dsa::kG)
 {
     dsa_status_t st;
     CUtensorMap map;
     {
-        const cuuint64_t dims[2] = {(cuuint64_t)dsa::kDI, (cuuint64_t)n_slots * dsa::kG};
+        const cuuint64_t dims[2] = {(cuuint64_t)dsa::kDI, (cuuint64_t)n_slots * ng};
         const cuuint64_t strides[1] = {(cuuint64_t)dsa::kDI};
         const cuuint32_t box[2] = {128, (cuuint32_t)dsa::idx::kChunk};
         if ((st = encode(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, summaries, dims, strides, box,
@@ -668,8 +729,13 @@ dsa_status_t scan_path(const void *index_q, const float *gate, const int32_t *q_
     p.cm_stride = cm_stride;
     p.n_slots = n_slots;
     p.ld = ld_scores;
-    p.units_per_query = (int)((ld_scores + dsa::idx::kChunk - 1) / dsa::idx::kChunk);
+    // stages per query: the (chunk, group) slabs of its row, four per stage
+    const int64_t chunks = (ld_scores + dsa::idx::kChunk - 1) / dsa::idx::kChunk;
+    p.units_per_query = (int)((chunks * ng + dsa::idx::kSlabs - 1) / dsa::idx::kSlabs);
     p.total_units = (int64_t)nq * p.units_per_query;
+    p.groups = ng;
+    p.gshift = gshift_of(ng);
+    p.g0 = g0;
     p.nq = nq;
     p.n_req = n_req;
     p.flags = flags;
@@ -734,16 +800,7 @@ dsa_status_t dsa_topk_regions(const float *scores, int64_t ld_scores, const int3
     if (nq == 0) return DSA_OK;
     DSA_REQUIRE(scores && q_pos && sel_idx && sel_count, "NULL pointer");
     DSA_REACHABLE({scores, "scores"}, {q_pos, "q_pos"}, {sel_idx, "sel_idx"}, {sel_count, "sel_count"}, {ws, "ws"});
-    int sms = 0;
-    dsa_status_t st = device_info(sms);
-    if (st != DSA_OK) return st;
-    const int rows = nq * dsa::kG;
-    const int cl = cluster_size_for(ld_scores);
-    if (cl > 0 && (int64_t)rows * cl <= 2 * sms) return topk_cluster_path(scores, ld_scores, q_pos, nq, k, sel_idx,
-                                                                           sel_count, cl, stream);
-    if (ld_scores <= dsa::topkr::kMaxLd) return topk_rows_path(scores, ld_scores, q_pos, nq, k, sel_idx, sel_count,
-                                                                stream);
-    return topk_workspace_path(scores, ld_scores, q_pos, nq, k, sel_idx, sel_count, ws, ws_bytes, stream);
+    return topk_dispatch(scores, ld_scores, q_pos, nq, k, sel_idx, sel_count, ws, ws_bytes, stream, dsa::kG);
 }
 
 dsa_status_t dsa_topk_regions_noalloc(const float *scores, int64_t ld_scores, const int32_t *q_pos, int nq, int k,
@@ -781,11 +838,51 @@ size_t dsa_decode_select_workspace_size(int nq, int64_t ld_scores, int k)
     return cm + dsa_topk_workspace_size(nq, ld_scores, k);
 }
 
-dsa_status_t dsa_decode_select(const void *index_q, const float *gate, const int32_t *q_req, const int32_t *q_pos,
-                               int nq, const uint8_t *summaries, const float *scales, int64_t n_slots,
-                               const int64_t *sum_base, int n_req, float *scores, int64_t ld_scores, uint32_t flags,
-                               int k, int32_t *sel_idx, int32_t *sel_count, void *ws, size_t ws_bytes,
-                               dsa_stream_t stream)
+namespace {
+// Scores and selection of the KV groups g0 .. g0 + ng - 1 (all four: g0 = 0, ng = 4); the
+// arguments are checked by the callers.
+dsa_status_t decode_select_impl(const void *index_q, const float *gate, const int32_t *q_req, const int32_t *q_pos,
+                                int nq, const uint8_t *summaries, const float *scales, int64_t n_slots,
+                                const int64_t *sum_base, int n_req, float *scores, int64_t ld_scores, uint32_t flags,
+                                int k, int32_t *sel_idx, int32_t *sel_count, void *ws, size_t ws_bytes,
+                                dsa_stream_t stream, int g0, int ng)
+{
+    const size_t need_ws = dsa_decode_select_workspace_size(nq, ld_scores, k);
+    if (!ws || ws_bytes < need_ws || !aligned(ws, 256))
+        return fail(DSA_ERR_WORKSPACE, "decode-select workspace too small or not 256-byte aligned (need " +
+                                           std::to_string(need_ws) + " bytes)");
+    int sms = 0;
+    dsa_status_t st = device_info(sms);
+    if (st != DSA_OK) return st;
+    const int64_t cm_stride = cm_stride_of(ld_scores);
+    float *chunk_max = static_cast<float *>(ws);
+    const size_t cm = round_up((size_t)nq * dsa::kG * (size_t)cm_stride * 4, 256);
+    const int cl = cluster_size_for(ld_scores);
+    const bool maxima = k <= 512 && cl > 1 && (int64_t)nq * ng * cl <= 2 * sms;
+    if ((st = scan_path(index_q, gate, q_req, q_pos, nq, summaries, scales, n_slots, sum_base, n_req, scores,
+                        ld_scores, flags, sms, stream, maxima ? chunk_max : nullptr, cm_stride, g0, ng)) != DSA_OK)
+        return st;
+    if (!maxima)
+        return topk_dispatch(scores, ld_scores, q_pos, nq, k, sel_idx, sel_count, static_cast<uint8_t *>(ws) + cm,
+                             ws_bytes - cm, stream, ng);
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(dsa::topkc::topk_cluster_kernel<false, true>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsa::topkc::kSmemBytes);
+    });
+    DSA_CUDA(attr_err, "cudaFuncSetAttribute(topk_cluster_kernel)");
+    return launch_k("topk_cluster_kernel", dsa::topkc::topk_cluster_kernel<false, true>,
+                    dim3((unsigned)cl, (unsigned)(nq * ng), 1), dim3(dsa::topkc::kThreads),
+                    dsa::topkc::kSmemBytes, stream, (unsigned)cl, scores, ld_scores, q_pos, k, sel_idx, sel_count,
+                    static_cast<const float *>(chunk_max), cm_stride, gshift_of(ng));
+}
+
+// Checks of the arguments dsa_decode_select and dsa_decode_select_groups share.
+dsa_status_t decode_select_args(const void *index_q, const float *gate, const int32_t *q_req, const int32_t *q_pos,
+                                int nq, const uint8_t *summaries, const float *scales, int64_t n_slots,
+                                const int64_t *sum_base, int n_req, float *scores, int64_t ld_scores, uint32_t flags,
+                                int k, int32_t *sel_idx, int32_t *sel_count, void *ws)
 {
     DSA_REQUIRE(nq >= 0, "nq must be >= 0");
     DSA_REQUIRE((flags & ~DSA_Q_FP8) == 0, "unknown flag");
@@ -800,35 +897,36 @@ dsa_status_t dsa_decode_select(const void *index_q, const float *gate, const int
     DSA_REACHABLE({index_q, "index_q"}, {gate, "gate"}, {q_req, "q_req"}, {q_pos, "q_pos"}, {summaries, "summaries"},
                   {scales, "scales"}, {sum_base, "sum_base"}, {scores, "scores"}, {sel_idx, "sel_idx"},
                   {sel_count, "sel_count"}, {ws, "ws"});
-    const size_t need_ws = dsa_decode_select_workspace_size(nq, ld_scores, k);
-    if (!ws || ws_bytes < need_ws || !aligned(ws, 256))
-        return fail(DSA_ERR_WORKSPACE, "decode-select workspace too small or not 256-byte aligned (need " +
-                                           std::to_string(need_ws) + " bytes)");
-    int sms = 0;
-    dsa_status_t st = device_info(sms);
+    return DSA_OK;
+}
+}  // namespace
+
+dsa_status_t dsa_decode_select(const void *index_q, const float *gate, const int32_t *q_req, const int32_t *q_pos,
+                               int nq, const uint8_t *summaries, const float *scales, int64_t n_slots,
+                               const int64_t *sum_base, int n_req, float *scores, int64_t ld_scores, uint32_t flags,
+                               int k, int32_t *sel_idx, int32_t *sel_count, void *ws, size_t ws_bytes,
+                               dsa_stream_t stream)
+{
+    dsa_status_t st = decode_select_args(index_q, gate, q_req, q_pos, nq, summaries, scales, n_slots, sum_base, n_req,
+                                         scores, ld_scores, flags, k, sel_idx, sel_count, ws);
+    if (st != DSA_OK || nq == 0) return st;
+    return decode_select_impl(index_q, gate, q_req, q_pos, nq, summaries, scales, n_slots, sum_base, n_req, scores,
+                              ld_scores, flags, k, sel_idx, sel_count, ws, ws_bytes, stream, 0, dsa::kG);
+}
+
+dsa_status_t dsa_decode_select_groups(const void *index_q, const float *gate, const int32_t *q_req,
+                                      const int32_t *q_pos, int nq, int g0, int ng, const uint8_t *summaries,
+                                      const float *scales, int64_t n_slots, const int64_t *sum_base, int n_req,
+                                      float *scores, int64_t ld_scores, uint32_t flags, int k, int32_t *sel_idx,
+                                      int32_t *sel_count, void *ws, size_t ws_bytes, dsa_stream_t stream)
+{
+    dsa_status_t st = group_range_args(g0, ng);
     if (st != DSA_OK) return st;
-    const int64_t cm_stride = cm_stride_of(ld_scores);
-    float *chunk_max = static_cast<float *>(ws);
-    const size_t cm = round_up((size_t)nq * dsa::kG * (size_t)cm_stride * 4, 256);
-    const int cl = cluster_size_for(ld_scores);
-    const bool maxima = k <= 512 && cl > 1 && (int64_t)nq * dsa::kG * cl <= 2 * sms;
-    if ((st = scan_path(index_q, gate, q_req, q_pos, nq, summaries, scales, n_slots, sum_base, n_req, scores,
-                        ld_scores, flags, sms, stream, maxima ? chunk_max : nullptr, cm_stride)) != DSA_OK)
-        return st;
-    if (!maxima)
-        return dsa_topk_regions(scores, ld_scores, q_pos, nq, k, sel_idx, sel_count, static_cast<uint8_t *>(ws) + cm,
-                                ws_bytes - cm, stream);
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(dsa::topkc::topk_cluster_kernel<false, true>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsa::topkc::kSmemBytes);
-    });
-    DSA_CUDA(attr_err, "cudaFuncSetAttribute(topk_cluster_kernel)");
-    return launch_k("topk_cluster_kernel", dsa::topkc::topk_cluster_kernel<false, true>,
-                    dim3((unsigned)cl, (unsigned)(nq * dsa::kG), 1), dim3(dsa::topkc::kThreads),
-                    dsa::topkc::kSmemBytes, stream, (unsigned)cl, scores, ld_scores, q_pos, k, sel_idx, sel_count,
-                    static_cast<const float *>(chunk_max), cm_stride);
+    st = decode_select_args(index_q, gate, q_req, q_pos, nq, summaries, scales, n_slots, sum_base, n_req, scores,
+                            ld_scores, flags, k, sel_idx, sel_count, ws);
+    if (st != DSA_OK || nq == 0) return st;
+    return decode_select_impl(index_q, gate, q_req, q_pos, nq, summaries, scales, n_slots, sum_base, n_req, scores,
+                              ld_scores, flags, k, sel_idx, sel_count, ws, ws_bytes, stream, g0, ng);
 }
 
 dsa_status_t dsa_copy(void *dst, const void *src, size_t bytes, dsa_stream_t stream)
@@ -861,6 +959,25 @@ dsa_status_t dsa_sparse_attn_decode(const void *q, const void *k_cache, const vo
 {
     return attn_common(q, k_cache, v_cache, n_pages, block_table, max_pages, nullptr, batch, q_pos, batch, sel_idx,
                        sel_count, k, out, lse, ws, ws_bytes, stream);
+}
+
+size_t dsa_attn_groups_workspace_size(int nq, int k, int ng)
+{
+    if (nq <= 0 || k < 1 || !(ng == 1 || ng == 2 || ng == 4)) return 0;
+    int sms = 0;
+    if (device_info(sms) != DSA_OK) sms = 148;
+    return attn_plan(nq, k, sms, ng).ws;
+}
+
+dsa_status_t dsa_sparse_attn_decode_groups(const void *q, const void *k_cache, const void *v_cache, int64_t n_pages,
+                                           const int32_t *block_table, int max_pages, const int32_t *q_pos, int batch,
+                                           int g0, int ng, const int32_t *sel_idx, const int32_t *sel_count, int k,
+                                           void *out, float *lse, void *ws, size_t ws_bytes, dsa_stream_t stream)
+{
+    dsa_status_t st = group_range_args(g0, ng);
+    if (st != DSA_OK) return st;
+    return attn_common(q, k_cache, v_cache, n_pages, block_table, max_pages, nullptr, batch, q_pos, batch, sel_idx,
+                       sel_count, k, out, lse, ws, ws_bytes, stream, 0, g0, ng);
 }
 
 dsa_status_t dsa_indexer_frontend(const void *hidden, int hid, int n_tok, const void *w, const void *gamma_q,

@@ -5,11 +5,14 @@
 // The scan streams the request's e4m3 summaries once (256 B per region and group: the
 // dominant HBM traffic of a decode step) and is built to run at HBM speed:
 //  * one producer warp issues TMA tile loads (2-D tensor map over the group-major pool,
-//    128-byte swizzle, no multicast) of 32 regions x 4 groups x 256 B = 32 KiB per stage
-//    into a ring of smem stages guarded by mbarriers;
-//  * four consumer warps, one per KV group, read their 32x256 tile with conflict-free
-//    ldmatrix and contract it on the tensor cores with mma.sync m16n8k32 e4m3, fp32
-//    accumulate.  A fp32 FFMA dot product would need 4 FMA per summary byte plus e4m3
+//    128-byte swizzle, no multicast) of four 32-region x 256 B slabs = 32 KiB per stage
+//    into a ring of smem stages guarded by mbarriers.  A query's slabs are its (32-region
+//    chunk, KV group) pairs in chunk-major order: with all 4 groups a stage is one chunk of
+//    every group; a call that holds fewer groups (a GPU of a KV-group-sharded decode, 1 or 2
+//    groups) packs 4 or 2 chunks per stage, so the consumers stay as busy;
+//  * four consumer warps, one per slab (warp w always meets local group w % groups), read
+//    their 32x256 tile with conflict-free ldmatrix and contract it on the tensor cores with
+//    mma.sync m16n8k32 e4m3, fp32 accumulate.  A fp32 FFMA dot product would need 4 FMA per summary byte plus e4m3
 //    conversions and run out of ALU before HBM; on the tensor pipe the summaries are fed
 //    as raw bytes;
 //  * the B operand (8 columns) holds the group's 4 heads, each split exactly into two
@@ -44,12 +47,13 @@ namespace idx {
 constexpr int kChunk = DSA_SCAN_CHUNK;             // regions per stage (multiple of 32)
 constexpr int kStages = DSA_SCAN_STAGES;
 constexpr int kCtasPerSm = DSA_SCAN_CTAS_PER_SM;
-constexpr int kHalfBytes = kChunk * 128;           // one 128-byte column half of a group tile
-constexpr int kGroupBytes = 2 * kHalfBytes;        // 8 KiB at 32 regions
-constexpr int kStageBytes = kG * kGroupBytes;      // 32 KiB at 32 regions
+constexpr int kSlabs = 4;                          // 32-region slabs per stage (= consumer warps)
+constexpr int kHalfBytes = kChunk * 128;           // one 128-byte column half of a slab
+constexpr int kGroupBytes = 2 * kHalfBytes;        // one slab: 8 KiB at 32 regions
+constexpr int kStageBytes = kSlabs * kGroupBytes;  // 32 KiB at 32 regions
 constexpr int kTiles = kChunk / 16;                // m16 tiles per group per stage
 constexpr int kThreads = 160;                      // 4 consumer warps + 1 producer warp
-constexpr int kScaleBytes = kG * kChunk * 4;       // fp32 scales of one stage (512 B)
+constexpr int kScaleBytes = kSlabs * kChunk * 4;   // fp32 scales of one stage (512 B)
 constexpr size_t kSmemBytes =
     (size_t)kStages * (kStageBytes + kScaleBytes) + 1024 /*align*/ + 64 /*barriers*/;
 
@@ -66,11 +70,25 @@ struct Params {
     int64_t n_slots;
     int64_t ld;
     int64_t total_units;
-    int units_per_query;
+    int units_per_query;       // stages per query: ceil(chunks * groups / 4)
     int nq;
     int n_req;
     uint32_t flags;
+    // KV groups of the call: g0 .. g0 + groups - 1 (groups 1, 2 or 4).  summaries / scales
+    // hold only these groups ([groups][n_slots][256]); scores and chunk_max are
+    // [nq][groups][..]; index_q and gate are the full [nq][16][..] (heads 4g .. 4g + 3).
+    int groups;
+    int gshift;                // log2(groups)
+    int g0;
 };
+
+// Slab j of stage unit `uu` of a query: its 32-region chunk and local group.
+__device__ __forceinline__ void slab_of(const Params &p, int uu, int j, int &chunk, int &gl)
+{
+    const int sidx = uu * kSlabs + j;
+    chunk = sidx >> p.gshift;
+    gl = sidx & (p.groups - 1);
+}
 
 // Checks one query; returns own (regions before the own region) or -1 if the query is
 // invalid.  base receives the request's first slot.
@@ -167,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1 + 32);   // expect_tx arrive + one arrive per producer lane (scales)
-            mbar_init(&empty[s], kG);
+            mbar_init(&empty[s], kSlabs);
         }
         fence_mbar_init();
     }
@@ -176,20 +194,23 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const int64_t u_begin = (int64_t)blockIdx.x * p.total_units / gridDim.x;
     const int64_t u_end = (int64_t)(blockIdx.x + 1) * p.total_units / gridDim.x;
 
-    if (warp == kG) {
+    if (warp == kSlabs) {
         // ---------------- producer warp: lane 0 issues the TMA loads of the summaries; every
         // lane copies 4 of the stage's 128 fp32 scales into smem asynchronously
         if (lane == 0) prefetch_tensormap(&tmap);
         const uint64_t pol = l2_evict_first_policy();     // the summaries are read once per query
         int it = 0;
-        constexpr int kScalesPerLane = kG * kChunk / 32;          // 4 at 32 regions per stage
+        constexpr int kScalesPerLane = kSlabs * kChunk / 32;      // 4 at 32 regions per stage
         const int sg = (lane * kScalesPerLane) / kChunk, sr = (lane * kScalesPerLane) % kChunk;
         for (int64_t u = u_begin; u < u_end; ++u) {
             const int qi = (int)(u / p.units_per_query);
-            const int64_t r0 = (u % p.units_per_query) * kChunk;
+            const int uu = (int)(u - (int64_t)qi * p.units_per_query);
             int64_t base;
             const int64_t own = query_own(p, qi, base);
-            if (own < 0 || r0 >= own) continue;
+            int c_first;
+            int gl_first;
+            slab_of(p, uu, 0, c_first, gl_first);
+            if (own < 0 || (int64_t)c_first * kChunk >= own) continue;
             const int s = it % kStages;
             const unsigned ph = (unsigned)(it / kStages) & 1u;
             if (!mbar_wait(&empty[s], ph ^ 1u)) break;
@@ -197,19 +218,26 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 mbar_arrive_expect_tx(&full[s], kStageBytes);
                 uint8_t *st = smem + s * kStageBytes;
 #pragma unroll
-                for (int g = 0; g < kG; ++g) {
-                    const int y = (int)(g * p.n_slots + base + r0);
-                    tma_load_2d_hint(st + g * kGroupBytes, &tmap, 0, y, &full[s], pol);
-                    tma_load_2d_hint(st + g * kGroupBytes + kHalfBytes, &tmap, 128, y, &full[s], pol);
+                for (int j = 0; j < kSlabs; ++j) {
+                    // slabs past the own region (the last stage of a query) are loaded and ignored
+                    int c;
+                    int gl;
+                    slab_of(p, uu, j, c, gl);
+                    const int y = (int)(gl * p.n_slots + base + (int64_t)c * kChunk);
+                    tma_load_2d_hint(st + j * kGroupBytes, &tmap, 0, y, &full[s], pol);
+                    tma_load_2d_hint(st + j * kGroupBytes + kHalfBytes, &tmap, 128, y, &full[s], pol);
                 }
             }
             // scales: asynchronous 4-byte copies that arrive on the stage's barrier when they
             // land, so the producer never waits for them
-            const float *srow = p.scales + sg * p.n_slots + base;
+            int c;
+            int gl;
+            slab_of(p, uu, sg, c, gl);
+            const float *srow = p.scales + gl * p.n_slots + base;
 #pragma unroll
             for (int e = 0; e < kScalesPerLane; ++e) {
-                const int64_t r = r0 + sr + e;
-                cp_async_4(sscale + (s * kG + sg) * kChunk + sr + e, srow + (r < own ? r : 0), r < own);
+                const int64_t r = (int64_t)c * kChunk + sr + e;
+                cp_async_4(sscale + (s * kSlabs + sg) * kChunk + sr + e, srow + (r < own ? r : 0), r < own);
             }
             cp_async_mbar_arrive(&full[s]);
             ++it;
@@ -217,8 +245,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         return;
     }
 
-    // ---------------- consumers: warp g contracts group g
-    const int g = warp;
+    // ---------------- consumers: warp j contracts slab j (local group j % groups)
+    const int g = warp % p.groups;
     const int n = lane >> 2, t = lane & 3;
     uint32_t bfrag[8][2];
     float sq_t = 0.0f, z_t = 0.0f;
@@ -226,16 +254,23 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     int it = 0;
     for (int64_t u = u_begin; u < u_end; ++u) {
         const int qi = (int)(u / p.units_per_query);
-        const int64_t r0 = (u % p.units_per_query) * kChunk;
+        const int uu = (int)(u - (int64_t)qi * p.units_per_query);
         int64_t base;
         const int64_t own = query_own(p, qi, base);
         if (own < 0) {
-            if (r0 == 0 && lane == 0) set_error(kErrIndexerQuery);
+            if (uu == 0 && warp == 0 && lane == 0) set_error(kErrIndexerQuery);
             continue;
         }
-        if (r0 >= own) continue;
+        int c_first;
+        int gl_first;
+        slab_of(p, uu, 0, c_first, gl_first);
+        if ((int64_t)c_first * kChunk >= own) continue;
+        int chunk;
+        int gl;
+        slab_of(p, uu, warp, chunk, gl);
+        const int64_t r0 = (int64_t)chunk * kChunk;
         if (qi != cached_q) {
-            load_query_fragments(p, qi, g, lane, bfrag, sq_t, z_t);
+            load_query_fragments(p, qi, p.g0 + g, lane, bfrag, sq_t, z_t);
             cached_q = qi;
         }
         const int s = it % kStages;
@@ -246,8 +281,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 #pragma unroll
         for (int m = 0; m < kTiles; ++m)
 #pragma unroll
-            for (int h = 0; h < 2; ++h) sc[m][h] = sscale[(s * kG + g) * kChunk + 16 * m + 8 * h + n];
-        const uint32_t tile = smem_u32(smem + s * kStageBytes + g * kGroupBytes);
+            for (int h = 0; h < 2; ++h) sc[m][h] = sscale[(s * kSlabs + warp) * kChunk + 16 * m + 8 * h + n];
+        const uint32_t tile = smem_u32(smem + s * kStageBytes + warp * kGroupBytes);
         float acc[kTiles][4];
 #pragma unroll
         for (int m = 0; m < kTiles; ++m) {
@@ -268,8 +303,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
         ++it;
+        if (r0 >= own) continue;                              // a slab past the own region
 
-        float *out = p.scores + ((int64_t)qi * kG + g) * p.ld;
+        float *out = p.scores + ((int64_t)qi * p.groups + g) * p.ld;
         float cmax = -1.0f;                                   // below every score (scores are >= +0)
 #pragma unroll
         for (int m = 0; m < kTiles; ++m) {
@@ -292,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             static_assert(kChunk == 32, "chunk maxima cover 32 regions");
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
-            if (lane == 0) p.chunk_max[((int64_t)qi * kG + g) * p.cm_stride + r0 / kChunk] = cmax;
+            if (lane == 0) p.chunk_max[((int64_t)qi * p.groups + g) * p.cm_stride + r0 / kChunk] = cmax;
         }
     }
 }

@@ -31,11 +31,12 @@ struct Ws {
     uint32_t *ctr;      // [rows][4]: sure count, candidate count, finished CTAs
     int32_t *sure;      // [rows][k]
     uint2 *cand;        // [rows][ld]: (key, region)
+    int gshift;         // rows per query = 2^gshift (the KV groups of the call)
 };
 
-__device__ __forceinline__ int64_t row_own(const int32_t *q_pos, int row)
+__device__ __forceinline__ int64_t row_own(const int32_t *q_pos, int row, int gshift)
 {
-    const int p = q_pos[row >> 2];
+    const int p = q_pos[row >> gshift];
     return p < 0 ? -1 : p / kRegion;
 }
 
@@ -104,7 +105,7 @@ __global__ void __launch_bounds__(kThreads) hist_kernel(const float *__restrict_
     pdl_wait();      // the previous kernel's results are visible from here on
     __shared__ uint32_t h[kBins];
     const int row = blockIdx.y;
-    const int64_t own = row_own(q_pos, row);
+    const int64_t own = row_own(q_pos, row, ws.gshift);
     if (own < 0 || own > ld) return;
     const int64_t need = min((int64_t)(k - 1), own);
     if (need == own || need == 0) return;             // all eligible selected, or only the own region
@@ -251,7 +252,7 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const float *__r
     constexpr int NT = kSelectThreads;
     const int row = blockIdx.y;
     const int tid = threadIdx.x;
-    const int64_t own = row_own(q_pos, row);
+    const int64_t own = row_own(q_pos, row, ws.gshift);
     if (own < 0 || own > ld) {
         if (blockIdx.x == 0) {
             if (tid == 0) {

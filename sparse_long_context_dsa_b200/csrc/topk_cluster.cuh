@@ -408,7 +408,7 @@ template <bool kSingle, bool kMaxima = false>
 __global__ void __launch_bounds__(kThreads, 1)
     topk_cluster_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ q_pos, int k,
                         int32_t *__restrict__ sel_idx, int32_t *__restrict__ sel_count,
-                        const float *__restrict__ chunk_max, int64_t cm_stride)
+                        const float *__restrict__ chunk_max, int64_t cm_stride, int gshift)
 {
     pdl_trigger();   // the next kernel may launch; it waits for this one itself
     pdl_wait();      // the previous kernel's results are visible from here on
@@ -441,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ---- loads: this thread's group is the CTA's entries tid, tid+512, ... (coalesced)
-    const int p = q_pos[row >> 2];
+    const int p = q_pos[row >> gshift];   // rows per query = 2^gshift (the call's KV groups)
     const int64_t part = ((ld + CL - 1) / CL + 31) / 32 * 32;              // whole 32-region chunks
     const int64_t lo = min(ld, (int64_t)rank * part), hi_ld = min(ld, lo + part);
     const float *src = scores + (int64_t)row * ld + lo;

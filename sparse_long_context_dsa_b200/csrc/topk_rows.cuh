@@ -47,7 +47,7 @@ static_assert(5 * kSmemBytes <= 227 * 1024, "five CTAs per SM");
 
 __global__ void __launch_bounds__(kThreads, 5)
     topk_rows_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ q_pos, int k,
-                     int32_t *__restrict__ sel_idx, int32_t *__restrict__ sel_count)
+                     int32_t *__restrict__ sel_idx, int32_t *__restrict__ sel_count, int gshift)
 {
     pdl_trigger();   // the next kernel may launch; it waits for this one itself
     pdl_wait();      // the previous kernel's results are visible from here on
@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(kThreads, 5)
 
     const int tid = threadIdx.x, lane = tid & 31;
     const int row = blockIdx.x;
-    const int p = q_pos[row >> 2];
+    const int p = q_pos[row >> gshift];   // rows per query = 2^gshift (the call's KV groups)
     const bool valid = p >= 0 && (int64_t)(p / kRegion) <= ld;
     const int64_t own = valid ? p / kRegion : 0;
     const int64_t need = valid ? min((int64_t)(k - 1), own) : 0;

@@ -54,6 +54,16 @@ _SIG = {
                                          _I64P, ctypes.c_int, _F32P, ctypes.c_int64, ctypes.c_uint32, ctypes.c_int,
                                          _I32P, _I32P, _VP, ctypes.c_size_t, _VP]),
     "dsa_copy": (ctypes.c_int, [_VP, _VP, ctypes.c_size_t, _VP]),
+    "dsa_compress_regions_groups": (ctypes.c_int, [_VP, ctypes.c_int64, ctypes.c_int64, _I64P, _I64P, ctypes.c_int,
+                                                   ctypes.c_int, ctypes.c_int, _U8P, _F32P, ctypes.c_int64, _VP]),
+    "dsa_decode_select_groups": (ctypes.c_int, [_VP, _F32P, _I32P, _I32P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                _U8P, _F32P, ctypes.c_int64, _I64P, ctypes.c_int, _F32P,
+                                                ctypes.c_int64, ctypes.c_uint32, ctypes.c_int, _I32P, _I32P, _VP,
+                                                ctypes.c_size_t, _VP]),
+    "dsa_attn_groups_workspace_size": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "dsa_sparse_attn_decode_groups": (ctypes.c_int, [_VP, _VP, _VP, ctypes.c_int64, _I32P, ctypes.c_int, _I32P,
+                                                     ctypes.c_int, ctypes.c_int, ctypes.c_int, _I32P, _I32P,
+                                                     ctypes.c_int, _VP, _F32P, _VP, ctypes.c_size_t, _VP]),
     "dsa_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_int64, _VP]),
     "dsa_attn_workspace_size": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int]),
     "dsa_sparse_attn_decode": (ctypes.c_int, [_VP, _VP, _VP, ctypes.c_int64, _I32P, ctypes.c_int, _I32P,
@@ -234,6 +244,88 @@ def topk_regions_noalloc(scores, q_pos, k, sel_idx, sel_count):
     _need(sel_count, torch.int32, (nq, G), "sel_count")
     _check(lib().dsa_topk_regions_noalloc(_p(scores), ld, _p(q_pos), nq, k, _p(sel_idx), _p(sel_count), _stream()))
     return sel_idx, sel_count
+
+
+def _group_range(g0, ng):
+    if ng not in (1, 2, 4) or g0 < 0 or g0 + ng > G:
+        raise ValueError("groups g0 .. g0 + ng - 1 must be 1, 2 or 4 consecutive groups of 0 .. 3")
+
+
+def compress_regions_groups(index_k, src_row, dst_slot, summaries, scales, g0):
+    """dsa_compress_regions_groups: groups g0 .. g0 + ng - 1 of index_k bf16 [rows][4][256]
+    into a shard's pool summaries uint8 [ng][n_slots][256], scales fp32 [ng][n_slots]."""
+    _need(index_k, torch.bfloat16, name="index_k")
+    _need(src_row, torch.int64, name="src_row")
+    _need(dst_slot, torch.int64, (src_row.numel(),), "dst_slot")
+    _need(summaries, torch.uint8, name="summaries")
+    ng, n_slots = summaries.shape[0], summaries.shape[1]
+    _group_range(g0, ng)
+    _need(scales, torch.float32, (ng, n_slots), "scales")
+    row_stride = index_k[0].numel() if index_k.shape[0] else G * DI
+    _check(lib().dsa_compress_regions_groups(_p(index_k), row_stride, index_k.shape[0], _p(src_row), _p(dst_slot),
+                                             src_row.numel(), g0, ng, _p(summaries), _p(scales), n_slots, _stream()))
+
+
+def decode_select_groups(index_q, gate, q_req, q_pos, summaries, scales, sum_base, scores, k, g0, flags=0,
+                         sel_idx=None, sel_count=None):
+    """dsa_decode_select_groups: scores [nq][ng][ld] and selection [nq][ng][k] of the shard
+    holding groups g0 .. g0 + ng - 1 (ng = summaries.shape[0])."""
+    nq = index_q.shape[0]
+    _need(index_q, torch.bfloat16, (nq, HI, DI), "index_q")
+    _need(gate, torch.float32, (nq, HI), "gate")
+    _need(q_req, torch.int32, (nq,), "q_req")
+    _need(q_pos, torch.int32, (nq,), "q_pos")
+    _need(summaries, torch.uint8, name="summaries")
+    ng, n_slots = summaries.shape[0], summaries.shape[1]
+    _group_range(g0, ng)
+    _need(scales, torch.float32, (ng, n_slots), "scales")
+    _need(sum_base, torch.int64, name="sum_base")
+    _need(scores, torch.float32, name="scores")
+    if scores.dim() != 3 or scores.shape[0] != nq or scores.shape[1] != ng:
+        raise ValueError("scores must be [nq][ng][ld]")
+    ld = scores.shape[2]
+    if sel_idx is None:
+        sel_idx = torch.empty((nq, ng, k), dtype=torch.int32, device=scores.device)
+    if sel_count is None:
+        sel_count = torch.empty((nq, ng), dtype=torch.int32, device=scores.device)
+    _need(sel_idx, torch.int32, (nq, ng, k), "sel_idx")
+    _need(sel_count, torch.int32, (nq, ng), "sel_count")
+    nbytes = lib().dsa_decode_select_workspace_size(nq, ld, k)
+    ws = _workspace(nbytes, scores.device)
+    _check(lib().dsa_decode_select_groups(_p(index_q), _p(gate), _p(q_req), _p(q_pos), nq, g0, ng, _p(summaries),
+                                          _p(scales), n_slots, _p(sum_base), sum_base.numel(), _p(scores), ld, flags,
+                                          k, _p(sel_idx), _p(sel_count), _p(ws), nbytes, _stream()))
+    return sel_idx, sel_count
+
+
+def sparse_attn_decode_groups(q, k_cache, v_cache, block_table, q_pos, sel_idx, sel_count, g0, out=None, lse=None):
+    """dsa_sparse_attn_decode_groups: the shard's caches [n_pages][ng][64][192] and selection
+    [B][ng][k]; returns out bf16 [B][16 ng][192] (the heads of groups g0 .. g0 + ng - 1)."""
+    nq = q.shape[0]
+    _need(q, torch.bfloat16, (nq, HQ, D), "q")
+    _need(k_cache, torch.bfloat16, name="k_cache")
+    ng = k_cache.shape[1]
+    _group_range(g0, ng)
+    if k_cache.dim() != 4 or tuple(k_cache.shape[2:]) != (PAGE, D):
+        raise ValueError("k_cache must be [n_pages][ng][64][192]")
+    _need(v_cache, torch.bfloat16, tuple(k_cache.shape), "v_cache")
+    _need(block_table, torch.int32, name="block_table")
+    _need(q_pos, torch.int32, (nq,), "q_pos")
+    k = sel_idx.shape[-1]
+    _need(sel_idx, torch.int32, (nq, ng, k), "sel_idx")
+    _need(sel_count, torch.int32, (nq, ng), "sel_count")
+    hq = 16 * ng
+    if out is None:
+        out = torch.empty((nq, hq, D), dtype=torch.bfloat16, device=q.device)
+    _need(out, torch.bfloat16, (nq, hq, D), "out")
+    if lse is not None:
+        _need(lse, torch.float32, (nq, hq), "lse")
+    nbytes = lib().dsa_attn_groups_workspace_size(nq, k, ng)
+    ws = _workspace(nbytes, q.device)
+    _check(lib().dsa_sparse_attn_decode_groups(_p(q), _p(k_cache), _p(v_cache), k_cache.shape[0], _p(block_table),
+                                               block_table.shape[1], _p(q_pos), nq, g0, ng, _p(sel_idx),
+                                               _p(sel_count), k, _p(out), _p(lse), _p(ws), nbytes, _stream()))
+    return out
 
 
 def selftest_wait_timeout(limit_cycles: int):

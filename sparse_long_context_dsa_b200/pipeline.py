@@ -40,12 +40,18 @@ class DecodeStep:
     summaries/scales: the group-major pool; sum_base int64 [B]; block_table int32 [B][P];
     k_cache/v_cache bf16 [pages][4][64][192]; ld: score row length (>= max own region).
     tail_tokens = 8 gives the step an input tail buffer (bf16 [B*8][4][256]) whose
-    regions are compressed when `set_compress` lists them."""
+    regions are compressed when `set_compress` lists them.
+    g0: first KV group of a group shard ([P2] §索引器打分: one GPU of a KV-group-sharded decode):
+    with summaries [ng][slots][256] and caches [pages][ng][64][192] of groups g0 .. g0+ng-1
+    the step runs the `_groups` calls and `out` holds those groups' 16*ng heads."""
 
     def __init__(self, summaries, scales, sum_base, block_table, k_cache, v_cache, ld, k=512,
-                 tail_tokens=0, flags=0):
+                 tail_tokens=0, flags=0, g0=0):
         dev = summaries.device
         self.B = B = int(block_table.shape[0])
+        self.g0, self.ng = int(g0), int(summaries.shape[0])
+        self.sharded = self.ng != G
+        ng = self.ng
         self.k = int(k)
         self.ld = int(ld)
         self.flags = flags
@@ -68,11 +74,11 @@ class DecodeStep:
         self.tail, off = _carve(self.arena, off, (B * max(tail_tokens, 1), G, DI), torch.bfloat16)
         self.tail_tokens = tail_tokens
         self.q_req = torch.arange(B, dtype=torch.int32, device=dev)
-        self.scores = torch.zeros((B, G, self.ld), dtype=torch.float32, device=dev)
-        self.sel_idx = torch.empty((B, G, self.k), dtype=torch.int32, device=dev)
-        self.sel_count = torch.empty((B, G), dtype=torch.int32, device=dev)
-        self.out = torch.empty((B, HQ, D), dtype=torch.bfloat16, device=dev)
-        self.lse = torch.empty((B, HQ), dtype=torch.float32, device=dev)
+        self.scores = torch.zeros((B, ng, self.ld), dtype=torch.float32, device=dev)
+        self.sel_idx = torch.empty((B, ng, self.k), dtype=torch.int32, device=dev)
+        self.sel_count = torch.empty((B, ng), dtype=torch.int32, device=dev)
+        self.out = torch.empty((B, 16 * ng, D), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((B, 16 * ng), dtype=torch.float32, device=dev)
         self.n_compress = 0
         self.src_row = torch.zeros(max(1, B), dtype=torch.int64, device=dev)
         self.dst_slot = torch.zeros(max(1, B), dtype=torch.int64, device=dev)
@@ -81,7 +87,8 @@ class DecodeStep:
         self.ws_idx_n = L.dsa_indexer_workspace_size(B, self.ld)
         self.ws_topk_n = L.dsa_topk_workspace_size(B, self.ld, self.k)
         self.ws_sel_n = L.dsa_decode_select_workspace_size(B, self.ld, self.k)
-        self.ws_attn_n = L.dsa_attn_workspace_size(B, self.k)
+        self.ws_attn_n = (L.dsa_attn_groups_workspace_size(B, self.k, ng) if self.sharded
+                          else L.dsa_attn_workspace_size(B, self.k))
         self.ws_idx = torch.empty(max(1, self.ws_idx_n), dtype=torch.uint8, device=dev)
         self.ws_topk = torch.empty(max(1, self.ws_topk_n), dtype=torch.uint8, device=dev)
         self.ws_attn = torch.empty(max(1, self.ws_attn_n), dtype=torch.uint8, device=dev)
@@ -117,7 +124,7 @@ class DecodeStep:
             out = self.out
         elif tuple(out.shape) != tuple(self.out.shape) or out.dtype != self.out.dtype or not (
                 out.is_cuda or out.is_pinned()):
-            raise ValueError("out must be bf16 [B][64][192], on the device or in pinned host memory")
+            raise ValueError("out must be bf16 [B][16*ng][192], on the device or in pinned host memory")
         L = dsa.lib()
         main = torch.cuda.current_stream()
         p = dsa._p
@@ -125,15 +132,29 @@ class DecodeStep:
             self.side.wait_stream(main)
             with torch.cuda.stream(self.side):
                 t = self.tail
-                dsa._check(L.dsa_compress_regions(p(t), t[0].numel(), t.shape[0], p(self.src_row), p(self.dst_slot),
-                                                  self.n_compress, p(self.summaries), p(self.scales),
-                                                  self.summaries.shape[1], dsa._stream()))
+                if self.sharded:
+                    dsa._check(L.dsa_compress_regions_groups(p(t), t[0].numel(), t.shape[0], p(self.src_row),
+                                                             p(self.dst_slot), self.n_compress, self.g0, self.ng,
+                                                             p(self.summaries), p(self.scales),
+                                                             self.summaries.shape[1], dsa._stream()))
+                else:
+                    dsa._check(L.dsa_compress_regions(p(t), t[0].numel(), t.shape[0], p(self.src_row),
+                                                      p(self.dst_slot), self.n_compress, p(self.summaries),
+                                                      p(self.scales), self.summaries.shape[1], dsa._stream()))
         st = dsa._stream()
         # scores and selection in one call (the scan's chunk maxima bound the selection)
-        dsa._check(L.dsa_decode_select(p(self.index_q), p(self.gate), p(self.q_req), p(self.q_pos), self.B,
-                                       p(self.summaries), p(self.scales), self.summaries.shape[1], p(self.sum_base),
-                                       self.sum_base.numel(), p(self.scores), self.ld, self.flags, self.k,
-                                       p(self.sel_idx), p(self.sel_count), p(self.ws_sel), self.ws_sel_n, st))
+        if self.sharded:
+            dsa._check(L.dsa_decode_select_groups(p(self.index_q), p(self.gate), p(self.q_req), p(self.q_pos), self.B,
+                                                  self.g0, self.ng, p(self.summaries), p(self.scales),
+                                                  self.summaries.shape[1], p(self.sum_base), self.sum_base.numel(),
+                                                  p(self.scores), self.ld, self.flags, self.k, p(self.sel_idx),
+                                                  p(self.sel_count), p(self.ws_sel), self.ws_sel_n, st))
+        else:
+            dsa._check(L.dsa_decode_select(p(self.index_q), p(self.gate), p(self.q_req), p(self.q_pos), self.B,
+                                           p(self.summaries), p(self.scales), self.summaries.shape[1],
+                                           p(self.sum_base), self.sum_base.numel(), p(self.scores), self.ld,
+                                           self.flags, self.k, p(self.sel_idx), p(self.sel_count), p(self.ws_sel),
+                                           self.ws_sel_n, st))
         self.run_attention(out)
         if self.n_compress:
             main.wait_stream(self.side)
@@ -143,10 +164,17 @@ class DecodeStep:
         """The step's attention alone, over the selection in sel_idx / sel_count."""
         L, p, st = dsa.lib(), dsa._p, dsa._stream()
         out = self.out if out is None else out
-        dsa._check(L.dsa_sparse_attn_decode(p(self.q), p(self.k_cache), p(self.v_cache), self.k_cache.shape[0],
-                                            p(self.block_table), self.block_table.shape[1], p(self.q_pos), self.B,
-                                            p(self.sel_idx), p(self.sel_count), self.k, p(out), p(self.lse),
-                                            p(self.ws_attn), self.ws_attn_n, st))
+        if self.sharded:
+            dsa._check(L.dsa_sparse_attn_decode_groups(p(self.q), p(self.k_cache), p(self.v_cache),
+                                                       self.k_cache.shape[0], p(self.block_table),
+                                                       self.block_table.shape[1], p(self.q_pos), self.B, self.g0,
+                                                       self.ng, p(self.sel_idx), p(self.sel_count), self.k, p(out),
+                                                       p(self.lse), p(self.ws_attn), self.ws_attn_n, st))
+        else:
+            dsa._check(L.dsa_sparse_attn_decode(p(self.q), p(self.k_cache), p(self.v_cache), self.k_cache.shape[0],
+                                                p(self.block_table), self.block_table.shape[1], p(self.q_pos), self.B,
+                                                p(self.sel_idx), p(self.sel_count), self.k, p(out), p(self.lse),
+                                                p(self.ws_attn), self.ws_attn_n, st))
         return out
 
 

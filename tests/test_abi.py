@@ -64,3 +64,21 @@ def test_bad_arguments_are_rejected_on_the_host(lib, call):
 def test_zero_sized_calls_are_noops(lib):
     assert lib.dsa_compress_regions(None, 1024, 8, None, None, 0, None, None, 1, None) == dsa.OK
     assert lib.dsa_topk_regions(None, 16, None, 0, 8, None, None, None, 0, None) == dsa.OK
+
+
+def test_group_ranges_are_checked_on_the_host(lib):
+    # a KV group shard is 1, 2 or 4 consecutive groups of 0 .. 3
+    for g0, ng in ((0, 3), (3, 2), (-1, 1), (2, 4), (0, 0)):
+        assert lib.dsa_decode_select_groups(None, None, None, None, 1, g0, ng, None, None, 1, None, 1, None, 8, 0, 8,
+                                            None, None, None, 0, None) == dsa.ERR_INVALID_ARG
+        assert lib.dsa_sparse_attn_decode_groups(None, None, None, 1, None, 1, None, 1, g0, ng, None, None, 8, None,
+                                                 None, None, 0, None) == dsa.ERR_INVALID_ARG
+        assert lib.dsa_compress_regions_groups(None, 1024, 8, None, None, 1, g0, ng, None, None, 1, None) == \
+            dsa.ERR_INVALID_ARG
+        assert "g0" in lib.dsa_last_error().decode() or "ng" in lib.dsa_last_error().decode()
+    assert lib.dsa_attn_groups_workspace_size(4, 512, 3) == 0
+
+
+def test_selftest_bound_is_checked_on_the_host(lib):
+    assert lib.dsa_selftest_wait_timeout(0, None) == dsa.ERR_INVALID_ARG
+    assert lib.dsa_selftest_wait_timeout((1 << 31) + 1, None) == dsa.ERR_INVALID_ARG

@@ -46,12 +46,6 @@ def test_a_wait_that_nothing_completes_gives_up_and_reports_it():
     assert torch.all(C > 0)
 
 
-def test_selftest_bound_is_checked_on_the_host():
-    L = dsa.lib()
-    assert L.dsa_selftest_wait_timeout(0, None) == dsa.ERR_INVALID_ARG
-    assert L.dsa_selftest_wait_timeout((1 << 31) + 1, None) == dsa.ERR_INVALID_ARG
-
-
 def _attr_pageable():
     from cuda.bindings import runtime as rt
     err, v = rt.cudaDeviceGetAttribute(rt.cudaDeviceAttr.cudaDevAttrPageableMemoryAccess, torch.cuda.current_device())

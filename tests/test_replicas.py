@@ -1,4 +1,4 @@
-"""Multi-rank host logic of the replica path (gloo, 2 processes on CPU)."""
+"""Multi-rank host logic of the replica and KV-group-shard paths (gloo, 2 processes on CPU)."""
 import os
 import socket
 
@@ -58,3 +58,50 @@ def test_two_ranks_agree_on_the_slowest_time():
     assert out[0][0] == out[1][0] == 15.0
     assert out[0][1] + out[1][1] == 33
     assert out[0][2] == out[1][2] == 2 * 17 / 0.015
+
+
+def test_group_plan_covers_every_group_of_every_replica():
+    for world, tp in ((1, 1), (2, 2), (4, 4), (4, 2), (8, 4), (8, 2)):
+        seen = {}
+        for r in range(world):
+            rep, g0, ng = replicas.group_plan(r, world, tp)
+            seen.setdefault(rep, []).extend(range(g0, g0 + ng))
+        assert len(seen) == world // tp
+        assert all(v == [0, 1, 2, 3] for v in seen.values())
+    for bad in ((0, 2, 3), (0, 3, 2), (2, 2, 2)):
+        with pytest.raises(ValueError):
+            replicas.group_plan(*bad)
+
+
+def _heads(nq, g0, ng):
+    """A deterministic stand-in output whose every element names its query, head and dim."""
+    q = torch.arange(nq, dtype=torch.float32)[:, None, None]
+    h = torch.arange(16 * g0, 16 * (g0 + ng), dtype=torch.float32)[None, :, None]
+    d = torch.arange(192, dtype=torch.float32)[None, None, :]
+    return q * 1e5 + h * 200 + d
+
+
+def _shard_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        rep, g0, ng = replicas.group_plan(rank, world, tp=world)
+        grp = replicas.tp_group(world, world)
+        full = replicas.gather_heads(_heads(3, g0, ng), grp, tp=world)
+        out[rank] = (g0, ng, bool(torch.equal(full, _heads(3, 0, 4))))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_group_shards_gather_the_64_heads():
+    world = 2
+    port = _free_port()
+    out = mp.Manager().dict()
+    mp.spawn(_shard_worker, args=(world, port, out), nprocs=world, join=True)
+    assert (out[0][0], out[0][1]) == (0, 2) and (out[1][0], out[1][1]) == (2, 2)
+    assert out[0][2] and out[1][2]
+
+
+def test_assemble_heads_rejects_partial_cover():
+    with pytest.raises(ValueError):
+        replicas.assemble_heads([_heads(2, 0, 2)])
