@@ -7,7 +7,9 @@ over those scores ([P2] Step-5-Preview 如何实现1M长上下文 §索引器打
 to the lower region).  Cases: decode batches whose rows take the chunk-maxima path (few long
 rows: 16,384 .. 131,071 regions) and rows that do not (short rows, k = 1024, many rows), all-
 zero queries (every score +0: the maxima tie in bulk and the selection falls back), identical
-summaries (every score of a row equal), and rows whose own region is below k.
+summaries (every score of a row equal), rows whose own region is below k, and rows whose best
+regions crowd into one stretch of the row (many chunk maxima tie near the bound, and whole
+chunks are candidates).
 """
 import numpy as np
 import pytest
@@ -102,3 +104,20 @@ def test_decode_step_uses_it():
     own = int(d["q_pos"][0]) // 8
     assert torch.equal(st.scores[:, :, :own], s2[:, :, :own])
     assert torch.equal(st.sel_idx, i2) and torch.equal(st.sel_count, c2)
+
+
+@pytest.mark.parametrize("lo,n", [(70000, 700), (0, 3000), (131071 - 600, 600)])
+def test_crowded_best_regions_fall_back_exactly(lo, n):
+    # scales of regions lo .. lo+n-1 times 64: their scores are 64x the others' (ReLU is
+    # positively homogeneous), so the selection crowds into a few hundred whole chunks
+    lengths = [1 << 20]
+    d, S, C = setup(lengths, seed=77 + lo)
+    C[:, lo:lo + n] *= 64.0
+    k = 512
+    ld = max(lengths) // 8
+    s1, i1, c1, s2, i2, c2 = both(d, S, C, k, ld)
+    assert torch.equal(s1, s2)
+    assert torch.equal(c1, c2) and torch.equal(i1, i2)
+    check_against_oracle(s1, i1, c1, d["q_pos"], k)
+    sel = i1.cpu().numpy()[0]
+    assert np.mean((sel[:, : k - 1] >= lo) & (sel[:, : k - 1] < lo + n)) > 0.9
