@@ -9,11 +9,12 @@
 // it) and one bit per tile that needs no mask (every query selected all its regions, all at or
 // before the earliest position).  The union streams in tiles of 8 regions (64 tokens),
 // flash-attention style:
-//  * two TMA warps load each region's K (one warp) and V (the other) as three 8 x 64 boxes
-//    (128-byte swizzle, laid out [block][8 rows][128 B] so that 8-token atoms sit 3 KiB
-//    apart) into separate 4-stage rings: a K stage frees as soon as S has read it, a V stage
-//    once P V has; a region that is invalid or past the union is loaded from rows past the
-//    cache, which fill zeros;
+//  * two TMA warps load each region's K (one warp) and V (the other) as ONE 3 KiB box of a
+//    3-D view of the cache whose dimensions are the 64 dims of a block, the token rows and the
+//    3 blocks (block stride 128 B below the row stride 384 B), so that it lands as [block]
+//    [8 rows][128 B] with the 128-byte swizzle (8-token atoms 3 KiB apart), into separate
+//    4-stage rings: a K stage frees as soon as S has read it, a V stage once P V has; a region
+//    that is invalid or past the union is loaded from rows past the cache, which fill zeros;
 //  * one thread issues S = Q K^T (M = 128, N = 64, K = 192: 12 tcgen05.mma.kind::f16, Q
 //    read from TMEM where the softmax warps put it at the start) into one of two 64-column
 //    TMEM buffers, and O += P V (M = 128, N = 192, K = 64: 4 MMAs with
@@ -139,9 +140,9 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16])
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// tmap_k / tmap_v: 2-D views [n_pages * 4 * 64 rows][192] of the caches, box 64 x 8 rows
-// (one 64-wide column block of a region), 128-byte swizzle.  kv_rows: the views' row count
-// (a load there reads zeros).
+// tmap_k / tmap_v: 3-D views (64 dims, n_pages * 4 * 64 rows, 3 blocks) of the caches, box
+// {64, 8, 3} (one region), 128-byte swizzle.  kv_rows: the views' row count (a load there
+// reads zeros).
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                           const Params p, int kv_rows)
@@ -358,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0 || warp == 2) {
         // ---------------- TMA producers: warp 0 loads K, warp 2 loads V; lane j < 8 issues
-        // region j of each tile (three 8 x 64 boxes)
+        // region j of each tile (one 3 KiB box)
         const bool is_k = warp == 0;
         const CUtensorMap *map = is_k ? &tmap_k : &tmap_v;
         uint8_t *ring = is_k ? ks : vs;
@@ -378,8 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int u = i * kTileRegions + lane;
                 const int y = u < U ? urow[u] : kv_rows;        // past the union: zeros
                 uint8_t *dst = ring + s * kTileBytes + lane * kRegionBox;
-#pragma unroll
-                for (int blk = 0; blk < 3; ++blk) tma_load_2d(dst + blk * 1024, map, blk * 64, y, &full[s]);
+                tma_load_3d(dst, map, 0, y, 0, &full[s]);
             }
             issued = i + 1;
         }

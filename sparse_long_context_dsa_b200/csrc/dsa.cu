@@ -203,14 +203,16 @@ dsa_status_t kv_map(CUtensorMap *m, const void *cache, int64_t n_pages, int ng =
     return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, cache, dims, strides, box, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 }
 
-// 2-D view [n_pages * 4 * 64 rows][192] of a K/V cache: one 64-wide column block of 8 rows
-// per box (the tcgen05 shared-selection attention's operand tiles).
-dsa_status_t kv_map_rows(CUtensorMap *m, const void *cache, int64_t n_pages)
+// 3-D view (64 dims, n_pages * 4 * 64 rows, 3 blocks) of a K/V cache with the row stride 384 B
+// and the block stride 128 B (a stride order the tensor map accepts): one box {64, 8, 3} is a
+// whole region, landing as [3 blocks][8 rows][128 B] with the 128-byte swizzle, the tcgen05
+// shared-selection attention's operand tiles.
+dsa_status_t kv_map_blocks(CUtensorMap *m, const void *cache, int64_t n_pages)
 {
-    const cuuint64_t dims[2] = {(cuuint64_t)dsa::kD, (cuuint64_t)n_pages * dsa::kG * dsa::kPage};
-    const cuuint64_t strides[1] = {(cuuint64_t)dsa::kD * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)dsa::kRegion};
-    return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, cache, dims, strides, box, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+    const cuuint64_t dims[3] = {64, (cuuint64_t)n_pages * dsa::kG * dsa::kPage, 3};
+    const cuuint64_t strides[2] = {(cuuint64_t)dsa::kD * 2, 128};
+    const cuuint32_t box[3] = {64, (cuuint32_t)dsa::kRegion, 3};
+    return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, cache, dims, strides, box, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 }
 
 struct TopkLayout {
@@ -389,8 +391,8 @@ dsa_status_t attn_common(const void *q, const void *k_cache, const void *v_cache
         });
         DSA_CUDA(sh_err, "cudaFuncSetAttribute(sparse_attn_tc_kernel)");
         CUtensorMap rk, rv;
-        if ((st = kv_map_rows(&rk, k_cache, n_pages)) != DSA_OK) return st;
-        if ((st = kv_map_rows(&rv, v_cache, n_pages)) != DSA_OK) return st;
+        if ((st = kv_map_blocks(&rk, k_cache, n_pages)) != DSA_OK) return st;
+        if ((st = kv_map_blocks(&rv, v_cache, n_pages)) != DSA_OK) return st;
         const unsigned blocks = (unsigned)((nq + dsa::attntc::kQueries - 1) / dsa::attntc::kQueries) * dsa::kG;
         if ((st = launch_k("sparse_attn_tc_kernel", dsa::attntc::sparse_attn_tc_kernel, dim3(blocks),
                            dim3(dsa::attntc::kThreads), dsa::attntc::kSmemBytes, stream, 0, rk, rv, p,

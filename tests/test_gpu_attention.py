@@ -174,3 +174,35 @@ def test_prefill_shared_block_running_max_grows():
             idx[8 * b: 8 * b + 8, g, :200] = sel
             cnt[8 * b: 8 * b + 8, g] = 200
     run(d, idx, cnt, q_req=d["q_req"], prefill=True)
+
+
+@pytest.mark.parametrize("grow", [False, True])
+def test_prefill_rows_on_tcgen05(grow):
+    # 96 queries x 4 groups = 384 rows (more than two per SM: the tcgen05 per-row kernel, each
+    # persistent CTA streaming two or three rows back to back), selections of 512 regions (32
+    # tiles of 128 tokens) beside ragged ones (1, 17, 129 regions) and empty rows; with grow, K
+    # of region r is scaled by 1 + r/64 so every row's running max
+    # passes the slack many times (O^T rescaled in TMEM)
+    ctx, n_new = 16384, 96
+    dev = "cuda"
+    d = W.prefill_chunk(ctx, n_new, seed=51 + grow, device=dev, permute=True)
+    if grow:
+        kc = d["k_cache"].float()
+        bt = d["block_table"][0].long()
+        rs = torch.zeros(kc.shape[0], device=dev)
+        rs[bt] = torch.arange(bt.numel(), device=dev, dtype=torch.float32)   # page -> its first region / 8
+        scale = 1.0 + (rs[:, None, None, None] * 8 + torch.arange(64, device=dev)[None, None, :, None] // 8) / 64.0
+        d["k_cache"] = (kc * scale).to(torch.bfloat16)
+    qp = d["q_pos"].cpu().numpy()
+    idx, cnt = random_selection(qp, 512, seed=7 + grow)
+    for i, n in ((3, 1), (10, 17), (20, 129), (33, 0), (47, 0)):
+        for g in range(G):
+            if n:
+                own = qp[i] // 8
+                keep = np.sort(np.concatenate([idx[i, g, : cnt[i, g] - 1][:n - 1], [own]]))
+                idx[i, g, :] = -1
+                idx[i, g, :n] = keep
+            else:
+                idx[i, g, :] = -1
+            cnt[i, g] = n
+    run(d, idx, cnt, q_req=d["q_req"], prefill=True)
