@@ -11,6 +11,9 @@ The region a decode token completes is always the query's own region (token p co
 region p/8 exactly when p % 8 == 7), and the own region is forced, never scored.  So this
 step's scan never reads what this step's compression writes, and the compression runs on
 a parallel branch (a side stream joined at the end of the step); the next step sees it.
+The branch forks after the selection, so the compression shares the GPU with the
+attention (64 CTAs at batch 1, most SMs idle) rather than with the scan, whose slowest
+CTAs it would delay.
 
 All buffers are allocated once, so a step can be captured in a CUDA graph and replayed.
 The per-step inputs live in one device arena (index_q, gate, q, q_pos and, optionally,
@@ -128,19 +131,6 @@ class DecodeStep:
         L = dsa.lib()
         main = torch.cuda.current_stream()
         p = dsa._p
-        if self.n_compress:
-            self.side.wait_stream(main)
-            with torch.cuda.stream(self.side):
-                t = self.tail
-                if self.sharded:
-                    dsa._check(L.dsa_compress_regions_groups(p(t), t[0].numel(), t.shape[0], p(self.src_row),
-                                                             p(self.dst_slot), self.n_compress, self.g0, self.ng,
-                                                             p(self.summaries), p(self.scales),
-                                                             self.summaries.shape[1], dsa._stream()))
-                else:
-                    dsa._check(L.dsa_compress_regions(p(t), t[0].numel(), t.shape[0], p(self.src_row),
-                                                      p(self.dst_slot), self.n_compress, p(self.summaries),
-                                                      p(self.scales), self.summaries.shape[1], dsa._stream()))
         st = dsa._stream()
         # scores and selection in one call (the scan's chunk maxima bound the selection)
         if self.sharded:
@@ -155,6 +145,19 @@ class DecodeStep:
                                            p(self.sum_base), self.sum_base.numel(), p(self.scores), self.ld,
                                            self.flags, self.k, p(self.sel_idx), p(self.sel_count), p(self.ws_sel),
                                            self.ws_sel_n, st))
+        if self.n_compress:
+            self.side.wait_stream(main)
+            with torch.cuda.stream(self.side):
+                t = self.tail
+                if self.sharded:
+                    dsa._check(L.dsa_compress_regions_groups(p(t), t[0].numel(), t.shape[0], p(self.src_row),
+                                                             p(self.dst_slot), self.n_compress, self.g0, self.ng,
+                                                             p(self.summaries), p(self.scales),
+                                                             self.summaries.shape[1], dsa._stream()))
+                else:
+                    dsa._check(L.dsa_compress_regions(p(t), t[0].numel(), t.shape[0], p(self.src_row),
+                                                      p(self.dst_slot), self.n_compress, p(self.summaries),
+                                                      p(self.scales), self.summaries.shape[1], dsa._stream()))
         self.run_attention(out)
         if self.n_compress:
             main.wait_stream(self.side)
