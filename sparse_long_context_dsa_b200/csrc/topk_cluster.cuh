@@ -17,7 +17,9 @@
 //  3. the keys >= L are pushed in region order, with each CTA's count, into rank 0's shared
 //     memory; rank 0 gathers them densely (still in region order), selects exactly the need
 //     largest (key desc, then region asc) and writes them with one ordered compaction, the
-//     own region last.
+//     own region last.  The exact step takes one 2048-bin histogram of the candidate keys
+//     over [L, row maximum] and one block scan from the top bin; the bin that holds the
+//     need-th largest key is either taken whole or ranked by one warp.
 // When the candidates do not fit (many equal scores, or k beyond the group count) every CTA
 // sees it in the pushed counts and the cluster runs an exact distributed radix select
 // instead: per digit every CTA histograms its keys that match the prefix found so far, the
@@ -399,6 +401,75 @@ __device__ void key_levels(Valid valid, Key key, uint32_t m, uint32_t cap, uint3
     __syncthreads();
 }
 
+// The m-th largest composite among a block's dense candidates, threshold form: afterwards a
+// candidate c is selected iff c >= *t_out, and exactly m are.  Thread t holds entries
+// d0 .. d0 + R - 1 of `total` (cv[u] = key << 32 | ~region, all distinct; every key in
+// [klo, khi]; 1 <= m <= total).  One 2048-bin histogram of the keys over [klo, khi] (`h`,
+// 2048 words, zeroed by the caller), one block scan from the top bin to the bin b holding
+// the m-th largest; b is taken whole when it holds exactly the count still missing, else one
+// warp ranks its members (key desc, then region asc) when they are at most 32.  Returns
+// false, with nothing decided, when b holds more than 32 candidates (equal keys in bulk):
+// the caller then runs the general levels.  `list`: 33 8-byte words; `res`: 3 words;
+// `sh_n`: one word.  Needs blockDim.x == kThreads == 512 (4 bins per thread).
+template <int R>
+__device__ bool dense_exact_threshold(const uint64_t (&cv)[R], uint32_t d0, uint32_t total, uint32_t m, uint32_t klo,
+                                      uint32_t khi, uint32_t *h, uint64_t *list, uint32_t *res, uint32_t *scan_ws,
+                                      uint32_t *sh_n, uint64_t *t_out)
+{
+    static_assert(kThreads * 4 == 2048, "4 bins per thread");
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const uint32_t range = khi - klo;
+    const int sh = range < 2048u ? 0 : (32 - __clz((int)range)) - 11;       // range >> sh < 2048
+    // a key above khi (a NaN score, which the chunk maxima skip) counts in the top bin: the
+    // same bin in both passes, so the counts stay exact and no index leaves the histogram
+    auto bin_of = [&](uint64_t c) { return min(2047u, ((uint32_t)(c >> 32) - klo) >> sh); };
+#pragma unroll
+    for (int u = 0; u < R; ++u)
+        if (d0 + u < total) atomicAdd(&h[bin_of(cv[u])], 1u);
+    __syncthreads();
+    // thread t: bins 2047 - 4t down to 2044 - 4t (thread 0 holds the top bins)
+    const uint4 q4 = reinterpret_cast<const uint4 *>(h)[kThreads - 1 - tid];
+    const uint32_t c[4] = {q4.w, q4.z, q4.y, q4.x};
+    const uint32_t s = c[0] + c[1] + c[2] + c[3];
+    const uint32_t incl = block_scan_incl<kThreads>(s, scan_ws);
+    const uint32_t excl = incl - s;
+    if (excl < m && incl >= m) {
+        uint32_t run = excl;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (run + c[u] >= m) {
+                res[0] = 2047u - 4u * (uint32_t)tid - (uint32_t)u;
+                res[1] = run;
+                res[2] = c[u];
+                break;
+            }
+            run += c[u];
+        }
+    }
+    if (tid == 0) *sh_n = 0u;
+    __syncthreads();
+    const uint32_t b = res[0], above = res[1], nb = res[2];
+    const uint32_t m_rem = m - above;                                        // 1 <= m_rem <= nb
+    if (nb == m_rem) {
+        *t_out = (uint64_t)(klo + (b << sh)) << 32;                          // every key of b and above
+        return true;
+    }
+    if (nb > 32u) return false;
+#pragma unroll
+    for (int u = 0; u < R; ++u)
+        if (d0 + u < total && bin_of(cv[u]) == b) list[atomicAdd(sh_n, 1u)] = cv[u];
+    __syncthreads();
+    if (warp == 0) {
+        const uint64_t e = lane < (int)nb ? list[lane] : 0ull;
+        uint32_t gt = 0;
+        for (int j = 0; j < (int)nb; ++j) gt += __shfl_sync(0xffffffffu, e, j) > e ? 1u : 0u;
+        if (lane < (int)nb && gt == m_rem - 1) list[32] = e;
+    }
+    __syncthreads();
+    *t_out = list[32];
+    return true;
+}
+
 // kSingle: one CTA per row (launched without a cluster; CL = 1), else a cluster of CL CTAs.
 // kMaxima: the indexer scan that wrote the scores also wrote chunk_max[row][c], the largest
 // score of regions 32c .. 32c+31 (row stride cm_stride, a multiple of 4): the cluster then
@@ -481,6 +552,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         sh_nin = 0u;
     }
     if (tid < 256) reinterpret_cast<uint32_t *>(smem_raw + kOffHs)[tid] = 0u;
+    if (rank == 0) reinterpret_cast<uint4 *>(smem_raw + kOffDense)[tid] = make_uint4(0u, 0u, 0u, 0u);   // 2048 bins
     __syncthreads();                                                        // keys staged
     auto key_at = [&](int i) -> uint32_t { return keys[padded(i)]; };
 
@@ -499,51 +571,58 @@ __global__ void __launch_bounds__(kThreads, 1)
     // after the candidate barrier: the fast-path decision (the same in every CTA from the pushed
     // counts) and, at rank 0, the exact selection among the gathered candidates, emitted in order
     uint64_t *slots = reinterpret_cast<uint64_t *>(smem_raw + kOffSlots);
-    auto finish_fast = [&](uint32_t Lk, int lg_slot, uint32_t slot_n) -> bool {
-        bool fast_ok = false;
+    auto finish_fast = [&](uint32_t Lk, uint32_t Kmax, int lg_slot, uint32_t slot_n) -> bool {
+        // the counts and each rank's first dense entry, in registers (the same in every thread)
+        uint32_t first[kMaxCluster];
         uint32_t total = 0;
         bool overflow = false;
-        for (int q = 0; q < CL; ++q) {
-            total += cand_cnt[q];
-            overflow |= cand_cnt[q] > slot_n;
+#pragma unroll
+        for (int q = 0; q < kMaxCluster; ++q) {
+            const uint32_t cq = q < CL ? cand_cnt[q] : 0u;
+            first[q] = total;
+            total += cq;
+            overflow |= cq > slot_n;
         }
-        fast_ok = !overflow && total >= (uint32_t)need && total <= (uint32_t)kDense;
+        const bool fast_ok = !overflow && total >= (uint32_t)need && total <= (uint32_t)kDense;
         if (fast_ok && rank == 0) {
-            // ---- dense gather in region order: thread t takes entries [t*kDPer, (t+1)*kDPer)
-            uint32_t *first = slice_tot;                                    // first dense entry of each rank
-            if (tid == 0) {
-                uint32_t run = 0;
-                for (int q = 0; q < CL; ++q) {
-                    first[q] = run;
-                    run += cand_cnt[q];
-                }
-            }
-            __syncthreads();
+            // ---- dense gather in region order: thread t takes entries [t*kDPer, (t+1)*kDPer);
+            // entry d is in the last rank whose first entry is <= d (ranks without candidates
+            // share their first entry with the next rank)
             uint64_t cv[kDPer];
             const uint32_t d0 = tid * kDPer;
-            int q = 0;
-            while (q + 1 < CL && d0 >= first[q + 1]) ++q;
 #pragma unroll
             for (int u = 0; u < kDPer; ++u) {
                 const uint32_t d = d0 + u;
-                while (q + 1 < CL && d >= first[q + 1]) ++q;
-                cv[u] = d < total ? slots[((uint32_t)q << lg_slot) + (d - first[q])] : 0ull;
+                uint32_t base = 0;
+#pragma unroll
+                for (int q = 0; q < kMaxCluster; ++q)
+                    if (q < CL && d >= first[q]) base = ((uint32_t)q << lg_slot) - first[q];
+                cv[u] = d < total ? slots[base + d] : 0ull;
             }
-            auto valid_u = [&](int u) { return d0 + (uint32_t)u < total; };
-            auto comp_u = [&](int u) { return cv[u]; };
-            uint64_t elo, ehi, cp, cm;
-            const bool ok = block_threshold<kDPer>(valid_u, comp_u, (uint32_t)need, Lk, hs, dense, hw, &sh_kmax,
-                                                   &sh_nin, scan_ws + 32, mm_ws, &elo, &ehi, &cp, &cm);
+            // ---- the need-th largest candidate: every key lies in [Lk, Kmax]
+            uint64_t T = 0;
+            bool ok = dense_exact_threshold<kDPer>(cv, d0, total, (uint32_t)need, Lk, Kmax,
+                                                   reinterpret_cast<uint32_t *>(dense), reinterpret_cast<uint64_t *>(hs),
+                                                   scan_ws + 32, scan_ws, &sh_nin, &T);
+            if (!ok) {
+                // more than 32 candidates in the threshold bin (equal keys in bulk): general levels
+                auto valid_u = [&](int u) { return d0 + (uint32_t)u < total; };
+                auto comp_u = [&](int u) { return cv[u]; };
+                uint64_t elo, ehi, cm;
+                __syncthreads();                                            // the bins are read
+                ok = block_threshold<kDPer>(valid_u, comp_u, (uint32_t)need, Lk, hs, dense, hw, &sh_kmax, &sh_nin,
+                                            scan_ws + 32, mm_ws, &elo, &ehi, &T, &cm);
+            }
             if (ok) {
-                // ---- ordered emit
+                // ---- ordered emit: the candidates >= T, exactly need of them
                 uint32_t cs = 0;
 #pragma unroll
-                for (int u = 0; u < kDPer; ++u) cs += (valid_u(u) && threshold_selects(cv[u], elo, ehi, cp, cm)) ? 1u : 0u;
+                for (int u = 0; u < kDPer; ++u) cs += (d0 + u < total && cv[u] >= T) ? 1u : 0u;
                 const uint32_t sincl = block_scan_incl<kThreads>(cs, scan_ws);
                 uint32_t opos = sincl - cs;
 #pragma unroll
                 for (int u = 0; u < kDPer; ++u) {
-                    if (valid_u(u) && threshold_selects(cv[u], elo, ehi, cp, cm)) {
+                    if (d0 + u < total && cv[u] >= T) {
                         if (opos < (uint32_t)need) out[opos] = (int32_t)(0xFFFFFFFFu - (uint32_t)cv[u]);
                         ++opos;
                     }
@@ -587,6 +666,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t above, n_in;
             key_levels<kM>(mvalid, mkey, (uint32_t)need, 64u, hs, &sh_kmin, &sh_kmax, scan_ws + 32, elo, ehi, above,
                            n_in);
+            const uint32_t Kmax = sh_kmax;                                  // the row's largest maximum
             mfast = n_in <= 64u;                                            // else maxima tie in bulk
             Lk = (uint32_t)elo;
             if (mfast) {
@@ -663,7 +743,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     sh_nin = 0u;
                 }
                 cluster.sync();                                             // candidates and counts in place
-                fast_ok = finish_fast(Lk, lg_slot, slot_n);
+                fast_ok = finish_fast(Lk, Kmax, lg_slot, slot_n);
             }
         }
         if (!fast_ok) {
@@ -807,7 +887,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             sh_nin = 0u;
         }
         cluster.sync();                                                     // candidates and counts in place
-        fast_ok = finish_fast(Lk, lg_slot, slot_n);
+        fast_ok = finish_fast(Lk, gmx, lg_slot, slot_n);
     }
     if (fast_ok) return;               // nothing reads another CTA's smem after the barrier
 

@@ -7,9 +7,11 @@ over those scores ([P2] Step-5-Preview 如何实现1M长上下文 §索引器打
 to the lower region).  Cases: decode batches whose rows take the chunk-maxima path (few long
 rows: 16,384 .. 131,071 regions) and rows that do not (short rows, k = 1024, many rows), all-
 zero queries (every score +0: the maxima tie in bulk and the selection falls back), identical
-summaries (every score of a row equal), rows whose own region is below k, and rows whose best
+summaries (every score of a row equal), rows whose own region is below k, rows whose best
 regions crowd into one stretch of the row (many chunk maxima tie near the bound, and whole
-chunks are candidates).
+chunks are candidates), and rows where a run of regions shares the threshold score exactly
+(copies of the summary at the threshold: the candidate bin at the threshold is taken whole,
+ranked by one warp, or narrowed by the general levels).
 """
 import numpy as np
 import pytest
@@ -121,3 +123,32 @@ def test_crowded_best_regions_fall_back_exactly(lo, n):
     check_against_oracle(s1, i1, c1, d["q_pos"], k)
     sel = i1.cpu().numpy()[0]
     assert np.mean((sel[:, : k - 1] >= lo) & (sel[:, : k - 1] < lo + n)) > 0.9
+
+
+@pytest.mark.parametrize("n_tied", [5, 31, 40])
+def test_ties_at_the_threshold(n_tied):
+    # each group's summary and scale at its (k-1)-th best region are copied over a run of
+    # n_tied regions: their scores equal the threshold score bit for bit
+    lengths = [1 << 20]
+    d, S, C = setup(lengths, seed=900 + n_tied)
+    k = 512
+    ld = max(lengths) // 8
+    own = int(d["q_pos"][0]) // 8
+    s0 = torch.zeros((1, G, ld), dtype=torch.float32, device="cuda")
+    dsa.indexer_scores(d["index_q"], d["gate"], d["q_req"], d["q_pos"], S, C, d["sum_base"], s0)
+    dsa.check_device()
+    base = int(d["sum_base"][0])
+    for g in range(G):
+        row = s0[0, g, :own].cpu().numpy()
+        r = int(np.argsort(-row, kind="stable")[k - 2])
+        x = 3000 + 20011 * g
+        S[g, base + x:base + x + n_tied] = S[g, base + r]
+        C[g, base + x:base + x + n_tied] = C[g, base + r]
+    s1, i1, c1, s2, i2, c2 = both(d, S, C, k, ld)
+    assert torch.equal(s1, s2)
+    assert torch.equal(c1, c2) and torch.equal(i1, i2)
+    check_against_oracle(s1, i1, c1, d["q_pos"], k)
+    sc = s1.cpu().numpy()[0]
+    for g in range(G):
+        x = 3000 + 20011 * g
+        assert np.all(sc[g, x:x + n_tied] == sc[g, x])       # the run is one tie

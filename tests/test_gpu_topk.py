@@ -150,3 +150,22 @@ def test_equal_scores_take_the_lowest_regions(ld):
     s[1] = 0.75
     s[2] = np.where((np.arange(ld) // 97) % 2 == 0, 1.5, 1.25).astype(np.float32)
     check(s, [8 * ld - 1, 8 * ld - 3, 8 * (ld - 5)], k)
+
+
+@pytest.mark.parametrize("n_tied", [5, 31, 33, 40])
+def test_cluster_path_ties_at_the_threshold(n_tied):
+    # n_tied regions take exactly the score of the need-th best one, so the bin of the
+    # candidate histogram that holds the threshold holds n_tied + 1 equal keys: taken whole,
+    # ranked by one warp (<= 32) or narrowed by the general levels (> 32); the lowest regions
+    # of the tie win
+    rng = np.random.default_rng(100 + n_tied)
+    ld, k = 120000, 512
+    s = rng.standard_normal((2, G, ld)).astype(np.float32)
+    q_pos = [8 * ld, 8 * ld - 5]                              # own regions ld and ld - 1
+    for b in range(2):
+        own = q_pos[b] // 8
+        for g in range(G):
+            v = np.sort(s[b, g, :own])[::-1][k - 2]           # the (k-1)-th largest: need = k - 1
+            x = 1000 + 7919 * (b * G + g)
+            s[b, g, x:x + n_tied] = v
+    check(s, q_pos, k)
