@@ -6,12 +6,15 @@
 // selected regions [32*rank, 32*rank + 32).  Every CTA issues all of its K/V loads at once
 // (32 regions x 6 KiB, TMA with the 128-byte swizzle into 16 pair buffers, one mbarrier per
 // pair), so a CTA waits for one memory round trip, not one per pair.  Its 8 warps take two
-// pairs each: S = Q K^T and O += P V on mma.sync m16n8k16 bf16 with fp32 accumulation and an
-// exp2 online softmax, tokens t <= p only.  The warps merge (max, sum, O) in smem and the
-// CTA pushes head h of its result into CTA h's inbox through distributed shared memory; after
-// one cluster barrier CTA r merges head r of the row from its own inbox (O = sum_c 2^(m_c - M)
-// O_c / sum_c 2^(m_c - M) l_c) and writes the bf16 output and the LSE.  No partials in global
-// memory, no second kernel.
+// pairs each for S = Q K^T (mma.sync m16n8k16 bf16, fp32 accumulate; tokens t <= p only, in
+// log2 units); the CTA's row maximum M of each head goes through smem, every warp writes
+// P = 2^(S - M) in bf16 to one [16 heads][256 tokens] tile, and warp w then computes the
+// output dims [24w, 24w + 24) of O = P V over all the CTA's tokens.  So no warp merges
+// another's O: each warp stores its dims of head h straight into CTA h's inbox through
+// distributed shared memory, beside the CTA's (M, l).  After one cluster barrier CTA r
+// merges head r of the row from its own inbox (O = sum_c 2^(m_c - M) O_c / sum_c
+// 2^(m_c - M) l_c) and writes the bf16 output and the LSE.  No partials in global memory,
+// no second kernel.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -33,14 +36,20 @@ constexpr int kRegionsPerCta = 32;
 constexpr int kPairs = kRegionsPerCta / 2;
 constexpr int kWarps = 8;
 constexpr int kThreads = 32 * kWarps;
-constexpr int kRow = kD + 8;                   // padded merge row (floats)
 constexpr size_t kPairArea = (size_t)kPairs * kPairBytes;                 // 192 KiB
-constexpr size_t kMergeO = (size_t)kWarps * 16 * kRow * 4;               // per-warp O for the merge
-constexpr size_t kMergeMl = (size_t)kWarps * 16 * 2 * 4;
-static_assert(kMergeO + kMergeMl + 16 * kWarps * 4 <= kPairArea, "merge buffers fit in the pair area");
 constexpr int kInRow = kD + 4;                 // inbox row per source CTA: O [kD], m, l, pad
 constexpr size_t kInbox = (size_t)kSplits * kInRow * 4;                  // outside the pair area
-constexpr size_t kSmemBytes = 1024 + kPairArea + kQBytes + 256 + kInbox;
+constexpr int kTokens = 8 * kRegionsPerCta;    // 256 tokens of a CTA
+constexpr int kPRow = 2 * kTokens + 16;        // P tile row (bytes): padded, conflict-free ldmatrix
+constexpr size_t kMl = (size_t)2 * kWarps * 16 * 4;                      // per-warp row maxima and sums
+constexpr size_t kPTile = (size_t)16 * kPRow;
+constexpr int kDimsPerWarp = kD / kWarps;      // 24: three n8 tiles of O per warp
+static_assert(kDimsPerWarp == 24, "three n8 tiles of output dims per warp");
+static_assert(kInbox % 16 == 0 && kMl % 16 == 0, "the P tile stays 16-byte aligned");
+static_assert((kInRow * 4) % 16 == 0 && (size_t)16 * kInRow * 4 <= kPairArea,
+              "inbox rows are whole 16-byte bulk copies; the staged rows fit the pair area");
+static_assert((kPairs + 1) * 8 <= 256, "pair barriers and the inbox barrier fit their 256 bytes");
+constexpr size_t kSmemBytes = 1024 + kPairArea + kQBytes + 256 + kInbox + kMl + kPTile;
 constexpr int kMaxK = kSplits * kRegionsPerCta;                            // 512
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -54,7 +63,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *qs = smem + kPairArea;
     uint64_t *bars = reinterpret_cast<uint64_t *>(qs + kQBytes);            // [kPairs]
     float *inbox = reinterpret_cast<float *>(qs + kQBytes + 256);           // [kSplits][kInRow]
+    float *mw = inbox + kSplits * kInRow;                                   // [kWarps][16] row maxima
+    float *lw = mw + kWarps * 16;                                           // [kWarps][16] row sums
+    uint8_t *ptile = reinterpret_cast<uint8_t *>(lw + kWarps * 16);         // P [16 heads][kPRow bytes]
     __shared__ int sh_y[kRegionsPerCta], sh_r[kRegionsPerCta], sh_v[kRegionsPerCta];   // per region of the CTA
+    __shared__ int sh_ok[kPairs];                                           // the pair's data landed
 
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
@@ -87,8 +100,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     // their barriers, resolves their coordinates (sel_idx -> block_table, lanes 0..3) and
     // issues their TMA loads itself, so the 8 warps issue in parallel.
     if (lane < 2) mbar_init(&bars[warp + 8 * lane], 1);
+    uint64_t *inbox_bar = &bars[kPairs];                                    // the 16 inbox rows landed
+    if (tid == 0) {
+        mbar_init(inbox_bar, 1);
+        mbar_arrive_expect_tx(inbox_bar, (unsigned)(kSplits * kInRow * 4));
+    }
     fence_mbar_init();
     __syncwarp();
+    // every CTA's inbox barrier is set up before any CTA copies into it: arrive now, wait
+    // before the copies (long after every CTA arrived)
+    cluster_arrive_relaxed();
     if (lane < 4) {
         const int j = reg_of(lane);
         int y = 0, r = -1, v = 0;
@@ -154,23 +175,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     const int gq = lane >> 2, t = lane & 3;
-    float o[24][4];
-#pragma unroll
-    for (int i = 0; i < 24; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
-    float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.0f, 0.0f};
     const int n_pairs = (nr + 1) / 2;
-    bool ok = true;
-    for (int pr = warp; pr < n_pairs && ok; pr += kWarps) {
+    // ---- S = Q K^T of this warp's pairs (warp, warp + 8), in log2 units, masked to t <= p
+    float s[2][2][4];
+    float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) s[i][nt][0] = s[i][nt][1] = s[i][nt][2] = s[i][nt][3] = -INFINITY;
+        const int pr = warp + kWarps * i;
+        if (pr >= n_pairs) continue;
+        const bool landed = mbar_wait(&bars[pr], 0u);                     // false: error set, pair skipped
+        if (lane == 0) sh_ok[pr] = landed ? 1 : 0;
+        if (!landed) continue;
         const int rr[2] = {sh_r[2 * pr], sh_r[2 * pr + 1]};
         const bool rv[2] = {sh_v[2 * pr] != 0, sh_v[2 * pr + 1] != 0};
-        ok = mbar_wait(&bars[pr], 0u);
-        if (!ok) break;
         const uint32_t kt = smem_u32(smem + (size_t)pr * kPairBytes);
-        const uint32_t vt = kt + 2 * kRegionBytes;
-        float s[2][4];
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
-            s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.0f;
+            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
             const uint32_t tile = kt + nt * kRegionBytes;
             const int r = lane & 7;
 #pragma unroll
@@ -178,140 +201,142 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int c = kp * 32 + 8 * (lane >> 3);
                 uint32_t b0, b1, b2, b3;
                 ldmatrix_x4(tile + swz(r, c), b0, b1, b2, b3);
-                mma_bf16_16816(s[nt], qa[2 * kp][0], qa[2 * kp][1], qa[2 * kp][2], qa[2 * kp][3], b0, b1);
-                mma_bf16_16816(s[nt], qa[2 * kp + 1][0], qa[2 * kp + 1][1], qa[2 * kp + 1][2], qa[2 * kp + 1][3],
-                               b2, b3);
+                mma_bf16_16816(acc, qa[2 * kp][0], qa[2 * kp][1], qa[2 * kp][2], qa[2 * kp][3], b0, b1);
+                mma_bf16_16816(acc, qa[2 * kp + 1][0], qa[2 * kp + 1][1], qa[2 * kp + 1][2], qa[2 * kp + 1][3], b2,
+                               b3);
             }
-        }
-        float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int tok = 8 * rr[nt] + 2 * t + (e & 1);
-                const bool keep = rv[nt] && tok <= pos;
-                const float v = keep ? s[nt][e] * p.scale_log2 : -INFINITY;
-                s[nt][e] = v;
+                const float v = (rv[nt] && tok <= pos) ? acc[e] * p.scale_log2 : -INFINITY;
+                s[i][nt][e] = v;
                 mx[e >> 1] = fmaxf(mx[e >> 1], v);
             }
-        // lazy rescaling: the reference max mrow moves only when a block's max exceeds it by
-        // more than kSlack (log2 units; P stays below 2^kSlack): the same softmax, rarely rescaled
-        float alpha[2], mref[2];
-        bool grow_any = false;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
-            mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
-            const bool grow = mx[h] > mrow[h] + attn::kSlack;
-            alpha[h] = grow ? exp2f(mrow[h] - mx[h]) : 1.0f;
-            if (grow) mrow[h] = mx[h];
-            grow_any |= grow;
-            mref[h] = (mrow[h] == -INFINITY) ? 0.0f : mrow[h];
-        }
-        float ps[2] = {0.0f, 0.0f};
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float pv = exp2f(s[nt][e] - mref[e >> 1]);
-                s[nt][e] = pv;
-                ps[e >> 1] += pv;
-            }
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            ps[h] += __shfl_xor_sync(0xffffffffu, ps[h], 1);
-            ps[h] += __shfl_xor_sync(0xffffffffu, ps[h], 2);
-            lrow[h] = lrow[h] * alpha[h] + ps[h];
-        }
-        if (__any_sync(0xffffffffu, grow_any)) {
-#pragma unroll
-            for (int nd = 0; nd < 24; ++nd) {
-                o[nd][0] *= alpha[0];
-                o[nd][1] *= alpha[0];
-                o[nd][2] *= alpha[1];
-                o[nd][3] *= alpha[1];
-            }
-        }
-        const uint32_t pa0 = pack_bf16x2(s[0][0], s[0][1]);
-        const uint32_t pa1 = pack_bf16x2(s[0][2], s[0][3]);
-        const uint32_t pa2 = pack_bf16x2(s[1][0], s[1][1]);
-        const uint32_t pa3 = pack_bf16x2(s[1][2], s[1][3]);
-        {
-            const int r = lane & 7;
-            const int reg = (lane >> 3) & 1;
-            const int dsub = 8 * (lane >> 4);
-#pragma unroll
-            for (int nd = 0; nd < 24; nd += 2) {
-                uint32_t b0, b1, b2, b3;
-                ldmatrix_x4_trans(vt + reg * kRegionBytes + swz(r, nd * 8 + dsub), b0, b1, b2, b3);
-                // a region that was not loaded holds stale smem: its P is 0, but 0 * NaN is not
-                if (!rv[0]) b0 = b2 = 0u;
-                if (!rv[1]) b1 = b3 = 0u;
-                mma_bf16_16816(o[nd], pa0, pa1, pa2, pa3, b0, b1);
-                mma_bf16_16816(o[nd + 1], pa0, pa1, pa2, pa3, b2, b3);
-            }
         }
     }
-
-    // ---- merge the 8 warps into this CTA's (m, l, O) (the pair area is free once every warp
-    // is done with its pairs; a warp that gave up on a wait still joins the barriers)
-    __syncthreads();
-    float *red_o = reinterpret_cast<float *>(smem);                          // [8][16][kRow]
-    float *red_ml = red_o + kWarps * 16 * kRow;                              // [8][16][2]
+    // ---- the CTA's row maximum of each head (rows gq and gq + 8 of this lane)
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-        const int hr = gq + 8 * h;
-        float *rowp = red_o + (warp * 16 + hr) * kRow + 2 * t;
-#pragma unroll
-        for (int nd = 0; nd < 24; ++nd)
-            *reinterpret_cast<float2 *>(rowp + nd * 8) = make_float2(o[nd][2 * h], o[nd][2 * h + 1]);
-        if (t == 0) {
-            red_ml[(warp * 16 + hr) * 2 + 0] = mrow[h];
-            red_ml[(warp * 16 + hr) * 2 + 1] = lrow[h];
-        }
+        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
+        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
+    }
+    if (t == 0) {
+        mw[warp * 16 + gq] = mx[0];
+        mw[warp * 16 + gq + 8] = mx[1];
     }
     __syncthreads();
-    float *wts = red_ml + kWarps * 16 * 2;                                   // [16][8]
-    // this CTA's (m, l) of head hr and its O row go to CTA hr's inbox row `rank`
-    if (tid < 16) {
-        const int hr = tid;
-        float M = -INFINITY;
+    float M[2], mref[2];
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, red_ml[(w * 16 + hr) * 2]);
-        const float Mref = (M == -INFINITY) ? 0.0f : M;
-        float L = 0.0f;
+    for (int h = 0; h < 2; ++h) {
+        M[h] = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-            const float wt = exp2f(red_ml[(w * 16 + hr) * 2] - Mref);
-            wts[hr * kWarps + w] = wt;
-            L += wt * red_ml[(w * 16 + hr) * 2 + 1];
+        for (int w = 0; w < kWarps; ++w) M[h] = fmaxf(M[h], mw[w * 16 + gq + 8 * h]);
+        mref[h] = (M[h] == -INFINITY) ? 0.0f : M[h];
+    }
+    // ---- P = 2^(S - M): bf16 into the P tile (token column 16 pr + 8 nt + 2t), fp32 row sums
+    float ps[2] = {0.0f, 0.0f};
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int pr = warp + kWarps * i;
+        if (pr >= n_pairs) continue;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const float p0 = exp2f(s[i][nt][0] - mref[0]), p1 = exp2f(s[i][nt][1] - mref[0]);
+            const float p2 = exp2f(s[i][nt][2] - mref[1]), p3 = exp2f(s[i][nt][3] - mref[1]);
+            ps[0] += p0 + p1;
+            ps[1] += p2 + p3;
+            const int col = 2 * (16 * pr + 8 * nt + 2 * t);
+            *reinterpret_cast<uint32_t *>(ptile + gq * kPRow + col) = pack_bf16x2(p0, p1);
+            *reinterpret_cast<uint32_t *>(ptile + (gq + 8) * kPRow + col) = pack_bf16x2(p2, p3);
         }
-        float *dst = cluster.map_shared_rank(inbox, hr) + rank * kInRow + kD;
-        dst[0] = M;
-        dst[1] = L;
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        ps[h] += __shfl_xor_sync(0xffffffffu, ps[h], 1);
+        ps[h] += __shfl_xor_sync(0xffffffffu, ps[h], 2);
+    }
+    if (t == 0) {
+        lw[warp * 16 + gq] = ps[0];
+        lw[warp * 16 + gq + 8] = ps[1];
     }
     __syncthreads();
-    for (int e = tid; e < 16 * kD / 4; e += kThreads) {
-        const int hr = e / (kD / 4), d = 4 * (e % (kD / 4));
-        float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+
+    // ---- O[:, 24 warp .. 24 warp + 24) = P V, one k-step per pair (16 tokens); the loop is
+    // unrolled over the 16 pairs with two accumulator sets (even and odd pairs), so the loads
+    // of later pairs overlap the MMAs of earlier ones
+    float o[2][3][4];
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-            const float4 v = *reinterpret_cast<const float4 *>(red_o + (w * 16 + hr) * kRow + d);
-            const float wt = wts[hr * kWarps + w];
-            acc.x += wt * v.x;
-            acc.y += wt * v.y;
-            acc.z += wt * v.z;
-            acc.w += wt * v.w;
+    for (int a2 = 0; a2 < 2; ++a2)
+#pragma unroll
+        for (int j = 0; j < 3; ++j) o[a2][j][0] = o[a2][j][1] = o[a2][j][2] = o[a2][j][3] = 0.0f;
+    {
+        // region j of the CTA takes part when its data landed and it is valid (bit j)
+        const unsigned use = __ballot_sync(0xffffffffu, (lane >> 1) < n_pairs && sh_v[lane] != 0 && sh_ok[lane >> 1] != 0);
+        const uint32_t pbase = smem_u32(ptile);
+        const int ar = (lane & 7) + 8 * ((lane >> 3) & 1);
+        const int r = lane & 7, reg = (lane >> 3) & 1, dsub = 8 * (lane >> 4);
+        const int nd0 = 3 * warp;
+        const uint32_t vbase = smem_u32(smem) + 2 * kRegionBytes + reg * kRegionBytes;
+        const uint32_t voff_b = swz(r, nd0 * 8 + dsub), voff_c = swz(r, (nd0 + 2) * 8);
+#pragma unroll
+        for (int pr = 0; pr < kPairs; ++pr) {
+            const unsigned u2 = (use >> (2 * pr)) & 3u;
+            if (u2 == 0u) continue;                                       // uniform: no token of the pair
+            uint32_t a0, a1, a2, a3;
+            ldmatrix_x4(pbase + ar * kPRow + 2 * (16 * pr + 8 * (lane >> 4)), a0, a1, a2, a3);
+            const uint32_t vt = vbase + (uint32_t)pr * kPairBytes;
+            uint32_t b0, b1, b2, b3, c0, c1;
+            ldmatrix_x4_trans(vt + voff_b, b0, b1, b2, b3);
+            ldmatrix_x2_trans(vt + voff_c, c0, c1);
+            // a region that was not loaded holds stale smem: its P is 0, but 0 * NaN is not
+            if (!(u2 & 1u)) b0 = b2 = c0 = 0u;
+            if (!(u2 & 2u)) b1 = b3 = c1 = 0u;
+            float(&oa)[3][4] = o[pr & 1];
+            mma_bf16_16816(oa[0], a0, a1, a2, a3, b0, b1);
+            mma_bf16_16816(oa[1], a0, a1, a2, a3, b2, b3);
+            mma_bf16_16816(oa[2], a0, a1, a2, a3, c0, c1);
         }
-        *reinterpret_cast<float4 *>(cluster.map_shared_rank(inbox, hr) + rank * kInRow + d) = acc;
+#pragma unroll
+        for (int j = 0; j < 3; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[0][j][e] += o[1][j][e];
     }
-    // every CTA's rows are in the inboxes; afterwards no CTA touches another's smem
-    asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
-    asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+    // ---- this CTA's (M, l, O) of head h goes to CTA h's inbox row `rank`: the rows are staged
+    // in the (now free) pair area and sent as 16 bulk copies of kInRow floats, each completing
+    // on the destination's inbox barrier, so a CTA waits for its own 16 rows and nothing else
+    __syncthreads();                                                        // every warp is done with P and V
+    float *stage = reinterpret_cast<float *>(smem);                         // [16][kInRow]
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+        const int col = (3 * warp + j) * 8 + 2 * t;
+        *reinterpret_cast<float2 *>(stage + gq * kInRow + col) = make_float2(o[0][j][0], o[0][j][1]);
+        *reinterpret_cast<float2 *>(stage + (gq + 8) * kInRow + col) = make_float2(o[0][j][2], o[0][j][3]);
+    }
+    if (warp == 0 && t == 0) {
+        float L[2] = {0.0f, 0.0f};
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) L[h] += lw[w * 16 + gq + 8 * h];
+        stage[gq * kInRow + kD] = M[0];
+        stage[gq * kInRow + kD + 1] = L[0];
+        stage[(gq + 8) * kInRow + kD] = M[1];
+        stage[(gq + 8) * kInRow + kD + 1] = L[1];
+    }
+    fence_proxy_async();                                                    // the rows, to the copy engine
+    __syncwarp();
+    cluster_wait();
+    __syncthreads();
+    if (warp == 0 && lane < kSplits) {
+        bulk_copy_to_cta(inbox + rank * kInRow, stage + lane * kInRow, (unsigned)(kInRow * 4), inbox_bar,
+                         (unsigned)lane);
+        bulk_commit();
+    }
+    const bool inbox_ok = mbar_wait(inbox_bar, 0u);                         // false: error set
 
     // ---- CTA `rank` merges head `rank` of the row from its inbox
     const int hr = rank;
-    if (tid < kD) {
+    if (inbox_ok && tid < kD) {
         float M = -INFINITY;
 #pragma unroll
         for (int c = 0; c < kSplits; ++c) M = fmaxf(M, inbox[c * kInRow + kD]);
@@ -328,6 +353,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         p.out[head * kD + d] = __float2bfloat16_rn(L > 0.0f ? acc / L : 0.0f);
         if (p.lse && d == 0) p.lse[head] = (L > 0.0f) ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
     }
+    // this CTA's copies have read their rows before its shared memory goes away
+    if (warp == 0 && lane < kSplits) bulk_wait_read_all();
 }
 
 }  // namespace attnc
