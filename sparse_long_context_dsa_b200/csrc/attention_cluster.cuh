@@ -10,11 +10,11 @@
 // log2 units); the CTA's row maximum M of each head goes through smem, every warp writes
 // P = 2^(S - M) in bf16 to one [16 heads][256 tokens] tile, and warp w then computes the
 // output dims [24w, 24w + 24) of O = P V over all the CTA's tokens.  So no warp merges
-// another's O: each warp stores its dims of head h straight into CTA h's inbox through
-// distributed shared memory, beside the CTA's (M, l).  After one cluster barrier CTA r
-// merges head r of the row from its own inbox (O = sum_c 2^(m_c - M) O_c / sum_c
-// 2^(m_c - M) l_c) and writes the bf16 output and the LSE.  No partials in global memory,
-// no second kernel.
+// another's O.  The CTA's (M, l, O) of head h goes to CTA h's inbox as one bulk copy that
+// completes on that CTA's inbox barrier; once its 16 rows are in, CTA r merges head r of
+// the row (O = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c) and writes the bf16 output and
+// the LSE.  No partials in global memory, no second kernel, no cluster barrier after the
+// start.
 #pragma once
 
 #include <cooperative_groups.h>
