@@ -795,6 +795,7 @@ def run_swa(args):
     ms = replicas.max_over_ranks(t0.elapsed_time(t1), dev)
     step_us = ms * 1e3 / n
     bytes_step = SWA_BATCH * swa_bytes_per_query()
+    launches = int(dsa.lib().dsa_window_decode_launches(SWA_BATCH, SWA_WINDOW))   # 1: append folded into the clustered kernel
     peak, kind = peaks()
     achieved = bytes_step / (step_us * 1e-6) / 1e9
     # e2e: per step the inputs from pinned host memory and the output back, through the calls
@@ -822,12 +823,14 @@ def run_swa(args):
         "config": {"workload": "swa_decode_b8", "batch": SWA_BATCH, "position": L_CTX - 1, "window": SWA_WINDOW,
                    "ring_pages": SWA_RING, "layers": SWA_LAYERS,
                    "l2": "69 layers' rings rotate (868 MB > L2)"},
-        "roofline": {"kernel": "window step (kv_append + sparse_attn_kernel + combine_kernel)", "bound": "hbm",
+        "roofline": {"kernel": ("window step (sparse_attn_cluster_kernel with the append folded in)" if launches == 1
+                                else "window step (kv_append_kernel + sparse_attn_kernel [+ combine_kernel])"),
+                     "bound": "hbm",
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_kind": kind, "bytes_per_step": bytes_step, "traffic": None},
         "e2e": {"value": world * SWA_BATCH * n_e2e / (e2e_ms / 1e3), "unit": "queries/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 3 * n,
+        "gpu_launches": launches * n,
         "clocks": sampler.summary(),
     }
     if rank == 0 and not args.no_cpu_baseline:

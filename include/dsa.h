@@ -267,9 +267,24 @@ dsa_status_t dsa_sparse_attn_prefill(const void *q, const void *k_cache, const v
  *   out[q][h] = sum_{t in T} softmax_t(q[q][h] . K_t / sqrt(192)) V_t   (bf16, fp32 math)
  *   lse[q][h] = ln sum_{t in T} exp(q[q][h] . K_t / sqrt(192))          (NULL: not written)
  * The caller keeps every token of the window in the cache (a ring of at least `window`
- * tokens).  1 <= window <= 2^20.  Runs on the per-row attention kernel (split across CTAs,
- * with a merge kernel, when there are few rows); workspace dsa_window_attn_workspace_size(
- * nq, window) bytes, 256-byte aligned (0: none needed).  Errors as for the sparse calls. */
+ * tokens).  1 <= window <= 2^20.  A window of at most 624 tokens, with every (query,
+ * group) row's 8-CTA cluster resident at once, runs in one kernel that merges the row's
+ * splits in distributed shared memory; other calls run on the per-row attention kernel
+ * (split across CTAs, with a merge kernel, when there are few rows).  Workspace
+ * dsa_window_attn_workspace_size(nq, window) bytes, 256-byte aligned (0: none needed).
+ * Errors as for the sparse calls.
+ *
+ * dsa_window_decode: one window-layer decode step, dsa_kv_append(new_k, new_v at q_pos)
+ * followed by dsa_window_attn over the window that now ends at the appended token, with the
+ * same arguments, results and errors as the two calls.  Where dsa_window_attn would run
+ * its clustered kernel the append is folded into it (one launch: the CTA that holds a row's
+ * newest region writes the token's K and V rows to the cache slot and attends them from
+ * new_k / new_v); elsewhere it makes the two calls.  As for dsa_kv_append, the queries of one
+ * call must be distinct requests (no query's window may hold another query's new token).
+ *
+ * dsa_window_decode_launches: the number of kernels dsa_window_decode(nq, window) launches
+ * on the current device (1 where the append is folded in, else 2 or 3; 0 for nq <= 0 or
+ * window < 1). */
 dsa_status_t dsa_kv_append(void *k_cache, void *v_cache, int64_t n_pages, const int32_t *block_table,
                            int max_pages, int n_req, const int32_t *q_req, const int32_t *q_pos, int n,
                            const void *new_k, const void *new_v, dsa_stream_t stream);
@@ -278,6 +293,11 @@ dsa_status_t dsa_window_attn(const void *q, const void *k_cache, const void *v_c
                              const int32_t *block_table, int max_pages, int n_req, const int32_t *q_req,
                              const int32_t *q_pos, int nq, int window, void *out, float *lse, void *ws,
                              size_t ws_bytes, dsa_stream_t stream);
+dsa_status_t dsa_window_decode(void *k_cache, void *v_cache, int64_t n_pages, const int32_t *block_table,
+                               int max_pages, int n_req, const int32_t *q_req, const int32_t *q_pos, int nq,
+                               const void *new_k, const void *new_v, const void *q, int window, void *out,
+                               float *lse, void *ws, size_t ws_bytes, dsa_stream_t stream);
+int dsa_window_decode_launches(int nq, int window);
 
 /* ------------------------------------------------------------------------------ */
 /* Indexer front end.  [P2 §索引器打分] the indexer projects the hidden state to index_q /

@@ -56,6 +56,12 @@ struct Params {
     // q is the full [nq][64][192] and out / lse hold the local groups' heads ([nq][16 ng][192]).
     int gshift;
     int g0;
+    // window decode with the append folded in (nullable): query q's token at q_pos[q], K and V
+    // rows new_k / new_v [nq][4][192], is written to its cache slot and attended from these rows
+    const __nv_bfloat16 *new_k;
+    const __nv_bfloat16 *new_v;
+    __nv_bfloat16 *k_cache;    // the caches the rows go to (with new_k)
+    __nv_bfloat16 *v_cache;
 };
 
 // Index of head hr of local group gl of query qi in out / lse ([nq][16 << gshift]).

@@ -1,20 +1,24 @@
-// A4 sparse GQA attention for a few long selections (decode of one or two requests), with
-// the split merge inside the kernel ([P1] kwkr.cn/news/601179 §DSA ④; [P3] 100 万 token
-// 上下文实测 §一: the hit regions are gathered from the paged cache through the block_table).
+// A4 sparse GQA attention for a few long selections (decode of one or two requests), and the
+// window layers' decode over each query's last `window` tokens (optionally appending the
+// query's own token to the cache in the same kernel), with the split merge inside the kernel ([P1] kwkr.cn/news/601179 §DSA ④ and §滑窗注意力; [P3] 100 万 token 上下文实测
+// §一: the hit regions are gathered from the paged cache through the block_table).
 //
-// A (query, group) row is attended by a cluster of kSplits CTAs; CTA `rank` takes the
-// selected regions [32*rank, 32*rank + 32).  Every CTA issues all of its K/V loads at once
-// (32 regions x 6 KiB, TMA with the 128-byte swizzle into 16 pair buffers, one mbarrier per
-// pair), so a CTA waits for one memory round trip, not one per pair.  Its 8 warps take two
-// pairs each for S = Q K^T (mma.sync m16n8k16 bf16, fp32 accumulate; tokens t <= p only, in
+// A (query, group) row is attended by a cluster of S CTAs; CTA `rank` takes the row's
+// regions [R*rank, R*rank + R) (the selection, or the window's regions in order).  Shapes:
+// S = 16, R = 32 for selections of up to 512 regions; S = 8, R = 10 for windows of up to 80
+// regions (a 512-token window touches at most 65), two CTAs per SM.  Every CTA issues all of
+// its K/V loads at once (R regions x 6 KiB, TMA with the 128-byte swizzle into R/2 pair
+// buffers, one mbarrier per pair), so a CTA waits for one memory round trip, not one per
+// pair.  Warp w takes pairs w and w + 8 (those that exist) for S = Q K^T (mma.sync
+// m16n8k16 bf16, fp32 accumulate; tokens t <= p only, and t > p - window for a window, in
 // log2 units); the CTA's row maximum M of each head goes through smem, every warp writes
-// P = 2^(S - M) in bf16 to one [16 heads][256 tokens] tile, and warp w then computes the
+// P = 2^(S - M) in bf16 to one [16 heads][8R tokens] tile, and warp w then computes the
 // output dims [24w, 24w + 24) of O = P V over all the CTA's tokens.  So no warp merges
-// another's O.  The CTA's (M, l, O) of head h goes to CTA h's inbox as one bulk copy that
-// completes on that CTA's inbox barrier; once its 16 rows are in, CTA r merges head r of
-// the row (O = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c) and writes the bf16 output and
-// the LSE.  No partials in global memory, no second kernel, no cluster barrier after the
-// start.
+// another's O.  The CTA's (M, l, O) of head h goes to CTA h mod S (slot h / S of its inbox
+// row for this CTA) as one bulk copy that completes on that CTA's inbox barrier; once its 16
+// rows are in, CTA r merges heads r, r + S, ... of the row (O = sum_c 2^(m_c - M) O_c /
+// sum_c 2^(m_c - M) l_c) and writes the bf16 output and the LSE.  No partials in global
+// memory, no second kernel, no cluster barrier after the start.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -31,39 +35,60 @@ using attn::kRegionBytes;
 using attn::Params;
 using attn::swz;
 
-constexpr int kSplits = 16;                    // CTAs per row (non-portable cluster size)
-constexpr int kRegionsPerCta = 32;
-constexpr int kPairs = kRegionsPerCta / 2;
 constexpr int kWarps = 8;
 constexpr int kThreads = 32 * kWarps;
-constexpr size_t kPairArea = (size_t)kPairs * kPairBytes;                 // 192 KiB
-constexpr int kInRow = kD + 4;                 // inbox row per source CTA: O [kD], m, l, pad
-constexpr size_t kInbox = (size_t)kSplits * kInRow * 4;                  // outside the pair area
-constexpr int kTokens = 8 * kRegionsPerCta;    // 256 tokens of a CTA
-constexpr int kPRow = 2 * kTokens + 16;        // P tile row (bytes): padded, conflict-free ldmatrix
-constexpr size_t kMl = (size_t)2 * kWarps * 16 * 4;                      // per-warp row maxima and sums
-constexpr size_t kPTile = (size_t)16 * kPRow;
+constexpr int kInRow = kD + 4;                 // inbox row per (source CTA, head slot): O [kD], m, l, pad
 constexpr int kDimsPerWarp = kD / kWarps;      // 24: three n8 tiles of O per warp
 static_assert(kDimsPerWarp == 24, "three n8 tiles of output dims per warp");
-static_assert(kInbox % 16 == 0 && kMl % 16 == 0, "the P tile stays 16-byte aligned");
-static_assert((kInRow * 4) % 16 == 0 && (size_t)16 * kInRow * 4 <= kPairArea,
-              "inbox rows are whole 16-byte bulk copies; the staged rows fit the pair area");
-static_assert((kPairs + 1) * 8 <= 256, "pair barriers and the inbox barrier fit their 256 bytes");
-constexpr size_t kSmemBytes = 1024 + kPairArea + kQBytes + 256 + kInbox + kMl + kPTile;
-constexpr int kMaxK = kSplits * kRegionsPerCta;                            // 512
 
-__global__ void __launch_bounds__(kThreads, 1)
+// The shape of a row's cluster: S CTAs of R regions each (R even, R <= 32, 16 % S == 0).
+template <int S, int R>
+struct Shape {
+    static constexpr int kSplits = S;
+    static constexpr int kRegionsPerCta = R;
+    static constexpr int kPairs = R / 2;
+    static constexpr int kOwn = (kPairs + kWarps - 1) / kWarps;             // pairs a warp owns, at most
+    static constexpr int kHeadsPerCta = kHeadsPerGroup / S;                 // heads a CTA merges
+    static constexpr size_t kPairArea = (size_t)kPairs * kPairBytes;
+    static constexpr size_t kInbox = (size_t)kHeadsPerGroup * kInRow * 4;   // 16 rows, outside the pair area
+    static constexpr int kTokens = 8 * R;
+    static constexpr int kPRow = 2 * kTokens + 16;                          // P tile row (bytes), padded
+    static constexpr size_t kMl = (size_t)2 * kWarps * 16 * 4;              // per-warp row maxima and sums
+    static constexpr size_t kPTile = (size_t)16 * kPRow;
+    static constexpr size_t kSmemBytes = 1024 + kPairArea + kQBytes + 256 + kInbox + kMl + kPTile;
+    static constexpr int kMaxK = S * R;
+    static_assert(R % 2 == 0 && R <= 32 && kHeadsPerGroup % S == 0, "shape");
+    static_assert(kInbox % 16 == 0 && kMl % 16 == 0, "the P tile stays 16-byte aligned");
+    static_assert((kInRow * 4) % 16 == 0 && (size_t)kHeadsPerGroup * kInRow * 4 <= kPairArea,
+                  "inbox rows are whole 16-byte bulk copies; the staged rows fit the pair area");
+    static_assert((kPairs + 1) * 8 <= 256, "pair barriers and the inbox barrier fit their 256 bytes");
+    // ldmatrix of 8 P rows: row r starts (r * kPRow / 4) mod 32 banks in; 16-byte chunks of the
+    // 8 rows fall in distinct 4-bank groups when that step is 4 or 12 modulo 32 (or 20, 28)
+    static_assert((kPRow / 4) % 8 == 4, "P rows land in distinct 16-byte bank groups");
+};
+using Decode = Shape<16, 32>;                  // selections of up to 512 regions
+using Window = Shape<8, 10>;                   // windows of up to 80 regions
+constexpr int kMaxK = Decode::kMaxK;           // 512
+
+// kWin: window mode (the row's regions are the window's, from the position) instead of a
+// selection (sel_idx, sel_count).
+template <int S, int R, int kMinBlocks, bool kWin>
+__global__ void __launch_bounds__(kThreads, kMinBlocks)
     sparse_attn_cluster_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                                const Params p)
 {
+    using Sh = Shape<S, R>;
+    constexpr int kSplits = S, kRegionsPerCta = R, kPairs = Sh::kPairs, kOwn = Sh::kOwn;
+    constexpr int kHpc = Sh::kHeadsPerCta, kPRow = Sh::kPRow;
+    constexpr size_t kPairArea = Sh::kPairArea;
     pdl_trigger();   // the next kernel may launch; it waits for this one itself
     pdl_wait();      // the previous kernel's results are visible from here on
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *qs = smem + kPairArea;
     uint64_t *bars = reinterpret_cast<uint64_t *>(qs + kQBytes);            // [kPairs]
-    float *inbox = reinterpret_cast<float *>(qs + kQBytes + 256);           // [kSplits][kInRow]
-    float *mw = inbox + kSplits * kInRow;                                   // [kWarps][16] row maxima
+    float *inbox = reinterpret_cast<float *>(qs + kQBytes + 256);           // [kSplits][kHpc][kInRow]
+    float *mw = inbox + kHeadsPerGroup * kInRow;                            // [kWarps][16] row maxima
     float *lw = mw + kWarps * 16;                                           // [kWarps][16] row sums
     uint8_t *ptile = reinterpret_cast<uint8_t *>(lw + kWarps * 16);         // P [16 heads][kPRow bytes]
     __shared__ int sh_y[kRegionsPerCta], sh_r[kRegionsPerCta], sh_v[kRegionsPerCta];   // per region of the CTA
@@ -85,32 +110,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int i = tid + u * kThreads;
         if (i < kQChunks) qv[u] = __ldg(reinterpret_cast<const uint4 *>(qsrc + (i / (kD / 8)) * kD + (i % (kD / 8)) * 8));
     }
-    auto reg_of = [&](int l) { return (l >> 1) * 16 + 2 * warp + (l & 1); };   // lane l < 4 -> region
+    // lane l < 2 kOwn of warp w -> region 2 (w + 8 (l / 2)) + l % 2 of the CTA (its owned pairs)
+    auto reg_of = [&](int l) { return (l >> 1) * 16 + 2 * warp + (l & 1); };
+    const bool reg_lane = lane < 2 * kOwn && reg_of(lane) < kRegionsPerCta;
     const int j0 = rank * kRegionsPerCta;
+    constexpr bool win = kWin;
     int rr_spec = -1;
-    if (lane < 4 && j0 + reg_of(lane) < p.k) rr_spec = p.sel_idx[(int64_t)row * p.k + j0 + reg_of(lane)];
+    if (!win && reg_lane && j0 + reg_of(lane) < p.k) rr_spec = p.sel_idx[(int64_t)row * p.k + j0 + reg_of(lane)];
     const int b = p.q_req ? p.q_req[qi] : qi;
     const int pos = p.q_pos[qi];
-    const int cnt_raw = p.sel_count[row];
-    const int cnt = min(max(cnt_raw, 0), p.k);
-    if (cnt != cnt_raw && rank == 0 && tid == 0) set_error(kErrAttnIndex);
+    // window mode: the regions holding tokens t_lo .. pos, tokens below t_lo masked
+    const int t_lo = win ? max(0, pos - p.window + 1) : 0;
+    int cnt;
+    const int newest = (pos >> 3) - (t_lo >> 3);                            // window mode: the token's region
+    if constexpr (win) {
+        cnt = pos < 0 ? 0 : min(newest + 1, p.k);
+        rr_spec = (t_lo >> 3) + j0 + reg_of(lane);
+    } else {
+        const int cnt_raw = p.sel_count[row];
+        cnt = min(max(cnt_raw, 0), p.k);
+        if (cnt != cnt_raw && rank == 0 && tid == 0) set_error(kErrAttnIndex);
+    }
     const int nr = max(0, min(kRegionsPerCta, cnt - j0));                   // regions of this CTA
     const bool bad_req = (b < 0 || b >= p.n_req || pos < 0);
     // Warp w owns pairs w and w + 8 (regions 2w, 2w+1, 2w+16, 2w+17 of the CTA): it sets up
     // their barriers, resolves their coordinates (sel_idx -> block_table, lanes 0..3) and
     // issues their TMA loads itself, so the 8 warps issue in parallel.
-    if (lane < 2) mbar_init(&bars[warp + 8 * lane], 1);
+    if (lane < kOwn && warp + 8 * lane < kPairs) mbar_init(&bars[warp + 8 * lane], 1);
     uint64_t *inbox_bar = &bars[kPairs];                                    // the 16 inbox rows landed
     if (tid == 0) {
         mbar_init(inbox_bar, 1);
-        mbar_arrive_expect_tx(inbox_bar, (unsigned)(kSplits * kInRow * 4));
+        mbar_arrive_expect_tx(inbox_bar, (unsigned)(kHeadsPerGroup * kInRow * 4));
     }
     fence_mbar_init();
     __syncwarp();
     // every CTA's inbox barrier is set up before any CTA copies into it: arrive now, wait
     // before the copies (long after every CTA arrived)
     cluster_arrive_relaxed();
-    if (lane < 4) {
+    if (reg_lane) {
         const int j = reg_of(lane);
         int y = 0, r = -1, v = 0;
         if (!bad_req && j < nr) {
@@ -131,15 +168,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         sh_y[j] = y;
         sh_r[j] = r;
         sh_v[j] = v;
-        if (warp == 0 && lane == 0) {
-            prefetch_tensormap(&tmap_k);
-            prefetch_tensormap(&tmap_v);
-        }
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmap_k);
+        prefetch_tensormap(&tmap_v);
     }
     __syncwarp();
-    if (lane < 2) {
+    if (lane < kOwn) {
         const int pr = warp + 8 * lane;
-        if (2 * pr < nr) {
+        if (pr < kPairs && 2 * pr < nr) {
             const int va = sh_v[2 * pr], vb = sh_v[2 * pr + 1];
             const unsigned bytes = (va ? 2u * kRegionBytes : 0u) + (vb ? 2u * kRegionBytes : 0u);
             if (bytes == 0) mbar_arrive(&bars[pr]);
@@ -147,7 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     __syncwarp();
-    if (lane < 4) {
+    if (reg_lane) {
         const int j = reg_of(lane), pr = j >> 1, half = j & 1;
         if (sh_v[j]) {
             uint8_t *dst = smem + (size_t)pr * kPairBytes;
@@ -177,10 +214,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int gq = lane >> 2, t = lane & 3;
     const int n_pairs = (nr + 1) / 2;
     // ---- S = Q K^T of this warp's pairs (warp, warp + 8), in log2 units, masked to t <= p
-    float s[2][2][4];
+    float s[kOwn][2][4];
     float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kOwn; ++i) {
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) s[i][nt][0] = s[i][nt][1] = s[i][nt][2] = s[i][nt][3] = -INFINITY;
         const int pr = warp + kWarps * i;
@@ -188,6 +225,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool landed = mbar_wait(&bars[pr], 0u);                     // false: error set, pair skipped
         if (lane == 0) sh_ok[pr] = landed ? 1 : 0;
         if (!landed) continue;
+        if constexpr (kWin) {
+            // the appended token (window decode with the append folded in): its K and V rows
+            // from new_k / new_v into this pair's tiles, whatever the load read for its slot,
+            // and into its cache slot for the steps to come (this group's rows; the CTA of the
+            // row's newest region writes them)
+            const int jn = newest - j0;
+            if (p.new_k && jn >= 0 && jn < kRegionsPerCta && (jn >> 1) == pr && sh_v[jn]) {
+                const int rt = pos & 7;                                     // the token's row in its region
+                const int64_t crow = (int64_t)sh_y[jn] + rt;                // and in the cache
+                const int64_t src = ((int64_t)qi * kG + p.g0 + g) * kD;
+                for (int c = lane; c < 2 * (kD / 8); c += 32) {             // 16-byte chunks: K, then V
+                    const int which = c / (kD / 8), cc = c % (kD / 8);
+                    const uint4 v = __ldg(reinterpret_cast<const uint4 *>((which ? p.new_v : p.new_k) + src + cc * 8));
+                    uint8_t *tile = smem + (size_t)pr * kPairBytes + (2 * which + (jn & 1)) * kRegionBytes;
+                    *reinterpret_cast<uint4 *>(tile + swz(rt, cc * 8)) = v;
+                    *reinterpret_cast<uint4 *>((which ? p.v_cache : p.k_cache) + crow * kD + cc * 8) = v;
+                }
+                __syncwarp();
+            }
+        }
         const int rr[2] = {sh_r[2 * pr], sh_r[2 * pr + 1]};
         const bool rv[2] = {sh_v[2 * pr] != 0, sh_v[2 * pr + 1] != 0};
         const uint32_t kt = smem_u32(smem + (size_t)pr * kPairBytes);
@@ -208,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int tok = 8 * rr[nt] + 2 * t + (e & 1);
-                const float v = (rv[nt] && tok <= pos) ? acc[e] * p.scale_log2 : -INFINITY;
+                const float v = (rv[nt] && tok <= pos && tok >= t_lo) ? acc[e] * p.scale_log2 : -INFINITY;
                 s[i][nt][e] = v;
                 mx[e >> 1] = fmaxf(mx[e >> 1], v);
             }
@@ -236,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- P = 2^(S - M): bf16 into the P tile (token column 16 pr + 8 nt + 2t), fp32 row sums
     float ps[2] = {0.0f, 0.0f};
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kOwn; ++i) {
         const int pr = warp + kWarps * i;
         if (pr >= n_pairs) continue;
 #pragma unroll
@@ -271,7 +328,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < 3; ++j) o[a2][j][0] = o[a2][j][1] = o[a2][j][2] = o[a2][j][3] = 0.0f;
     {
         // region j of the CTA takes part when its data landed and it is valid (bit j)
-        const unsigned use = __ballot_sync(0xffffffffu, (lane >> 1) < n_pairs && sh_v[lane] != 0 && sh_ok[lane >> 1] != 0);
+        const unsigned use = __ballot_sync(0xffffffffu, lane < kRegionsPerCta && (lane >> 1) < n_pairs &&
+                                                            sh_v[lane] != 0 && sh_ok[lane >> 1] != 0);
         const uint32_t pbase = smem_u32(ptile);
         const int ar = (lane & 7) + 8 * ((lane >> 3) & 1);
         const int r = lane & 7, reg = (lane >> 3) & 1, dsub = 8 * (lane >> 4);
@@ -301,9 +359,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 4; ++e) o[0][j][e] += o[1][j][e];
     }
-    // ---- this CTA's (M, l, O) of head h goes to CTA h's inbox row `rank`: the rows are staged
-    // in the (now free) pair area and sent as 16 bulk copies of kInRow floats, each completing
-    // on the destination's inbox barrier, so a CTA waits for its own 16 rows and nothing else
+    // ---- this CTA's (M, l, O) of head h goes to CTA h % S, inbox row (rank, h / S): the rows
+    // are staged in the (now free) pair area and sent as 16 bulk copies of kInRow floats, each
+    // completing on the destination's inbox barrier, so a CTA waits for its own 16 rows and
+    // nothing else
     __syncthreads();                                                        // every warp is done with P and V
     float *stage = reinterpret_cast<float *>(smem);                         // [16][kInRow]
 #pragma unroll
@@ -327,34 +386,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     cluster_wait();
     __syncthreads();
-    if (warp == 0 && lane < kSplits) {
-        bulk_copy_to_cta(inbox + rank * kInRow, stage + lane * kInRow, (unsigned)(kInRow * 4), inbox_bar,
-                         (unsigned)lane);
+    if (warp == 0 && lane < kHeadsPerGroup) {
+        bulk_copy_to_cta(inbox + (rank * kHpc + lane / kSplits) * kInRow, stage + lane * kInRow,
+                         (unsigned)(kInRow * 4), inbox_bar, (unsigned)(lane % kSplits));
         bulk_commit();
     }
     const bool inbox_ok = mbar_wait(inbox_bar, 0u);                         // false: error set
 
-    // ---- CTA `rank` merges head `rank` of the row from its inbox
-    const int hr = rank;
-    if (inbox_ok && tid < kD) {
+    // ---- CTA `rank` merges heads rank + S j (j < 16 / S) of the row from its inbox
+    for (int e = tid; inbox_ok && e < kHpc * kD; e += kThreads) {
+        const int j = e / kD, d = e % kD, hr = rank + kSplits * j;
         float M = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < kSplits; ++c) M = fmaxf(M, inbox[c * kInRow + kD]);
+        for (int c = 0; c < kSplits; ++c) M = fmaxf(M, inbox[(c * kHpc + j) * kInRow + kD]);
         const float Mref = (M == -INFINITY) ? 0.0f : M;
         float L = 0.0f, acc = 0.0f;
 #pragma unroll
         for (int c = 0; c < kSplits; ++c) {
-            const float wt = exp2f(inbox[c * kInRow + kD] - Mref);
-            L += wt * inbox[c * kInRow + kD + 1];
-            acc += wt * inbox[c * kInRow + tid];
+            const float *in = inbox + (c * kHpc + j) * kInRow;
+            const float wt = exp2f(in[kD] - Mref);
+            L += wt * in[kD + 1];
+            acc += wt * in[d];
         }
-        const int d = tid;
         const int64_t head = attn::out_head(p, qi, g, hr);
         p.out[head * kD + d] = __float2bfloat16_rn(L > 0.0f ? acc / L : 0.0f);
         if (p.lse && d == 0) p.lse[head] = (L > 0.0f) ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
     }
     // this CTA's copies have read their rows before its shared memory goes away
-    if (warp == 0 && lane < kSplits) bulk_wait_read_all();
+    if (warp == 0 && lane < kHeadsPerGroup) bulk_wait_read_all();
 }
 
 }  // namespace attnc

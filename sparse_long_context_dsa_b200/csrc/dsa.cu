@@ -264,49 +264,56 @@ AttnPlan attn_plan(int nq, int k, int sm_count, int ng = dsa::kG)
 }
 
 // The clustered attention kernel (splits merged in the kernel) serves rows that get one
-// 16-CTA cluster each with every cluster resident at once: k <= 512 and rows <= the number
-// of such clusters the device holds together (queried once per process; 0 when the kernel
-// cannot take the non-portable cluster size).
-int cluster_attn_capacity()
-{
-    static std::once_flag once;
-    static int capacity = 0;
-    std::call_once(once, [] {
-        auto *fn = dsa::attnc::sparse_attn_cluster_kernel;
-        if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsa::attnc::kSmemBytes) !=
-                cudaSuccess ||
-            cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
-            cudaGetLastError();
-            return;
-        }
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(dsa::attnc::kSplits, 1, 1);
-        cfg.blockDim = dim3(dsa::attnc::kThreads, 1, 1);
-        cfg.dynamicSmemBytes = dsa::attnc::kSmemBytes;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = dsa::attnc::kSplits;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
-            cudaGetLastError();
-            return;
-        }
-        capacity = n;
-    });
-    return capacity;
-}
-
-dsa_status_t attn_cluster_launch(const CUtensorMap &mk, const CUtensorMap &mv, const dsa::attn::Params &p, int nq,
-                                 dsa_stream_t stream)
-{
-    return launch_k("sparse_attn_cluster_kernel", dsa::attnc::sparse_attn_cluster_kernel,
-                    dim3(dsa::attnc::kSplits, (unsigned)(nq * ((int)1 << p.gshift))), dim3(dsa::attnc::kThreads),
-                    dsa::attnc::kSmemBytes, stream, (unsigned)dsa::attnc::kSplits, mk, mv, p);
-}
+// cluster each with every cluster resident at once: rows <= the number of such clusters the
+// device holds together (queried once per process and shape; 0 when the kernel cannot take
+// its cluster size).  Selections (k <= 512): 16-CTA clusters, one CTA per SM; windows of up
+// to 80 regions: 8-CTA clusters, two CTAs per SM.
+template <class Sh, int kMinBlocks, bool kWin>
+struct ClusterAttn {
+    static constexpr auto fn =
+        dsa::attnc::sparse_attn_cluster_kernel<Sh::kSplits, Sh::kRegionsPerCta, kMinBlocks, kWin>;
+    static int capacity()
+    {
+        static std::once_flag once;
+        static int cap = 0;
+        std::call_once(once, [] {
+            if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Sh::kSmemBytes) !=
+                    cudaSuccess ||
+                cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+                cudaGetLastError();
+                return;
+            }
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(Sh::kSplits, 1, 1);
+            cfg.blockDim = dim3(dsa::attnc::kThreads, 1, 1);
+            cfg.dynamicSmemBytes = Sh::kSmemBytes;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = Sh::kSplits;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
+                cudaGetLastError();
+                return;
+            }
+            cap = n;
+        });
+        return cap;
+    }
+    static dsa_status_t launch(const CUtensorMap &mk, const CUtensorMap &mv, const dsa::attn::Params &p, int nq,
+                               dsa_stream_t stream)
+    {
+        return launch_k("sparse_attn_cluster_kernel", fn,
+                        dim3(Sh::kSplits, (unsigned)(nq * ((int)1 << p.gshift))), dim3(dsa::attnc::kThreads),
+                        Sh::kSmemBytes, stream, (unsigned)Sh::kSplits, mk, mv, p);
+    }
+};
+using DecodeAttn = ClusterAttn<dsa::attnc::Decode, 1, false>;
+using WindowAttn = ClusterAttn<dsa::attnc::Window, 2, true>;
+int cluster_attn_capacity() { return DecodeAttn::capacity(); }
 
 // Regions a window of `window` tokens can touch: its first token may sit anywhere in a region.
 int window_regions(int window) { return window / dsa::kRegion + 2; }
@@ -317,7 +324,7 @@ dsa_status_t attn_common(const void *q, const void *k_cache, const void *v_cache
                          const int32_t *block_table, int max_pages, const int32_t *q_req, int n_req,
                          const int32_t *q_pos, int nq, const int32_t *sel_idx, const int32_t *sel_count, int k,
                          void *out, float *lse, void *ws, size_t ws_bytes, dsa_stream_t stream, int window = 0,
-                         int g0 = 0, int ng = dsa::kG)
+                         int g0 = 0, int ng = dsa::kG, const void *new_k = nullptr, const void *new_v = nullptr)
 {
     DSA_REQUIRE(nq >= 0, "nq must be >= 0");
     DSA_REQUIRE(window > 0 || (k >= 1 && k <= DSA_MAX_TOPK), "k out of [1, DSA_MAX_TOPK]");
@@ -339,13 +346,16 @@ dsa_status_t attn_common(const void *q, const void *k_cache, const void *v_cache
     // of the 4-group call)
     const bool clustered =
         window == 0 && k <= dsa::attnc::kMaxK && (int64_t)nq * dsa::kG <= cluster_attn_capacity();
+    // window layers: one 8-CTA cluster per row while every row's cluster is resident at once
+    const bool clustered_window = window > 0 && ng == dsa::kG && k <= dsa::attnc::Window::kMaxK &&
+                                  (int64_t)nq * dsa::kG <= WindowAttn::capacity();
     // prefill chunks: 8 neighbouring queries per CTA share one stream of their selections' union
     const bool shared = window == 0 && !clustered && ng == dsa::kG && q_req != nullptr && nq >= kSharedMinQueries &&
                         k <= dsa::attntc::kMaxK &&
                         (int64_t)max_pages * dsa::kPage / dsa::kRegion <= (int64_t)dsa::attntc::kMaxWords * 32;
     const AttnPlan plan = attn_plan(nq, k, sms, ng);
     const size_t need_ws = plan.ws + (shared ? round_up((size_t)nq * dsa::kG, 256) : 0);
-    if (need_ws > 0 && !clustered) {
+    if (need_ws > 0 && !clustered && !clustered_window) {
         if (!ws || ws_bytes < need_ws || !aligned(ws, 256))
             return fail(DSA_ERR_WORKSPACE, "attention workspace too small or not 256-byte aligned (need " +
                                                std::to_string(need_ws) + " bytes)");
@@ -378,8 +388,16 @@ dsa_status_t attn_common(const void *q, const void *k_cache, const void *v_cache
     p.scale_log2 = dsa::attn::kLog2e / sqrtf((float)dsa::kD);
     p.gshift = ng == 4 ? 2 : ng == 2 ? 1 : 0;
     p.g0 = g0;
+    if (new_k) {                       // the append folded in: only the clustered window kernel takes it
+        if (!clustered_window) return fail(DSA_ERR_UNSUPPORTED, "window append without the clustered kernel");
+        p.new_k = static_cast<const __nv_bfloat16 *>(new_k);
+        p.new_v = static_cast<const __nv_bfloat16 *>(new_v);
+        p.k_cache = static_cast<__nv_bfloat16 *>(const_cast<void *>(k_cache));
+        p.v_cache = static_cast<__nv_bfloat16 *>(const_cast<void *>(v_cache));
+    }
 
-    if (clustered) return attn_cluster_launch(mk, mv, p, nq, stream);
+    if (clustered) return DecodeAttn::launch(mk, mv, p, nq, stream);
+    if (clustered_window) return WindowAttn::launch(mk, mv, p, nq, stream);
     if (shared) {
         // 8 neighbouring queries of one request with a small union: tcgen05 tiles of 128 rows
         p.row_shared = static_cast<uint8_t *>(ws) + plan.ws;
@@ -1036,6 +1054,23 @@ dsa_status_t dsa_indexer_frontend(const void *hidden, int hid, int n_tok, const 
                     dim3(dsa::fe::kThreads), dsa::fe::kSmemBytes, stream, 0, map_h, map_w, p);
 }
 
+namespace {
+// The window call runs on the clustered kernel (splits merged in the kernel, one launch).
+bool window_clustered(int nq, int window)
+{
+    return window_regions(window) <= dsa::attnc::Window::kMaxK && (int64_t)nq * dsa::kG <= WindowAttn::capacity();
+}
+}  // namespace
+
+int dsa_window_decode_launches(int nq, int window)
+{
+    if (nq <= 0 || window < 1) return 0;
+    if (window_clustered(nq, window)) return 1;                            // the append folded in
+    int sms = 0;
+    if (device_info(sms) != DSA_OK) sms = 148;
+    return 1 + (attn_plan(nq, window_regions(window), sms).n_splits > 1 ? 2 : 1);
+}
+
 size_t dsa_window_attn_workspace_size(int nq, int window)
 {
     if (nq <= 0 || window < 1) return 0;
@@ -1052,6 +1087,30 @@ dsa_status_t dsa_window_attn(const void *q, const void *k_cache, const void *v_c
     DSA_REQUIRE(window >= 1 && window <= (1 << 20), "window out of [1, 2^20]");
     return attn_common(q, k_cache, v_cache, n_pages, block_table, max_pages, q_req, q_req ? n_req : nq, q_pos, nq,
                        nullptr, nullptr, window_regions(window), out, lse, ws, ws_bytes, stream, window);
+}
+
+dsa_status_t dsa_window_decode(void *k_cache, void *v_cache, int64_t n_pages, const int32_t *block_table,
+                               int max_pages, int n_req, const int32_t *q_req, const int32_t *q_pos, int nq,
+                               const void *new_k, const void *new_v, const void *q, int window, void *out,
+                               float *lse, void *ws, size_t ws_bytes, dsa_stream_t stream)
+{
+    DSA_REQUIRE(window >= 1 && window <= (1 << 20), "window out of [1, 2^20]");
+    DSA_REQUIRE(nq >= 0, "nq must be >= 0");
+    if (nq == 0) return DSA_OK;
+    DSA_REQUIRE(new_k && new_v, "NULL pointer");
+    DSA_REQUIRE(aligned(new_k, 16) && aligned(new_v, 16), "new rows must be 16-byte aligned");
+    DSA_REACHABLE({new_k, "new_k"}, {new_v, "new_v"});
+    if (!window_clustered(nq, window)) {
+        // the two calls it stands for
+        dsa_status_t st = dsa_kv_append(k_cache, v_cache, n_pages, block_table, max_pages, n_req, q_req, q_pos, nq,
+                                        new_k, new_v, stream);
+        if (st != DSA_OK) return st;
+        return dsa_window_attn(q, k_cache, v_cache, n_pages, block_table, max_pages, n_req, q_req, q_pos, nq, window,
+                               out, lse, ws, ws_bytes, stream);
+    }
+    return attn_common(q, k_cache, v_cache, n_pages, block_table, max_pages, q_req, q_req ? n_req : nq, q_pos, nq,
+                       nullptr, nullptr, window_regions(window), out, lse, ws, ws_bytes, stream, window, 0, dsa::kG,
+                       new_k, new_v);
 }
 
 dsa_status_t dsa_kv_append(void *k_cache, void *v_cache, int64_t n_pages, const int32_t *block_table, int max_pages,

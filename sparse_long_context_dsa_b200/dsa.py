@@ -50,6 +50,7 @@ _SIG = {
     "dsa_topk_regions_noalloc": (ctypes.c_int, [_F32P, ctypes.c_int64, _I32P, ctypes.c_int, ctypes.c_int, _I32P,
                                                 _I32P, _VP]),
     "dsa_decode_select_workspace_size": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int64, ctypes.c_int]),
+    "dsa_window_decode_launches": (ctypes.c_int, [ctypes.c_int, ctypes.c_int]),
     "dsa_decode_select": (ctypes.c_int, [_VP, _F32P, _I32P, _I32P, ctypes.c_int, _U8P, _F32P, ctypes.c_int64,
                                          _I64P, ctypes.c_int, _F32P, ctypes.c_int64, ctypes.c_uint32, ctypes.c_int,
                                          _I32P, _I32P, _VP, ctypes.c_size_t, _VP]),
@@ -79,6 +80,9 @@ _SIG = {
                                             _VP]),
     "dsa_window_attn": (ctypes.c_int, [_VP, _VP, _VP, ctypes.c_int64, _I32P, ctypes.c_int, ctypes.c_int, _I32P,
                                        _I32P, ctypes.c_int, ctypes.c_int, _VP, _F32P, _VP, ctypes.c_size_t, _VP]),
+    "dsa_window_decode": (ctypes.c_int, [_VP, _VP, ctypes.c_int64, _I32P, ctypes.c_int, ctypes.c_int, _I32P, _I32P,
+                                         ctypes.c_int, _VP, _VP, _VP, ctypes.c_int, _VP, _F32P, _VP,
+                                         ctypes.c_size_t, _VP]),
 }
 
 
@@ -436,6 +440,32 @@ def window_attn(q, k_cache, v_cache, block_table, q_pos, window=512, q_req=None,
     _check(lib().dsa_window_attn(_p(q), _p(k_cache), _p(v_cache), k_cache.shape[0], _p(block_table),
                                  block_table.shape[1], block_table.shape[0], _p(q_req), _p(q_pos), nq, int(window),
                                  _p(out), _p(lse), _p(ws), nbytes, _stream()))
+    return out
+
+
+def window_decode(q, k_cache, v_cache, block_table, q_pos, new_k, new_v, window=512, q_req=None, out=None,
+                  lse=None):
+    """One window-layer decode step: kv_append(new_k, new_v at q_pos), then window_attn over the
+    window ending at the appended token (one launch where the clustered kernel serves it).
+    The queries must be distinct requests.  Returns out bf16 [nq][64][192]."""
+    nq = q.shape[0]
+    _need(q, torch.bfloat16, (nq, HQ, D), "q")
+    _cache_args(k_cache, v_cache, block_table)
+    _need(q_pos, torch.int32, (nq,), "q_pos")
+    _need(new_k, torch.bfloat16, (nq, G, D), "new_k")
+    _need(new_v, torch.bfloat16, (nq, G, D), "new_v")
+    if q_req is not None:
+        _need(q_req, torch.int32, (nq,), "q_req")
+    if out is None:
+        out = torch.empty((nq, HQ, D), dtype=torch.bfloat16, device=q.device)
+    _need(out, torch.bfloat16, (nq, HQ, D), "out")
+    if lse is not None:
+        _need(lse, torch.float32, (nq, HQ), "lse")
+    nbytes = lib().dsa_window_attn_workspace_size(nq, window)
+    ws = _workspace(nbytes, q.device)
+    _check(lib().dsa_window_decode(_p(k_cache), _p(v_cache), k_cache.shape[0], _p(block_table), block_table.shape[1],
+                                   block_table.shape[0], _p(q_req), _p(q_pos), nq, _p(new_k), _p(new_v), _p(q),
+                                   int(window), _p(out), _p(lse), _p(ws), nbytes, _stream()))
     return out
 
 

@@ -244,8 +244,8 @@ def ring_block_table(batch: int, max_pages: int, ring_pages: int = 8, device="cu
 
 class WindowDecodeStep:
     """One decode step of a window layer for a batch of requests, one token each: the new
-    token's K/V into the request's ring (dsa_kv_append), then GQA over its last `window`
-    tokens (dsa_window_attn).  Buffers are allocated once (capturable in a CUDA graph).
+    token's K/V into the request's ring, then GQA over its last `window` tokens, in one call
+    (dsa_window_decode).  Buffers are allocated once (capturable in a CUDA graph).
 
     k_ring/v_ring: bf16 [B * ring_pages][4][64][192]; block_table: ring_block_table(...).
     Per-step inputs: q bf16 [B][64][192], new_k/new_v bf16 [B][4][192], q_pos int32 [B]."""
@@ -272,8 +272,8 @@ class WindowDecodeStep:
     def run(self):
         L, p, st = dsa.lib(), dsa._p, dsa._stream()
         kr, bt = self.k_ring, self.block_table
-        dsa._check(L.dsa_kv_append(p(kr), p(self.v_ring), kr.shape[0], p(bt), bt.shape[1], self.B, None,
-                                   p(self.q_pos), self.B, p(self.new_k), p(self.new_v), st))
-        dsa._check(L.dsa_window_attn(p(self.q), p(kr), p(self.v_ring), kr.shape[0], p(bt), bt.shape[1], self.B,
-                                     None, p(self.q_pos), self.B, self.window, p(self.out), None, p(self.ws),
-                                     self.ws_n, st))
+        # the append and the window attention in one call (one kernel where the clustered
+        # window kernel serves the batch)
+        dsa._check(L.dsa_window_decode(p(kr), p(self.v_ring), kr.shape[0], p(bt), bt.shape[1], self.B, None,
+                                       p(self.q_pos), self.B, p(self.new_k), p(self.new_v), p(self.q), self.window,
+                                       p(self.out), None, p(self.ws), self.ws_n, st))

@@ -6,7 +6,8 @@ write (dsa_kv_append) against the oracle's window attention.
 modulo of the position.  Bar as for the sparse attention: bf16 outputs within 2e-2
 absolute + 1e-2 relative of the oracle's, lse within 1e-3.  Cases: decode batches on a
 linear paged cache (windows shorter than, equal to and longer than the context, window
-sizes 1 .. 4,096, a 1M-token context), many queries of one request (the per-row kernel
+sizes 1 .. 4,096, a 1M-token context; up to 624 tokens the clustered kernel with its in-kernel
+merge, beyond it the split kernel and the combine), many queries of one request (the per-row kernel
 without splits, a prefill chunk's shape), a ring of 8 pages per request filled token by
 token through dsa_kv_append across several wraps, and an append beyond the block table
 (flagged, nothing written).
@@ -43,6 +44,8 @@ def check(q, kc, vc, bt, q_req, q_pos, window, out, lse):
     ([1500, 3000], 100),
     ([9000, 5000, 40000], 4096),
     ([1 << 20], 512),
+    ([5000, 700, 2000], 600),            # 77 regions: the clustered kernel's last CTAs partly filled
+    ([3000, 640, 625], 624),             # 80 regions: every region slot of the clustered kernel
 ])
 def test_decode_batch_matches_oracle(lengths, window):
     d = W.decode_batch(lengths, seed=sum(lengths) % 1000 + window, device="cuda", permute=True)
@@ -121,3 +124,48 @@ def test_append_beyond_the_block_table_is_flagged_and_skipped():
     with pytest.raises(dsa.DsaError):
         dsa.check_device()
     assert not kr.any() and not vr.any()
+
+
+@pytest.mark.parametrize("window", [512, 4096])
+def test_window_decode_equals_append_then_attention(window):
+    # dsa_window_decode (the append folded into the clustered kernel at 512 tokens; the two
+    # calls at 4,096) against kv_append + window_attn on a copy of the same rings, step by
+    # step: outputs, LSE and ring contents bit for bit, and the oracle on some steps
+    lengths = [700, 1030, 60, 4200]
+    steps = 12
+    d = W.decode_batch([L + steps for L in lengths], seed=57 + window, device="cuda", permute=True)
+    B = len(lengths)
+    ring_pages = (window + PAGE - 1) // PAGE + 1
+    max_pages = d["block_table"].shape[1]
+    cyc = (torch.arange(B, dtype=torch.int32)[:, None] * ring_pages +
+           torch.arange(max_pages, dtype=torch.int32)[None] % ring_pages).to("cuda")
+    bt = d["block_table"]
+
+    def token_rows(cache, b, t):
+        t = torch.as_tensor(t, device="cuda")
+        return cache[bt[b, t // PAGE].long(), :, t % PAGE, :]
+
+    kr = torch.zeros((B * ring_pages, G, PAGE, 192), dtype=torch.bfloat16, device="cuda")
+    vr = torch.zeros_like(kr)
+    slots = ring_pages * PAGE
+    for b, L in enumerate(lengths):
+        pos = torch.arange(max(0, L - slots), L, dtype=torch.int32, device="cuda")
+        dsa.kv_append(kr, vr, cyc, pos, token_rows(d["k_cache"], b, pos.long()).contiguous(),
+                      token_rows(d["v_cache"], b, pos.long()).contiguous(), q_req=torch.full_like(pos, b))
+    kr2, vr2 = kr.clone(), vr.clone()
+    dsa.check_device()
+    for step in range(steps):
+        pos = torch.tensor([L + step for L in lengths], dtype=torch.int32, device="cuda")
+        newk = torch.stack([token_rows(d["k_cache"], b, int(pos[b])) for b in range(B)]).contiguous()
+        newv = torch.stack([token_rows(d["v_cache"], b, int(pos[b])) for b in range(B)]).contiguous()
+        lse = torch.empty((B, 64), dtype=torch.float32, device="cuda")
+        out = dsa.window_decode(d["q"], kr, vr, cyc, pos, newk, newv, window, lse=lse)
+        dsa.kv_append(kr2, vr2, cyc, pos, newk, newv)
+        lse2 = torch.empty((B, 64), dtype=torch.float32, device="cuda")
+        out2 = dsa.window_attn(d["q"], kr2, vr2, cyc, pos, window, lse=lse2)
+        dsa.check_device()
+        assert torch.equal(out, out2) and torch.equal(lse, lse2)
+        assert torch.equal(kr, kr2) and torch.equal(vr, vr2)
+        if step in (0, steps - 1):
+            check(d["q"], d["k_cache"], d["v_cache"], bt, np.arange(B), pos.cpu().numpy(), window, out, lse)
+    assert dsa.lib().dsa_window_decode_launches(B, window) == (1 if window == 512 else 3)
