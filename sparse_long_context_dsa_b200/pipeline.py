@@ -252,12 +252,23 @@ class WindowDecodeStep:
 
     def __init__(self, k_ring, v_ring, block_table, window: int = 512):
         dev = k_ring.device
-        self.B = block_table.shape[0]
+        self.B = B = block_table.shape[0]
         self.k_ring, self.v_ring, self.block_table, self.window = k_ring, v_ring, block_table, window
-        self.q = torch.zeros((self.B, HQ, D), dtype=torch.bfloat16, device=dev)
-        self.new_k = torch.zeros((self.B, G, D), dtype=torch.bfloat16, device=dev)
-        self.new_v = torch.zeros_like(self.new_k)
-        self.q_pos = torch.zeros((self.B,), dtype=torch.int32, device=dev)
+        # per-step inputs in one arena (q, new_k, new_v, q_pos): one copy stages a step
+        shapes = (((B, HQ, D), torch.bfloat16), ((B, G, D), torch.bfloat16), ((B, G, D), torch.bfloat16),
+                  ((B,), torch.int32))
+        size = 0
+        for shape, dt in shapes:
+            n = 1
+            for x in shape:
+                n *= x
+            size += (n * torch.tensor([], dtype=dt).element_size() + 255) // 256 * 256
+        self.arena = torch.zeros(size, dtype=torch.uint8, device=dev)
+        off = 0
+        self.q, off = _carve(self.arena, off, (B, HQ, D), torch.bfloat16)
+        self.new_k, off = _carve(self.arena, off, (B, G, D), torch.bfloat16)
+        self.new_v, off = _carve(self.arena, off, (B, G, D), torch.bfloat16)
+        self.q_pos, off = _carve(self.arena, off, (B,), torch.int32)
         self.out = torch.empty((self.B, HQ, D), dtype=torch.bfloat16, device=dev)
         L = dsa.lib()
         self.ws_n = L.dsa_window_attn_workspace_size(self.B, window)
@@ -269,11 +280,24 @@ class WindowDecodeStep:
         self.new_v.copy_(new_v, non_blocking=True)
         self.q_pos.copy_(q_pos, non_blocking=True)
 
-    def run(self):
+    def stage(self, host_arena):
+        """Copies the step's inputs from a pinned host image of `arena` with one library
+        kernel, in the stream's kernel chain."""
+        dsa.copy(self.arena, host_arena)
+
+    def run(self, out=None):
+        """Launches the step (capturable).  out: bf16 [B][64][192] on the device (default
+        `self.out`) or in pinned host memory, which the kernel then writes directly."""
+        if out is None:
+            out = self.out
+        elif tuple(out.shape) != tuple(self.out.shape) or out.dtype != self.out.dtype or not (
+                out.is_cuda or out.is_pinned()):
+            raise ValueError("out must be bf16 [B][64][192], on the device or in pinned host memory")
         L, p, st = dsa.lib(), dsa._p, dsa._stream()
         kr, bt = self.k_ring, self.block_table
         # the append and the window attention in one call (one kernel where the clustered
         # window kernel serves the batch)
         dsa._check(L.dsa_window_decode(p(kr), p(self.v_ring), kr.shape[0], p(bt), bt.shape[1], self.B, None,
                                        p(self.q_pos), self.B, p(self.new_k), p(self.new_v), p(self.q), self.window,
-                                       p(self.out), None, p(self.ws), self.ws_n, st))
+                                       p(out), None, p(self.ws), self.ws_n, st))
+        return out

@@ -169,3 +169,34 @@ def test_window_decode_equals_append_then_attention(window):
         if step in (0, steps - 1):
             check(d["q"], d["k_cache"], d["v_cache"], bt, np.arange(B), pos.cpu().numpy(), window, out, lse)
     assert dsa.lib().dsa_window_decode_launches(B, window) == (1 if window == 512 else 3)
+
+
+def test_window_step_runner_from_pinned_host_memory():
+    # pipeline.WindowDecodeStep: inputs staged from a pinned host image of its arena by the
+    # library's copy kernel, the output written into pinned host memory by the attention
+    # kernel; equal to dsa.window_decode on a copy of the same rings
+    from sparse_long_context_dsa_b200 import pipeline
+    B, ring_pages, window = 3, 9, 512
+    g = torch.Generator(device="cuda")
+    g.manual_seed(7)
+    bt = pipeline.ring_block_table(B, 20000, ring_pages, "cuda")
+    kr = torch.randn((B * ring_pages, G, PAGE, 192), generator=g, device="cuda").to(torch.bfloat16)
+    vr = torch.randn(kr.shape, generator=g, device="cuda").to(torch.bfloat16)
+    kr2, vr2 = kr.clone(), vr.clone()
+    st = pipeline.WindowDecodeStep(kr, vr, bt, window)
+    q = torch.randn((B, 64, 192), generator=g, device="cuda").to(torch.bfloat16)
+    nk = torch.randn((B, G, 192), generator=g, device="cuda").to(torch.bfloat16)
+    nv = torch.randn((B, G, 192), generator=g, device="cuda").to(torch.bfloat16)
+    pos = torch.tensor([1000, 70000, 511], dtype=torch.int32, device="cuda")
+    st.load(q, nk, nv, pos)
+    host = st.arena.cpu().pin_memory()
+    st.arena.zero_()
+    out_host = torch.empty((B, 64, 192), dtype=torch.bfloat16).pin_memory()
+    st.stage(host)
+    st.run(out_host)
+    torch.cuda.synchronize()
+    dsa.check_device()
+    want = dsa.window_decode(q, kr2, vr2, bt, pos, nk, nv, window)
+    dsa.check_device()
+    assert torch.equal(out_host, want.cpu())
+    assert torch.equal(kr, kr2) and torch.equal(vr, vr2)
