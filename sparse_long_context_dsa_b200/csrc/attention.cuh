@@ -108,6 +108,12 @@ __global__ void __launch_bounds__(kThreads, 2)
                        const Params p)
 {
     pdl_trigger();   // the next kernel may launch; it waits for this one itself
+    // the tensor maps are kernel parameters: their descriptors are fetched while the previous
+    // kernel finishes, not in front of the first loads
+    if (threadIdx.x == 0) {
+        prefetch_tensormap(&tmap_k);
+        prefetch_tensormap(&tmap_v);
+    }
     pdl_wait();      // the previous kernel's results are visible from here on
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -208,10 +214,6 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     // prologue: resolve this warp's first region coordinates (sel_idx -> block_table) while
     // the Q tile loads, then issue the first pairs' TMA before building the Q fragments
-    if (lane == 0) {
-        prefetch_tensormap(&tmap_k);
-        prefetch_tensormap(&tmap_v);
-    }
     if (my_pairs > 0) refill(0);
     // Q tile [16 heads][192] into smem with the same swizzled layout as the K/V tiles
     const __nv_bfloat16 *qsrc = p.q + q_head(p, qi, g) * kD;

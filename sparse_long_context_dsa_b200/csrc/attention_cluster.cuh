@@ -82,6 +82,12 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks)
     constexpr int kHpc = Sh::kHeadsPerCta, kPRow = Sh::kPRow;
     constexpr size_t kPairArea = Sh::kPairArea;
     pdl_trigger();   // the next kernel may launch; it waits for this one itself
+    // the tensor maps are kernel parameters (no earlier kernel writes them): their descriptors
+    // are fetched while the previous kernel finishes, not in front of the first loads
+    if (threadIdx.x == 0) {
+        prefetch_tensormap(&tmap_k);
+        prefetch_tensormap(&tmap_v);
+    }
     pdl_wait();      // the previous kernel's results are visible from here on
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -168,10 +174,6 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks)
         sh_y[j] = y;
         sh_r[j] = r;
         sh_v[j] = v;
-    }
-    if (warp == 0 && lane == 0) {
-        prefetch_tensormap(&tmap_k);
-        prefetch_tensormap(&tmap_v);
     }
     __syncwarp();
     if (lane < kOwn) {

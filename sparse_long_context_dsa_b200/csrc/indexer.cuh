@@ -174,6 +174,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     scan_kernel(const __grid_constant__ CUtensorMap tmap, const Params p)
 {
     pdl_trigger();   // the next kernel may launch; it waits for this one itself
+    // the tensor map is a kernel parameter: its descriptor is fetched while the previous
+    // kernel finishes, not in front of the first stage's loads
+    if (threadIdx.x == 32 * kSlabs) prefetch_tensormap(&tmap);
     pdl_wait();      // the previous kernel's results are visible from here on
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -197,7 +200,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     if (warp == kSlabs) {
         // ---------------- producer warp: lane 0 issues the TMA loads of the summaries; every
         // lane copies 4 of the stage's 128 fp32 scales into smem asynchronously
-        if (lane == 0) prefetch_tensormap(&tmap);
         const uint64_t pol = l2_evict_first_policy();     // the summaries are read once per query
         int it = 0;
         constexpr int kScalesPerLane = kSlabs * kChunk / 32;      // 4 at 32 regions per stage
