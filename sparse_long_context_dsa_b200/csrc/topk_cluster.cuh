@@ -97,6 +97,32 @@ __device__ __forceinline__ uint32_t block_scan_incl(uint32_t v, uint32_t *ws)
 }
 
 
+// The same inclusive block scan with one barrier: every thread adds up the totals of the
+// warps before its own (NT / 32 broadcast reads) instead of waiting for one warp to scan
+// them.  *total receives the block's sum.  The caller separates consecutive uses of `ws`
+// with a barrier (the next writes to ws must not overtake this scan's reads).
+template <int NT>
+__device__ __forceinline__ uint32_t block_scan_incl1(uint32_t v, uint32_t *ws, uint32_t *total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t x = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += x;
+    }
+    if (lane == 31) ws[warp] = v;
+    __syncthreads();
+    uint32_t add = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w) {
+        const uint32_t x = ws[w];
+        add += w < warp ? x : 0u;
+        tot += x;
+    }
+    *total = tot;
+    return v + add;
+}
+
 // Block-wide min and max (every thread gets both); `ws` needs 2 * kWarps entries.
 template <typename T>
 __device__ __forceinline__ void block_minmax(T &mn, T &mx, T *ws)
@@ -431,7 +457,9 @@ __device__ bool dense_exact_threshold(const uint64_t (&cv)[R], uint32_t d0, uint
     const uint4 q4 = reinterpret_cast<const uint4 *>(h)[kThreads - 1 - tid];
     const uint32_t c[4] = {q4.w, q4.z, q4.y, q4.x};
     const uint32_t s = c[0] + c[1] + c[2] + c[3];
-    const uint32_t incl = block_scan_incl<kThreads>(s, scan_ws);
+    uint32_t all;
+    const uint32_t incl = block_scan_incl1<kThreads>(s, scan_ws, &all);   // the barrier below separates ws uses
+    (void)all;
     const uint32_t excl = incl - s;
     if (excl < m && incl >= m) {
         uint32_t run = excl;
@@ -618,7 +646,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t cs = 0;
 #pragma unroll
                 for (int u = 0; u < kDPer; ++u) cs += (d0 + u < total && cv[u] >= T) ? 1u : 0u;
-                const uint32_t sincl = block_scan_incl<kThreads>(cs, scan_ws);
+                uint32_t n_sel;
+                const uint32_t sincl = block_scan_incl1<kThreads>(cs, scan_ws, &n_sel);   // last use of ws here
+                (void)n_sel;
                 uint32_t opos = sincl - cs;
 #pragma unroll
                 for (int u = 0; u < kDPer; ++u) {
@@ -679,8 +709,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (mvalid(u) && mk[u] >= Lk && c * 32 >= lo && c * 32 < hi_ld) take |= 1u << u;
                 }
                 const uint32_t nc = __popc(take);
-                const uint32_t cincl = block_scan_incl<kThreads>(nc, scan_ws);
-                const int n_cc = (int)scan_ws[kWarps - 1];
+                uint32_t n_cc_u;
+                const uint32_t cincl = block_scan_incl1<kThreads>(nc, scan_ws, &n_cc_u);   // barrier below
+                const int n_cc = (int)n_cc_u;
                 {
                     uint32_t pos = cincl - nc;
 #pragma unroll
@@ -718,8 +749,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncthreads();
                 // region-order offsets: thread t takes staged chunks [2t, 2t + 2)
                 uint32_t cc0 = 2 * tid < nst ? ccnt[2 * tid] : 0u, cc1 = 2 * tid + 1 < nst ? ccnt[2 * tid + 1] : 0u;
-                const uint32_t oincl = block_scan_incl<kThreads>(cc0 + cc1, scan_ws);
-                const uint32_t cta_total = scan_ws[kWarps - 1];
+                uint32_t cta_total;
+                const uint32_t oincl = block_scan_incl1<kThreads>(cc0 + cc1, scan_ws, &cta_total);   // barrier below
                 if (2 * tid < nst) ccnt[2 * tid] = oincl - cc0 - cc1;
                 if (2 * tid + 1 < nst) ccnt[2 * tid + 1] = oincl - cc1;
                 __syncthreads();
