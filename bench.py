@@ -44,7 +44,7 @@ N_LAYERS = 4
 KERNELS_PER_STEP = 4      # compress, scan (+ chunk maxima), cluster top-k, clustered attention
 # DRAM bytes (read + write) of one scan launch on this workload, from one ncu capture of the
 # current scan kernel (dram__bytes_read.sum + dram__bytes_write.sum); None once the kernel changes
-SCAN_TRAFFIC_BYTES = 136_397_056 + 3_877_888
+SCAN_TRAFFIC_BYTES = 136_384_000 + 3_348_480
 PREFILL_CTX, PREFILL_NEW = 262144, 2048
 PREFILL_KERNELS = 6       # compress, quantize, GEMM, top-k, shared-selection attention, per-row attention
 # DRAM bytes (read + write) of one gemm_scores_kernel launch on the prefill workload, from one
