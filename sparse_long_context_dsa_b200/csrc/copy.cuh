@@ -17,10 +17,20 @@ __global__ void __launch_bounds__(256) copy_kernel(uint8_t *__restrict__ dst, co
     const bool vec = ((reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(src)) & 15) == 0;
     size_t done = 0;
     if (vec) {
+        // up to four 16-byte loads of a thread in flight before its stores: from pinned host
+        // memory every dependent load would cost a bus round trip of its own
         const size_t n16 = bytes / 16;
         const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
         uint4 *d4 = reinterpret_cast<uint4 *>(dst);
-        for (size_t i = tid; i < n16; i += nt) d4[i] = s4[i];
+        for (size_t i0 = tid; i0 < n16; i0 += 4 * nt) {
+            uint4 r[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (i0 + u * nt < n16) r[u] = s4[i0 + u * nt];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (i0 + u * nt < n16) d4[i0 + u * nt] = r[u];
+        }
         done = n16 * 16;
     }
     for (size_t i = done + tid; i < bytes; i += nt) dst[i] = src[i];

@@ -11,7 +11,7 @@ from sparse_long_context_dsa_b200 import workloads as W
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("n", [1, 15, 16, 4096 + 7, 49664, 1 << 22])
+@pytest.mark.parametrize("n", [1, 15, 16, 4096 + 7, 49664, 1 << 22, (1 << 26) + 37])
 def test_copy_between_pinned_host_and_device(n):
     rng = np.random.default_rng(n)
     host = torch.from_numpy(rng.integers(0, 256, n, dtype=np.uint8)).pin_memory()
