@@ -85,6 +85,12 @@ int dsa_version(void);
  * The pointer stays valid until the next call on this thread. */
 const char *dsa_last_error(void);
 
+/* The same message copied into a caller buffer, for callers that keep no pointer into the
+ * library: writes at most len - 1 bytes of it and a terminating NUL into buf (nothing when
+ * len is 0; buf may then be NULL) and returns the message's full length, so a return value
+ * >= len means it was cut short. */
+size_t dsa_get_last_error(char *buf, size_t len);
+
 /* Synchronises `stream`, then reads and clears the error word that kernels of this
  * library set on the current device.  Returns DSA_OK or DSA_ERR_DEVICE (message via
  * dsa_last_error), or DSA_ERR_CUDA if the synchronisation itself failed. */

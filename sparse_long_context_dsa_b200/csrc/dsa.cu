@@ -654,6 +654,17 @@ int dsa_version(void) { return DSA_VERSION; }
 
 const char *dsa_last_error(void) { return g_last_error.c_str(); }
 
+size_t dsa_get_last_error(char *buf, size_t len)
+{
+    const size_t n = g_last_error.size();
+    if (buf && len > 0) {
+        const size_t m = std::min(n, len - 1);
+        std::memcpy(buf, g_last_error.data(), m);
+        buf[m] = '\0';
+    }
+    return n;
+}
+
 dsa_status_t dsa_check_device(dsa_stream_t stream)
 {
     DSA_CUDA(cudaStreamSynchronize(stream), "cudaStreamSynchronize");

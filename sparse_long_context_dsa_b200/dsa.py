@@ -37,6 +37,7 @@ _VP, _I32P, _I64P, _F32P, _U8P = (ctypes.c_void_p,) * 5
 _SIG = {
     "dsa_version": (ctypes.c_int, []),
     "dsa_last_error": (ctypes.c_char_p, []),
+    "dsa_get_last_error": (ctypes.c_size_t, [ctypes.c_char_p, ctypes.c_size_t]),
     "dsa_check_device": (ctypes.c_int, [_VP]),
     "dsa_compress_regions": (ctypes.c_int, [_VP, ctypes.c_int64, ctypes.c_int64, _I64P, _I64P, ctypes.c_int,
                                             _U8P, _F32P, ctypes.c_int64, _VP]),

@@ -61,6 +61,19 @@ def test_bad_arguments_are_rejected_on_the_host(lib, call):
     assert lib.dsa_last_error().decode()
 
 
+def test_last_error_copied_into_a_caller_buffer(lib):
+    assert lib.dsa_topk_regions(None, 16, None, 1, 0, None, None, None, 0, None) == dsa.ERR_INVALID_ARG
+    msg = lib.dsa_last_error()
+    n = len(msg)
+    assert n > 8
+    assert lib.dsa_get_last_error(None, 0) == n                   # length only, nothing written
+    buf = ctypes.create_string_buffer(b"x" * 8)                   # 9 bytes with its own NUL
+    assert lib.dsa_get_last_error(buf, 5) == n                    # cut short: 4 bytes and a NUL
+    assert buf.raw[:5] == msg[:4] + b"\0" and buf.raw[5:8] == b"xxx"
+    big = ctypes.create_string_buffer(n + 1)
+    assert lib.dsa_get_last_error(big, n + 1) == n and big.value == msg
+
+
 def test_zero_sized_calls_are_noops(lib):
     assert lib.dsa_compress_regions(None, 1024, 8, None, None, 0, None, None, 1, None) == dsa.OK
     assert lib.dsa_topk_regions(None, 16, None, 0, 8, None, None, None, 0, None) == dsa.OK
