@@ -47,9 +47,10 @@ KERNELS_PER_STEP = 4      # compress, scan (+ chunk maxima), cluster top-k, clus
 SCAN_TRAFFIC_BYTES = 136_384_000 + 3_348_480
 PREFILL_CTX, PREFILL_NEW = 262144, 2048
 PREFILL_KERNELS = 6       # compress, quantize, GEMM, top-k, shared-selection attention, per-row attention
-# DRAM bytes (read + write) of one gemm_scores_kernel launch on the prefill workload, from one
-# ncu capture of the current kernel; None once the kernel changes
-GEMM_TRAFFIC_BYTES = 139_658_240 + 1_020_275_000
+# DRAM bytes (read + write) of one gemm_scores_kernel launch on the prefill workload: None, the
+# kernel changed (its roles now drain their last copies and MMAs before exiting) after the last
+# capture that counted them (139,658,240 read + 1,020,275,000 written)
+GEMM_TRAFFIC_BYTES = None
 
 
 def parse():
