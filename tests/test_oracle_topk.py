@@ -100,3 +100,22 @@ def test_k_at_least_region_count_selects_everything():
     idx, cnt = check(s, [39 * 8 + 2], 512)
     assert np.all(cnt == 40)
     assert list(idx[0, 2, :40]) == list(range(40))
+
+
+def test_property_random_small_rows():
+    """Random tiny cases (hypothesis): rows of up to 40 regions drawn from a handful of values
+    (with -0.0 beside +0.0), any query position inside the row, any k: the oracle equals the
+    sort-based brute force."""
+    hypothesis = pytest.importorskip("hypothesis")
+    st = hypothesis.strategies
+
+    @hypothesis.settings(max_examples=150, deadline=None, derandomize=True)
+    @hypothesis.given(st.integers(1, 40), st.integers(1, 45), st.data())
+    def run(ld, k, data):
+        vals = st.sampled_from([0.0, -0.0, 0.5, 1.0, 1.0 + 2.0 ** -23, 3.0])
+        s = np.array(data.draw(st.lists(vals, min_size=G * ld, max_size=G * ld)), dtype=np.float32)
+        s = s.reshape(1, G, ld)
+        pos = data.draw(st.integers(0, 8 * ld - 1))
+        check(s, [pos], k)
+
+    run()
